@@ -1,0 +1,297 @@
+"""fp64 restatement of the Tail-Replay hot path (test infrastructure only).
+
+Citations name the page and the section/equation on it:
+  RN = "Tail-Replay reading notes" (cc.laoqi.cc page), GS = "Tail-Replay
+  technical summary" (gist.science page).
+
+Readings where the pages are silent (the GDN layer internals are never given;
+RN section 2.3 says no model dimensions are to be made up from Eq. (1)):
+  * state layout M = S^T, [d_k][d_v]; readout o_t = scale * M_t^T q_t after the
+    update of token t;
+  * per LA layer: RMSNorm (eps 1e-6, gain ones unless given) -> one projection
+    x_hat W_in^T = [q | k | v | a_alpha | a_beta] (no bias, no short
+    convolution, no activation on v) -> q and k L2-normalised per head
+    (x / sqrt(sum x^2 + 1e-6)) -> alpha = exp(-softplus(a_alpha)),
+    beta = sigmoid(a_beta) -> Eq. (1) scan -> x <- x + o W_o^T; the FFN sublayer
+    is left out, so the next LA layer reads the residual after the attention
+    sublayer;
+  * bf16 cast points of the boundary (``emulate_casts``): the projection
+    operands x_hat and o and the stored q, k, v are rounded to bf16
+    (round-to-nearest-even); everything else stays fp64 here.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import List, Optional, Sequence, Tuple
+
+import numpy as np
+
+from . import _build
+
+_lib = None
+
+
+def _scan_lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        f = lib.oracle_gdn_scan_f64
+        P = ctypes.c_void_p
+        f.argtypes = [ctypes.c_int64] * 4 + [P] * 7 + [ctypes.c_double, P, P, ctypes.c_int]
+        f.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    """Exact fp64 values of an array-like (bf16/fp32 torch tensors included)."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return x.detach().to("cpu", torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(x, dtype=np.float64)
+
+
+# --------------------------------------------------------------------------- a0
+def tail_len(m: int, r_num: int, r_den: int) -> int:
+    """k = ceil(r * m) with r = r_num / r_den, in integers, clamped to [0, m].
+
+    RN section 2.1, symbol table: k = ceil(r m) replayed tokens, r in {0.05, 0.10}
+    in the experiments.  Integer arithmetic avoids 0.07 * 100 -> 7.000000000000001
+    rounding up to 8.
+    """
+    m, r_num, r_den = int(m), int(r_num), int(r_den)
+    if r_den <= 0:
+        raise ValueError("r_den must be positive")
+    if m <= 0 or r_num <= 0:
+        return 0
+    k = -((-r_num * m) // r_den)
+    return max(0, min(m, k))
+
+
+def tail_rows(m: int, k: int) -> Tuple[int, int]:
+    """0-based half-open row range of the tail h_{m-k+1..m} (RN section 2.2, step 2)."""
+    if not 0 <= k <= m:
+        raise ValueError("need 0 <= k <= m")
+    return m - k, m
+
+
+# ------------------------------------------------------------------- cast points
+def bf16_round(x) -> np.ndarray:
+    """Round fp64 values to the nearest bf16 value (ties to even), returned as fp64.
+
+    Goes through fp32 first (round-to-nearest) and then keeps the top 16 bits of
+    the fp32 pattern with round-to-nearest-even, as a device fp32 -> bf16
+    conversion does.
+    """
+    f = np.ascontiguousarray(_f64(x), dtype=np.float64).astype(np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    r = ((u + 0x7FFF + lsb) >> 16) << 16
+    nan = np.isnan(f)
+    out = r.astype(np.uint32).view(np.float32).astype(np.float64)
+    if nan.any():
+        out[nan] = np.nan
+    return out
+
+
+# ------------------------------------------------------------------------- a2
+def rmsnorm(x, gain=None, eps: float = 1e-6) -> np.ndarray:
+    """x_hat = x / sqrt(mean_j x_j^2 + eps) * gain, per row.
+
+    Not on the pages (layer internals are never given); the RMSNorm in front of
+    each LA layer is the reading stated in the module docstring.
+    """
+    x = _f64(x)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    y = x / np.sqrt(ms + eps)
+    if gain is not None:
+        y = y * _f64(gain)
+    return y
+
+
+# ------------------------------------------------------------------------- a3
+def in_projection(x_hat, W_in, n_heads: int, d_k: int, d_v: int):
+    """[q | k | v | a_alpha | a_beta] = x_hat W_in^T, split per head.
+
+    W_in is [2 H d_k + H d_v + 2 H, D] (output features x input features).
+    Reading (pages silent): one bias-free projection, no short convolution.
+    """
+    x_hat = _f64(x_hat)
+    W = _f64(W_in)
+    y = x_hat @ W.T
+    T = y.shape[0]
+    H = n_heads
+    o = 0
+    q = y[:, o:o + H * d_k].reshape(T, H, d_k); o += H * d_k
+    k = y[:, o:o + H * d_k].reshape(T, H, d_k); o += H * d_k
+    v = y[:, o:o + H * d_v].reshape(T, H, d_v); o += H * d_v
+    a_alpha = y[:, o:o + H]; o += H
+    a_beta = y[:, o:o + H]; o += H
+    assert o == W.shape[0]
+    return q, k, v, a_alpha, a_beta
+
+
+# ------------------------------------------------------------------------- a4
+def l2_normalize(x, eps: float = 1e-6) -> np.ndarray:
+    """x / sqrt(sum x^2 + eps) along the last axis.
+
+    RN section 2.3 (after Eq. (1)): unit-norm keys with beta in [0, 2] make
+    I - beta k k^T non-expansive; q is normalised the same way (reading).
+    """
+    x = _f64(x)
+    return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps)
+
+
+def gates(a_alpha, a_beta):
+    """log alpha = -softplus(a_alpha), beta = sigmoid(a_beta).
+
+    RN section 2.3 only fixes alpha in (0, 1]; the exp(-softplus) form gives
+    alpha in (0, 1) and beta in (0, 1), inside the [0, 2] range of the
+    non-expansive condition.  softplus(a) = max(a, 0) + log1p(exp(-|a|)) is the
+    overflow-free form of log(1 + e^a).
+    """
+    a = _f64(a_alpha)
+    b = _f64(a_beta)
+    softplus = np.maximum(a, 0.0) + np.log1p(np.exp(-np.abs(a)))
+    log_alpha = -softplus
+    beta = np.where(b >= 0, 1.0 / (1.0 + np.exp(-np.abs(b))),
+                    np.exp(-np.abs(b)) / (1.0 + np.exp(-np.abs(b))))
+    return log_alpha, beta
+
+
+# ------------------------------------------------------------------------- a5
+def gdn_scan(q, k, v, log_alpha, beta, cu_seqlens, S0=None, scale: float = 1.0,
+             want_o: bool = True, normalize_qk: bool = False, norm_eps: float = 1e-6,
+             n_threads: Optional[int] = None):
+    """Eq. (1) of RN section 2.3, token by token from S0 (zero when None).
+
+    Returns (o [T, H, d_v] or None, S_final [N, H, d_k, d_v]) in the M = S^T
+    layout.  With ``normalize_qk`` q and k are first L2-normalised per head
+    (step a4).  The recurrence itself runs in the plain C file eq1_scan.c.
+    """
+    q = _f64(q) if q is not None else None
+    k = _f64(k)
+    if normalize_qk:
+        k = l2_normalize(k, norm_eps)
+        if q is not None:
+            q = l2_normalize(q, norm_eps)
+    v = _f64(v)
+    la = _f64(log_alpha)
+    b = _f64(beta)
+    cu = np.ascontiguousarray(_f64(cu_seqlens).astype(np.int64))
+    T, H, dk = k.shape
+    dv = v.shape[2]
+    N = cu.shape[0] - 1
+    if cu[0] != 0 or cu[-1] != T or np.any(np.diff(cu) < 0):
+        raise ValueError("bad cu_seqlens")
+    S = np.zeros((N, H, dk, dv), dtype=np.float64)
+    o = np.zeros((T, H, dv), dtype=np.float64) if want_o else None
+    if want_o and q is None:
+        raise ValueError("q is needed for the readout")
+    qc = np.ascontiguousarray(q) if q is not None else None
+    kc, vc = np.ascontiguousarray(k), np.ascontiguousarray(v)
+    lac, bc = np.ascontiguousarray(la), np.ascontiguousarray(b)
+    S0c = np.ascontiguousarray(_f64(S0)) if S0 is not None else None
+    if S0c is not None and S0c.shape != S.shape:
+        raise ValueError("S0 shape")
+    if n_threads is None:
+        n_threads = os.cpu_count() or 1
+    P = lambda a: a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+    rc = _scan_lib().oracle_gdn_scan_f64(N, H, dk, dv, P(cu), P(qc), P(kc), P(vc), P(lac), P(bc),
+                                         P(S0c), float(scale), P(o), P(S), int(n_threads))
+    if rc != 0:
+        raise RuntimeError("oracle scan rejected its arguments")
+    return o, S
+
+
+# ------------------------------------------------------------------------- a6
+def out_projection_residual(x, o, W_o) -> np.ndarray:
+    """x + o W_o^T with o flattened to [T, H d_v] and W_o [D, H d_v].
+
+    Reading (pages silent on the layer internals): the LA layer's attention
+    sublayer adds its output projection to the residual stream.
+    """
+    x = _f64(x)
+    o = _f64(o)
+    T = o.shape[0]
+    return x + o.reshape(T, -1) @ _f64(W_o).T
+
+
+# ---------------------------------------------------------------------- a2..a6
+def replay_layer(x, W_in, W_o, rms_gain, cu_seqlens, n_heads: int, d_k: int, d_v: int,
+                 want_output: bool = True, emulate_casts: bool = True,
+                 rms_eps: float = 1e-6, norm_eps: float = 1e-6, n_threads=None):
+    """One LA layer of the replay from a zero state: returns (S_hat, x_next or None)."""
+    x = _f64(x)
+    cast = bf16_round if emulate_casts else (lambda a: a)
+    x_hat = cast(rmsnorm(x, rms_gain, rms_eps))
+    q, k, v, a_alpha, a_beta = in_projection(x_hat, W_in, n_heads, d_k, d_v)
+    q = cast(l2_normalize(q, norm_eps))
+    k = cast(l2_normalize(k, norm_eps))
+    v = cast(v)
+    log_alpha, beta = gates(a_alpha, a_beta)
+    o, S_hat = gdn_scan(q, k, v, log_alpha, beta, cu_seqlens, None, 1.0, want_o=want_output,
+                        n_threads=n_threads)
+    x_next = None
+    if want_output:
+        x_next = out_projection_residual(x, cast(o), W_o)
+    return S_hat, x_next
+
+
+def replay_group(h_tail, cu_seqlens, layers: Sequence, n_heads: int, d_k: int, d_v: int,
+                 emulate_casts: bool = True, skip_last_output: bool = False,
+                 rms_eps: float = 1e-6, norm_eps: float = 1e-6, n_threads=None):
+    """Replay one group's LA layers over the packed tails (RN section 2.2 steps 2-3).
+
+    Every LA state of the group starts at zero at the tail start (step 2, GS
+    "Key Mechanisms": initialise the replay state to zero); the tail hiddens
+    h_{m-k+1..m} go through the group's LA layers in order (step 3), each layer
+    feeding the next.  ``layers`` is a sequence of objects with W_in, W_o and
+    rms_gain.  Returns (S_hat [L, N, H, d_k, d_v], x_out [T, D] or None).
+    With ``skip_last_output`` the last layer's readout and output projection are
+    not computed (its output is not used to rebuild any state; RN section 2.5
+    makes the same argument for the tail FFN).
+    """
+    x = _f64(h_tail)
+    S_all = []
+    L = len(layers)
+    for i, lw in enumerate(layers):
+        want = not (skip_last_output and i == L - 1)
+        S_hat, x_next = replay_layer(x, lw.W_in, lw.W_o, lw.rms_gain, cu_seqlens, n_heads, d_k, d_v,
+                                     want_output=want, emulate_casts=emulate_casts,
+                                     rms_eps=rms_eps, norm_eps=norm_eps, n_threads=n_threads)
+        S_all.append(S_hat)
+        x = x_next
+    return np.stack(S_all, 0), x
+
+
+# ------------------------------------------------------------------------- a8
+def state_error(S, S_hat):
+    """||S - S_hat||_F / ||S||_F per d_k x d_v matrix and over the whole tensor.
+
+    RN section 2.3 defines E_m = S_m - S_hat_m; the relative Frobenius norm is
+    the measure the workloads ask for.  Reading for ||S|| = 0: the error is 0
+    when S_hat is 0 too, else +inf.
+    """
+    S = _f64(S)
+    Sh = _f64(S_hat)
+    dk, dv = S.shape[-2:]
+    d = (S - Sh).reshape(-1, dk * dv)
+    s = S.reshape(-1, dk * dv)
+    num = np.sum(d * d, axis=1)
+    den = np.sum(s * s, axis=1)
+
+    def ratio(n, dd):
+        with np.errstate(divide="ignore", invalid="ignore"):
+            r = np.sqrt(n / dd)
+        r = np.where(dd > 0, r, np.where(n > 0, np.inf, 0.0))
+        return r
+
+    per = ratio(num, den)
+    tot = float(ratio(np.array([num.sum()]), np.array([den.sum()]))[0])
+    return per, tot

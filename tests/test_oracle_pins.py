@@ -1,0 +1,368 @@
+"""Pins for the fp64 oracle: facts the pages and the mathematics fix, checked on the CPU.
+
+Each test states the passage or the mathematical fact it checks.  None of them
+re-types the oracle's own formula: they use explicit transition matrices in the
+paper's own (d_v x d_k) layout, closed forms, invariants, special cases, and an
+independent bf16 conversion.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(20260901)
+
+
+def _unit(x):
+    return x / np.linalg.norm(x, axis=-1, keepdims=True)
+
+
+def _rand_scan(T, H, dk, dv, alpha_lo=0.5, alpha_hi=1.0, seed=0):
+    r = np.random.default_rng(seed)
+    q = _unit(r.standard_normal((T, H, dk)))
+    k = _unit(r.standard_normal((T, H, dk)))
+    v = r.standard_normal((T, H, dv))
+    la = np.log(r.uniform(alpha_lo, alpha_hi, (T, H)))
+    b = 1.0 / (1.0 + np.exp(-r.standard_normal((T, H))))
+    return q, k, v, la, b
+
+
+def _explicit_T(alpha, beta, k):
+    """T_i = alpha_i (I - beta_i k_i k_i^T) as an explicit d_k x d_k matrix (Eq. (1))."""
+    return alpha * (np.eye(k.shape[0]) - beta * np.outer(k, k))
+
+
+# --------------------------------------------------------------- a0: tail length
+def test_worked_example_tail_positions():
+    """Reading notes section 2.2 worked example: m = 10,000, r = 5% -> positions 9,501..10,000."""
+    g = json.load(open(os.path.join(GOLDEN, "worked_example_tail.json")))
+    k = oracle.tail_len(g["m"], g["r_num"], g["r_den"])
+    assert k == g["k"]
+    a, b = oracle.tail_rows(g["m"], k)
+    assert (a + 1, b) == (g["first_position_1based"], g["last_position_1based"])
+
+
+@pytest.mark.parametrize("m,rn,rd,k", [
+    (4096, 5, 100, 205),        # ceil(204.8)
+    (32768, 5, 100, 1639),      # ceil(1638.4)
+    (32768, 10, 100, 3277),     # ceil(3276.8)
+    (131072, 20, 100, 26215),   # ceil(26214.4)
+    (100, 7, 100, 7),           # exact: 0.07 * 100 in floating point is 7.000000000000001
+    (4096, 1, 100, 41),         # ceil(40.96)
+    (10, 0, 1, 0),              # r = 0: the Zero-only baseline
+    (0, 5, 100, 0),
+    (1000, 1, 1, 1000),         # r = 1: full prefill
+    (1000, 3, 2, 1000),         # r > 1 is clamped to m
+])
+def test_tail_len_ceiling(m, rn, rd, k):
+    """Symbol table of reading notes section 2.1: k = ceil(r m)."""
+    assert oracle.tail_len(m, rn, rd) == k
+    # the ceiling: k-1 < r m <= k (in rationals), unless clamped
+    if 0 < k < m:
+        assert (k - 1) * rd < rn * m <= k * rd
+
+
+# ------------------------------------------------------------ a5: Eq. (1) scan
+@pytest.mark.parametrize("dk,dv,T", [(2, 3, 7), (5, 2, 12), (8, 8, 10), (3, 1, 5)])
+def test_eq1_brute_force_paper_layout(dk, dv, T):
+    """Eq. (1) (reading notes section 2.3) with explicit d_k x d_k matrices T_i in the
+    paper's own S in R^{d_v x d_k} layout, where the key-space operator acts from the
+    right (the remark after Eq. (1)): S_i = S_{i-1} T_i + beta_i v_i k_i^T, o_i = S_i q_i.
+    The oracle keeps M = S^T, so M must equal S^T and o must match."""
+    H = 2
+    q, k, v, la, b = _rand_scan(T, H, dk, dv, seed=dk * 100 + dv)
+    S0 = rng.standard_normal((1, H, dk, dv)) * 0.3
+    o, S = oracle.gdn_scan(q, k, v, la, b, [0, T], S0=S0)
+    for h in range(H):
+        Sp = S0[0, h].T.copy()                      # d_v x d_k
+        for t in range(T):
+            Ti = _explicit_T(math.exp(la[t, h]), b[t, h], k[t, h])
+            Sp = Sp @ Ti + b[t, h] * np.outer(v[t, h], k[t, h])
+            np.testing.assert_allclose(o[t, h], Sp @ q[t, h], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(S[0, h], Sp.T, rtol=1e-12, atol=1e-12)
+
+
+def test_error_identity_first_layer():
+    """Reading notes section 2.3: E_m = S_m - S_hat_m = (T_m ... T_{a+1}) S_a with a = m - k
+    (the notes' own derivation; exact for a single recurrence).  Explicit products."""
+    m, k, H, dk, dv = 40, 9, 2, 6, 4
+    a = m - k
+    q, kk, v, la, b = _rand_scan(m, H, dk, dv, alpha_lo=0.7, seed=3)
+    _, S_m = oracle.gdn_scan(q, kk, v, la, b, [0, m], want_o=False)
+    _, S_a = oracle.gdn_scan(q[:a], kk[:a], v[:a], la[:a], b[:a], [0, a], want_o=False)
+    _, S_hat = oracle.gdn_scan(q[a:], kk[a:], v[a:], la[a:], b[a:], [0, k], want_o=False)
+    for h in range(H):
+        P = np.eye(dk)
+        for i in range(a, m):                       # T_m ... T_{a+1}: later factors on the left
+            P = _explicit_T(math.exp(la[i, h]), b[i, h], kk[i, h]) @ P
+        E = S_m[0, h] - S_hat[0, h]
+        np.testing.assert_allclose(E, P @ S_a[0, h], rtol=1e-10, atol=1e-13)
+
+
+def test_contraction_bound():
+    """Reading notes section 2.3: with unit keys and beta in [0, 2], ||I - beta k k^T||_2 <= 1,
+    so ||E_m||_F <= (prod_{i>a} alpha_i) ||S_a||_F (the rho^k bound with per-step alphas)."""
+    m, k, H, dk, dv = 300, 30, 4, 16, 8
+    a = m - k
+    q, kk, v, la, b = _rand_scan(m, H, dk, dv, alpha_lo=0.85, seed=4)
+    b = b * 2.0 * 0.999                               # beta in (0, 2)
+    _, S_m = oracle.gdn_scan(q, kk, v, la, b, [0, m], want_o=False)
+    _, S_a = oracle.gdn_scan(q[:a], kk[:a], v[:a], la[:a], b[:a], [0, a], want_o=False)
+    _, S_hat = oracle.gdn_scan(q[a:], kk[a:], v[a:], la[a:], b[a:], [0, k], want_o=False)
+    for h in range(H):
+        E = np.linalg.norm(S_m[0, h] - S_hat[0, h])
+        bound = math.exp(la[a:, h].sum()) * np.linalg.norm(S_a[0, h])
+        assert E <= bound * (1 + 1e-9) + 1e-300
+
+
+def test_zero_tail_is_zero_state():
+    """k = 0 is the Zero-only baseline (reading notes section 3.1): S_hat = 0."""
+    q, k, v, la, b = _rand_scan(0, 3, 4, 5)
+    o, S = oracle.gdn_scan(q, k, v, la, b, [0, 0])
+    assert S.shape == (1, 3, 4, 5) and not S.any()
+
+
+def test_full_replay_equals_prefill():
+    """k = m replays every position: S_hat_m is the full-prefill S_m (reading notes 3.1, 'Full')."""
+    m = 57
+    assert oracle.tail_len(m, 1, 1) == m
+    q, k, v, la, b = _rand_scan(m, 2, 8, 8, seed=5)
+    a, e = oracle.tail_rows(m, m)
+    o1, S1 = oracle.gdn_scan(q, k, v, la, b, [0, m])
+    o2, S2 = oracle.gdn_scan(q[a:e], k[a:e], v[a:e], la[a:e], b[a:e], [0, e - a])
+    assert np.array_equal(S1, S2) and np.array_equal(o1, o2)
+
+
+def test_identity_transition():
+    """alpha = 1, beta = 0: T_i = I and the write term vanishes, so S stays S0 and o_t = S0^T q_t."""
+    T, H, dk, dv = 9, 2, 6, 5
+    q, k, v, la, b = _rand_scan(T, H, dk, dv, seed=6)
+    S0 = rng.standard_normal((1, H, dk, dv))
+    o, S = oracle.gdn_scan(q, k, v, np.zeros((T, H)), np.zeros((T, H)), [0, T], S0=S0)
+    np.testing.assert_array_equal(S, S0)
+    np.testing.assert_allclose(o, np.einsum("hdj,thd->thj", S0[0], q), rtol=1e-13, atol=1e-13)
+
+
+def test_delta_rule_recall():
+    """beta_t = 1 with a unit key: M_t^T k_t = alpha (M - k k^T M)^T k + v = v exactly (for any
+    alpha), the delta rule's write.  Read out with q_t = k_t."""
+    T, H, dk, dv = 20, 2, 8, 6
+    _, k, v, la, _ = _rand_scan(T, H, dk, dv, alpha_lo=0.3, seed=7)
+    o, _ = oracle.gdn_scan(k, k, v, la, np.ones((T, H)), [0, T])
+    np.testing.assert_allclose(o, v, rtol=1e-12, atol=1e-12)
+
+
+def test_orthonormal_keys_accumulate():
+    """alpha = beta = 1 with orthonormal keys: each write lands in a fresh direction, so
+    M_n = sum_j k_j v_j^T (closed form)."""
+    dk, dv, n, H = 8, 5, 6, 1
+    Qm, _ = np.linalg.qr(rng.standard_normal((dk, dk)))
+    k = Qm[:, :n].T.reshape(n, 1, dk)
+    v = rng.standard_normal((n, H, dv))
+    _, S = oracle.gdn_scan(k, k, v, np.zeros((n, H)), np.ones((n, H)), [0, n], want_o=False)
+    np.testing.assert_allclose(S[0, 0], sum(np.outer(k[j, 0], v[j, 0]) for j in range(n)),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_scalar_recurrence_closed_form():
+    """d_k = d_v = 1 reduces Eq. (1) to m_i = a_i m_{i-1} + b_i with a_i = alpha_i (1 - beta_i k_i^2),
+    b_i = beta_i k_i v_i, whose solution is m_n = sum_j (prod_{i>j} a_i) b_j + (prod a_i) m_0."""
+    T = 30
+    r = np.random.default_rng(8)
+    k = r.uniform(-1.2, 1.2, (T, 1, 1))
+    v = r.standard_normal((T, 1, 1))
+    la = np.log(r.uniform(0.6, 1.0, (T, 1)))
+    b = r.uniform(0.0, 1.0, (T, 1))
+    m0 = np.array([[[[0.7]]]])
+    _, S = oracle.gdn_scan(k, k, v, la, b, [0, T], S0=m0, want_o=False)
+    a = np.exp(la[:, 0]) * (1 - b[:, 0] * k[:, 0, 0] ** 2)
+    bb = b[:, 0] * k[:, 0, 0] * v[:, 0, 0]
+    expect = np.prod(a) * 0.7 + sum(np.prod(a[j + 1:]) * bb[j] for j in range(T))
+    assert abs(S[0, 0, 0, 0] - expect) < 1e-12
+
+
+def test_split_composition_and_varlen():
+    """Scanning x[:t] and then x[t:] from the state reached equals scanning x; packing two
+    sequences with cu_seqlens equals two separate calls (both exactly, in the oracle)."""
+    T, H, dk, dv = 45, 3, 8, 4
+    q, k, v, la, b = _rand_scan(T, H, dk, dv, seed=9)
+    o, S = oracle.gdn_scan(q, k, v, la, b, [0, T])
+    t = 17
+    o1, S1 = oracle.gdn_scan(q[:t], k[:t], v[:t], la[:t], b[:t], [0, t])
+    o2, S2 = oracle.gdn_scan(q[t:], k[t:], v[t:], la[t:], b[t:], [0, T - t], S0=S1)
+    assert np.array_equal(S2, S) and np.array_equal(np.concatenate([o1, o2]), o)
+    op, Sp = oracle.gdn_scan(q, k, v, la, b, [0, t, T])
+    assert np.array_equal(Sp[0], S1[0]) and np.array_equal(op[:t], o1)
+    _, Sb = oracle.gdn_scan(q[t:], k[t:], v[t:], la[t:], b[t:], [0, T - t])
+    assert np.array_equal(Sp[1], Sb[0])
+
+
+def test_scan_normalize_flag_matches_prenormalised():
+    T, H, d = 12, 2, 8
+    r = np.random.default_rng(10)
+    q, k = r.standard_normal((T, H, d)) * 3, r.standard_normal((T, H, d)) * 0.2
+    _, _, v, la, b = _rand_scan(T, H, d, d, seed=10)
+    o1, S1 = oracle.gdn_scan(q, k, v, la, b, [0, T], normalize_qk=True, norm_eps=0.0)
+    o2, S2 = oracle.gdn_scan(_unit(q), _unit(k), v, la, b, [0, T])
+    np.testing.assert_allclose(S1, S2, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-14)
+
+
+# -------------------------------------------------------- a2-a4, a6 layer pieces
+def test_bf16_round_matches_independent_conversion():
+    """The oracle's bit-level bf16 rounding agrees with torch's own fp32 -> bf16 conversion,
+    including ties to even: 1 + 2^-8 is halfway between 1 and 1 + 2^-7 and rounds to 1."""
+    x = np.concatenate([rng.standard_normal(10000) * 10.0 ** rng.integers(-20, 20, 10000),
+                        [1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 0.0, -0.0, 65504.0]])
+    x32 = x.astype(np.float32)
+    ref = torch.from_numpy(x32).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(oracle.bf16_round(x32), ref)
+    assert oracle.bf16_round(np.array([1 + 2 ** -8]))[0] == 1.0
+    assert oracle.bf16_round(np.array([1 + 3 * 2 ** -8]))[0] == 1 + 2 ** -6
+
+
+def test_rmsnorm_special_cases():
+    """x = +-c has mean square c^2, so x_hat = +-c / sqrt(c^2 + eps) * g; scale invariance."""
+    D = 64
+    c = 3.0
+    x = np.where(np.arange(D) % 2 == 0, c, -c)[None]
+    g = rng.uniform(0.5, 1.5, D)
+    y = oracle.rmsnorm(x, g, eps=1e-6)
+    np.testing.assert_allclose(y[0], np.sign(x[0]) * c / math.sqrt(c * c + 1e-6) * g, rtol=1e-14)
+    z = rng.standard_normal((5, D))
+    np.testing.assert_allclose(oracle.rmsnorm(z * 1e3, eps=0.0), oracle.rmsnorm(z, eps=0.0), rtol=1e-12)
+    np.testing.assert_allclose(np.mean(oracle.rmsnorm(z, eps=0.0) ** 2, axis=1), 1.0, rtol=1e-12)
+
+
+def test_l2_normalize():
+    y = oracle.l2_normalize(np.array([[3.0, 4.0]]), eps=0.0)
+    np.testing.assert_allclose(y, [[0.6, 0.8]], rtol=1e-15)
+    z = rng.standard_normal((7, 3, 16))
+    np.testing.assert_allclose(np.linalg.norm(oracle.l2_normalize(z, 0.0), axis=-1), 1.0, rtol=1e-13)
+
+
+def test_gates_identities():
+    """alpha = exp(-softplus(a)) = 1/(1 + e^a): alpha(0) = 1/2; log alpha(-a) - log alpha(a) = a;
+    beta(a) + beta(-a) = 1; alpha in (0, 1), beta in (0, 1); no overflow at |a| = 800."""
+    a = np.concatenate([rng.standard_normal(1000) * 5, [0.0, 30.0, -30.0, 800.0, -800.0]])
+    la, b = oracle.gates(a, a)
+    la_n, b_n = oracle.gates(-a, -a)
+    assert np.all(np.isfinite(la)) and np.all(la <= 0)
+    np.testing.assert_allclose(la_n - la, a, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(b + b_n, 1.0, rtol=0, atol=1e-15)
+    mid = np.abs(a) < 30
+    np.testing.assert_allclose(np.exp(la[mid]), 1.0 / (1.0 + np.exp(a[mid])), rtol=1e-13)
+    la0, b0 = oracle.gates(np.array([0.0]), np.array([0.0]))
+    assert abs(la0[0] + math.log(2)) < 1e-16 and b0[0] == 0.5
+    assert np.all((b >= 0) & (b <= 1))
+
+
+def test_in_projection_split_order():
+    """One-hot weight rows pick input columns: checks the [q | k | v | a_alpha | a_beta] split and
+    the head-major order inside q, k, v."""
+    H, dk, dv = 2, 3, 2
+    n = synth.in_features(H, dk, dv)
+    D = n
+    W = np.eye(n)[np.arange(n)[::-1]]            # row r picks input column n-1-r
+    x = rng.standard_normal((4, D))
+    q, k, v, aa, ab = oracle.in_projection(x, W, H, dk, dv)
+    col = lambda r: x[:, n - 1 - r]
+    np.testing.assert_array_equal(q[:, 1, 2], col(1 * dk + 2))
+    np.testing.assert_array_equal(k[:, 0, 1], col(H * dk + 1))
+    np.testing.assert_array_equal(v[:, 1, 0], col(2 * H * dk + dv))
+    np.testing.assert_array_equal(aa[:, 1], col(2 * H * dk + H * dv + 1))
+    np.testing.assert_array_equal(ab[:, 0], col(2 * H * dk + H * dv + H))
+
+
+def test_out_projection_residual():
+    T, H, dv, D = 3, 2, 4, 5
+    x = rng.standard_normal((T, D))
+    o = rng.standard_normal((T, H, dv))
+    np.testing.assert_array_equal(oracle.out_projection_residual(x, o, np.zeros((D, H * dv))), x)
+    onehot = np.zeros((T, H, dv)); onehot[:, 1, 2] = 1.0
+    W = rng.standard_normal((D, H * dv))
+    np.testing.assert_allclose(oracle.out_projection_residual(x, onehot, W), x + W[:, dv + 2][None],
+                               rtol=1e-15)
+
+
+# ---------------------------------------------------------------- a8 state error
+def test_state_error_cases():
+    S = rng.standard_normal((3, 4, 5))
+    per, tot = oracle.state_error(S, S)
+    assert tot == 0 and not per.any()
+    per, tot = oracle.state_error(S, np.zeros_like(S))
+    np.testing.assert_allclose(per, 1.0); assert abs(tot - 1.0) < 1e-15
+    Z = np.zeros((2, 4, 5))
+    per, tot = oracle.state_error(Z, Z)
+    assert tot == 0.0 and not per.any()
+    Y = Z.copy(); Y[1, 0, 0] = 1e-3
+    per, _ = oracle.state_error(Z, Y)
+    assert per[0] == 0.0 and per[1] == np.inf
+    per, tot = oracle.state_error(S, 0.5 * S)
+    np.testing.assert_allclose(per, 0.5, rtol=1e-15)
+
+
+# ------------------------------------------------------------ group replay (a2-a7)
+def _tiny_group(lengths, D=48, H=2, dk=8, dv=8, L=3, seed=11):
+    layers = synth.la_layers(L, D, H, dk, dv, seed=seed, std=0.2, with_gain=True)
+    h = torch.cat([synth.hidden_prefix(n, D, seed + i) for i, n in enumerate(lengths)])
+    return h, layers, synth.cu_seqlens_of(lengths)
+
+
+def test_replay_first_layer_error_identity():
+    """In the replay of a group, the first LA layer sees exact inputs (reading notes section 2.4),
+    so for it E_m = (T_m ... T_{a+1}) S_a holds with the gates and keys that layer computes; the
+    later layers see the replayed layers' outputs (the cross-layer recurrence of section 2.3) and
+    only have to stay finite."""
+    m, D, H, dk, dv = 30, 48, 2, 8, 8
+    kk = oracle.tail_len(m, 30, 100)                  # 9
+    a = m - kk
+    h, layers, _ = _tiny_group([m], D, H, dk, dv)
+    S_full, _ = oracle.replay_group(h, [0, m], layers, H, dk, dv)
+    S_tail, _ = oracle.replay_group(h[a:], [0, kk], layers, H, dk, dv)
+    S_a, _ = oracle.replay_group(h[:a], [0, a], layers, H, dk, dv)
+    # rebuild layer 0's keys and gates independently from the pieces
+    lw = layers[0]
+    x_hat = oracle.bf16_round(oracle.rmsnorm(h, lw.rms_gain))
+    _, k, _, aa, ab = oracle.in_projection(x_hat, lw.W_in, H, dk, dv)
+    k = oracle.bf16_round(oracle.l2_normalize(k))
+    la, b = oracle.gates(aa, ab)
+    for hh in range(H):
+        P = np.eye(dk)
+        for i in range(a, m):
+            P = _explicit_T(math.exp(la[i, hh]), b[i, hh], k[i, hh]) @ P
+        np.testing.assert_allclose(S_full[0, 0, hh] - S_tail[0, 0, hh], P @ S_a[0, 0, hh],
+                                   rtol=1e-9, atol=1e-12)
+    assert np.all(np.isfinite(S_full - S_tail))
+
+
+def test_replay_zero_and_full_and_skip():
+    lengths = [13, 0, 21]
+    h, layers, cu = _tiny_group(lengths)
+    S, x = oracle.replay_group(h, cu, layers, 2, 8, 8)
+    assert S.shape == (3, 3, 2, 8, 8)
+    assert not S[:, 1].any()                         # k = 0: Zero-only state
+    S2, x2 = oracle.replay_group(h, cu, layers, 2, 8, 8, skip_last_output=True)
+    assert x2 is None and np.array_equal(S, S2)      # the skipped output feeds no state
+    # packed requests equal separate replays (groups, heads and requests are independent)
+    Sa, xa = oracle.replay_group(h[:13], [0, 13], layers, 2, 8, 8)
+    Sb, xb = oracle.replay_group(h[13:], [0, 21], layers, 2, 8, 8)
+    np.testing.assert_allclose(S[:, 0], Sa[:, 0], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(S[:, 2], Sb[:, 0], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(x, np.concatenate([xa, xb]), rtol=1e-12, atol=1e-12)
+
+
+def test_replay_cast_points_are_small():
+    """The bf16 cast points of the boundary move the states by about bf16 precision only."""
+    h, layers, cu = _tiny_group([40, 25], D=64, H=2, dk=16, dv=16)
+    S_c, _ = oracle.replay_group(h, cu, layers, 2, 16, 16, emulate_casts=True)
+    S_e, _ = oracle.replay_group(h, cu, layers, 2, 16, 16, emulate_casts=False)
+    _, tot = oracle.state_error(S_e, S_c)
+    assert 0 < tot < 2e-2
