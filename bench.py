@@ -1,0 +1,400 @@
+#!/usr/bin/env python
+"""Benchmark of the Tail-Replay hot path on B200.
+
+Workload (one step): one hit on one group of 3 Gated DeltaNet layers after a full-attention
+layer; d_model 2048, 16 heads of d_k = d_v = 128; cached FA output hiddens h ~ N(0,1) (bf16),
+weights N(0, 0.02) (bf16); matched prefix m = 32768, r = 5% -> the last k = 1639 hiddens are
+replayed from a zero state through the 3 layers (RMSNorm -> projection + gates + key norm ->
+chunked scan -> output projection + residual; the last layer's readout is skipped), and the
+rebuilt states S_hat_m are compared with the full-prefill S_m (state error, fp64).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  N > 1 runs under torchrun: every rank replays its own
+independent request (no collective on the data path; weak scaling); the time is the max over
+ranks.  --impl reference times the fp64 CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "replayed tokens/s & GDN scan state-updates/s on 1 B200; % of HBM/TC roofline"
+D, H, DH, L, M_PREFIX, R_NUM, R_DEN = 2048, 16, 128, 3, 32768, 5, 100
+WORKLOAD = ("one group = 1 FA + 3 LA (Gated DeltaNet) layers, d_model 2048, 16 heads "
+            "d_k=d_v=128, bf16 cached h ~N(0,1), weights N(0,0.02), alpha=exp(-softplus), "
+            "m=32768, r=0.05 (k=1639), batch 1")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {k: float(pk[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def env_rank():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+# ------------------------------------------------------------------ flop/byte model
+def flops_inproj(T, skip_q):
+    n_in = 2 * H * DH + H * DH + 2 * H - (H * DH if skip_q else 0)
+    return 2.0 * T * D * n_in
+
+
+def flops_outproj(T):
+    return 2.0 * T * (H * DH) * D
+
+
+def scan_flops_per_token_head(C=64, dk=DH, dv=DH):
+    # chunked form: 6 C dk + 4 C dv + C^2/3 + 6 dk dv per token-head
+    return 6 * C * dk + 4 * C * dv + C * C / 3.0 + 6 * dk * dv
+
+
+def group_model(k):
+    """Algorithmic FLOPs and bytes of one step (last layer's readout skipped)."""
+    F = 0.0
+    Bw = 0.0
+    for l in range(L):
+        last = l == L - 1
+        F += flops_inproj(k, last)
+        n_in = 3 * H * DH + 2 * H - (H * DH if last else 0)
+        Bw += n_in * D * 2
+        if not last:
+            F += flops_outproj(k)
+            Bw += D * H * DH * 2
+    F += L * k * H * scan_flops_per_token_head()
+    B = Bw + k * D * 2 + L * H * DH * DH * 4
+    return F, B
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+            time.sleep(0.15)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        rows = [r for r in csv.reader(io.StringIO(self.tmp.read())) if len(r) >= 9]
+        os.unlink(self.tmp.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ reference
+def reference_arm(args):
+    rank, world, _ = env_rank()
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+    import oracle
+    import synth
+
+    k = oracle.tail_len(M_PREFIX, R_NUM, R_DEN)
+    seed = synth.SEED_BASE + 1
+    h_tail = synth.hidden_prefix(M_PREFIX, D, seed)[M_PREFIX - k:]
+    layers = synth.la_layers(L, D, H, DH, DH, seed=seed)
+    sample = 205  # tokens per step: the first 1/8 of the tail, through all 3 layers
+    cu = [0, sample]
+    times = []
+    for i in range(args.warmup + args.steps):
+        a = (i * sample) % (k - sample)
+        t0 = time.perf_counter()
+        oracle.replay_group(h_tail[a:a + sample], cu, layers, H, DH, DH, skip_last_output=True)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    mean = sum(times) / len(times)
+    value = sample / mean
+    cores = os.cpu_count()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "replayed tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "k": k, "sample_tokens": sample},
+        "cpu_baseline": {"value": value, "unit": "replayed tokens/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": "%d consecutive tail tokens through all 3 LA layers per step"
+                                   % sample},
+        "e2e": {"value": value, "unit": "replayed tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- our arm
+def cpu_baseline_sample(h_tail_cpu, layers_cpu, k):
+    import oracle
+    reps, t = 0, 0.0
+    oracle.replay_group(h_tail_cpu[:64], [0, 64], layers_cpu, H, DH, DH, skip_last_output=True)
+    while reps < 2 or (t < 10.0 and reps < 4):
+        t0 = time.perf_counter()
+        oracle.replay_group(h_tail_cpu, [0, k], layers_cpu, H, DH, DH, skip_last_output=True)
+        t += time.perf_counter() - t0
+        reps += 1
+    return {"value": k * reps / t, "unit": "replayed tokens/s", "cores": os.cpu_count(),
+            "kind": "oracle",
+            "sample": "full k=%d tail of the bench workload, %d repetitions (%.1f s)" % (k, reps, t)}
+
+
+def our_arm(args):
+    import torch
+    import torch.distributed as dist
+    import synth
+    import linear_attention_state_zero_b200 as tr
+
+    rank, world, local = env_rank()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    peaks, peak_src = load_peaks()
+
+    k = tr.tail_len(M_PREFIX, R_NUM, R_DEN)
+    seed = synth.SEED_BASE + 1 + 1000 * rank
+    h_full_cpu = synth.hidden_prefix(M_PREFIX, D, seed)
+    h_tail_cpu = h_full_cpu[M_PREFIX - k:].contiguous()
+    layers_cpu = synth.la_layers(L, D, H, DH, DH, seed=seed)
+    layers = [tr.Layer(l.W_in.to(dev), l.W_o.to(dev)) for l in layers_cpu]
+    h_full = h_full_cpu.to(dev)
+    h_tail = h_tail_cpu.to(dev)
+
+    # full-prefill reference states S_m (k = m), untimed
+    full = tr.GroupReplay(h_full, [0, M_PREFIX], layers, H, DH, DH, skip_last_output=True)
+    S_m = full.run()[0].clone()
+    del full
+    rep = tr.GroupReplay(h_tail, [0, k], layers, H, DH, DH, skip_last_output=True)
+    S_m_flat = S_m.reshape(-1, DH, DH)
+    S_hat_flat = rep.S_hat.reshape(-1, DH, DH)
+    n_k = rep.kernel_count()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    # one event before the replay, one after each of its kernels, one after the state error
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(n_k + 2)]
+    stream = torch.cuda.current_stream()
+    for e in events:
+        e.record(stream)
+    handles = [e.cuda_event for e in events]
+
+    def step():
+        rep.run_profiled(handles[:n_k + 1], stream)
+        per, tot = tr.state_error(S_m_flat, S_hat_flat, per_mat=False)
+        events[-1].record(stream)
+        return tot
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    tr.check()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms, kern_ms = [], [[] for _ in range(n_k)]
+    err_tot = None
+    for _ in range(args.steps):
+        flush.zero_()
+        err_tot = step()
+        torch.cuda.synchronize()  # read this step's events before they are re-recorded
+        step_ms.append(events[0].elapsed_time(events[-1]))
+        for i in range(n_k):
+            kern_ms[i].append(events[i].elapsed_time(events[i + 1]))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    tr.check()
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * k / (ms_per_step * 1e-3)
+
+    # per-kernel breakdown (launch order: per layer rmsnorm, in-proj, scan[, out-proj])
+    names = []
+    for l in range(L):
+        names += ["rmsnorm", "in_proj", "scan"] + ([] if l == L - 1 else ["out_proj"])
+    avg = [sum(x) / len(x) for x in kern_ms]
+    brk = {}
+    for n, a in zip(names, avg):
+        brk[n] = brk.get(n, 0.0) + a * 1e3
+    in_idx = [i for i, n in enumerate(names) if n == "in_proj"]
+    in_flops = sum(flops_inproj(k, l == L - 1) for l in range(L))
+    in_ms = sum(avg[i] for i in in_idx)
+    achieved_tf = in_flops / (in_ms * 1e-3) / 1e12
+    F, B = group_model(k)
+    t_roof = max(F / (peaks["bf16_tflops"] * 1e12), B / (peaks["hbm_gbs"] * 1e9))
+
+    # end to end through the public API with host buffers
+    h_host = h_tail_cpu.pin_memory()
+    S_host = torch.empty(rep.S_hat.shape, dtype=torch.float32).pin_memory()
+    err_host = torch.empty(1, dtype=torch.float64).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        e0.record(stream)
+        h_tail.copy_(h_host, non_blocking=True)
+        rep.run(stream)
+        _, tot = tr.state_error(S_m_flat, S_hat_flat, per_mat=False)
+        S_host.copy_(rep.S_hat, non_blocking=True)
+        err_host.copy_(tot, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(e0.elapsed_time(e1))
+    t = torch.tensor([sum(e2e_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_value = world * k / (float(t.item()) / args.steps * 1e-3)
+
+    # scan-only cell: 32 heads d=128, m=32768, r=0.10 (k=3277), bf16, alpha ~ U[0.97, 1]
+    k5 = tr.tail_len(32768, 10, 100)
+    case = synth.scan_case([k5], 32, 128, 128, torch.bfloat16, 0.97, 1.0, seed=synth.SEED_BASE + 4)
+    sq, sk, sv = case.q.to(dev), case.k.to(dev), case.v.to(dev)
+    sla, sb = case.log_alpha.to(dev), case.beta.to(dev)
+    so = torch.empty_like(sv)
+    sS = torch.empty(1, 32, 128, 128, dtype=torch.float32, device=dev)
+    for _ in range(3):
+        tr.gdn_scan(sq, sk, sv, sla, sb, case.cu_seqlens, o=so, S_final=sS)
+    scan_ms = []
+    for _ in range(max(5, min(args.steps, 50))):
+        flush.zero_()
+        e0.record(stream)
+        tr.gdn_scan(sq, sk, sv, sla, sb, case.cu_seqlens, o=so, S_final=sS)
+        e1.record(stream)
+        e1.synchronize()
+        scan_ms.append(e0.elapsed_time(e1))
+    scan_t = sum(scan_ms) / len(scan_ms) * 1e-3
+    upd = k5 * 32
+    scan_bytes = upd * (3 * 256 + 8 + 256) + 32 * 128 * 128 * 4
+    scan_gbs = scan_bytes / scan_t / 1e9
+    tr.check()
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline_sample(h_tail_cpu, layers_cpu, k)
+        line = {
+            "metric": METRIC, "value": value, "unit": "replayed tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "d_model": D, "n_heads": H, "d_head": DH,
+                       "la_layers": L, "m": M_PREFIX, "r": R_NUM / R_DEN, "k": k,
+                       "requests_per_gpu": 1, "parallelism": "independent requests per GPU",
+                       "l2": "flushed (256 MiB write) before every timed step"},
+            "token_layers_per_s": value * L,
+            "state_updates_per_s": value * L * H,
+            "state_error_vs_full_prefill": float(err_tot.item()),
+            "roofline": {"bound": "tensor", "kernel": "in_proj (tcgen05 GEMM + gate/norm epilogue)",
+                         "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"],
+                         "traffic": None, "peak_source": peak_src + " (burst bf16)",
+                         "flops_per_step": in_flops, "ms_per_step": in_ms},
+            "group_roofline": {"t_roof_us": t_roof * 1e6, "t_step_us": ms_per_step * 1e3,
+                               "frac": t_roof / (ms_per_step * 1e-3), "alg_flops": F,
+                               "alg_bytes": B},
+            "kernel_us_per_step": brk,
+            "scan": {"workload": "scan only: 32 heads d=128, bf16, alpha~U[0.97,1], m=32768, "
+                                 "r=0.10 (k=%d)" % k5,
+                     "state_updates_per_s": upd / scan_t, "us": scan_t * 1e6,
+                     "roofline": {"bound": "hbm", "achieved": scan_gbs, "peak": peaks["hbm_gbs"],
+                                  "unit": "GB/s", "frac": scan_gbs / peaks["hbm_gbs"],
+                                  "traffic": None, "alg_bytes": scan_bytes}},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "replayed tokens/s",
+                    "h2d_bytes_per_step": k * D * 2,
+                    "d2h_bytes_per_step": int(S_host.numel() * 4 + 8)},
+            "gpu_launches": args.steps * (n_k + 2),
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        our_arm(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,279 @@
+/*
+ * tr.h -- C ABI of libtr.so, the B200 (sm_100a) hot path of Tail-Replay:
+ * zero-initialised replay of the last k = ceil(r*m) tokens of a matched prefix
+ * through each group's Gated DeltaNet (linear-attention, LA) layers, rebuilding
+ * the recurrent states S_hat_m.
+ *
+ * Sources (web pages on the Tail-Replay paper, arXiv 2608.30310):
+ *   RN = "Tail-Replay reading notes" (cc.laoqi.cc): section 2.1 (cache record,
+ *        k = ceil(r m)), section 2.2 (the four-step hit path and its worked
+ *        example), section 2.3 (Eq. (1), the error identity), section 2.4
+ *        (per-group exact entry points), section 2.5 (tail-FFN skip).
+ *   GS = "Tail-Replay technical summary" (gist.science), "Key Mechanisms":
+ *        fetch the last k cached FA output hiddens, zero the replay state,
+ *        replay Eq. (1), independently per group.
+ *
+ * Conventions for every call
+ *   - Ownership: the caller owns every buffer.  Array arguments are DEVICE
+ *     pointers unless the name ends in _host.  Nothing here allocates device
+ *     memory: scratch space is the caller's workspace `ws` of at least the size
+ *     the matching *_workspace_size() returns (256-byte aligned).
+ *   - Asynchrony: work is enqueued on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream) and the call returns after enqueue.
+ *     Device-side failures (a bounded wait that ran out) are reported by
+ *     tr_check().
+ *   - Errors: every call returns a tr_status; TR_OK is 0.  On failure nothing
+ *     was enqueued (argument errors are found before any launch) and
+ *     tr_last_error() returns a thread-local message.  No call exits, traps or
+ *     prints.
+ *   - Layouts are row-major and packed unless a stride argument says otherwise.
+ *     bf16 means IEEE bfloat16 (round-to-nearest-even on every store); all
+ *     recurrent state is fp32.
+ *   - State layout: the pages leave the axis order open (RN section 2.3, remark
+ *     after Eq. (1)).  States are stored as M = S^T, a d_k x d_v matrix per
+ *     (sequence, head), so that Eq. (1) reads M_i = T_i M_{i-1} + beta_i k_i v_i^T
+ *     with T_i = alpha_i (I - beta_i k_i k_i^T) acting from the left.
+ */
+#ifndef TAIL_REPLAY_TR_H
+#define TAIL_REPLAY_TR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int tr_status;
+enum {
+  TR_OK = 0,
+  TR_ERR_INVALID_ARG = 1,   /* NULL where a buffer is required, negative size, bad flag */
+  TR_ERR_SHAPE = 2,         /* sizes inconsistent (e.g. cu_seqlens_host[N] != total_tokens) */
+  TR_ERR_DTYPE = 3,         /* unknown dtype code */
+  TR_ERR_ALIGNMENT = 4,     /* a pointer or row stride is not 16-byte aligned */
+  TR_ERR_UNSUPPORTED = 5,   /* a size outside what the kernels implement (see each call) */
+  TR_ERR_WORKSPACE = 6,     /* ws NULL or smaller than *_workspace_size() */
+  TR_ERR_CUDA = 7,          /* a CUDA runtime call or launch failed */
+  TR_ERR_TIMEOUT = 8        /* reported by tr_check(): a device-side bounded wait ran out */
+};
+
+/* element types */
+enum { TR_DTYPE_F32 = 0, TR_DTYPE_BF16 = 1 };
+
+/* flags */
+enum {
+  TR_NORMALIZE_QK = 1u,      /* tr_gdn_scan: L2-normalise q and k per head in the kernel */
+  TR_SKIP_LAST_OUTPUT = 2u,  /* tr_replay_group(s): skip the last LA layer's readout, q
+                                projection and output projection (its output rebuilds no
+                                state; RN section 2.5 makes the same point for the tail FFN) */
+  TR_SCAN_RECURRENT = 4u     /* force the token-sequential scan kernel (test path) */
+};
+
+/* Human-readable message for the last failing call on this host thread. */
+const char *tr_last_error(void);
+
+/* Library build string (compiler, target). */
+const char *tr_version(void);
+
+/*
+ * Tail length (RN section 2.1, symbol table; worked example RN section 2.2):
+ * k = ceil(r * m) for r = r_num / r_den, in exact integer arithmetic, clamped to
+ * [0, m].  Returns -1 if r_den <= 0 or m < 0.  Host-only, no device work.
+ * The tail is rows m-k .. m-1 (0-based) of the cached hiddens, positions
+ * m-k+1 .. m (1-based).
+ */
+int64_t tr_tail_len(int64_t m, int64_t r_num, int64_t r_den);
+
+/*
+ * ---------------------------------------------------------------- tr_gdn_scan
+ * The Gated DeltaNet recurrence, Eq. (1) of RN section 2.3, over a packed batch
+ * of sequences, per head, from S0 (zero start when S0 is NULL -- RN section 2.2
+ * step 2, GS "Key Mechanisms"):
+ *
+ *   M_t = alpha_t (M_{t-1} - beta_t k_t (k_t^T M_{t-1})) + beta_t k_t v_t^T,
+ *   o_t = scale * M_t^T q_t   (readout after the update; the pages do not define
+ *                              the readout, this is the reading used)
+ *   S_final = M at the last token of each sequence (S0, or 0, for empty ones).
+ *
+ * Arguments (T = total_tokens, N = n_seqs, H = n_heads):
+ *   q, k      [T, H, d_k] elements of `dtype`, token stride q_stride/k_stride
+ *             elements (0 = H*d_k).  q may be NULL when o is NULL.
+ *   v         [T, H, d_v], token stride v_stride (0 = H*d_v).
+ *   log_alpha [T, H] fp32, log of the decay alpha in (0, 1] (so <= 0).  Values
+ *             are not checked on the device.
+ *   beta      [T, H] fp32.
+ *   cu_seqlens      [N+1] int32 device offsets, cu[0] = 0, cu[N] = T, nondecreasing.
+ *   cu_seqlens_host the same N+1 values in host memory (validation and the
+ *                   longest-first schedule); must equal the device copy.
+ *   S0        [N, H, d_k, d_v] fp32 or NULL (zero start).
+ *   o         [T, H, d_v] of `dtype`, or NULL to skip the readout.
+ *   S_final   [N, H, d_k, d_v] fp32, required.  Must not alias S0.
+ *   scale     readout scale (1.0 in every workload here).
+ *   flags     TR_NORMALIZE_QK, TR_SCAN_RECURRENT.
+ * Supported: d_k, d_v in {64, 128}; dtype TR_DTYPE_BF16 (chunked tensor-core
+ * kernel) or TR_DTYPE_F32 (token-sequential fp32 FMA kernel, the test path);
+ * 16-byte aligned q/k/v/o with strides that keep every row 16-byte aligned.
+ * Workspace: tr_gdn_scan_workspace_size(args) bytes.
+ */
+typedef struct tr_scan_args {
+  int32_t n_seqs, n_heads, d_k, d_v;
+  int64_t total_tokens;
+  int32_t dtype;
+  uint32_t flags;
+  float scale;
+  int64_t q_stride, k_stride, v_stride;
+  const void *q, *k, *v;
+  const float *log_alpha, *beta;
+  const int32_t *cu_seqlens;
+  const int32_t *cu_seqlens_host;
+  const float *S0;
+  void *o;
+  float *S_final;
+} tr_scan_args;
+
+size_t tr_gdn_scan_workspace_size(const tr_scan_args *args);
+tr_status tr_gdn_scan(const tr_scan_args *args, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * ---------------------------------------------------------- tr_replay_group
+ * Replay of one group's LA layers over the packed k-token tails (RN section
+ * 2.2 steps 2-3; GS "Key Mechanisms"; the group is the run of LA layers after
+ * one FA layer, RN section 2.1 figure 1).  Each request's tail starts from the
+ * cached FA output hiddens h_{m-k+1..m} (exact, RN section 2.4) with every LA
+ * state zero; the hiddens pass through the LA layers in order, giving S_hat_m
+ * for every LA layer.  Passing the whole prefix (k = m) gives the full-prefill
+ * S_m (RN section 3.1, "Full").
+ *
+ * Per LA layer (the pages give no layer internals; this is the reading used):
+ *   x_hat = bf16(RMSNorm(x) * gain)            eps = rms_eps (0 -> 1e-6)
+ *   [q|k|v|a_alpha|a_beta] = x_hat W_in^T      fp32 accumulate
+ *   q, k <- bf16(x / sqrt(sum x^2 + norm_eps)) per head (norm_eps 0 -> 1e-6)
+ *   v <- bf16(v); log alpha = -softplus(a_alpha), beta = sigmoid(a_beta) (fp32)
+ *   o, S_hat[layer] = tr_gdn_scan(q, k, v, log alpha, beta), zero start
+ *   x <- x + bf16(o) W_o^T                     fp32 residual; no FFN sublayer
+ * x starts as h_tail.  The cast points above are part of this contract.
+ *
+ * Arguments (T = total_tokens, D = d_model, H = n_heads):
+ *   h_tail   [T, D] bf16, the N requests' tails packed by cu_seqlens.
+ *   layers   HOST array of n_layers tr_la_layer:
+ *              rms_gain [D] fp32 or NULL (ones)
+ *              W_in     [2 H d_k + H d_v + 2 H, D] bf16 (output x input features;
+ *                       rows: q heads, k heads, v heads, a_alpha, a_beta)
+ *              W_o      [D, H d_v] bf16
+ *   S_hat    [n_layers, N, H, d_k, d_v] fp32 output.
+ *   x_out    [T, D] fp32 output of the last layer, or NULL (then the last
+ *            layer's output projection is not run).  Must be NULL with
+ *            TR_SKIP_LAST_OUTPUT.
+ * Supported: d_k = d_v = 128 or 64; D a multiple of 64; 1 <= n_layers <= 64.
+ * Workspace: tr_replay_group_workspace_size(args) bytes.
+ */
+typedef struct tr_la_layer {
+  const float *rms_gain;
+  const void *W_in;
+  const void *W_o;
+} tr_la_layer;
+
+typedef struct tr_group_args {
+  int32_t n_seqs, n_heads, d_k, d_v, d_model, n_layers;
+  int64_t total_tokens;
+  uint32_t flags;
+  float rms_eps, norm_eps;
+  const void *h_tail;
+  const int32_t *cu_seqlens;
+  const int32_t *cu_seqlens_host;
+  const tr_la_layer *layers;
+  float *S_hat;
+  float *x_out;
+} tr_group_args;
+
+size_t tr_replay_group_workspace_size(const tr_group_args *args);
+tr_status tr_replay_group(const tr_group_args *args, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * The same replay with timing marks: `events` is a HOST array of n_events
+ * created cudaEvent_t handles (passed as void*).  events[0] is recorded on
+ * `stream` before the first kernel and events[i] after the i-th kernel launch,
+ * in launch order (per layer: RMSNorm, input projection, scan, then the output
+ * projection when it runs).  n_events must be at least
+ * 1 + tr_replay_group_kernel_count(args); the rest are left alone.
+ */
+int32_t tr_replay_group_kernel_count(const tr_group_args *args);
+tr_status tr_replay_group_profiled(const tr_group_args *args, void *ws, size_t ws_bytes,
+                                   void *stream, void *const *events, int32_t n_events);
+
+/*
+ * All groups of all hits in one call (groups are independent: RN section 2.4,
+ * GS "Key Mechanisms").  groups is a HOST array of n_groups tr_group_args; each
+ * group carries its own LA weights and its own tails (the hits of one group
+ * share its weights and are packed by that group's cu_seqlens).  The workspace
+ * is shared: tr_replay_groups_workspace_size() is the largest single group's.
+ */
+size_t tr_replay_groups_workspace_size(const tr_group_args *groups, int32_t n_groups);
+tr_status tr_replay_groups(const tr_group_args *groups, int32_t n_groups, void *ws,
+                           size_t ws_bytes, void *stream);
+
+/*
+ * ---------------------------------------------------------- tr_state_error
+ * Relative Frobenius error of a rebuilt state against the full-prefill state
+ * (E_m = S_m - S_hat_m, RN section 2.3):
+ *   err_per_mat[i] = ||S_i - S_hat_i||_F / ||S_i||_F  over each d_k x d_v matrix
+ *   err_total      = ||S - S_hat||_F / ||S||_F        over all n_mats matrices
+ * with fp64 accumulation of the fp32 data.  When a denominator is 0 the error
+ * is 0 if the numerator is 0, else +inf.
+ *   S, S_hat     [n_mats, d_k, d_v] fp32 (device).
+ *   err_per_mat  [n_mats] fp64 (device) or NULL.
+ *   err_total    [1] fp64 (device) or NULL.
+ * Workspace: tr_state_error_workspace_size(n_mats) bytes.
+ */
+size_t tr_state_error_workspace_size(int64_t n_mats);
+tr_status tr_state_error(const float *S, const float *S_hat, int64_t n_mats, int32_t d_k,
+                         int32_t d_v, double *err_per_mat, double *err_total, void *ws,
+                         size_t ws_bytes, void *stream);
+
+/*
+ * ---------------------------------------------- steps of one LA layer, alone
+ * The three dense steps of tr_replay_group, exposed so that each can be checked
+ * on its own.  Same arithmetic and cast points as inside tr_replay_group.
+ *
+ * tr_rmsnorm: x_hat[t] = bf16(x[t] / sqrt(mean_j x[t,j]^2 + eps) * gain)
+ *   x [n_rows, D] of x_dtype (bf16 or fp32); gain [D] fp32 or NULL;
+ *   x_hat [n_rows, D] bf16.  eps 0 -> 1e-6.  D a multiple of 8.
+ */
+tr_status tr_rmsnorm(const void *x, int32_t x_dtype, const float *gain, int64_t n_rows,
+                     int32_t d_model, float eps, void *x_hat, void *stream);
+
+/*
+ * tr_in_projection: y = x_hat W_in^T (tcgen05 tensor cores, fp32 accumulate) with
+ * the gate and key-norm epilogue:
+ *   qkv [T, 2 H d_k + H d_v] bf16 = [L2norm(q) | L2norm(k) | v] per head,
+ *   log_alpha [T, H] = -softplus(a_alpha), beta [T, H] = sigmoid(a_beta), fp32.
+ * With TR_SKIP_LAST_OUTPUT in flags the q columns are neither computed nor
+ * written.  x_hat [T, D] bf16, W_in as in tr_la_layer.  norm_eps 0 -> 1e-6.
+ */
+tr_status tr_in_projection(const void *x_hat, const void *W_in, int64_t n_tokens,
+                           int32_t d_model, int32_t n_heads, int32_t d_k, int32_t d_v,
+                           uint32_t flags, float norm_eps, void *qkv, float *log_alpha,
+                           float *beta, void *stream);
+
+/*
+ * tr_out_projection: x_out = x_res + o W_o^T (tcgen05, fp32 accumulate, fp32 out).
+ *   o [T, H d_v] bf16 (row stride o_stride elements, 0 = H d_v); W_o [D, H d_v] bf16;
+ *   x_res [T, D] of x_res_dtype (bf16 or fp32); x_out [T, D] fp32 (may equal x_res
+ *   when x_res is fp32).
+ */
+tr_status tr_out_projection(const void *o, int64_t o_stride, const void *W_o, const void *x_res,
+                            int32_t x_res_dtype, int64_t n_tokens, int32_t d_model,
+                            int32_t hv, float *x_out, void *stream);
+
+/*
+ * tr_check: waits for `stream`, then reads and clears the library's device error
+ * word.  Returns TR_ERR_TIMEOUT if a kernel gave up a bounded wait since the
+ * last check, TR_ERR_CUDA if the stream reports an error, else TR_OK.
+ */
+tr_status tr_check(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TAIL_REPLAY_TR_H */

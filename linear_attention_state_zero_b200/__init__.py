@@ -1,0 +1,335 @@
+"""Tail-Replay on B200: zero-initialised tail replay of Gated DeltaNet layers.
+
+Python binding of ``libtr.so`` (declared in ``include/tr.h``).  This module only
+marshals arguments: it checks devices, dtypes and strides of torch tensors,
+allocates outputs and workspaces with PyTorch, and calls the C ABI.  Every step
+of the computation runs in the library's CUDA kernels; there is no CPU path.
+Importing fails if the library has not been built
+(``python linear_attention_state_zero_b200/_build.py``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtr.so")
+
+TR_OK = 0
+TR_DTYPE_F32, TR_DTYPE_BF16 = 0, 1
+TR_NORMALIZE_QK, TR_SKIP_LAST_OUTPUT, TR_SCAN_RECURRENT = 1, 2, 4
+
+STATUS_NAMES = {0: "TR_OK", 1: "TR_ERR_INVALID_ARG", 2: "TR_ERR_SHAPE", 3: "TR_ERR_DTYPE",
+                4: "TR_ERR_ALIGNMENT", 5: "TR_ERR_UNSUPPORTED", 6: "TR_ERR_WORKSPACE",
+                7: "TR_ERR_CUDA", 8: "TR_ERR_TIMEOUT"}
+
+c_i32, c_i64, c_u32, c_f32, c_vp, c_sz = (ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32,
+                                          ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t)
+
+
+class ScanArgs(ctypes.Structure):
+    _fields_ = [("n_seqs", c_i32), ("n_heads", c_i32), ("d_k", c_i32), ("d_v", c_i32),
+                ("total_tokens", c_i64), ("dtype", c_i32), ("flags", c_u32), ("scale", c_f32),
+                ("q_stride", c_i64), ("k_stride", c_i64), ("v_stride", c_i64),
+                ("q", c_vp), ("k", c_vp), ("v", c_vp), ("log_alpha", c_vp), ("beta", c_vp),
+                ("cu_seqlens", c_vp), ("cu_seqlens_host", c_vp), ("S0", c_vp), ("o", c_vp),
+                ("S_final", c_vp)]
+
+
+class LALayer(ctypes.Structure):
+    _fields_ = [("rms_gain", c_vp), ("W_in", c_vp), ("W_o", c_vp)]
+
+
+class GroupArgs(ctypes.Structure):
+    _fields_ = [("n_seqs", c_i32), ("n_heads", c_i32), ("d_k", c_i32), ("d_v", c_i32),
+                ("d_model", c_i32), ("n_layers", c_i32), ("total_tokens", c_i64),
+                ("flags", c_u32), ("rms_eps", c_f32), ("norm_eps", c_f32),
+                ("h_tail", c_vp), ("cu_seqlens", c_vp), ("cu_seqlens_host", c_vp),
+                ("layers", ctypes.POINTER(LALayer)), ("S_hat", c_vp), ("x_out", c_vp)]
+
+
+# exported symbol -> (restype, argtypes)
+_SIGNATURES = {
+    "tr_last_error": (ctypes.c_char_p, []),
+    "tr_version": (ctypes.c_char_p, []),
+    "tr_tail_len": (c_i64, [c_i64, c_i64, c_i64]),
+    "tr_gdn_scan_workspace_size": (c_sz, [ctypes.POINTER(ScanArgs)]),
+    "tr_gdn_scan": (ctypes.c_int, [ctypes.POINTER(ScanArgs), c_vp, c_sz, c_vp]),
+    "tr_replay_group_workspace_size": (c_sz, [ctypes.POINTER(GroupArgs)]),
+    "tr_replay_group": (ctypes.c_int, [ctypes.POINTER(GroupArgs), c_vp, c_sz, c_vp]),
+    "tr_replay_group_kernel_count": (c_i32, [ctypes.POINTER(GroupArgs)]),
+    "tr_replay_group_profiled": (ctypes.c_int, [ctypes.POINTER(GroupArgs), c_vp, c_sz, c_vp,
+                                                ctypes.POINTER(c_vp), c_i32]),
+    "tr_replay_groups_workspace_size": (c_sz, [ctypes.POINTER(GroupArgs), c_i32]),
+    "tr_replay_groups": (ctypes.c_int, [ctypes.POINTER(GroupArgs), c_i32, c_vp, c_sz, c_vp]),
+    "tr_state_error_workspace_size": (c_sz, [c_i64]),
+    "tr_state_error": (ctypes.c_int, [c_vp, c_vp, c_i64, c_i32, c_i32, c_vp, c_vp, c_vp, c_sz,
+                                      c_vp]),
+    "tr_rmsnorm": (ctypes.c_int, [c_vp, c_i32, c_vp, c_i64, c_i32, c_f32, c_vp, c_vp]),
+    "tr_in_projection": (ctypes.c_int, [c_vp, c_vp, c_i64, c_i32, c_i32, c_i32, c_i32, c_u32,
+                                        c_f32, c_vp, c_vp, c_vp, c_vp]),
+    "tr_out_projection": (ctypes.c_int, [c_vp, c_i64, c_vp, c_vp, c_i32, c_i64, c_i32, c_i32,
+                                         c_vp, c_vp]),
+    "tr_check": (ctypes.c_int, [c_vp]),
+}
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libtr.so is not built (%s); run "
+                          "`python linear_attention_state_zero_b200/_build.py`" % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in _SIGNATURES.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+class TrError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = lib.tr_last_error().decode(errors="replace")
+        super().__init__("%s: %s (%s)" % (where, STATUS_NAMES.get(status, status), msg))
+        self.status = status
+
+
+def _ok(st: int, where: str) -> None:
+    if st != TR_OK:
+        raise TrError(st, where)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return TR_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return TR_DTYPE_F32
+    raise TypeError("unsupported dtype %s" % t.dtype)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device")
+
+
+def _seqlens(cu_seqlens, device):
+    """(host int32 tensor, device int32 tensor) for a cu_seqlens given either way."""
+    cu = torch.as_tensor(cu_seqlens, dtype=torch.int32)
+    host = cu.cpu().contiguous()
+    dev = cu.to(device).contiguous() if not (cu.is_cuda and cu.is_contiguous()) else cu
+    return host, dev
+
+
+def version() -> str:
+    return lib.tr_version().decode()
+
+
+def tail_len(m: int, r_num: int, r_den: int) -> int:
+    """k = ceil(r m) for r = r_num / r_den, exact, clamped to [0, m] (C ABI, host-only)."""
+    k = lib.tr_tail_len(int(m), int(r_num), int(r_den))
+    if k < 0:
+        raise ValueError("bad tail length arguments")
+    return int(k)
+
+
+def gdn_scan(q, k, v, log_alpha, beta, cu_seqlens, *, S0=None, want_o=True, scale=1.0,
+             normalize_qk=False, recurrent=False, o=None, S_final=None, stream=None):
+    """Eq. (1) scan over a packed batch: returns (o or None, S_final [N, H, d_k, d_v] fp32)."""
+    _need_cuda(k, v, log_alpha, beta)
+    T, H, dk = k.shape
+    dv = v.shape[2]
+    for t in (q, k, v):
+        if t is not None and (t.stride(2) != 1 or t.stride(1) != t.shape[2]):
+            raise ValueError("q/k/v must be [T, H, d] with contiguous heads")
+    la = log_alpha.contiguous()
+    be = beta.contiguous()
+    host, dev = _seqlens(cu_seqlens, k.device)
+    N = host.numel() - 1
+    if want_o and o is None:
+        o = torch.empty((T, H, dv), dtype=k.dtype, device=k.device)
+    if not want_o:
+        o = None
+    if S_final is None:
+        S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=k.device)
+    flags = (TR_NORMALIZE_QK if normalize_qk else 0) | (TR_SCAN_RECURRENT if recurrent else 0)
+    a = ScanArgs(N, H, dk, dv, T, _dtype_code(k), flags, float(scale),
+                 q.stride(0) if q is not None else 0, k.stride(0), v.stride(0),
+                 _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(be),
+                 _ptr(dev), host.data_ptr(), _ptr(S0), _ptr(o), _ptr(S_final))
+    ws_bytes = lib.tr_gdn_scan_workspace_size(ctypes.byref(a))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=k.device) if ws_bytes else None
+    _ok(lib.tr_gdn_scan(ctypes.byref(a), _ptr(ws), ws_bytes, _stream(stream)), "tr_gdn_scan")
+    return o, S_final
+
+
+@dataclass
+class Layer:
+    """One LA layer's weights, device tensors (W_in [2Hd_k + Hd_v + 2H, D], W_o [D, H d_v])."""
+    W_in: torch.Tensor
+    W_o: torch.Tensor
+    rms_gain: Optional[torch.Tensor] = None
+
+
+class GroupReplay:
+    """A prepared tr_replay_group call: fixed buffers, so repeated calls cost one C call.
+
+    ``h_tail`` [T, D] bf16 and ``cu_seqlens`` describe the packed tails of the
+    group's requests; ``layers`` the group's LA layers.  Outputs: ``S_hat``
+    [L, N, H, d_k, d_v] fp32 and, unless ``skip_last_output``, ``x_out`` [T, D].
+    """
+
+    def __init__(self, h_tail, cu_seqlens, layers: Sequence, n_heads: int, d_k: int, d_v: int,
+                 *, skip_last_output=False, want_x_out=True, rms_eps=0.0, norm_eps=0.0,
+                 S_hat=None, x_out=None, workspace=None):
+        _need_cuda(h_tail)
+        if h_tail.dtype != torch.bfloat16 or not h_tail.is_contiguous():
+            raise ValueError("h_tail must be contiguous bf16 [T, D]")
+        dev = h_tail.device
+        T, D = h_tail.shape
+        self.host, self.dev_cu = _seqlens(cu_seqlens, dev)
+        N = self.host.numel() - 1
+        L = len(layers)
+        self.layers = list(layers)
+        self._layer_arr = (LALayer * L)()
+        for i, lw in enumerate(self.layers):
+            _need_cuda(lw.W_in, lw.W_o)
+            self._layer_arr[i] = LALayer(_ptr(lw.rms_gain), _ptr(lw.W_in), _ptr(lw.W_o))
+        self.S_hat = S_hat if S_hat is not None else torch.empty(
+            (L, N, n_heads, d_k, d_v), dtype=torch.float32, device=dev)
+        if skip_last_output:
+            want_x_out = False
+        self.x_out = None
+        if want_x_out:
+            self.x_out = x_out if x_out is not None else torch.empty((T, D), dtype=torch.float32,
+                                                                     device=dev)
+        flags = TR_SKIP_LAST_OUTPUT if skip_last_output else 0
+        self.h_tail = h_tail
+        self.args = GroupArgs(N, n_heads, d_k, d_v, D, L, T, flags, float(rms_eps),
+                              float(norm_eps), _ptr(h_tail), _ptr(self.dev_cu),
+                              self.host.data_ptr(), self._layer_arr, _ptr(self.S_hat),
+                              _ptr(self.x_out))
+        self.ws_bytes = lib.tr_replay_group_workspace_size(ctypes.byref(self.args))
+        if workspace is None and self.ws_bytes:
+            workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev)
+        self.workspace = workspace
+
+    def run(self, stream=None):
+        _ok(lib.tr_replay_group(ctypes.byref(self.args), _ptr(self.workspace), self.ws_bytes,
+                                _stream(stream)), "tr_replay_group")
+        return self.S_hat, self.x_out
+
+    def kernel_count(self) -> int:
+        return int(lib.tr_replay_group_kernel_count(ctypes.byref(self.args)))
+
+    def run_profiled(self, event_handles, stream=None):
+        """Same as run(), recording the given raw cudaEvent_t handles between kernel launches."""
+        arr = (c_vp * len(event_handles))(*event_handles)
+        _ok(lib.tr_replay_group_profiled(ctypes.byref(self.args), _ptr(self.workspace),
+                                         self.ws_bytes, _stream(stream), arr, len(event_handles)),
+            "tr_replay_group_profiled")
+        return self.S_hat, self.x_out
+
+
+def replay_group(h_tail, cu_seqlens, layers, n_heads, d_k, d_v, **kw):
+    """One group's replay: returns (S_hat [L, N, H, d_k, d_v], x_out or None)."""
+    stream = kw.pop("stream", None)
+    return GroupReplay(h_tail, cu_seqlens, layers, n_heads, d_k, d_v, **kw).run(stream)
+
+
+class GroupsReplay:
+    """A prepared tr_replay_groups call over several GroupReplay descriptions (shared workspace)."""
+
+    def __init__(self, groups: Sequence[GroupReplay]):
+        self.groups = list(groups)
+        n = len(self.groups)
+        self._arr = (GroupArgs * n)()
+        for i, g in enumerate(self.groups):
+            self._arr[i] = g.args
+        self.ws_bytes = lib.tr_replay_groups_workspace_size(self._arr, n)
+        dev = self.groups[0].h_tail.device
+        self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev) \
+            if self.ws_bytes else None
+
+    def run(self, stream=None):
+        _ok(lib.tr_replay_groups(self._arr, len(self.groups), _ptr(self.workspace),
+                                 self.ws_bytes, _stream(stream)), "tr_replay_groups")
+        return [(g.S_hat, g.x_out) for g in self.groups]
+
+
+def state_error(S, S_hat, *, per_mat=True, stream=None):
+    """(err_per_mat [n_mats] fp64 or None, err_total [1] fp64), device tensors."""
+    _need_cuda(S, S_hat)
+    if S.shape != S_hat.shape or S.dtype != torch.float32 or S_hat.dtype != torch.float32:
+        raise ValueError("S and S_hat must be fp32 tensors of one shape")
+    dk, dv = S.shape[-2:]
+    S, S_hat = S.contiguous(), S_hat.contiguous()
+    n = S.numel() // (dk * dv)
+    per = torch.empty(n, dtype=torch.float64, device=S.device) if per_mat else None
+    tot = torch.empty(1, dtype=torch.float64, device=S.device)
+    ws_bytes = lib.tr_state_error_workspace_size(n)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=S.device) if ws_bytes else None
+    _ok(lib.tr_state_error(_ptr(S), _ptr(S_hat), n, dk, dv, _ptr(per), _ptr(tot), _ptr(ws),
+                           ws_bytes, _stream(stream)), "tr_state_error")
+    return per, tot
+
+
+def rmsnorm(x, gain=None, eps=0.0, stream=None):
+    _need_cuda(x, gain)
+    x = x.contiguous()
+    T, D = x.shape
+    out = torch.empty((T, D), dtype=torch.bfloat16, device=x.device)
+    _ok(lib.tr_rmsnorm(_ptr(x), _dtype_code(x), _ptr(gain), T, D, float(eps), _ptr(out),
+                       _stream(stream)), "tr_rmsnorm")
+    return out
+
+
+def in_projection(x_hat, W_in, n_heads, d_k, d_v, *, skip_q=False, norm_eps=0.0, stream=None):
+    """(qkv [T, 2Hd_k + Hd_v] bf16, log_alpha [T, H], beta [T, H])."""
+    _need_cuda(x_hat, W_in)
+    T, D = x_hat.shape
+    dev = x_hat.device
+    x_hat = x_hat.contiguous()
+    W_in = W_in.contiguous()
+    qkv = torch.zeros((T, 2 * n_heads * d_k + n_heads * d_v), dtype=torch.bfloat16, device=dev)
+    la = torch.empty((T, n_heads), dtype=torch.float32, device=dev)
+    be = torch.empty((T, n_heads), dtype=torch.float32, device=dev)
+    _ok(lib.tr_in_projection(_ptr(x_hat), _ptr(W_in), T, D, n_heads,
+                             d_k, d_v, TR_SKIP_LAST_OUTPUT if skip_q else 0, float(norm_eps),
+                             _ptr(qkv), _ptr(la), _ptr(be), _stream(stream)), "tr_in_projection")
+    return qkv, la, be
+
+
+def out_projection(o, W_o, x_res, stream=None):
+    """x_res + o W_o^T in fp32; o [T, H d_v] bf16 (rows may be strided)."""
+    _need_cuda(o, W_o, x_res)
+    T, hv = o.shape
+    D = W_o.shape[0]
+    W_o = W_o.contiguous()
+    x_res = x_res.contiguous()
+    out = torch.empty((T, D), dtype=torch.float32, device=o.device)
+    _ok(lib.tr_out_projection(_ptr(o), o.stride(0), _ptr(W_o),
+                              _ptr(x_res), _dtype_code(x_res), T, D, hv, _ptr(out),
+                              _stream(stream)), "tr_out_projection")
+    return out
+
+
+def check(stream=None) -> None:
+    """Wait for the stream and raise if a kernel reported a device-side failure."""
+    _ok(lib.tr_check(_stream(stream)), "tr_check")

@@ -1,0 +1,325 @@
+// gemm_tc.cu -- the two projection GEMMs of an LA layer on the 5th-generation
+// tensor cores (tcgen05 + TMEM), fed by TMA:
+//
+//   input projection  : [q|k|v|a_alpha|a_beta] = x_hat W_in^T, with the per-head
+//                       L2 norm of q and k, -softplus / sigmoid gates, bf16 q/k/v
+//   output projection : x <- x + o W_o^T (fp32 residual stream)
+//
+// C[M, N] = A[M, K] * B[N, K]^T, A and B bf16 with K contiguous (K-major).
+// One persistent CTA per SM walks the output tiles (128 x BN).  Warp roles:
+//   warp 0     TMA producer: 4-6 stage ring of (A 128x64, B BNx64) bf16 tiles,
+//              128-byte swizzled, one mbarrier pair per stage
+//   warp 1     TMEM owner + MMA issuer: one thread issues tcgen05.mma
+//              (M=128, N=BN, K=16) into a double-buffered fp32 accumulator in
+//              TMEM and commits each stage back to the producer
+//   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter of the accumulator,
+//              fused activation/residual, stores; overlaps the next tile's MMAs
+// Every mbarrier wait is bounded (see tr_ptx.cuh); a timeout ends all roles of
+// the CTA, frees its TMEM and raises the library's error word.
+#include <cuda_bf16.h>
+
+#include "tr_internal.h"
+#include "tr_ptx.cuh"
+
+namespace tr {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kThreads = 192;
+
+enum { EPI_INPROJ = 0, EPI_RESID = 1 };
+
+template <int BN>
+struct Cfg {
+  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+};
+
+struct Ctl {
+  uint64_t full[8];
+  uint64_t empty[8];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16 *dst, const float (&v)[32], float s) {
+  uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+  for (int w = 0; w < 4; ++w)
+    d[w] = make_uint4(pack_bf16x2(v[8 * w + 0] * s, v[8 * w + 1] * s),
+                      pack_bf16x2(v[8 * w + 2] * s, v[8 * w + 3] * s),
+                      pack_bf16x2(v[8 * w + 4] * s, v[8 * w + 5] * s),
+                      pack_bf16x2(v[8 * w + 6] * s, v[8 * w + 7] * s));
+}
+
+__device__ __forceinline__ float softplus_f(float a) {
+  return fmaxf(a, 0.f) + log1pf(expf(-fabsf(a)));
+}
+__device__ __forceinline__ float sigmoid_f(float a) { return 1.f / (1.f + expf(-a)); }
+
+// Input-projection epilogue for one 128 x BN tile; this thread owns `row`.
+template <int BN>
+__device__ __forceinline__ void epi_inproj(const InProjEpi &ep, uint32_t tbase, int n0, int N,
+                                           int row, int M) {
+  const int dk = ep.dk;
+  const int nq = 2 * ep.H * dk;          // q and k features
+  const int nv = nq + ep.H * ep.dv;      // end of the v features
+  const int nblk = BN / dk;
+  for (int blk = 0; blk < nblk; ++blk) {
+    const int c0 = n0 + blk * dk;  // GEMM column
+    if (c0 >= N) break;
+    const int g0 = c0 + ep.col_offset;  // feature index in W_in
+    const uint32_t tb = tbase + (uint32_t)(c0 - n0);
+    if (g0 < nq) {
+      // one q or k head: L2 norm over its d_k features (two passes over TMEM)
+      float ssq = 0.f;
+      for (int j = 0; j < dk / 32; ++j) {
+        float v[32];
+        tmem_ld32(tb + 32 * j, v);
+        tc_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ssq = fmaf(v[i], v[i], ssq);
+      }
+      const float inv = rsqrtf(ssq + ep.norm_eps);
+      for (int j = 0; j < dk / 32; ++j) {
+        float v[32];
+        tmem_ld32(tb + 32 * j, v);
+        tc_wait_ld();
+        if (row < M) store_bf16x32(ep.qkv + (int64_t)row * ep.ldq + g0 + 32 * j, v, inv);
+      }
+    } else {
+      for (int j = 0; j < dk / 32; ++j) {
+        const int c = c0 + 32 * j;
+        if (c >= N) break;
+        const int g = g0 + 32 * j;
+        float v[32];
+        tmem_ld32(tb + 32 * j, v);
+        tc_wait_ld();
+        if (row >= M) continue;
+        if (g + 32 <= nv) {
+          store_bf16x32(ep.qkv + (int64_t)row * ep.ldq + g, v, 1.f);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int gi = g + i - nv;
+            if (c + i >= N) break;
+            if (gi < ep.H)
+              ep.log_alpha[(int64_t)row * ep.H + gi] = -softplus_f(v[i]);
+            else if (gi < 2 * ep.H)
+              ep.beta[(int64_t)row * ep.H + (gi - ep.H)] = sigmoid_f(v[i]);
+          }
+        }
+      }
+    }
+  }
+}
+
+template <int BN>
+__device__ __forceinline__ void epi_resid(const ResidEpi &ep, uint32_t tbase, int n0, int N,
+                                          int row, int M) {
+#pragma unroll 1
+  for (int j = 0; j < BN / 32; ++j) {
+    const int c = n0 + 32 * j;
+    if (c >= N) break;
+    float v[32];
+    tmem_ld32(tbase + 32 * j, v);
+    tc_wait_ld();
+    if (row >= M) continue;
+    float4 *out = reinterpret_cast<float4 *>(ep.x_out + (int64_t)row * ep.ld + c);
+    if (ep.res_is_bf16) {
+      const uint4 *r = reinterpret_cast<const uint4 *>(
+          reinterpret_cast<const __nv_bfloat16 *>(ep.x_res) + (int64_t)row * ep.ld + c);
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint4 p = r[w];
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&p);
+        float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
+        float2 f2 = __bfloat1622float2(h[2]), f3 = __bfloat1622float2(h[3]);
+        out[2 * w] = make_float4(f0.x + v[8 * w + 0], f0.y + v[8 * w + 1], f1.x + v[8 * w + 2],
+                                 f1.y + v[8 * w + 3]);
+        out[2 * w + 1] = make_float4(f2.x + v[8 * w + 4], f2.y + v[8 * w + 5],
+                                     f3.x + v[8 * w + 6], f3.y + v[8 * w + 7]);
+      }
+    } else {
+      const float4 *r = reinterpret_cast<const float4 *>(
+          reinterpret_cast<const float *>(ep.x_res) + (int64_t)row * ep.ld + c);
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        float4 a = r[w];
+        out[w] = make_float4(a.x + v[4 * w], a.y + v[4 * w + 1], a.z + v[4 * w + 2],
+                             a.w + v[4 * w + 3]);
+      }
+    }
+  }
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, int M, int N, int K,
+                        InProjEpi ip, ResidEpi rs, unsigned *err_word) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  Ctl *ctl = reinterpret_cast<Ctl *>(smem + C::STAGES * C::STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_tiles = (M + BM - 1) / BM;
+  const int n_tiles = (N + BN - 1) / BN;
+  const int n_total = m_tiles * n_tiles;
+  const int kblocks = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(smem_u32(&ctl->full[s]), 1);
+      mbar_init(smem_u32(&ctl->empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&ctl->tfull[b]), 1);
+      mbar_init(smem_u32(&ctl->tempty[b]), 4);
+    }
+    ctl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ctl->tmem_base), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  const AbortFlag ab{&ctl->abort, err_word, ERRBIT_GEMM_TIMEOUT};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph = 0;
+      for (int t = blockIdx.x; t < n_total; t += gridDim.x) {
+        const int tm = t % m_tiles, tn = t / m_tiles;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(smem_u32(&ctl->empty[stage]), ph ^ 1u, ab)) goto producer_done;
+          const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t fb = smem_u32(&ctl->full[stage]);
+          mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+          tma_load_2d(sa, &tmA, kb * BK, tm * BM, fb);
+          tma_load_2d(sa + C::A_BYTES, &tmB, kb * BK, tn * BN, fb);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+    producer_done:;
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(BM, BN, 0, 0);
+      int stage = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      for (int t = blockIdx.x; t < n_total; t += gridDim.x, ++it) {
+        const int b = it & 1;
+        const uint32_t u = (uint32_t)(it >> 1);
+        if (!mbar_wait(smem_u32(&ctl->tempty[b]), (u & 1u) ^ 1u, ab)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(b * BN);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(smem_u32(&ctl->full[stage]), ph, ab)) goto mma_done;
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = sw128_desc(sa + kk * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(sb + kk * 32, 16, 1024);
+            tc_mma_bf16(d, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+          }
+          tc_commit(smem_u32(&ctl->empty[stage]));
+          if (++stage == C::STAGES) {
+            stage = 0;
+            ph ^= 1u;
+          }
+        }
+        tc_commit(smem_u32(&ctl->tfull[b]));
+      }
+    mma_done:;
+    }
+  } else {
+    const int q4 = warp & 3;  // TMEM lanes this warp may read: 32*q4 .. 32*q4+31
+    int it = 0;
+    for (int t = blockIdx.x; t < n_total; t += gridDim.x, ++it) {
+      const int b = it & 1;
+      const uint32_t u = (uint32_t)(it >> 1);
+      if (!mbar_wait(smem_u32(&ctl->tfull[b]), u & 1u, ab)) break;
+      tc_fence_after();
+      const int tm = t % m_tiles, tn = t / m_tiles;
+      const int row = tm * BM + q4 * 32 + lane;
+      const uint32_t tbase = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(b * BN);
+      if (EPI == EPI_INPROJ)
+        epi_inproj<BN>(ip, tbase, tn * BN, N, row, M);
+      else
+        epi_resid<BN>(rs, tbase, tn * BN, N, row, M);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->tempty[b]));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int BN, int EPI>
+cudaError_t launch(const void *A, int64_t lda, const void *B, int M, int N, int K,
+                   const InProjEpi &ip, const ResidEpi &rs, unsigned *err_word, cudaStream_t s,
+                   std::string *err) {
+  using C = Cfg<BN>;
+  if (M <= 0 || N <= 0) return cudaSuccess;
+  CUtensorMap ta, tb;
+  if (!make_tmap_bf16_2d(&ta, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 2, BK, BM, err) ||
+      !make_tmap_bf16_2d(&tb, B, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN, err))
+    return cudaErrorInvalidValue;
+  auto kern = gemm_bf16_tn_kernel<BN, EPI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  int grid = device_sm_count();
+  if (grid > tiles) grid = tiles;
+  kern<<<grid, kThreads, C::SMEM, s>>>(ta, tb, M, N, K, ip, rs, err_word);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_inproj(const void *A, const void *B, int M, int N, int K,
+                               const InProjEpi &ep, unsigned *err_word, cudaStream_t s,
+                               std::string *err) {
+  ResidEpi none{};
+  return launch<256, EPI_INPROJ>(A, K, B, M, N, K, ep, none, err_word, s, err);
+}
+
+cudaError_t launch_gemm_resid(const void *A, int64_t lda, const void *B, int M, int N, int K,
+                              const ResidEpi &ep, unsigned *err_word, cudaStream_t s,
+                              std::string *err) {
+  InProjEpi none{};
+  return launch<256, EPI_RESID>(A, lda, B, M, N, K, none, ep, err_word, s, err);
+}
+
+}  // namespace tr

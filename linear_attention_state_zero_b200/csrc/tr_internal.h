@@ -1,0 +1,85 @@
+// tr_internal.h -- host-side interfaces between the C ABI layer (tr_api.cu) and
+// the kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+namespace tr {
+
+// Device error word bits (OR-ed into the library's error word by the kernels).
+enum : unsigned {
+  ERRBIT_GEMM_TIMEOUT = 1u,
+  ERRBIT_SCAN_TIMEOUT = 2u,
+};
+
+// Epilogue of the input projection: per-head L2 norm of q and k, bf16 q/k/v,
+// gate activations in fp32.
+struct InProjEpi {
+  __nv_bfloat16 *qkv;  // [M, ldq] bf16
+  int64_t ldq;         // 2 H d_k + H d_v
+  float *log_alpha;    // [M, H]
+  float *beta;         // [M, H]
+  int H, dk, dv;
+  int col_offset;      // W_in row that is GEMM column 0 (H d_k when q is skipped)
+  float norm_eps;
+};
+
+// Epilogue of the output projection: x_out = x_res + acc (fp32 out).
+struct ResidEpi {
+  const void *x_res;   // [M, ld] bf16 or fp32
+  int res_is_bf16;
+  float *x_out;        // [M, ld] fp32
+  int64_t ld;
+};
+
+struct ScanLaunch {
+  int n_seqs, H, dk, dv;
+  int64_t T;
+  int dtype;           // TR_DTYPE_*
+  unsigned flags;
+  float scale;
+  int64_t q_stride, k_stride, v_stride, o_stride;  // elements per token
+  const void *q, *k, *v;
+  const float *log_alpha, *beta;
+  const int32_t *cu_seqlens;
+  const int32_t *cu_seqlens_host;
+  const float *S0;
+  void *o;
+  float *S_final;
+  unsigned *err_word;
+};
+
+int device_sm_count();
+
+// 2D bf16 tensor map, 128-byte swizzle: `outer` rows of `inner` elements with
+// `row_stride_bytes` between rows; box = box_inner x box_outer elements.
+bool make_tmap_bf16_2d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t outer,
+                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                       std::string *err);
+
+// C[M, N] = A[M, K] * B[N, K]^T with the input-projection epilogue.
+cudaError_t launch_gemm_inproj(const void *A, const void *B, int M, int N, int K,
+                               const InProjEpi &ep, unsigned *err_word, cudaStream_t s,
+                               std::string *err);
+// C[M, N] = A[M, K] * B[N, K]^T with the residual epilogue; A rows lda elements apart.
+cudaError_t launch_gemm_resid(const void *A, int64_t lda, const void *B, int M, int N, int K,
+                              const ResidEpi &ep, unsigned *err_word, cudaStream_t s,
+                              std::string *err);
+
+cudaError_t launch_rmsnorm(const void *x, int x_is_bf16, const float *gain, int64_t rows, int D,
+                           float eps, void *out, cudaStream_t s);
+
+cudaError_t launch_scan_recurrent(const ScanLaunch &p, cudaStream_t s);
+cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string *err);
+bool scan_chunked_supported(const ScanLaunch &p);
+
+cudaError_t launch_state_error(const float *S, const float *Sh, int64_t n_mats, int64_t mat_elems,
+                               double *partials, double *err_per, double *err_total,
+                               cudaStream_t s);
+
+}  // namespace tr

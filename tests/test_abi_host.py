@@ -1,0 +1,120 @@
+"""The C ABI without a GPU: the library loads, exports every function include/tr.h declares,
+computes the tail length exactly, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import random
+import re
+
+import pytest
+
+import oracle
+import linear_attention_state_zero_b200 as tr
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x10000  # a 16-byte aligned non-NULL address; never dereferenced by validation
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "tr.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tr_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_function_is_exported():
+    names = header_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(tr.lib, n), n
+        assert n in tr._SIGNATURES, "binding lacks a signature for " + n
+
+
+def test_struct_layouts_match_c():
+    # offsets follow the C declaration order with natural alignment
+    assert ctypes.sizeof(tr.ScanArgs) == 16 + 8 + 12 + 4 + 24 + 8 * 10
+    assert tr.ScanArgs.q_stride.offset == 40
+    assert ctypes.sizeof(tr.LALayer) == 24
+    assert tr.GroupArgs.h_tail.offset == 48
+    assert ctypes.sizeof(tr.GroupArgs) == 48 + 6 * 8
+
+
+def test_tail_len_matches_oracle():
+    r = random.Random(5)
+    for _ in range(2000):
+        m = r.randint(0, 1 << 20)
+        num = r.randint(0, 120)
+        den = r.choice([1, 10, 100, 1000, 7])
+        assert tr.tail_len(m, num, den) == oracle.tail_len(m, num, den)
+    assert tr.tail_len(10000, 5, 100) == 500
+    assert tr.tail_len(100, 7, 100) == 7
+    assert tr.lib.tr_tail_len(10, 1, 0) == -1
+    assert tr.lib.tr_tail_len(-1, 1, 2) == -1
+
+
+def _scan_args(**kw):
+    cu = (ctypes.c_int32 * 3)(0, 5, 9)
+    a = tr.ScanArgs(2, 4, 128, 128, 9, tr.TR_DTYPE_BF16, 0, 1.0, 0, 0, 0,
+                    FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.addressof(cu), None, FAKE, FAKE + 4096)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a, cu
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("n_heads", 0, 1), ("dtype", 7, 3), ("d_k", 96, 5), ("d_v", 32, 5), ("flags", 0x80, 1),
+    ("k", None, 1), ("S_final", None, 1), ("cu_seqlens", None, 1), ("total_tokens", 10, 2), ("q", FAKE + 2, 4),
+    ("k_stride", 100, 2), ("S0", FAKE + 4096, 1), ("cu_seqlens_host", None, 1),
+])
+def test_scan_rejects_bad_arguments(field, value, status):
+    a, cu = _scan_args(**{field: value})
+    st = tr.lib.tr_gdn_scan(ctypes.byref(a), None, 0, None)
+    assert st == status, (st, tr.lib.tr_last_error())
+    assert tr.lib.tr_last_error()
+
+
+def test_scan_rejects_bad_cu_seqlens():
+    a, _ = _scan_args()
+    bad = (ctypes.c_int32 * 3)(0, 6, 5)
+    a.cu_seqlens_host = ctypes.addressof(bad)
+    assert tr.lib.tr_gdn_scan(ctypes.byref(a), None, 0, None) == 2
+
+
+def _group_args(**kw):
+    cu = (ctypes.c_int32 * 2)(0, 16)
+    layers = (tr.LALayer * 3)(*[tr.LALayer(None, FAKE, FAKE) for _ in range(3)])
+    a = tr.GroupArgs(1, 16, 128, 128, 2048, 3, 16, 0, 0.0, 0.0, FAKE, FAKE,
+                     ctypes.addressof(cu), layers, FAKE, None)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a, (cu, layers)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("n_layers", 0, 5), ("n_layers", 65, 5), ("d_model", 100, 5), ("d_k", 32, 5),
+    ("flags", 8, 1), ("h_tail", None, 1), ("S_hat", FAKE + 8, 4), ("total_tokens", 17, 2),
+])
+def test_replay_rejects_bad_arguments(field, value, status):
+    a, keep = _group_args(**{field: value})
+    assert tr.lib.tr_replay_group(ctypes.byref(a), None, 0, None) == status
+
+
+def test_replay_skip_flag_forbids_x_out():
+    a, keep = _group_args(flags=tr.TR_SKIP_LAST_OUTPUT, x_out=FAKE)
+    assert tr.lib.tr_replay_group(ctypes.byref(a), None, 0, None) == 1
+
+
+def test_replay_workspace_checks():
+    a, keep = _group_args()
+    need = tr.lib.tr_replay_group_workspace_size(ctypes.byref(a))
+    T, D, H, d = 16, 2048, 16, 128
+    assert need >= T * D * 4 + T * D * 2 + T * (3 * H * d) * 2 + T * H * d * 2
+    assert tr.lib.tr_replay_group(ctypes.byref(a), None, 0, None) == 6
+    assert tr.lib.tr_replay_group(ctypes.byref(a), FAKE, need - 1, None) == 6
+    assert tr.lib.tr_replay_group(ctypes.byref(a), FAKE + 16, need, None) == 4
+
+
+def test_state_error_workspace_and_args():
+    assert tr.lib.tr_state_error_workspace_size(0) == 0
+    assert tr.lib.tr_state_error_workspace_size(100) >= 1600
+    assert tr.lib.tr_state_error(FAKE, FAKE, 100, 128, 128, FAKE, FAKE, None, 0, None) == 6
+    assert tr.lib.tr_state_error(FAKE, FAKE + 4, 1, 8, 8, None, FAKE, FAKE, 4096, None) == 4
+    assert tr.lib.tr_state_error(FAKE, FAKE, -1, 8, 8, None, FAKE, FAKE, 4096, None) == 1

@@ -1,0 +1,107 @@
+"""GPU parity of the group replay (tr_replay_group / tr_replay_groups) against the oracle.
+
+The oracle restates the boundary's cast points (bf16 x_hat, q, k, v, o); everything between
+them is fp64 there.  Tolerance: relative Frobenius error 5e-3 per output tensor."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import linear_attention_state_zero_b200 as tr
+from gpu_util import f64, per_matrix_rel_fro, rel_fro, to_dev
+
+pytestmark = pytest.mark.gpu
+
+TOL = 5e-3
+
+
+def make_group(lengths, D, H, d, L, seed, with_gain=False):
+    layers = synth.la_layers(L, D, H, d, d, seed=seed, with_gain=with_gain)
+    h = torch.cat([synth.hidden_prefix(max(n, 1), D, seed * 10 + i)[:n]
+                   for i, n in enumerate(lengths)]) if sum(lengths) else \
+        torch.zeros(0, D, dtype=torch.bfloat16)
+    return h, layers, synth.cu_seqlens_of(lengths)
+
+
+@pytest.mark.parametrize("skip", [False, True])
+def test_small_group_varlen(cuda_device, skip):
+    D, H, d, L = 256, 2, 128, 3
+    lengths = [37, 130, 0, 201, 64]
+    h, layers, cu = make_group(lengths, D, H, d, L, seed=301, with_gain=True)
+    S, x = tr.replay_group(h.to(cuda_device), cu, to_dev(layers, cuda_device), H, d, d,
+                           skip_last_output=skip)
+    wS, wx = oracle.replay_group(h, cu, layers, H, d, d, skip_last_output=skip)
+    for l in range(L):
+        assert rel_fro(S[l], wS[l]) < TOL, l
+    nz = [0, 1, 3, 4]
+    assert np.all(per_matrix_rel_fro(S[:, nz], wS[:, nz]) < 2 * TOL)
+    assert not f64(S[:, 2]).any()
+    if skip:
+        assert x is None
+    else:
+        assert rel_fro(x, wx) < TOL
+
+
+def test_one_group_paper_shape(cuda_device):
+    """One group of 3 LA layers, d_model 2048, 16 heads of 128, matched prefix m = 32768,
+    r = 5% -> the last 1639 cached hiddens are replayed from a zero state."""
+    D, H, d, L, m = 2048, 16, 128, 3, 32768
+    k = tr.tail_len(m, 5, 100)
+    assert k == 1639
+    seed = synth.SEED_BASE + 1
+    h = synth.hidden_prefix(m, D, seed)[m - k:].contiguous()
+    layers = synth.la_layers(L, D, H, d, d, seed=seed)
+    cu = synth.cu_seqlens_of([k])
+    S, x = tr.replay_group(h.to(cuda_device), cu, to_dev(layers, cuda_device), H, d, d)
+    wS, wx = oracle.replay_group(h, cu, layers, H, d, d)
+    for l in range(L):
+        assert rel_fro(S[l], wS[l]) < TOL, l
+    assert rel_fro(x, wx) < TOL
+    # the launch configuration the benchmark times (last layer's output skipped)
+    S2, x2 = tr.replay_group(h.to(cuda_device), cu, to_dev(layers, cuda_device), H, d, d,
+                             skip_last_output=True)
+    assert x2 is None
+    for l in range(L):
+        assert rel_fro(S2[l], wS[l]) < TOL, l
+
+
+def test_groups_call_equals_single_calls(cuda_device):
+    D, H, d, L = 256, 2, 128, 2
+    gs = []
+    singles = []
+    for g in range(3):
+        h, layers, cu = make_group([50 + 40 * g, 17], D, H, d, L, seed=310 + g)
+        dl = to_dev(layers, cuda_device)
+        gs.append(tr.GroupReplay(h.to(cuda_device), cu, dl, H, d, d))
+        singles.append(tr.replay_group(h.to(cuda_device), cu, dl, H, d, d))
+    outs = tr.GroupsReplay(gs).run()
+    torch.cuda.synchronize()
+    for (S, x), (S1, x1) in zip(outs, singles):
+        assert torch.equal(S, S1) and torch.equal(x, x1)
+
+
+def test_all_empty_tails_give_zero_states(cuda_device):
+    D, H, d = 128, 2, 64
+    layers = synth.la_layers(2, D, H, d, d, seed=320)
+    h = torch.zeros(0, D, dtype=torch.bfloat16, device=cuda_device)
+    S, x = tr.replay_group(h, [0, 0, 0], to_dev(layers, cuda_device), H, d, d)
+    assert S.shape == (2, 2, H, d, d) and not S.any()
+
+
+def test_full_prefill_equals_tail_when_decay_is_strong(cuda_device):
+    """k = m runs the same path over the whole prefix (the full-prefill S_m).  With these
+    weights alpha = exp(-softplus(a)) is about 1/2, so by the bound of the reading notes
+    (section 2.3) the tail replay's error is below prod(alpha) ~ 2^-400 for the first layer:
+    S_m and S_hat_m must agree to rounding, and the GPU error must be tiny."""
+    D, H, d, L, m = 512, 4, 128, 3, 4096
+    k = tr.tail_len(m, 10, 100)
+    seed = 330
+    hfull = synth.hidden_prefix(m, D, seed)
+    layers = to_dev(synth.la_layers(L, D, H, d, d, seed=seed), cuda_device)
+    S_m, _ = tr.replay_group(hfull.to(cuda_device), [0, m], layers, H, d, d,
+                             skip_last_output=True)
+    S_hat, _ = tr.replay_group(hfull[m - k:].contiguous().to(cuda_device), [0, k], layers, H, d,
+                               d, skip_last_output=True)
+    _, tot = tr.state_error(S_m.reshape(-1, d, d), S_hat.reshape(-1, d, d))
+    assert float(tot.item()) < 1e-5

@@ -1,0 +1,132 @@
+"""GPU parity of the Eq. (1) scan (tr_gdn_scan) against the fp64 oracle.
+
+Tolerances: relative Frobenius error 1e-5 on the fp32 path, 5e-3 with bf16 inputs and fp32
+state (per output tensor), as the workloads require.  The state error reported on the GPU is
+compared absolutely: |err_gpu - err_oracle| <= 2e-5 (fp32) / 1e-2 (bf16)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import linear_attention_state_zero_b200 as tr
+from gpu_util import f64, per_matrix_rel_fro, rel_fro
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32, TOL_BF16 = 1e-5, 5e-3
+
+
+def run_gpu(case, dev, **kw):
+    g = lambda t: None if t is None else t.to(dev)
+    return tr.gdn_scan(g(case.q), g(case.k), g(case.v), g(case.log_alpha), g(case.beta),
+                       case.cu_seqlens, S0=g(case.S0), **kw)
+
+
+def run_oracle(case, **kw):
+    return oracle.gdn_scan(case.q, case.k, case.v, case.log_alpha, case.beta, case.cu_seqlens,
+                           S0=case.S0, **kw)
+
+
+def test_single_head_fp32_prefix_and_tail(cuda_device):
+    """One head, d_k = d_v = 64, fp32, m = 4096, r = 5% (k = 205): S_m, S_hat_m, o and the error."""
+    m = 4096
+    k = tr.tail_len(m, 5, 100)
+    assert k == 205
+    full, tail = synth.scan_case_from_prefix(m, k, 1, 64, 64, torch.float32, 0.90, 1.00,
+                                             seed=synth.SEED_BASE + 0)
+    o_f, S_m = run_gpu(full, cuda_device)
+    o_t, S_hat = run_gpu(tail, cuda_device)
+    wo_f, wS_m = run_oracle(full)
+    wo_t, wS_hat = run_oracle(tail)
+    assert rel_fro(S_m, wS_m) < TOL_F32
+    assert rel_fro(S_hat, wS_hat) < TOL_F32
+    assert rel_fro(o_f, wo_f) < TOL_F32
+    assert rel_fro(o_t, wo_t) < TOL_F32
+    per, tot = tr.state_error(S_m, S_hat)
+    wper, wtot = oracle.state_error(wS_m, wS_hat)
+    assert abs(float(tot.item()) - wtot) <= 2e-5
+    np.testing.assert_allclose(f64(per), wper, atol=2e-5)
+
+
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 128), (128, 64)])
+@pytest.mark.parametrize("recurrent", [True, False])
+def test_bf16_varlen_ragged(cuda_device, dk, dv, recurrent):
+    lengths = [1, 63, 64, 65, 300, 0, 129]
+    case = synth.scan_case(lengths, 4, dk, dv, torch.bfloat16, 0.90, 1.00, seed=201)
+    o, S = run_gpu(case, cuda_device, recurrent=recurrent)
+    wo, wS = run_oracle(case)
+    assert rel_fro(o, wo) < TOL_BF16
+    assert rel_fro(S, wS) < TOL_BF16
+    assert np.all(per_matrix_rel_fro(S[[0, 1, 2, 3, 4, 6]], wS[[0, 1, 2, 3, 4, 6]]) < 1e-2)
+    assert not f64(S[5]).any()  # an empty sequence keeps the zero start
+
+
+@pytest.mark.parametrize("alpha_lo", [0.80, 0.97])
+def test_bf16_long_sequence(cuda_device, alpha_lo):
+    case = synth.scan_case([2500, 777], 8, 128, 128, torch.bfloat16, alpha_lo, 1.00, seed=202)
+    o, S = run_gpu(case, cuda_device)
+    wo, wS = run_oracle(case)
+    assert rel_fro(o, wo) < TOL_BF16
+    assert rel_fro(S, wS) < TOL_BF16
+
+
+@pytest.mark.parametrize("dtype,tol", [(torch.float32, TOL_F32), (torch.bfloat16, TOL_BF16)])
+def test_initial_state_and_split(cuda_device, dtype, tol):
+    """S0 is honoured, and scanning x[:t] then x[t:] from the state reached equals scanning x."""
+    case = synth.scan_case([400], 2, 128, 128, dtype, 0.9, 1.0, seed=203, with_S0=True)
+    o, S = run_gpu(case, cuda_device)
+    wo, wS = run_oracle(case)
+    assert rel_fro(S, wS) < tol and rel_fro(o, wo) < tol
+    t = 150
+    first = synth.ScanCase(case.q[:t], case.k[:t], case.v[:t], case.log_alpha[:t], case.beta[:t],
+                           synth.cu_seqlens_of([t]), case.S0)
+    o1, S1 = run_gpu(first, cuda_device)
+    second = synth.ScanCase(case.q[t:], case.k[t:], case.v[t:], case.log_alpha[t:],
+                            case.beta[t:], synth.cu_seqlens_of([400 - t]), S1.cpu())
+    o2, S2 = run_gpu(second, cuda_device)
+    assert rel_fro(S2, wS) < tol
+    assert rel_fro(torch.cat([o1, o2]), wo) < tol
+
+
+def test_identity_transition_keeps_state(cuda_device):
+    """alpha = 1, beta = 0: the state is S0 exactly and o_t = S0^T q_t."""
+    case = synth.scan_case([77, 5], 2, 128, 128, torch.float32, 0.9, 1.0, seed=204, with_S0=True)
+    case.log_alpha.zero_()
+    case.beta.zero_()
+    o, S = run_gpu(case, cuda_device)
+    assert torch.equal(S.cpu(), case.S0)
+    wo, _ = run_oracle(case)
+    assert rel_fro(o, wo) < TOL_F32
+
+
+def test_delta_rule_recall(cuda_device):
+    """beta = 1 and q_t = k_t (unit): o_t = M_t^T k_t = v_t exactly in exact arithmetic."""
+    case = synth.scan_case([200], 2, 128, 128, torch.float32, 0.5, 1.0, seed=205)
+    case.beta.fill_(1.0)
+    o, _ = tr.gdn_scan(case.k.to(cuda_device), case.k.to(cuda_device), case.v.to(cuda_device),
+                       case.log_alpha.to(cuda_device), case.beta.to(cuda_device), case.cu_seqlens)
+    assert rel_fro(o, case.v) < 1e-5
+
+
+@pytest.mark.parametrize("dtype,tol", [(torch.float32, TOL_F32), (torch.bfloat16, TOL_BF16)])
+def test_normalize_flag(cuda_device, dtype, tol):
+    case = synth.scan_case([100, 33], 2, 128, 128, dtype, 0.9, 1.0, seed=206)
+    raw_q = (synth.normal(case.q.shape, 206, 90) * 3).to(dtype)
+    raw_k = (synth.normal(case.k.shape, 206, 91) * 0.5).to(dtype)
+    raw = synth.ScanCase(raw_q, raw_k, case.v, case.log_alpha, case.beta, case.cu_seqlens)
+    o, S = run_gpu(raw, cuda_device, normalize_qk=True)
+    wo, wS = run_oracle(raw, normalize_qk=True)
+    assert rel_fro(S, wS) < tol and rel_fro(o, wo) < tol
+
+
+def test_no_readout(cuda_device):
+    case = synth.scan_case([300, 50], 4, 128, 128, torch.bfloat16, 0.9, 1.0, seed=207)
+    o, S = run_gpu(case, cuda_device, want_o=False)
+    assert o is None
+    _, wS = run_oracle(case, want_o=False)
+    assert rel_fro(S, wS) < TOL_BF16
+
+
+def test_check_reports_clean_state(cuda_device):
+    tr.check()
