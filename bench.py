@@ -284,9 +284,12 @@ def our_arm(args):
     value = world * k / (ms_per_step * 1e-3)
 
     # per-kernel breakdown (launch order: per layer rmsnorm, in-proj, scan[, out-proj])
+    per_scan = (n_k - (L - 1)) // L - 2
+    scan_names = ["scan_prep", "scan_chain"] if per_scan == 2 else ["scan"]
     names = []
     for l in range(L):
-        names += ["rmsnorm", "in_proj", "scan"] + ([] if l == L - 1 else ["out_proj"])
+        names += ["rmsnorm", "in_proj"] + scan_names + ([] if l == L - 1 else ["out_proj"])
+    assert len(names) == n_k
     avg = [sum(x) / len(x) for x in kern_ms]
     brk = {}
     for n, a in zip(names, avg):

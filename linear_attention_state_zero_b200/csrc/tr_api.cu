@@ -132,6 +132,33 @@ bool make_tmap_bf16_2d(CUtensorMap *tm, const void *base, uint64_t inner, uint64
   return true;
 }
 
+bool make_tmap_f32_2d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t outer,
+                      uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                      std::string *err) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    if (err) *err = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    if (err) {
+      char b[160];
+      snprintf(b, sizeof(b), "cuTensorMapEncodeTiled (fp32) failed (%d): dims %llu x %llu",
+               (int)r, (unsigned long long)inner, (unsigned long long)outer);
+      *err = b;
+    }
+    return false;
+  }
+  return true;
+}
+
 }  // namespace tr
 
 // ---------------------------------------------------------------- validation
@@ -206,6 +233,8 @@ tr_status validate_scan(const tr_scan_args *a, tr::ScanLaunch *out) {
   p.o = a->o;
   p.S_final = a->S_final;
   p.err_word = nullptr;
+  p.ws = nullptr;
+  p.ws_bytes = 0;
   return TR_OK;
 }
 
@@ -213,11 +242,21 @@ bool use_chunked(const tr::ScanLaunch &p) {
   return p.dtype == TR_DTYPE_BF16 && !(p.flags & TR_SCAN_RECURRENT) && tr::scan_chunked_supported(p);
 }
 
-tr_status run_scan(const tr::ScanLaunch &p, cudaStream_t s) {
+size_t scan_ws_bytes(const tr::ScanLaunch &p) {
+  if (!p.cu_seqlens_host) return 0;
+  return use_chunked(p) ? tr::scan_chunked_workspace(p) : 0;
+}
+
+int scan_kernel_count(const tr::ScanLaunch &p) {
+  return use_chunked(p) ? tr::scan_chunked_kernels() : 1;
+}
+
+tr_status run_scan(const tr::ScanLaunch &p, cudaStream_t s,
+                   const std::function<cudaError_t()> &between = nullptr) {
   cudaError_t e;
   if (use_chunked(p)) {
     std::string err;
-    e = tr::launch_scan_chunked(p, s, &err);
+    e = tr::launch_scan_chunked(p, s, &err, between);
     if (e != cudaSuccess)
       return err.empty() ? cuda_fail(e, "scan (chunked)") : fail(TR_ERR_CUDA, "%s", err.c_str());
   } else {
@@ -229,9 +268,24 @@ tr_status run_scan(const tr::ScanLaunch &p, cudaStream_t s) {
 
 // ------------------------------------------------------------- replay group
 struct GroupLayout {
-  size_t x, xhat, qkv, la, beta, o, total;
+  size_t x, xhat, qkv, la, beta, o, scan, total;
   int64_t ldq;
 };
+
+// The scan launch of one LA layer of a group (pointers filled in by the caller).
+tr::ScanLaunch group_scan_launch(const tr_group_args *a) {
+  tr::ScanLaunch sp{};
+  sp.n_seqs = a->n_seqs;
+  sp.H = a->n_heads;
+  sp.dk = a->d_k;
+  sp.dv = a->d_v;
+  sp.T = a->total_tokens;
+  sp.dtype = TR_DTYPE_BF16;
+  sp.flags = 0;
+  sp.scale = 1.f;
+  sp.cu_seqlens_host = a->cu_seqlens_host;
+  return sp;
+}
 
 GroupLayout group_layout(const tr_group_args *a) {
   GroupLayout L;
@@ -244,6 +298,7 @@ GroupLayout group_layout(const tr_group_args *a) {
   L.la = off;   off = align256(off + T * H * 4);
   L.beta = off; off = align256(off + T * H * 4);
   L.o = off;    off = align256(off + T * H * (size_t)a->d_v * 2);
+  L.scan = off; off = align256(off + scan_ws_bytes(group_scan_launch(a)));
   L.total = off;
   return L;
 }
@@ -293,7 +348,7 @@ int group_kernel_count(const tr_group_args *a) {
   for (int l = 0; l < a->n_layers; ++l) {
     const bool last = l == a->n_layers - 1;
     const bool skip = last && (a->flags & TR_SKIP_LAST_OUTPUT);
-    n += 3;
+    n += 2 + scan_kernel_count(group_scan_launch(a));
     if (!skip && (!last || a->x_out)) n += 1;
   }
   return n;
@@ -343,15 +398,9 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
     if (e != cudaSuccess)
       return err.empty() ? cuda_fail(e, "input projection") : fail(TR_ERR_CUDA, "%s", err.c_str());
     if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
-    tr::ScanLaunch sp;
-    sp.n_seqs = a->n_seqs;
-    sp.H = H;
-    sp.dk = dk;
-    sp.dv = dv;
-    sp.T = T;
-    sp.dtype = TR_DTYPE_BF16;
-    sp.flags = 0;
-    sp.scale = 1.f;
+    tr::ScanLaunch sp = group_scan_launch(a);
+    sp.ws = base + L.scan;
+    sp.ws_bytes = L.total - L.scan;
     sp.q_stride = sp.k_stride = sp.v_stride = L.ldq;
     sp.o_stride = (int64_t)H * dv;
     sp.q = skip ? nullptr : qkv;
@@ -365,7 +414,7 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
     sp.o = skip ? nullptr : obuf;
     sp.S_final = a->S_hat + (size_t)l * state_elems;
     sp.err_word = err_word;
-    tr_status st = run_scan(sp, s);
+    tr_status st = run_scan(sp, s, [&]() { return mk->mark(s); });
     if (st != TR_OK) return st;
     if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
     if (!skip) {
@@ -410,16 +459,22 @@ int64_t tr_tail_len(int64_t m, int64_t r_num, int64_t r_den) {
 }
 
 size_t tr_gdn_scan_workspace_size(const tr_scan_args *args) {
-  (void)args;
-  return 0;
+  tr::ScanLaunch p;
+  if (validate_scan(args, &p) != TR_OK) return 0;
+  return scan_ws_bytes(p);
 }
 
 tr_status tr_gdn_scan(const tr_scan_args *args, void *ws, size_t ws_bytes, void *stream) {
-  (void)ws;
-  (void)ws_bytes;
   tr::ScanLaunch p;
   tr_status st = validate_scan(args, &p);
   if (st != TR_OK) return st;
+  const size_t need = scan_ws_bytes(p);
+  if (need > 0 && (!ws || ws_bytes < need))
+    return fail(TR_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", ws_bytes, need);
+  if (need > 0 && (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(TR_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  p.ws = ws;
+  p.ws_bytes = ws_bytes;
   int dev;
   unsigned *errw;
   std::string err;
@@ -430,7 +485,7 @@ tr_status tr_gdn_scan(const tr_scan_args *args, void *ws, size_t ws_bytes, void 
 }
 
 size_t tr_replay_group_workspace_size(const tr_group_args *args) {
-  if (!args || args->total_tokens < 0 || args->d_model <= 0 || args->n_heads <= 0) return 0;
+  if (validate_group(args) != TR_OK) return 0;
   return group_layout(args).total;
 }
 

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <functional>
 #include <string>
 
 namespace tr {
@@ -52,6 +53,8 @@ struct ScanLaunch {
   void *o;
   float *S_final;
   unsigned *err_word;
+  void *ws;            // scan workspace (chunked kernels), ws_bytes long
+  size_t ws_bytes;
 };
 
 int device_sm_count();
@@ -74,9 +77,18 @@ cudaError_t launch_gemm_resid(const void *A, int64_t lda, const void *B, int M, 
 cudaError_t launch_rmsnorm(const void *x, int x_is_bf16, const float *gain, int64_t rows, int D,
                            float eps, void *out, cudaStream_t s);
 
+// 2D fp32 tensor map, 128-byte swizzle (box_inner * 4 must be <= 128).
+bool make_tmap_f32_2d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t outer,
+                      uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                      std::string *err);
+
 cudaError_t launch_scan_recurrent(const ScanLaunch &p, cudaStream_t s);
-cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string *err);
+// Two launches (prep, chain); `between` runs after the first one is enqueued.
+cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string *err,
+                                const std::function<cudaError_t()> &between);
 bool scan_chunked_supported(const ScanLaunch &p);
+size_t scan_chunked_workspace(const ScanLaunch &p);  // needs p.cu_seqlens_host, H, dv
+int scan_chunked_kernels();
 
 cudaError_t launch_state_error(const float *S, const float *Sh, int64_t n_mats, int64_t mat_elems,
                                double *partials, double *err_per, double *err_total,
