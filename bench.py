@@ -45,7 +45,36 @@ def parse():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--profile", choices=["scan", "group"], default=None,
+                   help="run only one workload a few times (for ncu captures), no JSON line")
     return p.parse_args()
+
+
+def profile_run(args):
+    """A short run of one workload for profilers: the scan cell or the group replay step."""
+    import torch
+    import synth
+    import linear_attention_state_zero_b200 as tr
+    dev = torch.device("cuda", 0)
+    if args.profile == "scan":
+        k5 = tr.tail_len(32768, 10, 100)
+        case = synth.scan_case([k5], 32, 128, 128, torch.bfloat16, 0.97, 1.0,
+                               seed=synth.SEED_BASE + 4)
+        t = [x.to(dev) for x in (case.q, case.k, case.v, case.log_alpha, case.beta)]
+        for _ in range(args.warmup + args.steps):
+            tr.gdn_scan(*t, case.cu_seqlens)
+    else:
+        k = tr.tail_len(M_PREFIX, R_NUM, R_DEN)
+        seed = synth.SEED_BASE + 1
+        h = synth.hidden_prefix(M_PREFIX, D, seed)[M_PREFIX - k:].contiguous().to(dev)
+        layers = [tr.Layer(l.W_in.to(dev), l.W_o.to(dev))
+                  for l in synth.la_layers(L, D, H, DH, DH, seed=seed)]
+        rep = tr.GroupReplay(h, [0, k], layers, H, DH, DH, skip_last_output=True)
+        for _ in range(args.warmup + args.steps):
+            rep.run()
+    torch.cuda.synchronize()
+    tr.check()
+    print("profile run done:", args.profile)
 
 
 def load_peaks():
@@ -284,12 +313,18 @@ def our_arm(args):
     value = world * k / (ms_per_step * 1e-3)
 
     # per-kernel breakdown (launch order: per layer rmsnorm, in-proj, scan[, out-proj])
-    per_scan = (n_k - (L - 1)) // L - 2
-    scan_names = ["scan_prep", "scan_chain"] if per_scan == 2 else ["scan"]
+    # launch order per layer: rmsnorm, in_proj, scan kernels, out_proj (not after the last
+    # layer, whose readout and output projection are skipped)
+    chunked = n_k == L * 4 + (L - 1) * 2
     names = []
     for l in range(L):
-        names += ["rmsnorm", "in_proj"] + scan_names + ([] if l == L - 1 else ["out_proj"])
-    assert len(names) == n_k
+        last = l == L - 1
+        if chunked:
+            scan_names = ["scan_prep", "scan_chain"] + ([] if last else ["scan_out"])
+        else:
+            scan_names = ["scan"]
+        names += ["rmsnorm", "in_proj"] + scan_names + ([] if last else ["out_proj"])
+    assert len(names) == n_k, (len(names), n_k)
     avg = [sum(x) / len(x) for x in kern_ms]
     brk = {}
     for n, a in zip(names, avg):
@@ -393,7 +428,9 @@ def our_arm(args):
 
 def main():
     args = parse()
-    if args.impl == "reference":
+    if args.profile:
+        profile_run(args)
+    elif args.impl == "reference":
         reference_arm(args)
     else:
         our_arm(args)

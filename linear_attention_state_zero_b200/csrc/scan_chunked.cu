@@ -40,18 +40,23 @@ namespace {
 constexpr int C = 64;      // chunk length
 constexpr int DK = 128;    // key dimension handled here
 constexpr int DVS = 64;    // d_v columns per chain CTA
-constexpr int kThreads = 128;
 
 // --------------------------------------------------------------- helpers
-__device__ __forceinline__ uint64_t desc_k(uint32_t base, int kk, uint32_t half_stride) {
-  // K-major operand: 128-byte rows, 64-column halves `half_stride` bytes apart; K step kk
-  // (16 elements) starts 32 bytes further inside the 128-byte swizzle atom.
-  return sw128_desc(base + (uint32_t)(kk >> 2) * half_stride + (uint32_t)(kk & 3) * 32u, 16, 1024);
+// Shared-memory descriptors are built once per operand (sw128_desc) and advanced
+// per K step by adding to the 16-byte start-address field only.
+//   K-major operand: 128-byte rows, 64-column halves `half_stride` bytes apart; K step kk
+//   (16 elements) starts 32 bytes further inside the 128-byte swizzle atom.
+//   MN-major operand: rows are the K dimension, 128-byte rows hold 64 M/N elements
+//   (64-element blocks LBO bytes apart); K step kk = 16 rows = 2048 bytes.
+__device__ __forceinline__ uint64_t kmaj(uint32_t base) { return sw128_desc(base, 16, 1024); }
+__device__ __forceinline__ uint64_t mnmaj(uint32_t base, uint32_t lbo) {
+  return sw128_desc(base, lbo, 1024);
 }
-__device__ __forceinline__ uint64_t desc_mn(uint32_t base, int kk, uint32_t lbo) {
-  // MN-major operand: rows are the K dimension, 128-byte rows hold 64 M/N elements,
-  // 64-element M/N blocks `lbo` bytes apart; K step kk = 16 rows = 2048 bytes.
-  return sw128_desc(base + (uint32_t)kk * 2048u, lbo, 1024);
+__device__ __forceinline__ uint64_t desc_k(uint64_t d0, int kk, uint32_t half_stride) {
+  return d0 + (((uint32_t)(kk >> 2) * half_stride + (uint32_t)(kk & 3) * 32u) >> 4);
+}
+__device__ __forceinline__ uint64_t desc_mn(uint64_t d0, int kk) {
+  return d0 + (uint64_t)kk * 128u;
 }
 
 // 32 consecutive bf16 (v[i] * s) into row `row` of a 128-byte-row swizzled tile at col0.
@@ -80,16 +85,6 @@ __device__ __forceinline__ void load_row8_bf16(const uint8_t *tile, int row, int
   }
 }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
-  float a[16], b[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    a[i] = v[i];
-    b[i] = v[16 + i];
-  }
-  tmem_st16(taddr, a);
-  tmem_st16(taddr + 16, b);
-}
 
 // sum over sequences i < seq of ceil(len_i / C); every thread of the CTA gets the value
 __device__ int chunk_base(const int32_t *cu, int seq, int *red) {
@@ -133,6 +128,7 @@ struct ScanWs {
   float *B;          // [slots][128][dv]   B_c = K^T diag(gamma') U~
   float *O;          // [slots][64][dv]    O0 = P U~
   float *G;          // [slots]            gamma_C
+  __nv_bfloat16 *M;  // [slots][128][dv]   bf16 state at the chunk start (chain -> readout)
   int64_t slots;
 };
 
@@ -160,6 +156,7 @@ ScanWs ws_layout(const ScanLaunch &p, void *base, size_t *total) {
   const size_t oB = off; off = align256(off + S * 128 * (size_t)p.dv * 4);
   const size_t oO = off; off = align256(off + S * 64 * (size_t)p.dv * 4);
   const size_t oG = off; off = align256(off + S * 4);
+  const size_t oM = off; off = align256(off + S * 128 * (size_t)p.dv * 2);
   if (total) *total = off;
   uint8_t *b = static_cast<uint8_t *>(base);
   if (b) {
@@ -168,59 +165,92 @@ ScanWs ws_layout(const ScanLaunch &p, void *base, size_t *total) {
     w.B = reinterpret_cast<float *>(b + oB);
     w.O = reinterpret_cast<float *>(b + oO);
     w.G = reinterpret_cast<float *>(b + oG);
+    w.M = reinterpret_cast<__nv_bfloat16 *>(b + oM);
   }
   return w;
 }
 
 // ============================================================ prep kernel
-// shared memory (bytes from a 1024-aligned base)
-constexpr uint32_t P_KQ = 0;        // [half][K rows 0-63 | Q rows 64-127]      32 KB
-constexpr uint32_t P_V = 32768;     // [64-col block][64 t][128 B]              16 KB
-constexpr uint32_t P_AP = 49152;    // 128 x 64: rows 0-63 zero, 64-127 = P     16 KB
-constexpr uint32_t P_TS = 65536;    // 128 x 64: rows 0-63 = -T'', 64-127 = T'  16 KB
-constexpr uint32_t P_W = 81920;     // [half][64 t][128 B]  W                   16 KB
-constexpr uint32_t P_WG = 98304;    // gamma' W                                  16 KB
-constexpr uint32_t P_UT = 114688;   // [block][64 t][128 B]  U~                 16 KB
-constexpr uint32_t P_UG = 131072;   // gamma' U~                                 16 KB
-constexpr uint32_t P_AS = 147456;   // 64 x 65 fp32: A
-constexpr int AS_LD = 65;
-constexpr uint32_t P_CTL = 164096;
-constexpr size_t PREP_SMEM = P_CTL + 1024 + 1024;
+// 256 threads, persistent over work items (slot order: chunk-major, head-minor), with
+// the next items' K/Q/V tiles prefetched by TMA into a second buffer.
+// shared memory (bytes from a 1024-aligned base):
+constexpr uint32_t P_IN = 0;          // 2 x 48 KB: [KQ 32 KB: half x (K rows 0-63 | Q rows 64-127)][V 16 KB]
+constexpr uint32_t P_IN_BYTES = 49152;
+constexpr uint32_t P_AP = 98304;      // 128 x 64 bf16: rows 0-63 zero, 64-127 = P
+constexpr uint32_t P_TSH = 114688;    // [-T''; T'] high bf16 parts   (after P2: gamma' U~ high)
+constexpr uint32_t P_TSL = 131072;    // [-T''; T'] low bf16 parts    (after P2: gamma' U~ low)
+constexpr uint32_t P_AW = 147456;     // A fp32 [64][68] during the inverse; then W (16 KB) + gamma' W
+constexpr uint32_t P_TU = 180224;     // T fp32 [64][68] + X fp32 [32][36]; then U~ high + U~ low
+constexpr uint32_t P_END = 212992;
+constexpr int LDA = 68;               // fp32 row stride of A and T (16-byte aligned rows)
+constexpr int LDX = 36;
+constexpr size_t PREP_SMEM = P_END + 1024 + 1024;
+constexpr int kPrepThreads = 256;
+constexpr int kMaxSeqsChunked = 1024;
 
 struct PrepCtl {
-  uint64_t tma_bar;
+  uint64_t tma_bar[2];
   uint64_t mma_bar;
   uint32_t tmem;
   int abort;
-  float g[C];
+  float g[C];      // inclusive cumsum of log alpha over the chunk
   float beta[C];
-  int red[4];
+  float bg[C];     // beta * gamma
+  int cu_chunks[kMaxSeqsChunked + 1];
 };
 
+// hi + lo bf16 split of 32 values (v[i] * s) into two 128-byte-row swizzled tiles.
+__device__ __forceinline__ void store_row_split(uint8_t *hi, uint8_t *lo, int row, int col0,
+                                                const float *v, float s) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float a = v[8 * w + 2 * i] * s, b = v[8 * w + 2 * i + 1] * s;
+      const __nv_bfloat162 hh = __floats2bfloat162_rn(a, b);
+      const float2 hf = __bfloat1622float2(hh);
+      const __nv_bfloat162 ll = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+      h[i] = *reinterpret_cast<const uint32_t *>(&hh);
+      l[i] = *reinterpret_cast<const uint32_t *>(&ll);
+    }
+    const uint32_t off = sw128_offset((uint32_t)row, (uint32_t)(col0 + 8 * w) * 2u);
+    st_shared_v4(smem_u32(hi + off), h[0], h[1], h[2], h[3]);
+    st_shared_v4(smem_u32(lo + off), l[0], l[1], l[2], l[3]);
+  }
+}
+
 template <int DV>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kPrepThreads, 1)
     scan_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, ScanLaunch p, ScanWs ws) {
+                     const __grid_constant__ CUtensorMap tm_v, ScanLaunch p, ScanWs ws,
+                     int total_chunks) {
   extern __shared__ uint8_t smem_raw[];
+  __shared__ PrepCtl ctl_s;
+  PrepCtl *ctl = &ctl_s;
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
-  PrepCtl *ctl = reinterpret_cast<PrepCtl *>(sm + P_CTL);
-  float *As = reinterpret_cast<float *>(sm + P_AS);
+  float *As = reinterpret_cast<float *>(sm + P_AW);
+  float *Ts = reinterpret_cast<float *>(sm + P_TU);
+  float *Xs = Ts + C * LDA;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q4 = warp & 3, hsel = warp >> 2;   // TMEM lane quarter, column half
+  const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+  const int row = q4 * 32 + lane;              // TMEM lane = row of a 128-row result
   const int H = p.H;
-  const int c = blockIdx.x;
-  const int seq = blockIdx.y / H, head = blockIdx.y % H;
-  const int t_begin = p.cu_seqlens[seq], t_end = p.cu_seqlens[seq + 1];
-  if (c * C >= t_end - t_begin) return;  // uniform: this sequence has fewer chunks
-  const int t0 = t_begin + c * C;
-  const int nv = min(C, t_end - t0);
   const bool want_o = p.o != nullptr;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  const int cb = chunk_base(p.cu_seqlens, seq, ctl->red);
-  const int64_t slot = ((int64_t)cb + c) * H + head;
+  const int64_t n_items = (int64_t)total_chunks * H;
 
+  // first chunk of every sequence
   if (tid == 0) {
-    mbar_init(smem_u32(&ctl->tma_bar), 1);
+    int acc = 0;
+    for (int i = 0; i < p.n_seqs; ++i) {
+      ctl->cu_chunks[i] = acc;
+      acc += (p.cu_seqlens[i + 1] - p.cu_seqlens[i] + C - 1) / C;
+    }
+    ctl->cu_chunks[p.n_seqs] = acc;
+    mbar_init(smem_u32(&ctl->tma_bar[0]), 1);
+    mbar_init(smem_u32(&ctl->tma_bar[1]), 1);
     mbar_init(smem_u32(&ctl->mma_bar), 1);
     ctl->abort = 0;
     fence_mbar_init();
@@ -229,51 +259,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_u32(&ctl->tmem), 512);
     tmem_relinquish();
   }
-  for (int i = tid; i < 8192 / 16; i += kThreads) st_shared_v4(smem_u32(sm + P_AP) + 16 * i, 0, 0, 0, 0);
+  for (int i = tid; i < 8192 / 16; i += kPrepThreads) st_shared_v4(smem_u32(sm + P_AP) + 16 * i, 0, 0, 0, 0);
   if (!want_o)
-    for (int i = tid; i < 2 * 8192 / 16; i += kThreads)
-      st_shared_v4(smem_u32(sm + P_KQ + (i >> 9) * 16384 + 8192) + 16 * (i & 511), 0, 0, 0, 0);
+    for (int i = tid; i < 4 * 8192 / 16; i += kPrepThreads) {
+      const int blk = i >> 9;  // (buffer, half)
+      st_shared_v4(smem_u32(sm + P_IN + (blk >> 1) * P_IN_BYTES + (blk & 1) * 16384 + 8192) +
+                       16 * (i & 511), 0, 0, 0, 0);
+    }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem;
   const AbortFlag ab{&ctl->abort, p.err_word, ERRBIT_SCAN_TIMEOUT};
-  const uint32_t kq_u = smem_u32(sm + P_KQ);
 
-  if (tid == 0) {
-    const uint32_t bar = smem_u32(&ctl->tma_bar);
-    fence_proxy_async_smem();
+  // (sequence, chunk) of an item
+  auto locate = [&](int64_t item, int &seq, int &cc) {
+    const int chunk = (int)(item / H);
+    int lo = 0, hi = p.n_seqs - 1;
+    while (lo < hi) {  // last sequence whose first chunk is <= chunk
+      const int mid = (lo + hi + 1) >> 1;
+      if (ctl->cu_chunks[mid] <= chunk) lo = mid; else hi = mid - 1;
+    }
+    seq = lo;
+    cc = chunk - ctl->cu_chunks[lo];
+  };
+  auto issue = [&](int64_t item, int buf) {
+    int seq, cc;
+    locate(item, seq, cc);
+    const int head = (int)(item % H);
+    const int t0 = p.cu_seqlens[seq] + cc * C;
+    const uint32_t bar = smem_u32(&ctl->tma_bar[buf]);
+    const uint32_t kq = smem_u32(sm + P_IN + buf * P_IN_BYTES);
     mbar_arrive_expect_tx(bar, 16384u + (want_o ? 16384u : 0u) + (uint32_t)DV * 128u);
-    tma_load_2d(kq_u, &tm_k, head * DK, t0, bar);
-    tma_load_2d(kq_u + 16384, &tm_k, head * DK + 64, t0, bar);
+    tma_load_2d(kq, &tm_k, head * DK, t0, bar);
+    tma_load_2d(kq + 16384, &tm_k, head * DK + 64, t0, bar);
     if (want_o) {
-      tma_load_2d(kq_u + 8192, &tm_q, head * DK, t0, bar);
-      tma_load_2d(kq_u + 16384 + 8192, &tm_q, head * DK + 64, t0, bar);
+      tma_load_2d(kq + 8192, &tm_q, head * DK, t0, bar);
+      tma_load_2d(kq + 16384 + 8192, &tm_q, head * DK + 64, t0, bar);
     }
 #pragma unroll
     for (int b = 0; b < DV / 64; ++b)
-      tma_load_2d(smem_u32(sm + P_V) + 8192 * b, &tm_v, head * DV + 64 * b, t0, bar);
+      tma_load_2d(kq + 32768 + 8192 * b, &tm_v, head * DV + 64 * b, t0, bar);
+  };
+  if (tid == 0) {
+    fence_proxy_async_smem();
+    if ((int64_t)blockIdx.x < n_items) issue(blockIdx.x, 0);
+    if ((int64_t)blockIdx.x + gridDim.x < n_items) issue(blockIdx.x + gridDim.x, 1);
   }
-  // gates: g = inclusive cumsum of log alpha over the chunk, beta; 0 past the end
-  if (tid < C) {
-    float la = 0.f, b = 0.f;
-    if (tid < nv) {
-      la = p.log_alpha[(size_t)(t0 + tid) * H + head];
-      b = p.beta[(size_t)(t0 + tid) * H + head];
-    }
-    float s = la;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float y = __shfl_up_sync(0xffffffffu, s, o);
-      if (lane >= o) s += y;
-    }
-    ctl->g[tid] = s;
-    ctl->beta[tid] = b;
-  }
-  __syncthreads();
-  if (tid >= 32 && tid < C) ctl->g[tid] += ctl->g[31];
-  const bool ok_tma = mbar_wait(smem_u32(&ctl->tma_bar), 0, ab);
-  bool failed = __syncthreads_or(!ok_tma);
   const uint32_t mma_bar = smem_u32(&ctl->mma_bar);
   uint32_t mma_phase = 0;
   auto mma_wait = [&]() -> bool {
@@ -284,67 +316,96 @@ __global__ void __launch_bounds__(kThreads, 1)
     return true;
   };
 
-  do {
-    if (failed) break;
+  int n = 0;
+  for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x, ++n) {
+    const int buf = n & 1;
+    int seq, cc;
+    locate(item, seq, cc);
+    const int head = (int)(item % H);
+    const int t0 = p.cu_seqlens[seq] + cc * C;
+    const int nv = min(C, p.cu_seqlens[seq + 1] - t0);
+    uint8_t *KQ = sm + P_IN + buf * P_IN_BYTES;
+    const uint32_t kq_u = smem_u32(KQ);
+    const uint32_t v_u = kq_u + 32768;
+
+    // gates: g = inclusive cumsum of log alpha (0 past the end), beta, beta * gamma
+    if (tid < C) {
+      float la = 0.f, b = 0.f;
+      if (tid < nv) {
+        la = p.log_alpha[(size_t)(t0 + tid) * H + head];
+        b = p.beta[(size_t)(t0 + tid) * H + head];
+      }
+      float s = la;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += y;
+      }
+      ctl->g[tid] = s;
+      ctl->beta[tid] = b;
+    }
+    __syncthreads();
+    if (tid >= 32 && tid < C) ctl->g[tid] += ctl->g[31];
+    __syncthreads();
+    if (tid < C) ctl->bg[tid] = ctl->beta[tid] * exp_ftz(ctl->g[tid]);
+    const bool ok_tma = mbar_wait(smem_u32(&ctl->tma_bar[buf]), (uint32_t)(n >> 1) & 1u, ab);
+    if (__syncthreads_or(!ok_tma)) break;
     if (p.flags & TR_NORMALIZE_QK) {
-      if (tid < C || want_o) normalize_row(sm + P_KQ, tid);
+      if (tid < C || (tid < 2 * C && want_o)) normalize_row(KQ, tid);
       fence_proxy_async_smem();
       __syncthreads();
     }
-    // P1: [K; Q] K^T -> S (cols 0-63)
+
+    // P1: [K; Q] K^T -> TMEM cols [0, 64)
     if (tid == 0) {
       tc_fence_after();
+      const uint64_t dkq = kmaj(kq_u);
 #pragma unroll
       for (int kk = 0; kk < DK / 16; ++kk)
-        tc_mma_bf16(tmem + 0, desc_k(kq_u, kk, 16384), desc_k(kq_u, kk, 16384),
+        tc_mma_bf16(tmem, desc_k(dkq, kk, 16384), desc_k(dkq, kk, 16384),
                     idesc_bf16(128, 64, 0, 0), kk > 0);
       tc_commit(mma_bar);
     }
-    if (!mma_wait()) { failed = true; break; }
+    if (!mma_wait()) break;
 
-    // A (strictly lower, fp32) from K K^T, P (lower incl. diagonal) from Q K^T
+    // A (strictly lower, fp32) and P (lower incl. diagonal, bf16); columns split by hsel
     {
-      const int t = tid & 63;
-      const float gt = ctl->g[t];
       float v[32];
-      if (tid < C) {
+      tmem_ld32(tmem + lane_base + 32 * hsel, v);
+      tc_wait_ld();
+      const int t = row & 63;
+      const float gt = ctl->g[t];
+      if (row < C) {
         const float bt = ctl->beta[t];
-        float *Arow = As + t * AS_LD;
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          tmem_ld32(tmem + lane_base + 32 * hh, v);
-          tc_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int s = 32 * hh + i;
-            Arow[s] = (s < t) ? bt * __expf(gt - ctl->g[s]) * v[i] : 0.f;
-          }
+        for (int i = 0; i < 32; ++i) {
+          const int s = 32 * hsel + i;
+          v[i] = (s < t) ? bt * exp_ftz(gt - ctl->g[s]) * v[i] : 0.f;
         }
-      } else {
+        float4 *dst = reinterpret_cast<float4 *>(As + t * LDA + 32 * hsel);
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          tmem_ld32(tmem + lane_base + 32 * hh, v);
-          tc_wait_ld();
+        for (int w = 0; w < 8; ++w) dst[w] = make_float4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]);
+      } else if (want_o) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int s = 32 * hh + i;
-            v[i] = (s <= t) ? __expf(gt - ctl->g[s]) * v[i] : 0.f;
-          }
-          if (want_o) store_row_bf16(sm + P_AP, 64 + t, 32 * hh, v, 1.f);
+        for (int i = 0; i < 32; ++i) {
+          const int s = 32 * hsel + i;
+          v[i] = (s <= t) ? exp_ftz(gt - ctl->g[s]) * v[i] : 0.f;
         }
+        store_row_bf16(sm + P_AP, row, 32 * hsel, v, 1.f);
       }
     }
     __syncthreads();
 
-    // T = (I + A)^{-1}: thread j builds column j row by row (forward substitution, fp32);
-    // four partial sums keep the dependent FMA chains short.
+    // T = (I + A)^{-1}, blocked: T11 = (I + A11)^{-1}, T22 = (I + A22)^{-1} by forward
+    // substitution (thread = column, fp32 registers), then T21 = -T22 (A21 T11).
     if (tid < C) {
-      const int j = tid;
-      float Tc[C];
+      const int blk = tid >> 5, c = lane;
+      const int base = 32 * blk;
+      float Tc[32];
 #pragma unroll
-      for (int i = 0; i < C; ++i) {
+      for (int i = 0; i < 32; ++i) {
+        const float *Ar = As + (base + i) * LDA + base;
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-        const float *Ar = As + i * AS_LD;
 #pragma unroll
         for (int s = 0; s + 3 < i; s += 4) {
           a0 = fmaf(Ar[s], Tc[s], a0);
@@ -354,58 +415,105 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int s = i & ~3; s < i; ++s) a0 = fmaf(Ar[s], Tc[s], a0);
-        const float acc = (a0 + a1) + (a2 + a3);
-        Tc[i] = (i == j) ? 1.f : ((i < j) ? 0.f : -acc);
+        Tc[i] = (i == c) ? 1.f : ((i < c) ? 0.f : -((a0 + a1) + (a2 + a3)));
       }
-      const float bj = ctl->beta[j];
-      const float bgj = bj * __expf(ctl->g[j]);
-      __nv_bfloat16 *ts = reinterpret_cast<__nv_bfloat16 *>(sm + P_TS);
 #pragma unroll
-      for (int i = 0; i < C; ++i) {
-        ts[sw128_offset((uint32_t)i, (uint32_t)j * 2u) / 2] = __float2bfloat16_rn(-Tc[i] * bj);
-        ts[sw128_offset((uint32_t)(64 + i), (uint32_t)j * 2u) / 2] =
-            __float2bfloat16_rn(Tc[i] * bgj);
+      for (int i = 0; i < 32; ++i) Ts[(base + i) * LDA + base + c] = Tc[i];
+    }
+    __syncthreads();
+    {  // X = A21 T11 (32 x 32): thread -> row r, columns c0..c0+3
+      const int r = tid >> 3, c0 = (tid & 7) * 4;
+      float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+      const float *Ar = As + (32 + r) * LDA;
+#pragma unroll 4
+      for (int s = 0; s < 32; s += 4) {
+        const float4 a = *reinterpret_cast<const float4 *>(Ar + s);
+        const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 t = *reinterpret_cast<const float4 *>(Ts + (s + u) * LDA + c0);
+          x0 = fmaf(av[u], t.x, x0); x1 = fmaf(av[u], t.y, x1);
+          x2 = fmaf(av[u], t.z, x2); x3 = fmaf(av[u], t.w, x3);
+        }
       }
+      *reinterpret_cast<float4 *>(Xs + r * LDX + c0) = make_float4(x0, x1, x2, x3);
+    }
+    __syncthreads();
+    {  // T21 = -T22 X
+      const int r = tid >> 3, c0 = (tid & 7) * 4;
+      float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+      const float *Tr = Ts + (32 + r) * LDA + 32;
+#pragma unroll 4
+      for (int s = 0; s < 32; s += 4) {
+        const float4 a = *reinterpret_cast<const float4 *>(Tr + s);
+        const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 t = *reinterpret_cast<const float4 *>(Xs + (s + u) * LDX + c0);
+          x0 = fmaf(av[u], t.x, x0); x1 = fmaf(av[u], t.y, x1);
+          x2 = fmaf(av[u], t.z, x2); x3 = fmaf(av[u], t.w, x3);
+        }
+      }
+      *reinterpret_cast<float4 *>(Ts + (32 + r) * LDA + c0) = make_float4(-x0, -x1, -x2, -x3);
+    }
+    __syncthreads();
+    {  // [-T diag(beta); T diag(beta gamma)] as high + low bf16 parts
+      const int rr = tid >> 1, half = tid & 1, t = rr & 63;
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int s = 32 * half + i;
+        const float tv = (t < 32 && s >= 32) ? 0.f : Ts[t * LDA + s];
+        v[i] = (rr < C) ? -tv * ctl->beta[s] : tv * ctl->bg[s];
+      }
+      store_row_split(sm + P_TSH, sm + P_TSL, rr, 32 * half, v, 1.f);
     }
     fence_proxy_async_smem();
     __syncthreads();
 
-    // P2: [-T''; T'] V -> cols [64, 64+DV) (lanes 0-63: -U~), [-T''; T'] K -> [192, 320) (lanes 64-127: W)
+    // P2: [-T''; T'] V -> cols [64, 64+DV) (lanes 0-63: -U~); [-T''; T'] K -> [192, 320) (lanes 64-127: W)
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t ts_u = smem_u32(sm + P_TS);
+      const uint64_t th = kmaj(smem_u32(sm + P_TSH)), tl = kmaj(smem_u32(sm + P_TSL));
+      const uint64_t dv_ = mnmaj(v_u, 8192), dk_ = mnmaj(kq_u, 16384);
 #pragma unroll
       for (int kk = 0; kk < C / 16; ++kk)
-        tc_mma_bf16(tmem + 64, desc_k(ts_u, kk, 0), desc_mn(smem_u32(sm + P_V), kk, 8192),
-                    idesc_bf16(128, DV, 0, 1), kk > 0);
+        tc_mma_bf16(tmem + 64, desc_k(th, kk, 0), desc_mn(dv_, kk), idesc_bf16(128, DV, 0, 1), kk > 0);
 #pragma unroll
       for (int kk = 0; kk < C / 16; ++kk)
-        tc_mma_bf16(tmem + 192, desc_k(ts_u, kk, 0), desc_mn(kq_u, kk, 16384),
-                    idesc_bf16(128, 128, 0, 1), kk > 0);
+        tc_mma_bf16(tmem + 64, desc_k(tl, kk, 0), desc_mn(dv_, kk), idesc_bf16(128, DV, 0, 1), 1u);
+#pragma unroll
+      for (int kk = 0; kk < C / 16; ++kk)
+        tc_mma_bf16(tmem + 192, desc_k(th, kk, 0), desc_mn(dk_, kk), idesc_bf16(128, 128, 0, 1), kk > 0);
+#pragma unroll
+      for (int kk = 0; kk < C / 16; ++kk)
+        tc_mma_bf16(tmem + 192, desc_k(tl, kk, 0), desc_mn(dk_, kk), idesc_bf16(128, 128, 0, 1), 1u);
       tc_commit(mma_bar);
     }
-    if (!mma_wait()) { failed = true; break; }
+    if (!mma_wait()) break;
 
     const float gC = ctl->g[C - 1];
     {
       float v[32];
-      const int t = tid & 63;
-      const float gp = __expf(gC - ctl->g[t]);
-      if (tid >= C) {  // W row t -> W and gamma' W (natural [t][d] layout, 8 KB halves)
+      const int t = row & 63;
+      const float gp = exp_ftz(gC - ctl->g[t]);
+      if (row >= C) {  // W row t, columns 64*hsel..+63 -> W and gamma' W ([t][d], 8 KB halves)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          tmem_ld32(tmem + 192 + lane_base + 32 * q, v);
+        for (int j = 0; j < 2; ++j) {
+          tmem_ld32(tmem + 192 + lane_base + 64 * hsel + 32 * j, v);
           tc_wait_ld();
-          store_row_bf16(sm + P_W + (q >> 1) * 8192, t, 32 * (q & 1), v, 1.f);
-          store_row_bf16(sm + P_WG + (q >> 1) * 8192, t, 32 * (q & 1), v, gp);
+          store_row_bf16(sm + P_AW + hsel * 8192, t, 32 * j, v, 1.f);
+          store_row_bf16(sm + P_AW + 16384 + hsel * 8192, t, 32 * j, v, gp);
         }
-      } else {  // -U~ row t -> U~ and gamma' U~
+      } else {  // -U~ row t, columns (DV/2)*hsel.. -> U~ (hi, lo) and gamma' U~ (hi, lo)
 #pragma unroll
-        for (int q = 0; q < DV / 32; ++q) {
-          tmem_ld32(tmem + 64 + lane_base + 32 * q, v);
+        for (int j = 0; j < DV / 64; ++j) {
+          const int col = (DV / 2) * hsel + 32 * j;
+          tmem_ld32(tmem + 64 + lane_base + col, v);
           tc_wait_ld();
-          store_row_bf16(sm + P_UT + (q >> 1) * 8192, t, 32 * (q & 1), v, -1.f);
-          store_row_bf16(sm + P_UG + (q >> 1) * 8192, t, 32 * (q & 1), v, -gp);
+          const int blkoff = (col >> 6) * 8192, c0 = col & 63;
+          store_row_split(sm + P_TU + blkoff, sm + P_TU + 16384 + blkoff, t, c0, v, -1.f);
+          store_row_split(sm + P_TSH + blkoff, sm + P_TSL + blkoff, t, c0, v, -gp);
         }
       }
     }
@@ -413,95 +521,109 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
 
-    // one batch: P W -> [0,128), P U~ -> [128, 128+DV), A_c -> [256, 384), B_c -> [384, 384+DV)
+    // batch: P W -> [0,128), P U~ -> [128,128+DV), A_c -> [256,384), B_c -> [384,384+DV)
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t ap_u = smem_u32(sm + P_AP), w_u = smem_u32(sm + P_W);
-      const uint32_t ut_u = smem_u32(sm + P_UT), wg_u = smem_u32(sm + P_WG);
-      const uint32_t ug_u = smem_u32(sm + P_UG);
+      const uint64_t ap = kmaj(smem_u32(sm + P_AP));
+      const uint32_t w_u = smem_u32(sm + P_AW), uh_u = smem_u32(sm + P_TU);
+      const uint64_t w_d = mnmaj(w_u, 8192), wg_d = mnmaj(w_u + 16384, 8192);
+      const uint64_t uh = mnmaj(uh_u, 8192), ul = mnmaj(uh_u + 16384, 8192);
+      const uint64_t gh = mnmaj(smem_u32(sm + P_TSH), 8192), gl = mnmaj(smem_u32(sm + P_TSL), 8192);
+      const uint64_t kt = mnmaj(kq_u, 16384);
       if (want_o) {
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk)
-          tc_mma_bf16(tmem + 0, desc_k(ap_u, kk, 0), desc_mn(w_u, kk, 8192),
-                      idesc_bf16(128, 128, 0, 1), kk > 0);
+          tc_mma_bf16(tmem + 0, desc_k(ap, kk, 0), desc_mn(w_d, kk), idesc_bf16(128, 128, 0, 1), kk > 0);
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk)
-          tc_mma_bf16(tmem + 128, desc_k(ap_u, kk, 0), desc_mn(ut_u, kk, 8192),
-                      idesc_bf16(128, DV, 0, 1), kk > 0);
+          tc_mma_bf16(tmem + 128, desc_k(ap, kk, 0), desc_mn(uh, kk), idesc_bf16(128, DV, 0, 1), kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk)
+          tc_mma_bf16(tmem + 128, desc_k(ap, kk, 0), desc_mn(ul, kk), idesc_bf16(128, DV, 0, 1), 1u);
       }
 #pragma unroll
       for (int kk = 0; kk < C / 16; ++kk)
-        tc_mma_bf16(tmem + 256, desc_mn(kq_u, kk, 16384), desc_mn(wg_u, kk, 8192),
-                    idesc_bf16(128, 128, 1, 1), kk > 0);
+        tc_mma_bf16(tmem + 256, desc_mn(kt, kk), desc_mn(wg_d, kk), idesc_bf16(128, 128, 1, 1), kk > 0);
 #pragma unroll
       for (int kk = 0; kk < C / 16; ++kk)
-        tc_mma_bf16(tmem + 384, desc_mn(kq_u, kk, 16384), desc_mn(ug_u, kk, 8192),
-                    idesc_bf16(128, DV, 1, 1), kk > 0);
+        tc_mma_bf16(tmem + 384, desc_mn(kt, kk), desc_mn(gh, kk), idesc_bf16(128, DV, 1, 1), kk > 0);
+#pragma unroll
+      for (int kk = 0; kk < C / 16; ++kk)
+        tc_mma_bf16(tmem + 384, desc_mn(kt, kk), desc_mn(gl, kk), idesc_bf16(128, DV, 1, 1), 1u);
       tc_commit(mma_bar);
     }
-    if (!mma_wait()) { failed = true; break; }
+    if (!mma_wait()) break;
 
     {
       float v[32];
-      // A_c row d = -(K^T gamma' W)[d][:] (bf16), B_c row d (fp32): all 128 lanes
-      const int d = tid;
-      __nv_bfloat16 *Ad = ws.A + (size_t)slot * 128 * 128 + (size_t)d * 128;
+      const int64_t slot = item;
+      // A_c row d = -(K^T gamma' W)[d] (bf16), columns 64*hsel..+63
+      {
+        __nv_bfloat16 *Ad = ws.A + (size_t)slot * 128 * 128 + (size_t)row * 128 + 64 * hsel;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        tmem_ld32(tmem + 256 + lane_base + 32 * q, v);
-        tc_wait_ld();
-        uint4 *dst = reinterpret_cast<uint4 *>(Ad + 32 * q);
-#pragma unroll
-        for (int w = 0; w < 4; ++w)
-          dst[w] = make_uint4(pack_bf16x2(-v[8 * w], -v[8 * w + 1]),
-                              pack_bf16x2(-v[8 * w + 2], -v[8 * w + 3]),
-                              pack_bf16x2(-v[8 * w + 4], -v[8 * w + 5]),
-                              pack_bf16x2(-v[8 * w + 6], -v[8 * w + 7]));
-      }
-      float *Bd = ws.B + (size_t)slot * 128 * DV + (size_t)d * DV;
-#pragma unroll
-      for (int q = 0; q < DV / 32; ++q) {
-        tmem_ld32(tmem + 384 + lane_base + 32 * q, v);
-        tc_wait_ld();
-        float4 *dst = reinterpret_cast<float4 *>(Bd + 32 * q);
-#pragma unroll
-        for (int w = 0; w < 8; ++w)
-          dst[w] = make_float4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]);
-      }
-      if (want_o && tid >= C) {
-        // R row t = gamma_t q_t - (P W)_t (bf16), O0 row t (fp32)
-        const int t = tid - C;
-        const float gam = __expf(ctl->g[t]);
-        __nv_bfloat16 *Rt = ws.R + (size_t)slot * 64 * 128 + (size_t)t * 128;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          tmem_ld32(tmem + 0 + lane_base + 32 * q, v);
+        for (int j = 0; j < 2; ++j) {
+          tmem_ld32(tmem + 256 + lane_base + 64 * hsel + 32 * j, v);
           tc_wait_ld();
-          uint4 *dst = reinterpret_cast<uint4 *>(Rt + 32 * q);
+          uint4 *dst = reinterpret_cast<uint4 *>(Ad + 32 * j);
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            dst[w] = make_uint4(pack_bf16x2(-v[8 * w], -v[8 * w + 1]), pack_bf16x2(-v[8 * w + 2], -v[8 * w + 3]),
+                                pack_bf16x2(-v[8 * w + 4], -v[8 * w + 5]), pack_bf16x2(-v[8 * w + 6], -v[8 * w + 7]));
+        }
+      }
+      // B_c row d (fp32), columns (DV/2)*hsel..
+      {
+        float *Bd = ws.B + (size_t)slot * 128 * DV + (size_t)row * DV + (DV / 2) * hsel;
+#pragma unroll
+        for (int j = 0; j < DV / 64; ++j) {
+          tmem_ld32(tmem + 384 + lane_base + (DV / 2) * hsel + 32 * j, v);
+          tc_wait_ld();
+          float4 *dst = reinterpret_cast<float4 *>(Bd + 32 * j);
+#pragma unroll
+          for (int w = 0; w < 8; ++w) dst[w] = make_float4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]);
+        }
+      }
+      if (want_o && row >= C) {
+        const int t = row - C;
+        const float gam = exp_ftz(ctl->g[t]);
+        // R row t = gamma_t q_t - (P W)_t (bf16), columns 64*hsel..+63
+        __nv_bfloat16 *Rt = ws.R + (size_t)slot * 64 * 128 + (size_t)t * 128 + 64 * hsel;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          tmem_ld32(tmem + 0 + lane_base + 64 * hsel + 32 * j, v);
+          tc_wait_ld();
+          uint4 *dst = reinterpret_cast<uint4 *>(Rt + 32 * j);
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
             float f[8];
-            load_row8_bf16(sm + P_KQ + (q >> 1) * 16384, 64 + t, 32 * (q & 1) + 8 * w, f);
+            load_row8_bf16(KQ + hsel * 16384, 64 + t, 32 * j + 8 * w, f);
             dst[w] = make_uint4(pack_bf16x2(gam * f[0] - v[8 * w], gam * f[1] - v[8 * w + 1]),
                                 pack_bf16x2(gam * f[2] - v[8 * w + 2], gam * f[3] - v[8 * w + 3]),
                                 pack_bf16x2(gam * f[4] - v[8 * w + 4], gam * f[5] - v[8 * w + 5]),
                                 pack_bf16x2(gam * f[6] - v[8 * w + 6], gam * f[7] - v[8 * w + 7]));
           }
         }
-        float *Ot = ws.O + (size_t)slot * 64 * DV + (size_t)t * DV;
+        // O0 row t (fp32), columns (DV/2)*hsel..
+        float *Ot = ws.O + (size_t)slot * 64 * DV + (size_t)t * DV + (DV / 2) * hsel;
 #pragma unroll
-        for (int q = 0; q < DV / 32; ++q) {
-          tmem_ld32(tmem + 128 + lane_base + 32 * q, v);
+        for (int j = 0; j < DV / 64; ++j) {
+          tmem_ld32(tmem + 128 + lane_base + (DV / 2) * hsel + 32 * j, v);
           tc_wait_ld();
-          float4 *dst = reinterpret_cast<float4 *>(Ot + 32 * q);
+          float4 *dst = reinterpret_cast<float4 *>(Ot + 32 * j);
 #pragma unroll
-          for (int w = 0; w < 8; ++w)
-            dst[w] = make_float4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]);
+          for (int w = 0; w < 8; ++w) dst[w] = make_float4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]);
         }
       }
-      if (tid == 0) ws.G[slot] = __expf(gC);
+      if (tid == 0) ws.G[slot] = exp_ftz(gC);
     }
-  } while (false);
+    tc_fence_before();
+    __syncthreads();
+    // this buffer's K/Q/V are no longer read: prefetch the item after next into it
+    if (tid == 0 && item + 2 * (int64_t)gridDim.x < n_items) {
+      fence_proxy_async_smem();
+      issue(item + 2 * (int64_t)gridDim.x, buf);
+    }
+  }
 
   tc_fence_before();
   __syncthreads();
@@ -512,20 +634,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // =========================================================== chain kernel
-constexpr uint32_t H_A = 0;          // 2 x 32 KB  A_c  [half][128 rows][128 B]
-constexpr uint32_t H_R = 65536;      // 2 x 16 KB  R    [half][64 rows][128 B] (MMA rows 64-127 unused)
-constexpr uint32_t H_B = 98304;      // 2 x 32 KB  B_c slice, fp32 [box][128 rows][32 floats]
-constexpr uint32_t H_O = 163840;     // 2 x 16 KB  O0 slice,  fp32 [box][64 rows][32 floats]
-constexpr uint32_t H_MB = 196608;    // 16 KB      bf16 state slice [d][64]
-constexpr uint32_t H_CTL = 212992;
-constexpr size_t CHAIN_SMEM = H_CTL + 1024 + 1024;
+// One CTA per (sequence, head, 64-column slice of d_v), 288 threads.  Warps 0-7:
+// thread (quarter q4 = warp % 4, half hsel = warp / 4) owns row d = 32 q4 + lane of
+// the fp32 state slice and its columns 32 hsel .. +31.  Warp 8 only refills the TMA
+// ring (a tensor load can stall its issuing thread while many are in flight, so the
+// state-owning threads never issue them).  Per chunk: one tcgen05 product
+// Z = A_c M (M in bf16 in shared memory, 8 MMAs of K = 16), then
+// M <- gamma_C M + Z + B_c in registers.  A_c and the B_c slice arrive through a
+// 2-stage TMA ring; all gamma_C of the sequence are read into shared memory at the
+// start.  The bf16 state at the start of every chunk (double buffered by chunk
+// parity) is the operand of the next product and goes to the workspace, for the
+// readout kernel, by a TMA store.
+constexpr int kStages = 2;
+constexpr uint32_t H_STAGE = 65536;             // A_c [half][128 rows][128 B] + B_c [box][128][32 fp32]
+constexpr uint32_t H_MB = kStages * H_STAGE;    // 2 x bf16 state slice [128 d][128 B]
+constexpr int kMaxChunksPerSeq = 4096;
+constexpr size_t CHAIN_SMEM = H_MB + 2 * 16384 + 1024;
 
 struct ChainCtl {
-  uint64_t tma_bar[2];
-  uint64_t mma_bar;
+  uint64_t tma_bar[kStages];
+  uint64_t empty_bar[kStages];  // stage consumed (arrived by thread 0 after the barrier)
+  uint64_t bar_z;
   uint32_t tmem;
   int abort;
-  int red[4];
+  float gC[kMaxChunksPerSeq];
 };
 
 __device__ __forceinline__ void load_row32_f32(const uint8_t *tile, int row, float *f) {
@@ -538,184 +670,290 @@ __device__ __forceinline__ void load_row32_f32(const uint8_t *tile, int row, flo
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-    scan_chain_kernel(const __grid_constant__ CUtensorMap tm_A, const __grid_constant__ CUtensorMap tm_R,
-                      const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_O,
-                      ScanLaunch p, ScanWs ws) {
+constexpr int kChainThreads = 288;
+
+__global__ void __launch_bounds__(kChainThreads, 1)
+    scan_chain_kernel(const __grid_constant__ CUtensorMap tm_A, const __grid_constant__ CUtensorMap tm_B,
+                      const __grid_constant__ CUtensorMap tm_M, ScanLaunch p, ScanWs ws) {
   extern __shared__ uint8_t smem_raw[];
+  __shared__ ChainCtl ctl_s;
+  __shared__ int red[8];
+  ChainCtl *ctl = &ctl_s;
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
-  ChainCtl *ctl = reinterpret_cast<ChainCtl *>(sm + H_CTL);
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int H = p.H;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q4 = warp & 3, hsel = warp >> 2;
+  const int d = q4 * 32 + lane;
+  const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+  const int H = p.H, DV = p.dv;
   const int seq = blockIdx.x / H, head = blockIdx.x % H;
   const int slice = blockIdx.y;
+  const int col = slice * DVS + 32 * hsel;   // this thread's first d_v column
   const int t_begin = p.cu_seqlens[seq], t_end = p.cu_seqlens[seq + 1];
   const int nch = (t_end - t_begin + C - 1) / C;
-  const bool want_o = p.o != nullptr;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  const int cb = chunk_base(p.cu_seqlens, seq, ctl->red);
+  const int cb = chunk_base(p.cu_seqlens, seq, red);
+  auto slot_of = [&](int c) -> int64_t { return ((int64_t)cb + c) * H + head; };
 
   if (tid == 0) {
-    mbar_init(smem_u32(&ctl->tma_bar[0]), 1);
-    mbar_init(smem_u32(&ctl->tma_bar[1]), 1);
-    mbar_init(smem_u32(&ctl->mma_bar), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&ctl->tma_bar[s]), 1);
+      mbar_init(smem_u32(&ctl->empty_bar[s]), 1);
+    }
+    mbar_init(smem_u32(&ctl->bar_z), 1);
     ctl->abort = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(&ctl->tmem), 128);
+    tmem_alloc(smem_u32(&ctl->tmem), 64);
     tmem_relinquish();
   }
+  for (int c = tid; c < nch; c += kChainThreads) ctl->gC[c] = ws.G[slot_of(c)];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = ctl->tmem;  // Z: cols [0, 64), O: [64, 128)
+  const uint32_t tmem = ctl->tmem;
   const AbortFlag ab{&ctl->abort, p.err_word, ERRBIT_SCAN_TIMEOUT};
+  // bf16 state copy par (chunk parity) -> workspace slot of chunk c, by one TMA store
+  auto store_mc = [&](int c, int par) {
+    tma_store_2d(&tm_M, smem_u32(sm + H_MB + 16384 * par), slice * DVS, (int32_t)(slot_of(c) * 128));
+    bulk_commit();
+  };
 
-  float Mr[DVS];
-  bool m_zero = p.S0 == nullptr;
-  const size_t s_base = ((size_t)seq * H + head) * DK * p.dv + (size_t)tid * p.dv + (size_t)slice * DVS;
-  if (!m_zero) {
+  float Mr[32];
+  const bool m_zero = p.S0 == nullptr;
+  const bool producer = warp == 8;
+  const size_t s_off = ((size_t)seq * H + head) * DK * DV + (size_t)d * DV + col;
+  if (!m_zero && !producer) {
 #pragma unroll
-    for (int j = 0; j < DVS; j += 4) {
-      const float4 a = *reinterpret_cast<const float4 *>(p.S0 + s_base + j);
+    for (int j = 0; j < 32; j += 4) {
+      const float4 a = *reinterpret_cast<const float4 *>(p.S0 + s_off + j);
       Mr[j] = a.x; Mr[j + 1] = a.y; Mr[j + 2] = a.z; Mr[j + 3] = a.w;
     }
-    store_row_bf16(sm + H_MB, tid, 0, Mr, 1.f);
-    store_row_bf16(sm + H_MB, tid, 32, Mr + 32, 1.f);
   } else {
 #pragma unroll
-    for (int j = 0; j < DVS; ++j) Mr[j] = 0.f;
+    for (int j = 0; j < 32; ++j) Mr[j] = 0.f;
   }
+  if (nch > 0 && !producer) store_row_bf16(sm + H_MB, d, 32 * hsel, Mr, 1.f);
 
-  const uint32_t tx = 32768u + 32768u + (want_o ? 16384u + 16384u : 0u);
-  auto issue = [&](int c, int buf) {
-    const int64_t slot = ((int64_t)cb + c) * H + head;
-    const uint32_t bar = smem_u32(&ctl->tma_bar[buf]);
-    mbar_arrive_expect_tx(bar, tx);
-    const uint32_t a_u = smem_u32(sm + H_A + buf * 32768);
+  auto issue_tma = [&](int c) {
+    const int st = c % kStages;
+    const int64_t slot = slot_of(c);
+    const uint32_t bar = smem_u32(&ctl->tma_bar[st]);
+    const uint32_t a_u = smem_u32(sm + st * H_STAGE);
+    mbar_arrive_expect_tx(bar, 65536u);
     tma_load_2d(a_u, &tm_A, 0, (int32_t)(slot * 128), bar);
     tma_load_2d(a_u + 16384, &tm_A, 64, (int32_t)(slot * 128), bar);
-    const uint32_t b_u = smem_u32(sm + H_B + buf * 32768);
-    tma_load_2d(b_u, &tm_B, slice * DVS, (int32_t)(slot * 128), bar);
-    tma_load_2d(b_u + 16384, &tm_B, slice * DVS + 32, (int32_t)(slot * 128), bar);
-    if (want_o) {
-      const uint32_t r_u = smem_u32(sm + H_R + buf * 16384);
-      tma_load_2d(r_u, &tm_R, 0, (int32_t)(slot * 64), bar);
-      tma_load_2d(r_u + 8192, &tm_R, 64, (int32_t)(slot * 64), bar);
-      const uint32_t o_u = smem_u32(sm + H_O + buf * 16384);
-      tma_load_2d(o_u, &tm_O, slice * DVS, (int32_t)(slot * 64), bar);
-      tma_load_2d(o_u + 8192, &tm_O, slice * DVS + 32, (int32_t)(slot * 64), bar);
-    }
+    tma_load_2d(a_u + 32768, &tm_B, slice * DVS, (int32_t)(slot * 128), bar);
+    tma_load_2d(a_u + 49152, &tm_B, slice * DVS + 32, (int32_t)(slot * 128), bar);
   };
+  auto issue_mma = [&](int c) -> bool {
+    const int st = c % kStages;
+    if (!mbar_wait(smem_u32(&ctl->tma_bar[st]), (uint32_t)(c / kStages) & 1u, ab)) return false;
+    tc_fence_after();
+    const uint64_t ad = kmaj(smem_u32(sm + st * H_STAGE));
+    const uint64_t md = mnmaj(smem_u32(sm + H_MB + 16384 * (c & 1)), 16384);
+#pragma unroll
+    for (int kk = 0; kk < DK / 16; ++kk)
+      tc_mma_bf16(tmem, desc_k(ad, kk, 16384), desc_mn(md, kk), idesc_bf16(128, DVS, 0, 1), kk > 0);
+    tc_commit(smem_u32(&ctl->bar_z));
+    return true;
+  };
+
+  bool failed = false;
   if (tid == 0) {
     fence_proxy_async_smem();
-    if (nch > 0) issue(0, 0);
-    if (nch > 1) issue(1, 1);
+    for (int c = 0; c < kStages && c < nch; ++c) issue_tma(c);
   }
-  const uint32_t mma_bar = smem_u32(&ctl->mma_bar);
-  uint32_t mma_phase = 0;
-  bool failed = false;
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (tid == 0 && nch > 0) store_mc(0, 0);
 
-  for (int c = 0; c < nch; ++c) {
-    const int buf = c & 1;
-    const int t0 = t_begin + c * C;
-    const int64_t slot = ((int64_t)cb + c) * H + head;
-    const float gC = ws.G[slot];
-    const bool ok_tma = mbar_wait(smem_u32(&ctl->tma_bar[buf]), (uint32_t)(c >> 1) & 1u, ab);
-    if (__syncthreads_or(!ok_tma)) { failed = true; break; }
-    if (!m_zero) {
-      if (tid == 0) {
-        tc_fence_after();
-        const uint32_t a_u = smem_u32(sm + H_A + buf * 32768);
-        const uint32_t r_u = smem_u32(sm + H_R + buf * 16384);
-        const uint32_t mb_u = smem_u32(sm + H_MB);
-#pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk)
-          tc_mma_bf16(tmem + 0, desc_k(a_u, kk, 16384), desc_mn(mb_u, kk, 8192),
-                      idesc_bf16(128, DVS, 0, 1), kk > 0);
-        if (want_o) {
-#pragma unroll
-          for (int kk = 0; kk < DK / 16; ++kk)
-            tc_mma_bf16(tmem + 64, desc_k(r_u, kk, 8192), desc_mn(mb_u, kk, 8192),
-                        idesc_bf16(128, DVS, 0, 1), kk > 0);
-        }
-        tc_commit(mma_bar);
+  if (producer) {
+    // refill stage c % kStages with chunk c once chunk c - kStages has consumed it
+    if (lane == 0) {
+      for (int c = kStages; c < nch; ++c) {
+        const int st = c % kStages;
+        if (!mbar_wait(smem_u32(&ctl->empty_bar[st]), (uint32_t)((c - kStages) / kStages) & 1u, ab))
+          break;
+        issue_tma(c);
       }
-      const bool ok = mbar_wait(mma_bar, mma_phase, ab);
-      mma_phase ^= 1u;
-      if (__syncthreads_or(!ok)) { failed = true; break; }
-      tc_fence_after();
     }
-    // M <- gamma_C M + Z + B_c ; o = O + O0
-    {
-      const uint8_t *bt = sm + H_B + buf * 32768;
+  } else {
+    if (tid == 0 && !m_zero && nch > 0 && !issue_mma(0)) failed = true;
+    bool mma_for_c = !m_zero;
+    uint32_t z_phase = 0;
+    for (int c = 0; c < nch; ++c) {
+      const int st = c % kStages;
       float v[32], b[32];
+      if (mma_for_c) {
+        if (!mbar_wait(smem_u32(&ctl->bar_z), z_phase, ab)) failed = true;
+        z_phase ^= 1u;
+        tc_fence_after();
+        tmem_ld32(tmem + lane_base + 32 * hsel, v);
+      } else {
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        if (!m_zero) {
-          tmem_ld32(tmem + 0 + lane_base + 32 * hh, v);
-          tc_wait_ld();
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = 0.f;
-        }
-        load_row32_f32(bt + hh * 16384, tid, b);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) Mr[32 * hh + i] = fmaf(gC, Mr[32 * hh + i], v[i] + b[i]);
+        for (int j = 0; j < 32; ++j) v[j] = 0.f;
       }
-      if (want_o && tid < C) {
-        const int t = tid;
-        const uint8_t *ot = sm + H_O + buf * 16384;
+      // the stage's B_c has landed (its A_c did, for the product); read this thread's row
+      if (!mbar_wait(smem_u32(&ctl->tma_bar[st]), (uint32_t)(c / kStages) & 1u, ab)) failed = true;
+      load_row32_f32(sm + st * H_STAGE + 32768 + hsel * 16384, d, b);
+      if (mma_for_c) tc_wait_ld();
+      const float gC = ctl->gC[c];
+      // M <- gamma_C M + A_c M + B_c (fp32); bf16 copy for the next product and the readout
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          if (!m_zero) {
-            tmem_ld32(tmem + 64 + lane_base + 32 * hh, v);
-            tc_wait_ld();
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0.f;
-          }
-          load_row32_f32(ot + hh * 8192, t, b);
-          if (t0 + t < t_end) {
-            uint4 *d4 = reinterpret_cast<uint4 *>(
-                reinterpret_cast<__nv_bfloat16 *>(p.o) + (size_t)(t0 + t) * p.o_stride +
-                (size_t)head * p.dv + slice * DVS + 32 * hh);
-            const float sc = p.scale;
-#pragma unroll
-            for (int w = 0; w < 4; ++w)
-              d4[w] = make_uint4(pack_bf16x2((v[8 * w] + b[8 * w]) * sc, (v[8 * w + 1] + b[8 * w + 1]) * sc),
-                                 pack_bf16x2((v[8 * w + 2] + b[8 * w + 2]) * sc, (v[8 * w + 3] + b[8 * w + 3]) * sc),
-                                 pack_bf16x2((v[8 * w + 4] + b[8 * w + 4]) * sc, (v[8 * w + 5] + b[8 * w + 5]) * sc),
-                                 pack_bf16x2((v[8 * w + 6] + b[8 * w + 6]) * sc, (v[8 * w + 7] + b[8 * w + 7]) * sc));
-          }
-        }
-      }
-      store_row_bf16(sm + H_MB, tid, 0, Mr, 1.f);
-      store_row_bf16(sm + H_MB, tid, 32, Mr + 32, 1.f);
-      m_zero = false;
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0 && c + 2 < nch) {
+      for (int j = 0; j < 32; ++j) Mr[j] = fmaf(gC, Mr[j], v[j] + b[j]);
+      if (c + 1 < nch) store_row_bf16(sm + H_MB + 16384 * ((c + 1) & 1), d, 32 * hsel, Mr, 1.f);
       fence_proxy_async_smem();
-      issue(c + 2, buf);
+      tc_fence_before();
+      // copy (c + 1) & 1 was last stored to global two chunks ago: that store must have
+      // finished reading it before anyone rewrites it (after the barrier below)
+      if (tid == 0) bulk_wait_read<0>();
+      // named barrier over the 256 state-owning threads, voting on `failed` so that all
+      // of them leave the loop together
+      uint32_t any_failed;
+      asm volatile(
+          "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+          "bar.red.or.pred p, 1, 256, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+          : "=r"(any_failed)
+          : "r"((uint32_t)(failed || *ab.flag))
+          : "memory");
+      if (any_failed) { failed = true; break; }
+      if (tid == 0) {
+        // chunk c's stage is consumed: its product completed and its B_c rows were read
+        mbar_arrive(smem_u32(&ctl->empty_bar[st]));
+        if (c + 1 < nch) {
+          tc_fence_after();
+          if (!issue_mma(c + 1)) failed = true;
+          store_mc(c + 1, (c + 1) & 1);
+        }
+      }
+      mma_for_c = true;
     }
   }
 
-  if (!failed) {
-    float *dst = p.S_final + s_base;
+  if (tid == 0) bulk_wait<0>();
+  if (!failed && !producer) {
+    float *dst = p.S_final + s_off;
 #pragma unroll
-    for (int j = 0; j < DVS; j += 4)
+    for (int j = 0; j < 32; j += 4)
       *reinterpret_cast<float4 *>(dst + j) = make_float4(Mr[j], Mr[j + 1], Mr[j + 2], Mr[j + 3]);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, 64);
+  }
+}
+
+// ========================================================= readout kernel
+// o_c = R_c M_c + O0_c for every (chunk, head) in parallel: one tcgen05 product
+// ([R; unused rows] (128 x 128) times the bf16 chunk-start state M_c (128 x DV)),
+// plus the fp32 O0, scaled and stored as bf16.  128 threads; thread t < 64 owns
+// token row t.
+constexpr uint32_t O_R = 0;          // [half][128 rows][128 B]: rows 0-63 = R
+constexpr uint32_t O_M = 32768;      // [DV/64 blocks][128 d][128 B]: M_c
+constexpr uint32_t O_O = 65536;      // [DV/32 boxes][64 rows][32 fp32]: O0
+constexpr size_t OUT_SMEM = O_O + 32768 + 1024;
+
+template <int DV>
+__global__ void __launch_bounds__(128)
+    scan_out_kernel(const __grid_constant__ CUtensorMap tm_R, const __grid_constant__ CUtensorMap tm_M,
+                    const __grid_constant__ CUtensorMap tm_O, ScanLaunch p, ScanWs ws,
+                    int total_chunks) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar_t, bar_m;
+  __shared__ uint32_t tmem_s;
+  __shared__ int abort_s;
+  __shared__ int cu_chunks[kMaxSeqsChunked + 1];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = p.H;
+  const int64_t item = blockIdx.x;
+  const int chunk = (int)(item / H), head = (int)(item % H);
+  if (tid == 0) {
+    int acc = 0;
+    for (int i = 0; i < p.n_seqs; ++i) {
+      cu_chunks[i] = acc;
+      acc += (p.cu_seqlens[i + 1] - p.cu_seqlens[i] + C - 1) / C;
+    }
+    cu_chunks[p.n_seqs] = acc;
+    mbar_init(smem_u32(&bar_t), 1);
+    mbar_init(smem_u32(&bar_m), 1);
+    abort_s = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&tmem_s), DV);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_s;
+  const AbortFlag ab{&abort_s, p.err_word, ERRBIT_SCAN_TIMEOUT};
+  int lo = 0, hi = p.n_seqs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (cu_chunks[mid] <= chunk) lo = mid; else hi = mid - 1;
+  }
+  const int seq = lo;
+  const int t0 = p.cu_seqlens[seq] + (chunk - cu_chunks[seq]) * C;
+  const int nv = min(C, p.cu_seqlens[seq + 1] - t0);
+  if (tid == 0) {
+    const uint32_t r_u = smem_u32(sm + O_R), m_u = smem_u32(sm + O_M);
+    mbar_arrive_expect_tx(smem_u32(&bar_t), 16384u + (uint32_t)DV * 256u + (uint32_t)DV * 256u);
+#pragma unroll
+    for (int b = 0; b < DV / 32; ++b)
+      tma_load_2d(smem_u32(sm + O_O) + 8192 * b, &tm_O, 32 * b, (int32_t)(item * 64), smem_u32(&bar_t));
+    tma_load_2d(r_u, &tm_R, 0, (int32_t)(item * 64), smem_u32(&bar_t));
+    tma_load_2d(r_u + 16384, &tm_R, 64, (int32_t)(item * 64), smem_u32(&bar_t));
+#pragma unroll
+    for (int b = 0; b < DV / 64; ++b)
+      tma_load_2d(m_u + 16384 * b, &tm_M, 64 * b, (int32_t)(item * 128), smem_u32(&bar_t));
+  }
+  bool ok = mbar_wait(smem_u32(&bar_t), 0, ab);
+  if (tid == 0 && ok) {
+    tc_fence_after();
+    const uint64_t rd = kmaj(smem_u32(sm + O_R)), md = mnmaj(smem_u32(sm + O_M), 16384);
+#pragma unroll
+    for (int kk = 0; kk < DK / 16; ++kk)
+      tc_mma_bf16(tmem, desc_k(rd, kk, 16384), desc_mn(md, kk), idesc_bf16(128, DV, 0, 1), kk > 0);
+    tc_commit(smem_u32(&bar_m));
+  }
+  ok = ok && mbar_wait(smem_u32(&bar_m), 0, ab);
+  if (__syncthreads_or(!ok)) {
+    // a wait ran out: leave the outputs alone
+  } else {
+    tc_fence_after();
+    if (tid < C) {
+      const float sc = p.scale;
+#pragma unroll 1
+      for (int j = 0; j < DV / 32; ++j) {
+        float v[32], b[32];
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 32 * j, v);
+        load_row32_f32(sm + O_O + 8192 * j, tid, b);
+        tc_wait_ld();
+        if (tid < nv) {
+          uint4 *d4 = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.o) +
+                                                (size_t)(t0 + tid) * p.o_stride + (size_t)head * DV + 32 * j);
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            d4[w] = make_uint4(pack_bf16x2((v[8 * w] + b[8 * w]) * sc, (v[8 * w + 1] + b[8 * w + 1]) * sc),
+                               pack_bf16x2((v[8 * w + 2] + b[8 * w + 2]) * sc, (v[8 * w + 3] + b[8 * w + 3]) * sc),
+                               pack_bf16x2((v[8 * w + 4] + b[8 * w + 4]) * sc, (v[8 * w + 5] + b[8 * w + 5]) * sc),
+                               pack_bf16x2((v[8 * w + 6] + b[8 * w + 6]) * sc, (v[8 * w + 7] + b[8 * w + 7]) * sc));
+        }
+      }
+    }
+  }
+  (void)lane;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, DV);
   }
 }
 
@@ -726,8 +964,12 @@ bool make_tmap_f32_2d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_
                       std::string *err);
 
 bool scan_chunked_supported(const ScanLaunch &p) {
-  return p.dtype == TR_DTYPE_BF16 && p.dk == DK && (p.dv == 64 || p.dv == 128) &&
-         (p.o == nullptr || p.o_stride % 8 == 0);
+  if (!(p.dtype == TR_DTYPE_BF16 && p.dk == DK && (p.dv == 64 || p.dv == 128) &&
+        p.n_seqs <= kMaxSeqsChunked && (p.o == nullptr || p.o_stride % 8 == 0)))
+    return false;
+  for (int i = 0; p.cu_seqlens_host && i < p.n_seqs; ++i)
+    if ((p.cu_seqlens_host[i + 1] - p.cu_seqlens_host[i] + C - 1) / C > kMaxChunksPerSeq) return false;
+  return true;
 }
 
 size_t scan_chunked_workspace(const ScanLaunch &p) {
@@ -736,7 +978,7 @@ size_t scan_chunked_workspace(const ScanLaunch &p) {
   return total;
 }
 
-int scan_chunked_kernels() { return 2; }
+int scan_chunked_kernels(bool with_readout) { return with_readout ? 3 : 2; }
 
 cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string *err,
                                 const std::function<cudaError_t()> &between) {
@@ -747,34 +989,39 @@ cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string
     if (err) *err = "scan workspace too small";
     return cudaErrorInvalidValue;
   }
-  int max_chunks = 0;
-  count_slots(p, &max_chunks);
+  const int64_t items = ws.slots;
+  const int total_chunks = (int)(items / p.H);
+  if (items > 0x7fffffffLL) {
+    if (err) *err = "too many (chunk, head) work items";
+    return cudaErrorInvalidValue;
+  }
   const uint64_t T = (uint64_t)(p.T > 0 ? p.T : 1);
-  const uint64_t slots = (uint64_t)(ws.slots > 0 ? ws.slots : 1);
-  CUtensorMap tq, tk, tv, tA, tR, tB, tO;
+  const uint64_t slots = (uint64_t)(items > 0 ? items : 1);
+  CUtensorMap tq, tk, tv, tA, tR;
   const void *qb = p.q ? p.q : p.k;
   if (!make_tmap_bf16_2d(&tk, p.k, (uint64_t)p.H * DK, T, (uint64_t)p.k_stride * 2, 64, C, err) ||
       !make_tmap_bf16_2d(&tq, qb, (uint64_t)p.H * DK, T,
                          (uint64_t)(p.q ? p.q_stride : p.k_stride) * 2, 64, C, err) ||
       !make_tmap_bf16_2d(&tv, p.v, (uint64_t)p.H * p.dv, T, (uint64_t)p.v_stride * 2, 64, C, err) ||
       !make_tmap_bf16_2d(&tA, ws.A, 128, slots * 128, 256, 64, 128, err) ||
-      !make_tmap_bf16_2d(&tR, ws.R, 128, slots * 64, 256, 64, 64, err) ||
-      !make_tmap_f32_2d(&tB, ws.B, (uint64_t)p.dv, slots * 128, (uint64_t)p.dv * 4, 32, 128, err) ||
-      !make_tmap_f32_2d(&tO, ws.O, (uint64_t)p.dv, slots * 64, (uint64_t)p.dv * 4, 32, 64, err))
+      !make_tmap_bf16_2d(&tR, ws.R, 128, slots * 64, 256, 64, 64, err))
     return cudaErrorInvalidValue;
   cudaError_t e;
-  if (max_chunks > 0) {
-    dim3 pg((unsigned)max_chunks, (unsigned)(p.n_seqs * p.H));
+  if (items > 0) {
+    int64_t grid = device_sm_count();
+    if (grid > items) grid = items;
     if (p.dv == 128) {
       e = cudaFuncSetAttribute(scan_prep_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)PREP_SMEM);
       if (e != cudaSuccess) return e;
-      scan_prep_kernel<128><<<pg, kThreads, PREP_SMEM, s>>>(tq, tk, tv, p, ws);
+      scan_prep_kernel<128><<<(unsigned)grid, kPrepThreads, PREP_SMEM, s>>>(tq, tk, tv, p, ws,
+                                                                             total_chunks);
     } else {
       e = cudaFuncSetAttribute(scan_prep_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)PREP_SMEM);
       if (e != cudaSuccess) return e;
-      scan_prep_kernel<64><<<pg, kThreads, PREP_SMEM, s>>>(tq, tk, tv, p, ws);
+      scan_prep_kernel<64><<<(unsigned)grid, kPrepThreads, PREP_SMEM, s>>>(tq, tk, tv, p, ws,
+                                                                           total_chunks);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -783,11 +1030,36 @@ cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string
     e = between();
     if (e != cudaSuccess) return e;
   }
+  CUtensorMap tB, tM;
+  if (!make_tmap_f32_2d(&tB, ws.B, (uint64_t)p.dv, slots * 128, (uint64_t)p.dv * 4, 32, 128, err) ||
+      !make_tmap_bf16_2d(&tM, ws.M, (uint64_t)p.dv, slots * 128, (uint64_t)p.dv * 2, 64, 128, err))
+    return cudaErrorInvalidValue;
   e = cudaFuncSetAttribute(scan_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)CHAIN_SMEM);
   if (e != cudaSuccess) return e;
-  dim3 cg((unsigned)(p.n_seqs * p.H), (unsigned)(p.dv / DVS));
-  scan_chain_kernel<<<cg, kThreads, CHAIN_SMEM, s>>>(tA, tR, tB, tO, p, ws);
+  scan_chain_kernel<<<dim3((unsigned)(p.n_seqs * p.H), (unsigned)(p.dv / DVS)), kChainThreads,
+                      CHAIN_SMEM, s>>>(
+      tA, tB, tM, p, ws);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || !p.o || items == 0) return e;
+  if (between) {
+    e = between();
+    if (e != cudaSuccess) return e;
+  }
+  CUtensorMap tO;
+  if (!make_tmap_f32_2d(&tO, ws.O, (uint64_t)p.dv, slots * 64, (uint64_t)p.dv * 4, 32, 64, err))
+    return cudaErrorInvalidValue;
+  if (p.dv == 128) {
+    e = cudaFuncSetAttribute(scan_out_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)OUT_SMEM);
+    if (e != cudaSuccess) return e;
+    scan_out_kernel<128><<<(unsigned)items, 128, OUT_SMEM, s>>>(tR, tM, tO, p, ws, total_chunks);
+  } else {
+    e = cudaFuncSetAttribute(scan_out_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)OUT_SMEM);
+    if (e != cudaSuccess) return e;
+    scan_out_kernel<64><<<(unsigned)items, 128, OUT_SMEM, s>>>(tR, tM, tO, p, ws, total_chunks);
+  }
   return cudaGetLastError();
 }
 

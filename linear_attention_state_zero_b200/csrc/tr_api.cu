@@ -247,8 +247,8 @@ size_t scan_ws_bytes(const tr::ScanLaunch &p) {
   return use_chunked(p) ? tr::scan_chunked_workspace(p) : 0;
 }
 
-int scan_kernel_count(const tr::ScanLaunch &p) {
-  return use_chunked(p) ? tr::scan_chunked_kernels() : 1;
+int scan_kernel_count(const tr::ScanLaunch &p, bool with_readout) {
+  return use_chunked(p) ? tr::scan_chunked_kernels(with_readout) : 1;
 }
 
 tr_status run_scan(const tr::ScanLaunch &p, cudaStream_t s,
@@ -348,7 +348,7 @@ int group_kernel_count(const tr_group_args *a) {
   for (int l = 0; l < a->n_layers; ++l) {
     const bool last = l == a->n_layers - 1;
     const bool skip = last && (a->flags & TR_SKIP_LAST_OUTPUT);
-    n += 2 + scan_kernel_count(group_scan_launch(a));
+    n += 2 + scan_kernel_count(group_scan_launch(a), !skip);
     if (!skip && (!last || a->x_out)) n += 1;
   }
   return n;

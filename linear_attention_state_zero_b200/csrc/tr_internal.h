@@ -83,12 +83,13 @@ bool make_tmap_f32_2d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_
                       std::string *err);
 
 cudaError_t launch_scan_recurrent(const ScanLaunch &p, cudaStream_t s);
-// Two launches (prep, chain); `between` runs after the first one is enqueued.
+// Two or three launches (prep, chain, and the readout when o is requested); `between`
+// runs after every launch but the last.
 cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string *err,
                                 const std::function<cudaError_t()> &between);
 bool scan_chunked_supported(const ScanLaunch &p);
 size_t scan_chunked_workspace(const ScanLaunch &p);  // needs p.cu_seqlens_host, H, dv
-int scan_chunked_kernels();
+int scan_chunked_kernels(bool with_readout);
 
 cudaError_t launch_state_error(const float *S, const float *Sh, int64_t n_mats, int64_t mat_elems,
                                double *partials, double *err_per, double *err_total,
