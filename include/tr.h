@@ -231,6 +231,23 @@ tr_status tr_state_error(const float *S, const float *S_hat, int64_t n_mats, int
                          size_t ws_bytes, void *stream);
 
 /*
+ * tr_state_error_noalloc: the same result as tr_state_error, for callers that
+ * cannot allocate device memory when they make the call (an engine whose
+ * allocator owns all device memory, or code where cudaMalloc would synchronize
+ * the device).  The paper has no counterpart: this is a deployment variant.
+ *   - Scratch space is a fixed array inside the library (2 x 65536 doubles, 1 MiB
+ *     per GPU that loads the library, held until the process exits); n_mats above
+ *     65536 is rejected with TR_ERR_UNSUPPORTED.  Nothing is allocated.
+ *   - The first call on a device looks up the array's device address for that
+ *     device (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls share the array: calls whose kernels may overlap on the GPU race.
+ *     Each call writes every scratch entry it reads, so nothing needs clearing.
+ */
+tr_status tr_state_error_noalloc(const float *S, const float *S_hat, int64_t n_mats, int32_t d_k,
+                                 int32_t d_v, double *err_per_mat, double *err_total,
+                                 void *stream);
+
+/*
  * ---------------------------------------------- steps of one LA layer, alone
  * The three dense steps of tr_replay_group, exposed so that each can be checked
  * on its own.  Same arithmetic and cast points as inside tr_replay_group.

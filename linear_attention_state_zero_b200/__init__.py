@@ -69,6 +69,7 @@ _SIGNATURES = {
     "tr_state_error_workspace_size": (c_sz, [c_i64]),
     "tr_state_error": (ctypes.c_int, [c_vp, c_vp, c_i64, c_i32, c_i32, c_vp, c_vp, c_vp, c_sz,
                                       c_vp]),
+    "tr_state_error_noalloc": (ctypes.c_int, [c_vp, c_vp, c_i64, c_i32, c_i32, c_vp, c_vp, c_vp]),
     "tr_rmsnorm": (ctypes.c_int, [c_vp, c_i32, c_vp, c_i64, c_i32, c_f32, c_vp, c_vp]),
     "tr_in_projection": (ctypes.c_int, [c_vp, c_vp, c_i64, c_i32, c_i32, c_i32, c_i32, c_u32,
                                         c_f32, c_vp, c_vp, c_vp, c_vp]),
@@ -287,6 +288,22 @@ def state_error(S, S_hat, *, per_mat=True, stream=None):
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=S.device) if ws_bytes else None
     _ok(lib.tr_state_error(_ptr(S), _ptr(S_hat), n, dk, dv, _ptr(per), _ptr(tot), _ptr(ws),
                            ws_bytes, _stream(stream)), "tr_state_error")
+    return per, tot
+
+
+def state_error_noalloc(S, S_hat, *, per_mat=True, stream=None):
+    """Same as state_error, through the entry point that allocates no scratch
+    (for callers that cannot allocate device memory at the call; see include/tr.h)."""
+    _need_cuda(S, S_hat)
+    if S.shape != S_hat.shape or S.dtype != torch.float32 or S_hat.dtype != torch.float32:
+        raise ValueError("S and S_hat must be fp32 tensors of one shape")
+    dk, dv = S.shape[-2:]
+    S, S_hat = S.contiguous(), S_hat.contiguous()
+    n = S.numel() // (dk * dv)
+    per = torch.empty(n, dtype=torch.float64, device=S.device) if per_mat else None
+    tot = torch.empty(1, dtype=torch.float64, device=S.device)
+    _ok(lib.tr_state_error_noalloc(_ptr(S), _ptr(S_hat), n, dk, dv, _ptr(per), _ptr(tot),
+                                   _stream(stream)), "tr_state_error_noalloc")
     return per, tot
 
 

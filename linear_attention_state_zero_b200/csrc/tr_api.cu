@@ -98,6 +98,16 @@ EncodeTiledFn encode_fn() {
 
 namespace tr {
 
+int record_error(int status, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = status == TR_OK ? std::string() : std::string(buf);
+  return status;
+}
+
 int device_sm_count() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;

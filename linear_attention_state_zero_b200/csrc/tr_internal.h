@@ -59,6 +59,10 @@ struct ScanLaunch {
 
 int device_sm_count();
 
+// Set the thread-local message tr_last_error() returns (cleared for TR_OK) and
+// return `status`; printf-style.
+int record_error(int status, const char *fmt, ...);
+
 // 2D bf16 tensor map, 128-byte swizzle: `outer` rows of `inner` elements with
 // `row_stride_bytes` between rows; box = box_inner x box_outer elements.
 bool make_tmap_bf16_2d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t outer,
