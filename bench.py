@@ -45,6 +45,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--sample-tokens", type=int, default=205,
+                   help="reference arm: tail tokens per timed step (a bounded sample)")
     p.add_argument("--profile", choices=["scan", "group"], default=None,
                    help="run only one workload a few times (for ncu captures), no JSON line")
     return p.parse_args()
@@ -90,6 +92,30 @@ def load_peaks():
 def env_rank():
     return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
             int(os.environ.get("LOCAL_RANK", "0")))
+
+
+# ------------------------------------------------------------ multi-rank host logic
+# Every rank replays its own independent request (weak scaling): nothing but the
+# timing crosses ranks.
+def rank_seed(rank):
+    """Seed of the request a rank replays: distinct per rank, the same on every run."""
+    import synth
+    return synth.SEED_BASE + 1 + 1000 * rank
+
+
+def max_over_ranks(x, world, device):
+    """Largest x over all ranks (the slowest rank sets the job time)."""
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, world, ms_per_step):
+    """Units processed by all ranks per second, given the max-over-ranks step time."""
+    return world * units_per_rank / (ms_per_step * 1e-3)
 
 
 # ------------------------------------------------------------------ flop/byte model
@@ -189,7 +215,7 @@ def reference_arm(args):
     seed = synth.SEED_BASE + 1
     h_tail = synth.hidden_prefix(M_PREFIX, D, seed)[M_PREFIX - k:]
     layers = synth.la_layers(L, D, H, DH, DH, seed=seed)
-    sample = 205  # tokens per step: the first 1/8 of the tail, through all 3 layers
+    sample = args.sample_tokens  # tokens per step (default 205 = 1/8 of the tail), all 3 layers
     cu = [0, sample]
     times = []
     for i in range(args.warmup + args.steps):
@@ -248,7 +274,7 @@ def our_arm(args):
     peaks, peak_src = load_peaks()
 
     k = tr.tail_len(M_PREFIX, R_NUM, R_DEN)
-    seed = synth.SEED_BASE + 1 + 1000 * rank
+    seed = rank_seed(rank)
     h_full_cpu = synth.hidden_prefix(M_PREFIX, D, seed)
     h_tail_cpu = h_full_cpu[M_PREFIX - k:].contiguous()
     layers_cpu = synth.la_layers(L, D, H, DH, DH, seed=seed)
@@ -304,13 +330,9 @@ def our_arm(args):
         dist.barrier()
     clk = clocks.stop()
     tr.check()
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * k / (ms_per_step * 1e-3)
+    value = job_throughput(k, world, ms_per_step)
 
     # per-kernel breakdown (launch order: per layer rmsnorm, in-proj, scan[, out-proj])
     # launch order per layer: rmsnorm, in_proj, scan kernels, out_proj (not after the last
@@ -354,10 +376,7 @@ def our_arm(args):
         e1.synchronize()
         if i >= args.warmup:
             e2e_ms.append(e0.elapsed_time(e1))
-    t = torch.tensor([sum(e2e_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_value = world * k / (float(t.item()) / args.steps * 1e-3)
+    e2e_value = job_throughput(k, world, max_over_ranks(sum(e2e_ms), world, dev) / args.steps)
 
     # scan-only cell: 32 heads d=128, m=32768, r=0.10 (k=3277), bf16, alpha ~ U[0.97, 1]
     k5 = tr.tail_len(32768, 10, 100)
