@@ -150,6 +150,86 @@ def group_model(k):
     return F, B
 
 
+KERNEL_DESC = {
+    "rmsnorm": "RMSNorm (bytes: x in, x_hat out)",
+    "in_proj": "in-proj tcgen05 GEMM + gate/key-norm epilogue (flops)",
+    "scan_prep": "chunked scan, per-(chunk, head) prep (bytes: q, k, v, log alpha, beta in)",
+    "scan_chain": "chunked scan, chunk-to-chunk state chain (bytes: final state out)",
+    "scan_out": "chunked scan, readout (bytes: o out)",
+    "out_proj": "out-proj tcgen05 GEMM + residual (flops)",
+    "scan": "token-recurrent scan (bytes: q, k, v, gates in, o out)",
+}
+
+
+def kernel_work(name, layer, k):
+    """Algorithmic work of one launch: ("tensor", FLOPs) or ("hbm", bytes)."""
+    last = layer == L - 1
+    if name == "rmsnorm":
+        return "hbm", k * D * ((2 if layer == 0 else 4) + 2)
+    if name == "in_proj":
+        return "tensor", flops_inproj(k, last)
+    if name == "scan_prep":
+        return "hbm", k * H * ((2 if last else 3) * DH * 2 + 8)
+    if name == "scan_chain":
+        return "hbm", H * DH * DH * 4
+    if name == "scan_out":
+        return "hbm", k * H * DH * 2
+    if name == "out_proj":
+        return "tensor", flops_outproj(k)
+    if name == "scan":
+        return "hbm", k * H * ((2 if last else 3) * DH * 2 + 8 + (0 if last else DH * 2))
+    raise KeyError(name)
+
+
+def kernel_rooflines(names, avg_ms, k, peaks):
+    """Per kernel (summed over the layers): achieved algorithmic rate / measured peak."""
+    out = {}
+    layer, seen = 0, set()
+    work, ms, launches, bound = {}, {}, {}, {}
+    for n, t in zip(names, avg_ms):
+        if n in seen and n == "rmsnorm":
+            layer += 1
+        seen.add(n)
+        b, w = kernel_work(n, layer, k)
+        bound[n] = b
+        work[n] = work.get(n, 0.0) + w
+        ms[n] = ms.get(n, 0.0) + t
+        launches[n] = launches.get(n, 0) + 1
+    for n in work:
+        if bound[n] == "tensor":
+            ach, peak, unit = work[n] / (ms[n] * 1e-3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+        else:
+            ach, peak, unit = work[n] / (ms[n] * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
+        out[n] = {"bound": bound[n], "achieved": ach, "peak": peak, "unit": unit,
+                  "frac": ach / peak, "launches_per_step": launches[n],
+                  "us_per_step": ms[n] * 1e3,
+                  ("flops" if bound[n] == "tensor" else "bytes") + "_per_launch":
+                      work[n] / launches[n],
+                  "what": KERNEL_DESC[n]}
+    return out
+
+
+def load_traffic():
+    """DRAM bytes per launch (read + write) from the committed ncu summary, per kernel; a
+    kernel whose source changed since the capture gets None."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "dram_traffic_group_step.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return {}
+    out = {}
+    for n, r in rec.get("kernels", {}).items():
+        try:
+            with open(os.path.join(ROOT, r["source"]), "rb") as f:
+                sha = hashlib.sha256(f.read()).hexdigest()
+        except OSError:
+            continue
+        out[n] = r["bytes_per_launch"] if sha == r["sha256"] else None
+    return out
+
+
 # --------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -300,14 +380,25 @@ def our_arm(args):
     handles = [e.cuda_event for e in events]
 
     def step():
+        # the production path: every kernel launched back to back (programmatic
+        # dependent launch between them)
+        rep.run(stream)
+        per, tot = tr.state_error(S_m_flat, S_hat_flat, per_mat=False)
+        return tot
+
+    def step_profiled():
+        # the same kernels with an event recorded after each one (no overlap of launches)
         rep.run_profiled(handles[:n_k + 1], stream)
         per, tot = tr.state_error(S_m_flat, S_hat_flat, per_mat=False)
         events[-1].record(stream)
         return tot
 
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for _ in range(args.warmup):
         flush.zero_()
         step()
+        flush.zero_()
+        step_profiled()
     torch.cuda.synchronize()
     tr.check()
 
@@ -316,15 +407,15 @@ def our_arm(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    step_ms, kern_ms = [], [[] for _ in range(n_k)]
+    step_ms = []
     err_tot = None
     for _ in range(args.steps):
-        flush.zero_()
+        flush.zero_()  # L2 flush outside the timed interval
+        e0.record(stream)
         err_tot = step()
-        torch.cuda.synchronize()  # read this step's events before they are re-recorded
-        step_ms.append(events[0].elapsed_time(events[-1]))
-        for i in range(n_k):
-            kern_ms[i].append(events[i].elapsed_time(events[i + 1]))
+        e1.record(stream)
+        e1.synchronize()
+        step_ms.append(e0.elapsed_time(e1))
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -333,6 +424,17 @@ def our_arm(args):
     total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps
     value = job_throughput(k, world, ms_per_step)
+
+    # per-kernel CUDA-event times over the same number of steps (profiled launches)
+    prof_ms, kern_ms = [], [[] for _ in range(n_k)]
+    for _ in range(args.steps):
+        flush.zero_()
+        step_profiled()
+        torch.cuda.synchronize()  # read this step's events before they are re-recorded
+        prof_ms.append(events[0].elapsed_time(events[-1]))
+        for i in range(n_k):
+            kern_ms[i].append(events[i].elapsed_time(events[i + 1]))
+    tr.check()
 
     # per-kernel breakdown (launch order: per layer rmsnorm, in-proj, scan[, out-proj])
     # launch order per layer: rmsnorm, in_proj, scan kernels, out_proj (not after the last
@@ -351,10 +453,9 @@ def our_arm(args):
     brk = {}
     for n, a in zip(names, avg):
         brk[n] = brk.get(n, 0.0) + a * 1e3
-    in_idx = [i for i, n in enumerate(names) if n == "in_proj"]
-    in_flops = sum(flops_inproj(k, l == L - 1) for l in range(L))
-    in_ms = sum(avg[i] for i in in_idx)
-    achieved_tf = in_flops / (in_ms * 1e-3) / 1e12
+    kernels = kernel_rooflines(names, avg, k, peaks)
+    dominant = max(kernels, key=lambda n: kernels[n]["us_per_step"])
+    traffic = load_traffic()
     F, B = group_model(k)
     t_roof = max(F / (peaks["bf16_tflops"] * 1e12), B / (peaks["hbm_gbs"] * 1e9))
 
@@ -362,7 +463,6 @@ def our_arm(args):
     h_host = h_tail_cpu.pin_memory()
     S_host = torch.empty(rep.S_hat.shape, dtype=torch.float32).pin_memory()
     err_host = torch.empty(1, dtype=torch.float64).pin_memory()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e_ms = []
     for i in range(args.warmup + args.steps):
         flush.zero_()
@@ -417,11 +517,12 @@ def our_arm(args):
             "token_layers_per_s": value * L,
             "state_updates_per_s": value * L * H,
             "state_error_vs_full_prefill": float(err_tot.item()),
-            "roofline": {"bound": "tensor", "kernel": "in_proj (tcgen05 GEMM + gate/norm epilogue)",
-                         "achieved": achieved_tf, "peak": peaks["bf16_tflops"],
-                         "unit": "TFLOP/s", "frac": achieved_tf / peaks["bf16_tflops"],
-                         "traffic": None, "peak_source": peak_src + " (burst bf16)",
-                         "flops_per_step": in_flops, "ms_per_step": in_ms},
+            "roofline": dict(kernels[dominant], kernel=dominant,
+                             traffic=traffic.get(dominant),
+                             peak_source=peak_src + (" (burst bf16)" if kernels[dominant]["bound"] ==
+                                                     "tensor" else " (HBM copy)")),
+            "kernel_rooflines": {n: dict(r, traffic=traffic.get(n)) for n, r in kernels.items()},
+            "profiled_ms_per_step": sum(prof_ms) / len(prof_ms),
             "group_roofline": {"t_roof_us": t_roof * 1e6, "t_step_us": ms_per_step * 1e3,
                                "frac": t_roof / (ms_per_step * 1e-3), "alg_flops": F,
                                "alg_bytes": B},

@@ -123,42 +123,73 @@ __device__ __forceinline__ void epi_inproj(const InProjEpi &ep, uint32_t tbase, 
   }
 }
 
+// 32 residual values of `row` at column c: fp32, or bf16 widened
+struct Res32 {
+  uint4 u[8];
+};
+__device__ __forceinline__ void load_res32(const ResidEpi &ep, int64_t row, int c, Res32 &r) {
+  if (ep.res_is_bf16) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(
+        reinterpret_cast<const __nv_bfloat16 *>(ep.x_res) + row * ep.ld + c);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) r.u[w] = src[w];
+  } else {
+    const uint4 *src = reinterpret_cast<const uint4 *>(
+        reinterpret_cast<const float *>(ep.x_res) + row * ep.ld + c);
+#pragma unroll
+    for (int w = 0; w < 8; ++w) r.u[w] = src[w];
+  }
+}
+__device__ __forceinline__ void res32_to_f32(const ResidEpi &ep, const Res32 &r, float (&f)[32]) {
+  if (ep.res_is_bf16) {
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&r.u[w]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 t = __bfloat1622float2(h[i]);
+        f[8 * w + 2 * i] = t.x;
+        f[8 * w + 2 * i + 1] = t.y;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      f[4 * w] = __uint_as_float(r.u[w].x);
+      f[4 * w + 1] = __uint_as_float(r.u[w].y);
+      f[4 * w + 2] = __uint_as_float(r.u[w].z);
+      f[4 * w + 3] = __uint_as_float(r.u[w].w);
+    }
+  }
+}
+
+// Output-projection epilogue for one 128 x BN tile; this thread owns `row`.  The
+// residual of the next 32 columns is requested before the current ones are added, so
+// one global-load latency is in flight behind every TMEM load.
 template <int BN>
 __device__ __forceinline__ void epi_resid(const ResidEpi &ep, uint32_t tbase, int n0, int N,
                                           int row, int M) {
+  const bool live = row < M;
+  Res32 cur, nxt;
+  if (live && n0 < N) load_res32(ep, row, n0, cur);
 #pragma unroll 1
   for (int j = 0; j < BN / 32; ++j) {
     const int c = n0 + 32 * j;
     if (c >= N) break;
+    if (live && j + 1 < BN / 32 && c + 32 < N) load_res32(ep, row, c + 32, nxt);
     float v[32];
     tmem_ld32(tbase + 32 * j, v);
     tc_wait_ld();
-    if (row >= M) continue;
-    float4 *out = reinterpret_cast<float4 *>(ep.x_out + (int64_t)row * ep.ld + c);
-    if (ep.res_is_bf16) {
-      const uint4 *r = reinterpret_cast<const uint4 *>(
-          reinterpret_cast<const __nv_bfloat16 *>(ep.x_res) + (int64_t)row * ep.ld + c);
+    if (live) {
+      float r[32];
+      res32_to_f32(ep, cur, r);
+      float4 *out = reinterpret_cast<float4 *>(ep.x_out + (int64_t)row * ep.ld + c);
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        uint4 p = r[w];
-        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&p);
-        float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
-        float2 f2 = __bfloat1622float2(h[2]), f3 = __bfloat1622float2(h[3]);
-        out[2 * w] = make_float4(f0.x + v[8 * w + 0], f0.y + v[8 * w + 1], f1.x + v[8 * w + 2],
-                                 f1.y + v[8 * w + 3]);
-        out[2 * w + 1] = make_float4(f2.x + v[8 * w + 4], f2.y + v[8 * w + 5],
-                                     f3.x + v[8 * w + 6], f3.y + v[8 * w + 7]);
-      }
-    } else {
-      const float4 *r = reinterpret_cast<const float4 *>(
-          reinterpret_cast<const float *>(ep.x_res) + (int64_t)row * ep.ld + c);
-#pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        float4 a = r[w];
-        out[w] = make_float4(a.x + v[4 * w], a.y + v[4 * w + 1], a.z + v[4 * w + 2],
-                             a.w + v[4 * w + 3]);
-      }
+      for (int w = 0; w < 8; ++w)
+        out[w] = make_float4(r[4 * w] + v[4 * w], r[4 * w + 1] + v[4 * w + 1],
+                             r[4 * w + 2] + v[4 * w + 2], r[4 * w + 3] + v[4 * w + 3]);
     }
+    cur = nxt;
   }
 }
 
@@ -203,6 +234,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
   const AbortFlag ab{&ctl->abort, err_word, ERRBIT_GEMM_TIMEOUT};
+  // TMEM is held: the next kernel may start launching; the inputs are the previous
+  // kernel's outputs, so wait for it before the first load
+  pdl_trigger();
+  pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -289,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int BN, int EPI>
 cudaError_t launch(const void *A, int64_t lda, const void *B, int M, int N, int K,
                    const InProjEpi &ip, const ResidEpi &rs, unsigned *err_word, cudaStream_t s,
-                   std::string *err) {
+                   bool pdl, std::string *err) {
   using C = Cfg<BN>;
   if (M <= 0 || N <= 0) return cudaSuccess;
   CUtensorMap ta, tb;
@@ -303,24 +338,26 @@ cudaError_t launch(const void *A, int64_t lda, const void *B, int M, int N, int 
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   int grid = device_sm_count();
   if (grid > tiles) grid = tiles;
-  kern<<<grid, kThreads, C::SMEM, s>>>(ta, tb, M, N, K, ip, rs, err_word);
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3((unsigned)grid), dim3(kThreads), C::SMEM, s, pdl, ta, tb, M, N, K,
+                       ip, rs, err_word);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_inproj(const void *A, const void *B, int M, int N, int K,
                                const InProjEpi &ep, unsigned *err_word, cudaStream_t s,
-                               std::string *err) {
+                               bool pdl, std::string *err) {
   ResidEpi none{};
-  return launch<256, EPI_INPROJ>(A, K, B, M, N, K, ep, none, err_word, s, err);
+  return launch<256, EPI_INPROJ>(A, K, B, M, N, K, ep, none, err_word, s, pdl, err);
 }
 
 cudaError_t launch_gemm_resid(const void *A, int64_t lda, const void *B, int M, int N, int K,
-                              const ResidEpi &ep, unsigned *err_word, cudaStream_t s,
+                              const ResidEpi &ep, unsigned *err_word, cudaStream_t s, bool pdl,
                               std::string *err) {
   InProjEpi none{};
-  return launch<256, EPI_RESID>(A, lda, B, M, N, K, none, ep, err_word, s, err);
+  // 128-column tiles: the output is narrow (d_model), so twice the tiles spread over
+  // the SMs and a CTA with two tiles hides one tile's epilogue behind the other's MMAs
+  return launch<128, EPI_RESID>(A, lda, B, M, N, K, none, ep, err_word, s, pdl, err);
 }
 
 }  // namespace tr

@@ -23,7 +23,8 @@ namespace {
 
 constexpr int64_t kStaticMats = 65536;  // largest n_mats one call accepts
 
-// Per-matrix (sum (S - S_hat)^2, sum S^2) partials of the last call.
+// (sum (S - S_hat)^2, sum S^2) of each matrix piece of the last call (at most
+// kStaticMats pieces: a matrix is cut into fewer pieces when n_mats is large).
 static __device__ __align__(256) double g_noalloc_scratch[2 * kStaticMats];
 
 constexpr int kMaxDevices = 64;
@@ -70,8 +71,10 @@ extern "C" tr_status tr_state_error_noalloc(const float *S, const float *S_hat, 
   cudaError_t e = scratch_for_current_device(&scratch);
   if (e != cudaSuccess)
     return tr::record_error(TR_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
-  e = tr::launch_state_error(S, S_hat, n_mats, (int64_t)d_k * d_v, scratch, err_per_mat, err_total,
-                             static_cast<cudaStream_t>(stream));
+  const int64_t elems = (int64_t)d_k * d_v;
+  e = tr::launch_state_error(S, S_hat, n_mats, elems, tr::state_error_splits(n_mats, elems, kStaticMats),
+                             scratch, err_per_mat, err_total, static_cast<cudaStream_t>(stream),
+                             true);
   if (e != cudaSuccess)
     return tr::record_error(TR_ERR_CUDA, "state error: %s", cudaGetErrorString(e));
   return tr::record_error(TR_OK, "");

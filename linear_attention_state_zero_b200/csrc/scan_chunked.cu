@@ -72,6 +72,15 @@ __device__ __forceinline__ void store_row_bf16(uint8_t *tile, int row, int col0,
   }
 }
 
+// 32 fp32 values (v[i] * s) as row `row` (128 bytes) of a 128-byte-row swizzled tile.
+__device__ __forceinline__ void store_row32_f32(uint8_t *tile, int row, const float *v, float s) {
+#pragma unroll
+  for (int ch = 0; ch < 8; ++ch)
+    st_shared_v4(smem_u32(tile + sw128_offset((uint32_t)row, (uint32_t)ch * 16u)),
+                 __float_as_uint(v[4 * ch] * s), __float_as_uint(v[4 * ch + 1] * s),
+                 __float_as_uint(v[4 * ch + 2] * s), __float_as_uint(v[4 * ch + 3] * s));
+}
+
 // 8 consecutive bf16 of row `row` starting at column col0 (multiple of 8).
 __device__ __forceinline__ void load_row8_bf16(const uint8_t *tile, int row, int col0, float *f) {
   const uint4 u = *reinterpret_cast<const uint4 *>(
@@ -197,6 +206,7 @@ struct PrepCtl {
   float beta[C];
   float bg[C];     // beta * gamma
   int cu_chunks[kMaxSeqsChunked + 1];
+  int cu_tok[kMaxSeqsChunked + 1];  // the sequence offsets (cu_seqlens)
 };
 
 // hi + lo bf16 split of 32 values (v[i] * s) into two 128-byte-row swizzled tiles.
@@ -220,10 +230,23 @@ __device__ __forceinline__ void store_row_split(uint8_t *hi, uint8_t *lo, int ro
   }
 }
 
+// Output staging after the last product of an item (every region below is free by then;
+// each tile is 128-byte swizzled, one TMA box):
+//   A_c  [2 halves][128 rows][64 bf16]  at P_TU
+//   B_c  [DV/32 boxes][128 rows][32 fp32] at P_TSH (spans TSH, TSL, AW)
+//   R    [2 halves][64 rows][64 bf16]   at P_AP
+//   O0   [DV/32 boxes][64 rows][32 fp32] in the item's input buffer, over the K rows and V
+//        (the Q rows stay intact: R reads them)
+__device__ __forceinline__ uint32_t o0_box_offset(int b) {
+  return b < 2 ? (uint32_t)b * 16384u : 32768u + (uint32_t)(b - 2) * 8192u;
+}
+
 template <int DV>
 __global__ void __launch_bounds__(kPrepThreads, 1)
     scan_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, ScanLaunch p, ScanWs ws,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_A,
+                     const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_R,
+                     const __grid_constant__ CUtensorMap tm_O, ScanLaunch p, ScanWs ws,
                      int total_chunks) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ PrepCtl ctl_s;
@@ -241,14 +264,14 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   const bool want_o = p.o != nullptr;
   const int64_t n_items = (int64_t)total_chunks * H;
 
-  // first chunk of every sequence
   if (tid == 0) {
-    int acc = 0;
-    for (int i = 0; i < p.n_seqs; ++i) {
-      ctl->cu_chunks[i] = acc;
-      acc += (p.cu_seqlens[i + 1] - p.cu_seqlens[i] + C - 1) / C;
-    }
-    ctl->cu_chunks[p.n_seqs] = acc;
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_A);
+    tma_prefetch_desc(&tm_B);
+    tma_prefetch_desc(&tm_R);
+    tma_prefetch_desc(&tm_O);
     mbar_init(smem_u32(&ctl->tma_bar[0]), 1);
     mbar_init(smem_u32(&ctl->tma_bar[1]), 1);
     mbar_init(smem_u32(&ctl->mma_bar), 1);
@@ -271,6 +294,20 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ctl->tmem;
   const AbortFlag ab{&ctl->abort, p.err_word, ERRBIT_SCAN_TIMEOUT};
+  // TMEM is held: let the next kernel launch; then wait for the previous one's outputs
+  pdl_trigger();
+  pdl_wait();
+  // first chunk of every sequence
+  if (tid == 0) {
+    int acc = 0;
+    for (int i = 0; i < p.n_seqs; ++i) {
+      ctl->cu_chunks[i] = acc;
+      acc += (p.cu_seqlens[i + 1] - p.cu_seqlens[i] + C - 1) / C;
+    }
+    ctl->cu_chunks[p.n_seqs] = acc;
+  }
+  for (int i = tid; i <= p.n_seqs; i += kPrepThreads) ctl->cu_tok[i] = p.cu_seqlens[i];
+  __syncthreads();
 
   // (sequence, chunk) of an item
   auto locate = [&](int64_t item, int &seq, int &cc) {
@@ -287,7 +324,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     int seq, cc;
     locate(item, seq, cc);
     const int head = (int)(item % H);
-    const int t0 = p.cu_seqlens[seq] + cc * C;
+    const int t0 = ctl->cu_tok[seq] + cc * C;
     const uint32_t bar = smem_u32(&ctl->tma_bar[buf]);
     const uint32_t kq = smem_u32(sm + P_IN + buf * P_IN_BYTES);
     mbar_arrive_expect_tx(bar, 16384u + (want_o ? 16384u : 0u) + (uint32_t)DV * 128u);
@@ -306,6 +343,22 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     if ((int64_t)blockIdx.x < n_items) issue(blockIdx.x, 0);
     if ((int64_t)blockIdx.x + gridDim.x < n_items) issue(blockIdx.x + gridDim.x, 1);
   }
+  // log alpha and beta of an item's 64 tokens (thread tid < C: token tid; 0 past the end)
+  auto load_gates = [&](int64_t it, float &la, float &b) {
+    int sq, cq;
+    locate(it, sq, cq);
+    const int hd = (int)(it % H);
+    const int tt = ctl->cu_tok[sq] + cq * C;
+    la = 0.f;
+    b = 0.f;
+    if (tid < min(C, ctl->cu_tok[sq + 1] - tt)) {
+      la = p.log_alpha[(size_t)(tt + tid) * H + hd];
+      b = p.beta[(size_t)(tt + tid) * H + hd];
+    }
+  };
+  // the next item's gates are loaded during the current item
+  float la_next = 0.f, b_next = 0.f;
+  if (tid < C && (int64_t)blockIdx.x < n_items) load_gates(blockIdx.x, la_next, b_next);
   const uint32_t mma_bar = smem_u32(&ctl->mma_bar);
   uint32_t mma_phase = 0;
   auto mma_wait = [&]() -> bool {
@@ -319,22 +372,14 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   int n = 0;
   for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x, ++n) {
     const int buf = n & 1;
-    int seq, cc;
-    locate(item, seq, cc);
-    const int head = (int)(item % H);
-    const int t0 = p.cu_seqlens[seq] + cc * C;
-    const int nv = min(C, p.cu_seqlens[seq + 1] - t0);
     uint8_t *KQ = sm + P_IN + buf * P_IN_BYTES;
     const uint32_t kq_u = smem_u32(KQ);
     const uint32_t v_u = kq_u + 32768;
 
     // gates: g = inclusive cumsum of log alpha (0 past the end), beta, beta * gamma
     if (tid < C) {
-      float la = 0.f, b = 0.f;
-      if (tid < nv) {
-        la = p.log_alpha[(size_t)(t0 + tid) * H + head];
-        b = p.beta[(size_t)(t0 + tid) * H + head];
-      }
+      const float la = la_next, b = b_next;
+      if (item + (int64_t)gridDim.x < n_items) load_gates(item + gridDim.x, la_next, b_next);
       float s = la;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -365,6 +410,10 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         tc_mma_bf16(tmem, desc_k(dkq, kk, 16384), desc_k(dkq, kk, 16384),
                     idesc_bf16(128, 64, 0, 0), kk > 0);
       tc_commit(mma_bar);
+      // the previous item's output stores of R and B_c boxes 2, 3 must have read their
+      // staging before the A/P phase overwrites it (all threads pass the barrier in
+      // mma_wait after this); A_c and B_c boxes 0, 1 are waited for before the inverse
+      bulk_wait_read<1>();
     }
     if (!mma_wait()) break;
 
@@ -394,6 +443,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         store_row_bf16(sm + P_AP, row, 32 * hsel, v, 1.f);
       }
     }
+    if (tid == 0) bulk_wait_read<0>();  // the staging of A_c, B_c boxes 0, 1 is free
     __syncthreads();
 
     // T = (I + A)^{-1}, blocked: T11 = (I + A11)^{-1}, T22 = (I + A22)^{-1} by forward
@@ -457,14 +507,21 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       *reinterpret_cast<float4 *>(Ts + (32 + r) * LDA + c0) = make_float4(-x0, -x1, -x2, -x3);
     }
     __syncthreads();
-    {  // [-T diag(beta); T diag(beta gamma)] as high + low bf16 parts
-      const int rr = tid >> 1, half = tid & 1, t = rr & 63;
+    {  // [-T diag(beta); T diag(beta gamma)] as high + low bf16 parts; consecutive lanes
+       // take consecutive rows (conflict-free reads of T and swizzled stores)
+      const int rr = tid & 127, half = tid >> 7, t = rr & 63;
+      const bool zero = t < 32 && half == 1;  // T is lower triangular: T12 = 0
       float v[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int s = 32 * half + i;
-        const float tv = (t < 32 && s >= 32) ? 0.f : Ts[t * LDA + s];
-        v[i] = (rr < C) ? -tv * ctl->beta[s] : tv * ctl->bg[s];
+      for (int w = 0; w < 8; ++w) {
+        const float4 tv = zero ? make_float4(0.f, 0.f, 0.f, 0.f)
+                               : *reinterpret_cast<const float4 *>(Ts + t * LDA + 32 * half + 4 * w);
+        const float te[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int s = 32 * half + 4 * w + u;
+          v[4 * w + u] = (rr < C) ? -te[u] * ctl->beta[s] : te[u] * ctl->bg[s];
+        }
       }
       store_row_split(sm + P_TSH, sm + P_TSL, rr, 32 * half, v, 1.f);
     }
@@ -498,7 +555,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       const int t = row & 63;
       const float gp = exp_ftz(gC - ctl->g[t]);
       if (row >= C) {  // W row t, columns 64*hsel..+63 -> W and gamma' W ([t][d], 8 KB halves)
-#pragma unroll
+#pragma unroll 1
         for (int j = 0; j < 2; ++j) {
           tmem_ld32(tmem + 192 + lane_base + 64 * hsel + 32 * j, v);
           tc_wait_ld();
@@ -506,7 +563,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
           store_row_bf16(sm + P_AW + 16384 + hsel * 8192, t, 32 * j, v, gp);
         }
       } else {  // -U~ row t, columns (DV/2)*hsel.. -> U~ (hi, lo) and gamma' U~ (hi, lo)
-#pragma unroll
+#pragma unroll 1
         for (int j = 0; j < DV / 64; ++j) {
           const int col = (DV / 2) * hsel + 32 * j;
           tmem_ld32(tmem + 64 + lane_base + col, v);
@@ -556,75 +613,88 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
 
     {
       float v[32];
-      const int64_t slot = item;
       // A_c row d = -(K^T gamma' W)[d] (bf16), columns 64*hsel..+63
-      {
-        __nv_bfloat16 *Ad = ws.A + (size_t)slot * 128 * 128 + (size_t)row * 128 + 64 * hsel;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          tmem_ld32(tmem + 256 + lane_base + 64 * hsel + 32 * j, v);
-          tc_wait_ld();
-          uint4 *dst = reinterpret_cast<uint4 *>(Ad + 32 * j);
-#pragma unroll
-          for (int w = 0; w < 4; ++w)
-            dst[w] = make_uint4(pack_bf16x2(-v[8 * w], -v[8 * w + 1]), pack_bf16x2(-v[8 * w + 2], -v[8 * w + 3]),
-                                pack_bf16x2(-v[8 * w + 4], -v[8 * w + 5]), pack_bf16x2(-v[8 * w + 6], -v[8 * w + 7]));
-        }
+#pragma unroll 1
+      for (int j = 0; j < 2; ++j) {
+        tmem_ld32(tmem + 256 + lane_base + 64 * hsel + 32 * j, v);
+        tc_wait_ld();
+        store_row_bf16(sm + P_TU + hsel * 16384, row, 32 * j, v, -1.f);
       }
-      // B_c row d (fp32), columns (DV/2)*hsel..
-      {
-        float *Bd = ws.B + (size_t)slot * 128 * DV + (size_t)row * DV + (DV / 2) * hsel;
-#pragma unroll
-        for (int j = 0; j < DV / 64; ++j) {
-          tmem_ld32(tmem + 384 + lane_base + (DV / 2) * hsel + 32 * j, v);
-          tc_wait_ld();
-          float4 *dst = reinterpret_cast<float4 *>(Bd + 32 * j);
-#pragma unroll
-          for (int w = 0; w < 8; ++w) dst[w] = make_float4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]);
-        }
+      // B_c row d (fp32), columns (DV/2)*hsel.. (one 32-column box per 32 columns)
+#pragma unroll 1
+      for (int j = 0; j < DV / 64; ++j) {
+        tmem_ld32(tmem + 384 + lane_base + (DV / 2) * hsel + 32 * j, v);
+        tc_wait_ld();
+        store_row32_f32(sm + P_TSH + 16384 * (((DV / 2) * hsel + 32 * j) >> 5), row, v, 1.f);
       }
       if (want_o && row >= C) {
         const int t = row - C;
         const float gam = exp_ftz(ctl->g[t]);
         // R row t = gamma_t q_t - (P W)_t (bf16), columns 64*hsel..+63
-        __nv_bfloat16 *Rt = ws.R + (size_t)slot * 64 * 128 + (size_t)t * 128 + 64 * hsel;
-#pragma unroll
+#pragma unroll 1
         for (int j = 0; j < 2; ++j) {
           tmem_ld32(tmem + 0 + lane_base + 64 * hsel + 32 * j, v);
           tc_wait_ld();
-          uint4 *dst = reinterpret_cast<uint4 *>(Rt + 32 * j);
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
             float f[8];
             load_row8_bf16(KQ + hsel * 16384, 64 + t, 32 * j + 8 * w, f);
-            dst[w] = make_uint4(pack_bf16x2(gam * f[0] - v[8 * w], gam * f[1] - v[8 * w + 1]),
-                                pack_bf16x2(gam * f[2] - v[8 * w + 2], gam * f[3] - v[8 * w + 3]),
-                                pack_bf16x2(gam * f[4] - v[8 * w + 4], gam * f[5] - v[8 * w + 5]),
-                                pack_bf16x2(gam * f[6] - v[8 * w + 6], gam * f[7] - v[8 * w + 7]));
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[8 * w + i] = gam * f[i] - v[8 * w + i];
           }
+          store_row_bf16(sm + P_AP + hsel * 8192, t, 32 * j, v, 1.f);
         }
         // O0 row t (fp32), columns (DV/2)*hsel..
-        float *Ot = ws.O + (size_t)slot * 64 * DV + (size_t)t * DV + (DV / 2) * hsel;
-#pragma unroll
+#pragma unroll 1
         for (int j = 0; j < DV / 64; ++j) {
           tmem_ld32(tmem + 128 + lane_base + (DV / 2) * hsel + 32 * j, v);
           tc_wait_ld();
-          float4 *dst = reinterpret_cast<float4 *>(Ot + 32 * j);
-#pragma unroll
-          for (int w = 0; w < 8; ++w) dst[w] = make_float4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]);
+          store_row32_f32(KQ + o0_box_offset(((DV / 2) * hsel + 32 * j) >> 5), t, v, 1.f);
         }
       }
-      if (tid == 0) ws.G[slot] = exp_ftz(gC);
+      fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
-    // this buffer's K/Q/V are no longer read: prefetch the item after next into it
-    if (tid == 0 && item + 2 * (int64_t)gridDim.x < n_items) {
-      fence_proxy_async_smem();
-      issue(item + 2 * (int64_t)gridDim.x, buf);
+    if (tid == 0) {
+      const int64_t slot = item;
+      // three bulk groups, in the order the staging tiles are needed again:
+      //   1. O0 (this item's input buffer: the prefetch below refills it)
+      //   2. R (P_AP) and B_c boxes 2, 3 (P_AW): the next item's A/P phase writes there
+      //   3. A_c (P_TU) and B_c boxes 0, 1 (P_TSH, P_TSL): its inverse and split write there
+      if (want_o) {
+#pragma unroll
+        for (int b = 0; b < DV / 32; ++b)
+          tma_store_2d(&tm_O, smem_u32(KQ + o0_box_offset(b)), 32 * b, (int32_t)(slot * 64));
+      }
+      bulk_commit();
+      if (want_o) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          tma_store_2d(&tm_R, smem_u32(sm + P_AP + h * 8192), 64 * h, (int32_t)(slot * 64));
+      }
+#pragma unroll
+      for (int b = 2; b < DV / 32; ++b)
+        tma_store_2d(&tm_B, smem_u32(sm + P_TSH + 16384 * b), 32 * b, (int32_t)(slot * 128));
+      bulk_commit();
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        tma_store_2d(&tm_A, smem_u32(sm + P_TU + h * 16384), 64 * h, (int32_t)(slot * 128));
+#pragma unroll
+      for (int b = 0; b < 2; ++b)
+        tma_store_2d(&tm_B, smem_u32(sm + P_TSH + 16384 * b), 32 * b, (int32_t)(slot * 128));
+      bulk_commit();
+      ws.G[slot] = exp_ftz(gC);
+      // this buffer's K/Q/V are no longer read: prefetch the item after next into it
+      if (item + 2 * (int64_t)gridDim.x < n_items) {
+        bulk_wait_read<2>();
+        fence_proxy_async_smem();
+        issue(item + 2 * (int64_t)gridDim.x, buf);
+      }
     }
   }
 
+  if (tid == 0) bulk_wait<0>();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -635,9 +705,10 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
 
 // =========================================================== chain kernel
 // One CTA per (sequence, head, 64-column slice of d_v), 288 threads.  Warps 0-7:
-// thread (quarter q4 = warp % 4, half hsel = warp / 4) owns row d = 32 q4 + lane of
-// the fp32 state slice and its columns 32 hsel .. +31.  Warp 8 only refills the TMA
-// ring (a tensor load can stall its issuing thread while many are in flight, so the
+// thread (quarter q4 = warp % 4, column group cg = warp / 4) owns row d = 32 q4 + lane
+// of the fp32 state slice and its columns kCols cg .. +kCols-1 (the per-chunk update is
+// latency-bound: 16 state warps with half the columns each measured no faster).  Warp 8
+// only refills the TMA ring (a tensor load can stall its issuing thread while many are in flight, so the
 // state-owning threads never issue them).  Per chunk: one tcgen05 product
 // Z = A_c M (M in bf16 in shared memory, 8 MMAs of K = 16), then
 // M <- gamma_C M + Z + B_c in registers.  A_c and the B_c slice arrive through a
@@ -670,31 +741,35 @@ __device__ __forceinline__ void load_row32_f32(const uint8_t *tile, int row, flo
   }
 }
 
-constexpr int kChainThreads = 288;
+constexpr int kStateWarps = 8;
+constexpr int kChainThreads = 32 * (kStateWarps + 1);
+constexpr int kCols = DVS * 4 / kStateWarps;  // state columns per thread
+static_assert(kCols == 32, "state columns per thread");
+
+
 
 __global__ void __launch_bounds__(kChainThreads, 1)
     scan_chain_kernel(const __grid_constant__ CUtensorMap tm_A, const __grid_constant__ CUtensorMap tm_B,
                       const __grid_constant__ CUtensorMap tm_M, ScanLaunch p, ScanWs ws) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ ChainCtl ctl_s;
-  __shared__ int red[8];
+  __shared__ int red[32];  // one entry per warp (chunk_base)
   ChainCtl *ctl = &ctl_s;
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int q4 = warp & 3, hsel = warp >> 2;
+  const int q4 = warp & 3, cg = warp >> 2;
   const int d = q4 * 32 + lane;
   const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
   const int H = p.H, DV = p.dv;
   const int seq = blockIdx.x / H, head = blockIdx.x % H;
   const int slice = blockIdx.y;
-  const int col = slice * DVS + 32 * hsel;   // this thread's first d_v column
-  const int t_begin = p.cu_seqlens[seq], t_end = p.cu_seqlens[seq + 1];
-  const int nch = (t_end - t_begin + C - 1) / C;
-  const int cb = chunk_base(p.cu_seqlens, seq, red);
-  auto slot_of = [&](int c) -> int64_t { return ((int64_t)cb + c) * H + head; };
+  const int col = slice * DVS + kCols * cg;   // this thread's first d_v column
 
   if (tid == 0) {
+    tma_prefetch_desc(&tm_A);
+    tma_prefetch_desc(&tm_B);
+    tma_prefetch_desc(&tm_M);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&ctl->tma_bar[s]), 1);
       mbar_init(smem_u32(&ctl->empty_bar[s]), 1);
@@ -707,6 +782,16 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     tmem_alloc(smem_u32(&ctl->tmem), 64);
     tmem_relinquish();
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // TMEM is held: let the next kernel launch; then wait for the previous one's outputs
+  pdl_trigger();
+  pdl_wait();
+  const int t_begin = p.cu_seqlens[seq], t_end = p.cu_seqlens[seq + 1];
+  const int nch = (t_end - t_begin + C - 1) / C;
+  const int cb = chunk_base(p.cu_seqlens, seq, red);
+  auto slot_of = [&](int c) -> int64_t { return ((int64_t)cb + c) * H + head; };
   for (int c = tid; c < nch; c += kChainThreads) ctl->gC[c] = ws.G[slot_of(c)];
   tc_fence_before();
   __syncthreads();
@@ -719,21 +804,22 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     bulk_commit();
   };
 
-  float Mr[32];
+  float Mr[kCols];
   const bool m_zero = p.S0 == nullptr;
-  const bool producer = warp == 8;
+  const bool producer = warp == kStateWarps;
   const size_t s_off = ((size_t)seq * H + head) * DK * DV + (size_t)d * DV + col;
   if (!m_zero && !producer) {
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
+    for (int j = 0; j < kCols; j += 4) {
       const float4 a = *reinterpret_cast<const float4 *>(p.S0 + s_off + j);
       Mr[j] = a.x; Mr[j + 1] = a.y; Mr[j + 2] = a.z; Mr[j + 3] = a.w;
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) Mr[j] = 0.f;
+    for (int j = 0; j < kCols; ++j) Mr[j] = 0.f;
   }
-  if (nch > 0 && !producer) store_row_bf16(sm + H_MB, d, 32 * hsel, Mr, 1.f);
+  auto store_state = [&](uint8_t *tile) { store_row_bf16(tile, d, kCols * cg, Mr, 1.f); };
+  if (nch > 0 && !producer) store_state(sm + H_MB);
 
   auto issue_tma = [&](int c) {
     const int st = c % kStages;
@@ -784,38 +870,48 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     uint32_t z_phase = 0;
     for (int c = 0; c < nch; ++c) {
       const int st = c % kStages;
-      float v[32], b[32];
+      float v[kCols], b[kCols];
       if (mma_for_c) {
         if (!mbar_wait(smem_u32(&ctl->bar_z), z_phase, ab)) failed = true;
         z_phase ^= 1u;
         tc_fence_after();
-        tmem_ld32(tmem + lane_base + 32 * hsel, v);
+        tmem_ld32(tmem + lane_base + kCols * cg, v);
       } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = 0.f;
+        for (int j = 0; j < kCols; ++j) v[j] = 0.f;
       }
-      // the stage's B_c has landed (its A_c did, for the product); read this thread's row
+      // the stage's B_c has landed (its A_c did, for the product); read this thread's
+      // columns of row d from the 32-column box that holds them
       if (!mbar_wait(smem_u32(&ctl->tma_bar[st]), (uint32_t)(c / kStages) & 1u, ab)) failed = true;
-      load_row32_f32(sm + st * H_STAGE + 32768 + hsel * 16384, d, b);
+      {
+        const int c0 = kCols * cg;
+        const uint8_t *bt = sm + st * H_STAGE + 32768 + (c0 >> 5) * 16384;
+#pragma unroll
+        for (int ch = 0; ch < kCols / 4; ++ch) {
+          const float4 u = *reinterpret_cast<const float4 *>(
+              bt + sw128_offset((uint32_t)d, (uint32_t)(((c0 & 31) >> 2) + ch) * 16u));
+          b[4 * ch] = u.x; b[4 * ch + 1] = u.y; b[4 * ch + 2] = u.z; b[4 * ch + 3] = u.w;
+        }
+      }
       if (mma_for_c) tc_wait_ld();
       const float gC = ctl->gC[c];
       // M <- gamma_C M + A_c M + B_c (fp32); bf16 copy for the next product and the readout
 #pragma unroll
-      for (int j = 0; j < 32; ++j) Mr[j] = fmaf(gC, Mr[j], v[j] + b[j]);
-      if (c + 1 < nch) store_row_bf16(sm + H_MB + 16384 * ((c + 1) & 1), d, 32 * hsel, Mr, 1.f);
+      for (int j = 0; j < kCols; ++j) Mr[j] = fmaf(gC, Mr[j], v[j] + b[j]);
+      if (c + 1 < nch) store_state(sm + H_MB + 16384 * ((c + 1) & 1));
       fence_proxy_async_smem();
       tc_fence_before();
       // copy (c + 1) & 1 was last stored to global two chunks ago: that store must have
       // finished reading it before anyone rewrites it (after the barrier below)
       if (tid == 0) bulk_wait_read<0>();
-      // named barrier over the 256 state-owning threads, voting on `failed` so that all
-      // of them leave the loop together
+      // named barrier over the state-owning threads, voting on `failed` so that all of
+      // them leave the loop together
       uint32_t any_failed;
       asm volatile(
           "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
-          "bar.red.or.pred p, 1, 256, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+          "bar.red.or.pred p, 1, %2, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
           : "=r"(any_failed)
-          : "r"((uint32_t)(failed || *ab.flag))
+          : "r"((uint32_t)(failed || *ab.flag)), "n"(32 * kStateWarps)
           : "memory");
       if (any_failed) { failed = true; break; }
       if (tid == 0) {
@@ -835,7 +931,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
   if (!failed && !producer) {
     float *dst = p.S_final + s_off;
 #pragma unroll
-    for (int j = 0; j < 32; j += 4)
+    for (int j = 0; j < kCols; j += 4)
       *reinterpret_cast<float4 *>(dst + j) = make_float4(Mr[j], Mr[j + 1], Mr[j + 2], Mr[j + 3]);
   }
   tc_fence_before();
@@ -873,12 +969,9 @@ __global__ void __launch_bounds__(128)
   const int64_t item = blockIdx.x;
   const int chunk = (int)(item / H), head = (int)(item % H);
   if (tid == 0) {
-    int acc = 0;
-    for (int i = 0; i < p.n_seqs; ++i) {
-      cu_chunks[i] = acc;
-      acc += (p.cu_seqlens[i + 1] - p.cu_seqlens[i] + C - 1) / C;
-    }
-    cu_chunks[p.n_seqs] = acc;
+    tma_prefetch_desc(&tm_R);
+    tma_prefetch_desc(&tm_M);
+    tma_prefetch_desc(&tm_O);
     mbar_init(smem_u32(&bar_t), 1);
     mbar_init(smem_u32(&bar_m), 1);
     abort_s = 0;
@@ -891,6 +984,18 @@ __global__ void __launch_bounds__(128)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // TMEM is held: let the next kernel launch; then wait for the previous one's outputs
+  pdl_trigger();
+  pdl_wait();
+  if (tid == 0) {
+    int acc = 0;
+    for (int i = 0; i < p.n_seqs; ++i) {
+      cu_chunks[i] = acc;
+      acc += (p.cu_seqlens[i + 1] - p.cu_seqlens[i] + C - 1) / C;
+    }
+    cu_chunks[p.n_seqs] = acc;
+  }
+  __syncthreads();
   const uint32_t tmem = tmem_s;
   const AbortFlag ab{&abort_s, p.err_word, ERRBIT_SCAN_TIMEOUT};
   int lo = 0, hi = p.n_seqs - 1;
@@ -1006,6 +1111,11 @@ cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string
       !make_tmap_bf16_2d(&tA, ws.A, 128, slots * 128, 256, 64, 128, err) ||
       !make_tmap_bf16_2d(&tR, ws.R, 128, slots * 64, 256, 64, 64, err))
     return cudaErrorInvalidValue;
+  CUtensorMap tB, tM, tO;
+  if (!make_tmap_f32_2d(&tB, ws.B, (uint64_t)p.dv, slots * 128, (uint64_t)p.dv * 4, 32, 128, err) ||
+      !make_tmap_bf16_2d(&tM, ws.M, (uint64_t)p.dv, slots * 128, (uint64_t)p.dv * 2, 64, 128, err) ||
+      !make_tmap_f32_2d(&tO, ws.O, (uint64_t)p.dv, slots * 64, (uint64_t)p.dv * 4, 32, 64, err))
+    return cudaErrorInvalidValue;
   cudaError_t e;
   if (items > 0) {
     int64_t grid = device_sm_count();
@@ -1014,53 +1124,44 @@ cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string
       e = cudaFuncSetAttribute(scan_prep_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)PREP_SMEM);
       if (e != cudaSuccess) return e;
-      scan_prep_kernel<128><<<(unsigned)grid, kPrepThreads, PREP_SMEM, s>>>(tq, tk, tv, p, ws,
-                                                                             total_chunks);
+      e = launch_kernel(scan_prep_kernel<128>, dim3((unsigned)grid), dim3(kPrepThreads), PREP_SMEM,
+                        s, p.pdl, tq, tk, tv, tA, tB, tR, tO, p, ws, total_chunks);
     } else {
       e = cudaFuncSetAttribute(scan_prep_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)PREP_SMEM);
       if (e != cudaSuccess) return e;
-      scan_prep_kernel<64><<<(unsigned)grid, kPrepThreads, PREP_SMEM, s>>>(tq, tk, tv, p, ws,
-                                                                           total_chunks);
+      e = launch_kernel(scan_prep_kernel<64>, dim3((unsigned)grid), dim3(kPrepThreads), PREP_SMEM,
+                        s, p.pdl, tq, tk, tv, tA, tB, tR, tO, p, ws, total_chunks);
     }
-    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   if (between) {
     e = between();
     if (e != cudaSuccess) return e;
   }
-  CUtensorMap tB, tM;
-  if (!make_tmap_f32_2d(&tB, ws.B, (uint64_t)p.dv, slots * 128, (uint64_t)p.dv * 4, 32, 128, err) ||
-      !make_tmap_bf16_2d(&tM, ws.M, (uint64_t)p.dv, slots * 128, (uint64_t)p.dv * 2, 64, 128, err))
-    return cudaErrorInvalidValue;
   e = cudaFuncSetAttribute(scan_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)CHAIN_SMEM);
   if (e != cudaSuccess) return e;
-  scan_chain_kernel<<<dim3((unsigned)(p.n_seqs * p.H), (unsigned)(p.dv / DVS)), kChainThreads,
-                      CHAIN_SMEM, s>>>(
-      tA, tB, tM, p, ws);
-  e = cudaGetLastError();
+  e = launch_kernel(scan_chain_kernel, dim3((unsigned)(p.n_seqs * p.H), (unsigned)(p.dv / DVS)),
+                    dim3(kChainThreads), CHAIN_SMEM, s, p.pdl, tA, tB, tM, p, ws);
   if (e != cudaSuccess || !p.o || items == 0) return e;
   if (between) {
     e = between();
     if (e != cudaSuccess) return e;
   }
-  CUtensorMap tO;
-  if (!make_tmap_f32_2d(&tO, ws.O, (uint64_t)p.dv, slots * 64, (uint64_t)p.dv * 4, 32, 64, err))
-    return cudaErrorInvalidValue;
   if (p.dv == 128) {
     e = cudaFuncSetAttribute(scan_out_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)OUT_SMEM);
     if (e != cudaSuccess) return e;
-    scan_out_kernel<128><<<(unsigned)items, 128, OUT_SMEM, s>>>(tR, tM, tO, p, ws, total_chunks);
+    return launch_kernel(scan_out_kernel<128>, dim3((unsigned)items), dim3(128), OUT_SMEM, s, p.pdl,
+                         tR, tM, tO, p, ws, total_chunks);
   } else {
     e = cudaFuncSetAttribute(scan_out_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)OUT_SMEM);
     if (e != cudaSuccess) return e;
-    scan_out_kernel<64><<<(unsigned)items, 128, OUT_SMEM, s>>>(tR, tM, tO, p, ws, total_chunks);
+    return launch_kernel(scan_out_kernel<64>, dim3((unsigned)items), dim3(128), OUT_SMEM, s, p.pdl,
+                         tR, tM, tO, p, ws, total_chunks);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace tr

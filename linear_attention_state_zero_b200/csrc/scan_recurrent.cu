@@ -16,6 +16,7 @@
 
 #include "../../include/tr.h"
 #include "tr_internal.h"
+#include "tr_ptx.cuh"
 
 namespace tr {
 namespace {
@@ -47,6 +48,8 @@ __global__ void __launch_bounds__(128) scan_recurrent_kernel(ScanLaunch p) {
   __shared__ float vs[TT][32];
   __shared__ float las[TT], bes[TT];
 
+  pdl_trigger();
+  pdl_wait();
   const int sh = blockIdx.x;
   const int seq = sh / p.H, head = sh % p.H;
   const int col0 = blockIdx.y * 32;
@@ -148,13 +151,11 @@ cudaError_t launch_scan_recurrent(const ScanLaunch &p, cudaStream_t s) {
   dim3 grid((unsigned)(p.n_seqs * p.H), (unsigned)(p.dv / 32));
   const bool bf = p.dtype == TR_DTYPE_BF16;
   if (p.dk == 128) {
-    if (bf) scan_recurrent_kernel<128, __nv_bfloat16><<<grid, 128, 0, s>>>(p);
-    else scan_recurrent_kernel<128, float><<<grid, 128, 0, s>>>(p);
-  } else {
-    if (bf) scan_recurrent_kernel<64, __nv_bfloat16><<<grid, 128, 0, s>>>(p);
-    else scan_recurrent_kernel<64, float><<<grid, 128, 0, s>>>(p);
+    return bf ? launch_kernel(scan_recurrent_kernel<128, __nv_bfloat16>, grid, dim3(128), 0, s, p.pdl, p)
+              : launch_kernel(scan_recurrent_kernel<128, float>, grid, dim3(128), 0, s, p.pdl, p);
   }
-  return cudaGetLastError();
+  return bf ? launch_kernel(scan_recurrent_kernel<64, __nv_bfloat16>, grid, dim3(128), 0, s, p.pdl, p)
+            : launch_kernel(scan_recurrent_kernel<64, float>, grid, dim3(128), 0, s, p.pdl, p);
 }
 
 }  // namespace tr

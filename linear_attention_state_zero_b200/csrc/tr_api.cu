@@ -245,6 +245,7 @@ tr_status validate_scan(const tr_scan_args *a, tr::ScanLaunch *out) {
   p.err_word = nullptr;
   p.ws = nullptr;
   p.ws_bytes = 0;
+  p.pdl = true;
   return TR_OK;
 }
 
@@ -368,6 +369,9 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
                                cudaStream_t s, Marks *mk = nullptr) {
   Marks none;
   if (!mk) mk = &none;
+  // programmatic dependent launch between the kernels, except when events are recorded
+  // between them (the per-kernel timing path)
+  const bool pdl = mk->ev == nullptr;
   if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
   const GroupLayout L = group_layout(a);
   uint8_t *base = static_cast<uint8_t *>(ws);
@@ -390,7 +394,7 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
     const bool skip = last && (a->flags & TR_SKIP_LAST_OUTPUT);
     const void *x_in = l == 0 ? a->h_tail : static_cast<const void *>(x);
     const int in_bf16 = l == 0 ? 1 : 0;
-    e = tr::launch_rmsnorm(x_in, in_bf16, w.rms_gain, T, D, rms_eps, xhat, s);
+    e = tr::launch_rmsnorm(x_in, in_bf16, w.rms_gain, T, D, rms_eps, xhat, s, pdl);
     if (e != cudaSuccess) return cuda_fail(e, "rmsnorm");
     if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
     tr::InProjEpi ep;
@@ -404,7 +408,7 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
     ep.col_offset = skip ? H * dk : 0;
     ep.norm_eps = norm_eps;
     const void *Wb = static_cast<const __nv_bfloat16 *>(w.W_in) + (size_t)ep.col_offset * D;
-    e = tr::launch_gemm_inproj(xhat, Wb, T, n_in - ep.col_offset, D, ep, err_word, s, &err);
+    e = tr::launch_gemm_inproj(xhat, Wb, T, n_in - ep.col_offset, D, ep, err_word, s, pdl, &err);
     if (e != cudaSuccess)
       return err.empty() ? cuda_fail(e, "input projection") : fail(TR_ERR_CUDA, "%s", err.c_str());
     if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
@@ -424,6 +428,7 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
     sp.o = skip ? nullptr : obuf;
     sp.S_final = a->S_hat + (size_t)l * state_elems;
     sp.err_word = err_word;
+    sp.pdl = pdl;
     tr_status st = run_scan(sp, s, [&]() { return mk->mark(s); });
     if (st != TR_OK) return st;
     if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
@@ -436,7 +441,7 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
         rp.x_out = out;
         rp.ld = D;
         e = tr::launch_gemm_resid(obuf, (int64_t)H * dv, w.W_o, T, D, H * dv, rp, err_word, s,
-                                  &err);
+                                  pdl, &err);
         if (e != cudaSuccess)
           return err.empty() ? cuda_fail(e, "output projection")
                              : fail(TR_ERR_CUDA, "%s", err.c_str());
@@ -581,7 +586,8 @@ tr_status tr_replay_groups(const tr_group_args *groups, int32_t n_groups, void *
 }
 
 size_t tr_state_error_workspace_size(int64_t n_mats) {
-  return n_mats > 0 ? align256((size_t)n_mats * 2 * sizeof(double)) : 0;
+  // 2 doubles per matrix piece, up to 16 pieces per matrix
+  return n_mats > 0 ? align256((size_t)n_mats * 16 * 2 * sizeof(double)) : 0;
 }
 
 tr_status tr_state_error(const float *S, const float *S_hat, int64_t n_mats, int32_t d_k,
@@ -598,9 +604,11 @@ tr_status tr_state_error(const float *S, const float *S_hat, int64_t n_mats, int
   unsigned *errw;
   std::string err;
   if (!device_state(&dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
-  cudaError_t e = tr::launch_state_error(S, S_hat, n_mats, (int64_t)d_k * d_v,
+  const int64_t elems = (int64_t)d_k * d_v;
+  const int splits = tr::state_error_splits(n_mats, elems, (int64_t)(ws_bytes / (2 * sizeof(double))));
+  cudaError_t e = tr::launch_state_error(S, S_hat, n_mats, elems, splits,
                                          static_cast<double *>(ws), err_per_mat, err_total,
-                                         static_cast<cudaStream_t>(stream));
+                                         static_cast<cudaStream_t>(stream), true);
   if (e != cudaSuccess) return cuda_fail(e, "state error");
   return ok();
 }
@@ -614,7 +622,7 @@ tr_status tr_rmsnorm(const void *x, int32_t x_dtype, const float *gain, int64_t 
     return fail(TR_ERR_ALIGNMENT, "x/x_hat/gain must be 16-byte aligned");
   cudaError_t e = tr::launch_rmsnorm(x, x_dtype == TR_DTYPE_BF16, gain, n_rows, d_model,
                                      eps > 0.f ? eps : 1e-6f, x_hat,
-                                     static_cast<cudaStream_t>(stream));
+                                     static_cast<cudaStream_t>(stream), true);
   if (e != cudaSuccess) return cuda_fail(e, "rmsnorm");
   return ok();
 }
@@ -650,7 +658,7 @@ tr_status tr_in_projection(const void *x_hat, const void *W_in, int64_t n_tokens
   ep.norm_eps = norm_eps > 0.f ? norm_eps : 1e-6f;
   const void *Wb = static_cast<const __nv_bfloat16 *>(W_in) + (size_t)ep.col_offset * d_model;
   cudaError_t e = tr::launch_gemm_inproj(x_hat, Wb, (int)n_tokens, n_in - ep.col_offset, d_model,
-                                         ep, errw, static_cast<cudaStream_t>(stream), &err);
+                                         ep, errw, static_cast<cudaStream_t>(stream), true, &err);
   if (e != cudaSuccess)
     return err.empty() ? cuda_fail(e, "input projection") : fail(TR_ERR_CUDA, "%s", err.c_str());
   return ok();
@@ -679,7 +687,7 @@ tr_status tr_out_projection(const void *o, int64_t o_stride, const void *W_o, co
   rp.x_out = x_out;
   rp.ld = d_model;
   cudaError_t e = tr::launch_gemm_resid(o, ld, W_o, (int)n_tokens, d_model, hv, rp, errw,
-                                        static_cast<cudaStream_t>(stream), &err);
+                                        static_cast<cudaStream_t>(stream), true, &err);
   if (e != cudaSuccess)
     return err.empty() ? cuda_fail(e, "output projection") : fail(TR_ERR_CUDA, "%s", err.c_str());
   return ok();

@@ -55,9 +55,29 @@ struct ScanLaunch {
   unsigned *err_word;
   void *ws;            // scan workspace (chunked kernels), ws_bytes long
   size_t ws_bytes;
+  bool pdl;            // launch with programmatic dependent launch
 };
 
 int device_sm_count();
+
+// Launch `kern` on `s`; with `pdl` the launch carries programmatic stream serialization
+// (the kernel may start before its predecessor in the stream completes and must call
+// pdl_wait() before touching global data).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t s, bool pdl, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
 
 // Set the thread-local message tr_last_error() returns (cleared for TR_OK) and
 // return `status`; printf-style.
@@ -72,14 +92,14 @@ bool make_tmap_bf16_2d(CUtensorMap *tm, const void *base, uint64_t inner, uint64
 // C[M, N] = A[M, K] * B[N, K]^T with the input-projection epilogue.
 cudaError_t launch_gemm_inproj(const void *A, const void *B, int M, int N, int K,
                                const InProjEpi &ep, unsigned *err_word, cudaStream_t s,
-                               std::string *err);
+                               bool pdl, std::string *err);
 // C[M, N] = A[M, K] * B[N, K]^T with the residual epilogue; A rows lda elements apart.
 cudaError_t launch_gemm_resid(const void *A, int64_t lda, const void *B, int M, int N, int K,
-                              const ResidEpi &ep, unsigned *err_word, cudaStream_t s,
+                              const ResidEpi &ep, unsigned *err_word, cudaStream_t s, bool pdl,
                               std::string *err);
 
 cudaError_t launch_rmsnorm(const void *x, int x_is_bf16, const float *gain, int64_t rows, int D,
-                           float eps, void *out, cudaStream_t s);
+                           float eps, void *out, cudaStream_t s, bool pdl);
 
 // 2D fp32 tensor map, 128-byte swizzle (box_inner * 4 must be <= 128).
 bool make_tmap_f32_2d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t outer,
@@ -95,8 +115,11 @@ bool scan_chunked_supported(const ScanLaunch &p);
 size_t scan_chunked_workspace(const ScanLaunch &p);  // needs p.cu_seqlens_host, H, dv
 int scan_chunked_kernels(bool with_readout);
 
+// Pieces per matrix of the state error's first pass (partials holds 2 doubles per piece;
+// at most max_pieces pieces in all).
+int state_error_splits(int64_t n_mats, int64_t mat_elems, int64_t max_pieces);
 cudaError_t launch_state_error(const float *S, const float *Sh, int64_t n_mats, int64_t mat_elems,
-                               double *partials, double *err_per, double *err_total,
-                               cudaStream_t s);
+                               int splits, double *partials, double *err_per, double *err_total,
+                               cudaStream_t s, bool pdl);
 
 }  // namespace tr

@@ -16,6 +16,16 @@ namespace tr {
 // Every legitimate wait in these kernels completes in microseconds.
 constexpr unsigned long long WAIT_LIMIT_NS = 4000000000ull;
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel of the stream still runs; it must
+// execute pdl_wait() (wait for that kernel's completion and its memory) before it reads
+// or writes any global data the previous kernels touch.  pdl_trigger() lets the next
+// kernel of the stream start launching; every kernel here calls it only after it holds
+// all of its TMEM, so a waiting dependent never takes TMEM its primary still needs.
+// Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

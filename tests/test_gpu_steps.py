@@ -13,7 +13,7 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("in_dtype", [torch.bfloat16, torch.float32])
-@pytest.mark.parametrize("T,D", [(300, 512), (1, 64), (1639, 2048)])
+@pytest.mark.parametrize("T,D", [(300, 512), (1, 64), (1639, 2048), (37, 1024), (130, 4096), (5, 2056)])
 def test_rmsnorm(cuda_device, in_dtype, T, D):
     x = synth.normal((T, D), 101, 1).to(in_dtype)
     g = 1.0 + synth.normal((D,), 101, 2, 0.1)
