@@ -443,6 +443,7 @@ def our_arm(args):
     # per-kernel breakdown (launch order: per layer rmsnorm, in-proj, scan[, out-proj])
     # launch order per layer: rmsnorm, in_proj, scan kernels, out_proj (not after the last
     # layer, whose readout and output projection are skipped)
+    # the chunked scan is prep + chain + readout (the last layer has no readout)
     chunked = n_k == L * 4 + (L - 1) * 2
     names = []
     for l in range(L):

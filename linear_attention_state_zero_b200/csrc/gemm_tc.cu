@@ -32,11 +32,12 @@ enum { EPI_INPROJ = 0, EPI_RESID = 1 };
 
 template <int BN>
 struct Cfg {
-  static constexpr int STAGES = (BN == 256) ? 4 : 6;
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t B_BYTES = BN * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr uint32_t TMEM_COLS = 2 * BN;
+  // as many stages as fit next to the control block (at most 6)
+  static constexpr int STAGES = (200 * 1024 / STAGE_BYTES) < 6 ? (200 * 1024 / STAGE_BYTES) : 6;
+  static constexpr uint32_t TMEM_COLS = BN <= 128 ? 2 * BN : 512;  // double buffer, power of 2
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
 };
 
@@ -355,9 +356,9 @@ cudaError_t launch_gemm_resid(const void *A, int64_t lda, const void *B, int M, 
                               const ResidEpi &ep, unsigned *err_word, cudaStream_t s, bool pdl,
                               std::string *err) {
   InProjEpi none{};
-  // 128-column tiles: the output is narrow (d_model), so twice the tiles spread over
-  // the SMs and a CTA with two tiles hides one tile's epilogue behind the other's MMAs
-  return launch<128, EPI_RESID>(A, lda, B, M, N, K, none, ep, err_word, s, pdl, err);
+  // 192-column tiles: the output is narrow (d_model), so 128 x 256 tiles would leave SMs
+  // idle and N = 128 MMAs are issue-bound; d_model 2048 gives 11 x 13 = 143 tiles, one wave
+  return launch<192, EPI_RESID>(A, lda, B, M, N, K, none, ep, err_word, s, pdl, err);
 }
 
 }  // namespace tr

@@ -241,13 +241,15 @@ __device__ __forceinline__ uint32_t o0_box_offset(int b) {
   return b < 2 ? (uint32_t)b * 16384u : 32768u + (uint32_t)(b - 2) * 8192u;
 }
 
+// The prep work of one CTA: items first, then second, second + stride, ... (256 threads;
+// every barrier is the named barrier 1 over those threads).
 template <int DV>
-__global__ void __launch_bounds__(kPrepThreads, 1)
-    scan_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_A,
-                     const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_R,
-                     const __grid_constant__ CUtensorMap tm_O, ScanLaunch p, ScanWs ws,
-                     int total_chunks) {
+__device__ __forceinline__ void prep_body(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                                          const CUtensorMap &tm_v, const CUtensorMap &tm_A,
+                                          const CUtensorMap &tm_B, const CUtensorMap &tm_R,
+                                          const CUtensorMap &tm_O, const ScanLaunch &p,
+                                          const ScanWs &ws, int total_chunks, int64_t first,
+                                          int64_t second, int64_t stride) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ PrepCtl ctl_s;
   PrepCtl *ctl = &ctl_s;
@@ -290,7 +292,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
                        16 * (i & 511), 0, 0, 0, 0);
     }
   tc_fence_before();
-  __syncthreads();
+  bar_sync_n(1, kPrepThreads);
   tc_fence_after();
   const uint32_t tmem = ctl->tmem;
   const AbortFlag ab{&ctl->abort, p.err_word, ERRBIT_SCAN_TIMEOUT};
@@ -307,7 +309,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     ctl->cu_chunks[p.n_seqs] = acc;
   }
   for (int i = tid; i <= p.n_seqs; i += kPrepThreads) ctl->cu_tok[i] = p.cu_seqlens[i];
-  __syncthreads();
+  bar_sync_n(1, kPrepThreads);
 
   // (sequence, chunk) of an item
   auto locate = [&](int64_t item, int &seq, int &cc) {
@@ -340,8 +342,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   };
   if (tid == 0) {
     fence_proxy_async_smem();
-    if ((int64_t)blockIdx.x < n_items) issue(blockIdx.x, 0);
-    if ((int64_t)blockIdx.x + gridDim.x < n_items) issue(blockIdx.x + gridDim.x, 1);
+    if (first < n_items) issue(first, 0);
+    if (second < n_items) issue(second, 1);
   }
   // log alpha and beta of an item's 64 tokens (thread tid < C: token tid; 0 past the end)
   auto load_gates = [&](int64_t it, float &la, float &b) {
@@ -358,19 +360,20 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   };
   // the next item's gates are loaded during the current item
   float la_next = 0.f, b_next = 0.f;
-  if (tid < C && (int64_t)blockIdx.x < n_items) load_gates(blockIdx.x, la_next, b_next);
+  if (tid < C && first < n_items) load_gates(first, la_next, b_next);
+  auto next_item = [&](int64_t it) -> int64_t { return it == first ? second : it + stride; };
   const uint32_t mma_bar = smem_u32(&ctl->mma_bar);
   uint32_t mma_phase = 0;
   auto mma_wait = [&]() -> bool {
     const bool ok = mbar_wait(mma_bar, mma_phase, ab);
     mma_phase ^= 1u;
-    if (__syncthreads_or(!ok)) return false;
+    if (bar_or_n(1, kPrepThreads, !ok)) return false;
     tc_fence_after();
     return true;
   };
 
   int n = 0;
-  for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x, ++n) {
+  for (int64_t item = first; item < n_items; item = next_item(item), ++n) {
     const int buf = n & 1;
     uint8_t *KQ = sm + P_IN + buf * P_IN_BYTES;
     const uint32_t kq_u = smem_u32(KQ);
@@ -379,7 +382,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     // gates: g = inclusive cumsum of log alpha (0 past the end), beta, beta * gamma
     if (tid < C) {
       const float la = la_next, b = b_next;
-      if (item + (int64_t)gridDim.x < n_items) load_gates(item + gridDim.x, la_next, b_next);
+      if (next_item(item) < n_items) load_gates(next_item(item), la_next, b_next);
       float s = la;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -389,16 +392,16 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       ctl->g[tid] = s;
       ctl->beta[tid] = b;
     }
-    __syncthreads();
+    bar_sync_n(1, kPrepThreads);
     if (tid >= 32 && tid < C) ctl->g[tid] += ctl->g[31];
-    __syncthreads();
+    bar_sync_n(1, kPrepThreads);
     if (tid < C) ctl->bg[tid] = ctl->beta[tid] * exp_ftz(ctl->g[tid]);
     const bool ok_tma = mbar_wait(smem_u32(&ctl->tma_bar[buf]), (uint32_t)(n >> 1) & 1u, ab);
-    if (__syncthreads_or(!ok_tma)) break;
+    if (bar_or_n(1, kPrepThreads, !ok_tma)) break;
     if (p.flags & TR_NORMALIZE_QK) {
       if (tid < C || (tid < 2 * C && want_o)) normalize_row(KQ, tid);
       fence_proxy_async_smem();
-      __syncthreads();
+      bar_sync_n(1, kPrepThreads);
     }
 
     // P1: [K; Q] K^T -> TMEM cols [0, 64)
@@ -443,8 +446,16 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         store_row_bf16(sm + P_AP, row, 32 * hsel, v, 1.f);
       }
     }
-    if (tid == 0) bulk_wait_read<0>();  // the staging of A_c, B_c boxes 0, 1 is free
-    __syncthreads();
+    if (tid == 0) {
+      bulk_wait_read<0>();  // the staging of A_c, B_c boxes 0, 1 is free
+      // the previous item's input buffer (its K/Q/V, then its O0 staging) is free now:
+      // prefetch the next item into it (items 0 and 1 were loaded before the loop)
+      if (n >= 1 && next_item(item) < n_items) {
+        fence_proxy_async_smem();
+        issue(next_item(item), buf ^ 1);
+      }
+    }
+    bar_sync_n(1, kPrepThreads);
 
     // T = (I + A)^{-1}, blocked: T11 = (I + A11)^{-1}, T22 = (I + A22)^{-1} by forward
     // substitution (thread = column, fp32 registers), then T21 = -T22 (A21 T11).
@@ -454,23 +465,27 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       float Tc[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float *Ar = As + (base + i) * LDA + base;
+        // row i of A (16-byte aligned: 68-float rows, 32-float block offset), 4 at a time;
+        // entries at columns >= i are zeros of the strictly lower A and are skipped
+        const float4 *Ar4 = reinterpret_cast<const float4 *>(As + (base + i) * LDA + base);
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-        for (int s = 0; s + 3 < i; s += 4) {
-          a0 = fmaf(Ar[s], Tc[s], a0);
-          a1 = fmaf(Ar[s + 1], Tc[s + 1], a1);
-          a2 = fmaf(Ar[s + 2], Tc[s + 2], a2);
-          a3 = fmaf(Ar[s + 3], Tc[s + 3], a3);
+        for (int s4 = 0; s4 < 8; ++s4) {
+          const int s = 4 * s4;
+          if (s < i) {
+            const float4 a = Ar4[s4];
+            a0 = fmaf(a.x, Tc[s], a0);
+            if (s + 1 < i) a1 = fmaf(a.y, Tc[s + 1], a1);
+            if (s + 2 < i) a2 = fmaf(a.z, Tc[s + 2], a2);
+            if (s + 3 < i) a3 = fmaf(a.w, Tc[s + 3], a3);
+          }
         }
-#pragma unroll
-        for (int s = i & ~3; s < i; ++s) a0 = fmaf(Ar[s], Tc[s], a0);
         Tc[i] = (i == c) ? 1.f : ((i < c) ? 0.f : -((a0 + a1) + (a2 + a3)));
       }
 #pragma unroll
       for (int i = 0; i < 32; ++i) Ts[(base + i) * LDA + base + c] = Tc[i];
     }
-    __syncthreads();
+    bar_sync_n(1, kPrepThreads);
     {  // X = A21 T11 (32 x 32): thread -> row r, columns c0..c0+3
       const int r = tid >> 3, c0 = (tid & 7) * 4;
       float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
@@ -488,7 +503,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       }
       *reinterpret_cast<float4 *>(Xs + r * LDX + c0) = make_float4(x0, x1, x2, x3);
     }
-    __syncthreads();
+    bar_sync_n(1, kPrepThreads);
     {  // T21 = -T22 X
       const int r = tid >> 3, c0 = (tid & 7) * 4;
       float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
@@ -506,7 +521,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       }
       *reinterpret_cast<float4 *>(Ts + (32 + r) * LDA + c0) = make_float4(-x0, -x1, -x2, -x3);
     }
-    __syncthreads();
+    bar_sync_n(1, kPrepThreads);
     {  // [-T diag(beta); T diag(beta gamma)] as high + low bf16 parts; consecutive lanes
        // take consecutive rows (conflict-free reads of T and swizzled stores)
       const int rr = tid & 127, half = tid >> 7, t = rr & 63;
@@ -526,7 +541,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       store_row_split(sm + P_TSH, sm + P_TSL, rr, 32 * half, v, 1.f);
     }
     fence_proxy_async_smem();
-    __syncthreads();
+    bar_sync_n(1, kPrepThreads);
 
     // P2: [-T''; T'] V -> cols [64, 64+DV) (lanes 0-63: -U~); [-T''; T'] K -> [192, 320) (lanes 64-127: W)
     if (tid == 0) {
@@ -576,7 +591,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    bar_sync_n(1, kPrepThreads);
 
     // batch: P W -> [0,128), P U~ -> [128,128+DV), A_c -> [256,384), B_c -> [384,384+DV)
     if (tid == 0) {
@@ -655,7 +670,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       fence_proxy_async_smem();
     }
     tc_fence_before();
-    __syncthreads();
+    bar_sync_n(1, kPrepThreads);
     if (tid == 0) {
       const int64_t slot = item;
       // three bulk groups, in the order the staging tiles are needed again:
@@ -685,22 +700,27 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         tma_store_2d(&tm_B, smem_u32(sm + P_TSH + 16384 * b), 32 * b, (int32_t)(slot * 128));
       bulk_commit();
       ws.G[slot] = exp_ftz(gC);
-      // this buffer's K/Q/V are no longer read: prefetch the item after next into it
-      if (item + 2 * (int64_t)gridDim.x < n_items) {
-        bulk_wait_read<2>();
-        fence_proxy_async_smem();
-        issue(item + 2 * (int64_t)gridDim.x, buf);
-      }
     }
   }
 
   if (tid == 0) bulk_wait<0>();
   tc_fence_before();
-  __syncthreads();
+  bar_sync_n(1, kPrepThreads);
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+template <int DV>
+__global__ void __launch_bounds__(kPrepThreads, 1)
+    scan_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_A,
+                     const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_R,
+                     const __grid_constant__ CUtensorMap tm_O, const __grid_constant__ ScanLaunch p,
+                     const __grid_constant__ ScanWs ws, int total_chunks) {
+  prep_body<DV>(tm_q, tm_k, tm_v, tm_A, tm_B, tm_R, tm_O, p, ws, total_chunks, blockIdx.x,
+                (int64_t)blockIdx.x + gridDim.x, gridDim.x);
 }
 
 // =========================================================== chain kernel
@@ -719,17 +739,17 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
 constexpr int kStages = 2;
 constexpr uint32_t H_STAGE = 65536;             // A_c [half][128 rows][128 B] + B_c [box][128][32 fp32]
 constexpr uint32_t H_MB = kStages * H_STAGE;    // 2 x bf16 state slice [128 d][128 B]
-constexpr int kMaxChunksPerSeq = 4096;
-constexpr size_t CHAIN_SMEM = H_MB + 2 * 16384 + 1024;
 
 struct ChainCtl {
+  alignas(16) float g4[kStages][4];  // the 16-byte aligned group of G holding the stage's gamma_C
   uint64_t tma_bar[kStages];
   uint64_t empty_bar[kStages];  // stage consumed (arrived by thread 0 after the barrier)
   uint64_t bar_z;
   uint32_t tmem;
   int abort;
-  float gC[kMaxChunksPerSeq];
 };
+constexpr uint32_t H_CTL = H_MB + 2 * 16384;    // the control block, in dynamic shared memory
+constexpr size_t CHAIN_SMEM = H_CTL + sizeof(ChainCtl) + 1024;
 
 __device__ __forceinline__ void load_row32_f32(const uint8_t *tile, int row, float *f) {
   // one row (32 floats = 128 B) of a 128-byte-swizzled fp32 tile
@@ -748,22 +768,23 @@ static_assert(kCols == 32, "state columns per thread");
 
 
 
-__global__ void __launch_bounds__(kChainThreads, 1)
-    scan_chain_kernel(const __grid_constant__ CUtensorMap tm_A, const __grid_constant__ CUtensorMap tm_B,
-                      const __grid_constant__ CUtensorMap tm_M, ScanLaunch p, ScanWs ws) {
+// The chain of one (sequence * H + head, slice) task (kChainThreads threads).  The
+// loads of chunk c (A_c, the B_c slice and gamma_C, into stage c % kStages) are issued
+// by the producer warp.
+__device__ __forceinline__ void chain_body(const CUtensorMap &tm_A, const CUtensorMap &tm_B,
+                                           const CUtensorMap &tm_M, const ScanLaunch &p,
+                                           const ScanWs &ws, int seqhead, int slice) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ ChainCtl ctl_s;
   __shared__ int red[32];  // one entry per warp (chunk_base)
-  ChainCtl *ctl = &ctl_s;
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
+  ChainCtl *ctl = reinterpret_cast<ChainCtl *>(sm + H_CTL);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, cg = warp >> 2;
   const int d = q4 * 32 + lane;
   const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
   const int H = p.H, DV = p.dv;
-  const int seq = blockIdx.x / H, head = blockIdx.x % H;
-  const int slice = blockIdx.y;
+  const int seq = seqhead / H, head = seqhead % H;
   const int col = slice * DVS + kCols * cg;   // this thread's first d_v column
 
   if (tid == 0) {
@@ -792,7 +813,6 @@ __global__ void __launch_bounds__(kChainThreads, 1)
   const int nch = (t_end - t_begin + C - 1) / C;
   const int cb = chunk_base(p.cu_seqlens, seq, red);
   auto slot_of = [&](int c) -> int64_t { return ((int64_t)cb + c) * H + head; };
-  for (int c = tid; c < nch; c += kChainThreads) ctl->gC[c] = ws.G[slot_of(c)];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -826,12 +846,15 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     const int64_t slot = slot_of(c);
     const uint32_t bar = smem_u32(&ctl->tma_bar[st]);
     const uint32_t a_u = smem_u32(sm + st * H_STAGE);
-    mbar_arrive_expect_tx(bar, 65536u);
+    mbar_arrive_expect_tx(bar, 65536u + 16u);
     tma_load_2d(a_u, &tm_A, 0, (int32_t)(slot * 128), bar);
     tma_load_2d(a_u + 16384, &tm_A, 64, (int32_t)(slot * 128), bar);
     tma_load_2d(a_u + 32768, &tm_B, slice * DVS, (int32_t)(slot * 128), bar);
     tma_load_2d(a_u + 49152, &tm_B, slice * DVS + 32, (int32_t)(slot * 128), bar);
+    // gamma_C: the 16-byte group of G that holds it (G is padded to 256 bytes)
+    bulk_load(smem_u32(&ctl->g4[st][0]), ws.G + (slot & ~(int64_t)3), 16u, bar);
   };
+
   auto issue_mma = [&](int c) -> bool {
     const int st = c % kStages;
     if (!mbar_wait(smem_u32(&ctl->tma_bar[st]), (uint32_t)(c / kStages) & 1u, ab)) return false;
@@ -846,20 +869,17 @@ __global__ void __launch_bounds__(kChainThreads, 1)
   };
 
   bool failed = false;
-  if (tid == 0) {
-    fence_proxy_async_smem();
-    for (int c = 0; c < kStages && c < nch; ++c) issue_tma(c);
-  }
   fence_proxy_async_smem();
   __syncthreads();
   if (tid == 0 && nch > 0) store_mc(0, 0);
 
   if (producer) {
-    // refill stage c % kStages with chunk c once chunk c - kStages has consumed it
+    // fill stage c % kStages with chunk c once chunk c - kStages has consumed it
     if (lane == 0) {
-      for (int c = kStages; c < nch; ++c) {
+      for (int c = 0; c < nch; ++c) {
         const int st = c % kStages;
-        if (!mbar_wait(smem_u32(&ctl->empty_bar[st]), (uint32_t)((c - kStages) / kStages) & 1u, ab))
+        if (c >= kStages &&
+            !mbar_wait(smem_u32(&ctl->empty_bar[st]), (uint32_t)((c - kStages) / kStages) & 1u, ab))
           break;
         issue_tma(c);
       }
@@ -894,7 +914,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
         }
       }
       if (mma_for_c) tc_wait_ld();
-      const float gC = ctl->gC[c];
+      const float gC = ctl->g4[st][slot_of(c) & 3];
       // M <- gamma_C M + A_c M + B_c (fp32); bf16 copy for the next product and the readout
 #pragma unroll
       for (int j = 0; j < kCols; ++j) Mr[j] = fmaf(gC, Mr[j], v[j] + b[j]);
@@ -940,6 +960,13 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 64);
   }
+}
+
+__global__ void __launch_bounds__(kChainThreads, 1)
+    scan_chain_kernel(const __grid_constant__ CUtensorMap tm_A, const __grid_constant__ CUtensorMap tm_B,
+                      const __grid_constant__ CUtensorMap tm_M, const __grid_constant__ ScanLaunch p,
+                      const __grid_constant__ ScanWs ws) {
+  chain_body(tm_A, tm_B, tm_M, p, ws, blockIdx.x, blockIdx.y);
 }
 
 // ========================================================= readout kernel
@@ -1069,12 +1096,8 @@ bool make_tmap_f32_2d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_
                       std::string *err);
 
 bool scan_chunked_supported(const ScanLaunch &p) {
-  if (!(p.dtype == TR_DTYPE_BF16 && p.dk == DK && (p.dv == 64 || p.dv == 128) &&
-        p.n_seqs <= kMaxSeqsChunked && (p.o == nullptr || p.o_stride % 8 == 0)))
-    return false;
-  for (int i = 0; p.cu_seqlens_host && i < p.n_seqs; ++i)
-    if ((p.cu_seqlens_host[i + 1] - p.cu_seqlens_host[i] + C - 1) / C > kMaxChunksPerSeq) return false;
-  return true;
+  return p.dtype == TR_DTYPE_BF16 && p.dk == DK && (p.dv == 64 || p.dv == 128) &&
+         p.n_seqs <= kMaxSeqsChunked && (p.o == nullptr || p.o_stride % 8 == 0);
 }
 
 size_t scan_chunked_workspace(const ScanLaunch &p) {
@@ -1083,7 +1106,10 @@ size_t scan_chunked_workspace(const ScanLaunch &p) {
   return total;
 }
 
-int scan_chunked_kernels(bool with_readout) { return with_readout ? 3 : 2; }
+int scan_chunked_kernels(const ScanLaunch &p, bool with_readout) {
+  (void)p;
+  return with_readout ? 3 : 2;
+}
 
 cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string *err,
                                 const std::function<cudaError_t()> &between) {

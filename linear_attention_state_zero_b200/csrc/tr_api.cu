@@ -259,7 +259,7 @@ size_t scan_ws_bytes(const tr::ScanLaunch &p) {
 }
 
 int scan_kernel_count(const tr::ScanLaunch &p, bool with_readout) {
-  return use_chunked(p) ? tr::scan_chunked_kernels(with_readout) : 1;
+  return use_chunked(p) ? tr::scan_chunked_kernels(p, with_readout) : 1;
 }
 
 tr_status run_scan(const tr::ScanLaunch &p, cudaStream_t s,
