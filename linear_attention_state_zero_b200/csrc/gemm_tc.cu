@@ -12,8 +12,9 @@
 //   warp 1     TMEM owner + MMA issuer: one thread issues tcgen05.mma
 //              (M=128, N=BN, K=16) into a double-buffered fp32 accumulator in
 //              TMEM and commits each stage back to the producer
-//   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter of the accumulator,
-//              fused activation/residual, stores; overlaps the next tile's MMAs
+//   warps 2-9  epilogue: two warps per 32-lane quarter of the accumulator, each taking
+//              half of the tile's columns: tcgen05.ld, fused activation/residual,
+//              stores; overlaps the next tile's MMAs
 // Every mbarrier wait is bounded (see tr_ptx.cuh); a timeout ends all roles of
 // the CTA, frees its TMEM and raises the library's error word.
 #include <cuda_bf16.h>
@@ -26,7 +27,8 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 
 enum { EPI_INPROJ = 0, EPI_RESID = 1 };
 
@@ -67,15 +69,15 @@ __device__ __forceinline__ float softplus_f(float a) {
 }
 __device__ __forceinline__ float sigmoid_f(float a) { return 1.f / (1.f + exp_ftz(-a)); }
 
-// Input-projection epilogue for one 128 x BN tile; this thread owns `row`.
+// Input-projection epilogue for tile columns [lo, hi) of one 128 x BN tile (lo, hi multiples
+// of d_k); this thread owns `row`.
 template <int BN>
 __device__ __forceinline__ void epi_inproj(const InProjEpi &ep, uint32_t tbase, int n0, int N,
-                                           int row, int M) {
+                                           int row, int M, int lo, int hi) {
   const int dk = ep.dk;
   const int nq = 2 * ep.H * dk;          // q and k features
   const int nv = nq + ep.H * ep.dv;      // end of the v features
-  const int nblk = BN / dk;
-  for (int blk = 0; blk < nblk; ++blk) {
+  for (int blk = lo / dk; blk < hi / dk; ++blk) {
     const int c0 = n0 + blk * dk;  // GEMM column
     if (c0 >= N) break;
     const int g0 = c0 + ep.col_offset;  // feature index in W_in
@@ -164,20 +166,21 @@ __device__ __forceinline__ void res32_to_f32(const ResidEpi &ep, const Res32 &r,
   }
 }
 
-// Output-projection epilogue for one 128 x BN tile; this thread owns `row`.  The
-// residual of the next 32 columns is requested before the current ones are added, so
-// one global-load latency is in flight behind every TMEM load.
+// Output-projection epilogue for tile columns [lo, hi) of one 128 x BN tile (multiples of
+// 32); this thread owns `row`.  The residual of the next 32 columns is requested before
+// the current ones are added, so one global-load latency is in flight behind every TMEM
+// load.
 template <int BN>
 __device__ __forceinline__ void epi_resid(const ResidEpi &ep, uint32_t tbase, int n0, int N,
-                                          int row, int M) {
+                                          int row, int M, int lo, int hi) {
   const bool live = row < M;
   Res32 cur, nxt;
-  if (live && n0 < N) load_res32(ep, row, n0, cur);
+  if (live && n0 + lo < N) load_res32(ep, row, n0 + lo, cur);
 #pragma unroll 1
-  for (int j = 0; j < BN / 32; ++j) {
+  for (int j = lo / 32; j < hi / 32; ++j) {
     const int c = n0 + 32 * j;
     if (c >= N) break;
-    if (live && j + 1 < BN / 32 && c + 32 < N) load_res32(ep, row, c + 32, nxt);
+    if (live && j + 1 < hi / 32 && c + 32 < N) load_res32(ep, row, c + 32, nxt);
     float v[32];
     tmem_ld32(tbase + 32 * j, v);
     tc_wait_ld();
@@ -217,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&ctl->tfull[b]), 1);
-      mbar_init(smem_u32(&ctl->tempty[b]), 4);
+      mbar_init(smem_u32(&ctl->tempty[b]), kEpiWarps);
     }
     ctl->abort = 0;
     fence_mbar_init();
@@ -295,6 +298,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     const int q4 = warp & 3;  // TMEM lanes this warp may read: 32*q4 .. 32*q4+31
+    const int half = (warp - 2) >> 2;  // which half of the tile's columns
+    static_assert(BN % 64 == 0, "half tiles of whole 32-column groups");
+    const int lo = half * (BN / 2), hi = lo + BN / 2;
     int it = 0;
     for (int t = blockIdx.x; t < n_total; t += gridDim.x, ++it) {
       const int b = it & 1;
@@ -305,9 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = tm * BM + q4 * 32 + lane;
       const uint32_t tbase = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(b * BN);
       if (EPI == EPI_INPROJ)
-        epi_inproj<BN>(ip, tbase, tn * BN, N, row, M);
+        epi_inproj<BN>(ip, tbase, tn * BN, N, row, M, lo, hi);
       else
-        epi_resid<BN>(rs, tbase, tn * BN, N, row, M);
+        epi_resid<BN>(rs, tbase, tn * BN, N, row, M, lo, hi);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&ctl->tempty[b]));

@@ -457,20 +457,21 @@ __device__ __forceinline__ void prep_body(const CUtensorMap &tm_q, const CUtenso
     }
     bar_sync_n(1, kPrepThreads);
 
-    // T = (I + A)^{-1}, blocked: T11 = (I + A11)^{-1}, T22 = (I + A22)^{-1} by forward
-    // substitution (thread = column, fp32 registers), then T21 = -T22 (A21 T11).
+    // T = (I + A)^{-1}, blocked.  (a) the four 16 x 16 diagonal blocks by forward
+    // substitution (thread = column, fp32 registers); (b) each 32 x 32 diagonal block from
+    // its two 16-blocks: T21 = -T22 (A21 T11); (c) the 64 x 64 from the two 32-blocks the
+    // same way.
     if (tid < C) {
-      const int blk = tid >> 5, c = lane;
-      const int base = 32 * blk;
-      float Tc[32];
+      const int base = 16 * (tid >> 4), c = tid & 15;
+      float Tc[16];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        // row i of A (16-byte aligned: 68-float rows, 32-float block offset), 4 at a time;
-        // entries at columns >= i are zeros of the strictly lower A and are skipped
+      for (int i = 0; i < 16; ++i) {
+        // row i of the block's A (16-byte aligned), 4 at a time; entries at columns >= i
+        // are zeros of the strictly lower A and are skipped
         const float4 *Ar4 = reinterpret_cast<const float4 *>(As + (base + i) * LDA + base);
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-        for (int s4 = 0; s4 < 8; ++s4) {
+        for (int s4 = 0; s4 < 4; ++s4) {
           const int s = 4 * s4;
           if (s < i) {
             const float4 a = Ar4[s4];
@@ -483,7 +484,48 @@ __device__ __forceinline__ void prep_body(const CUtensorMap &tm_q, const CUtenso
         Tc[i] = (i == c) ? 1.f : ((i < c) ? 0.f : -((a0 + a1) + (a2 + a3)));
       }
 #pragma unroll
-      for (int i = 0; i < 32; ++i) Ts[(base + i) * LDA + base + c] = Tc[i];
+      for (int i = 0; i < 16; ++i) Ts[(base + i) * LDA + base + c] = Tc[i];
+    }
+    bar_sync_n(1, kPrepThreads);
+    // (b) thread -> 32-block J, row r of its lower 16 x 16 block, columns c0, c0 + 1
+    const int mJ = tid >> 7, mr = (tid >> 3) & 15, mc = (tid & 7) * 2;
+    {  // X16 = A21 T11 within block J
+      const float *Ar = As + (32 * mJ + 16 + mr) * LDA + 32 * mJ;
+      float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+      for (int s = 0; s < 16; s += 4) {
+        const float4 a = *reinterpret_cast<const float4 *>(Ar + s);
+        const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 t = *reinterpret_cast<const float2 *>(Ts + (32 * mJ + s + u) * LDA + 32 * mJ + mc);
+          x0 = fmaf(av[u], t.x, x0);
+          x1 = fmaf(av[u], t.y, x1);
+        }
+      }
+      *reinterpret_cast<float2 *>(Xs + (16 * mJ + mr) * LDX + mc) = make_float2(x0, x1);
+      // the upper-right 16 x 16 of the 32-block is zero (T is lower triangular); nothing
+      // in this step reads it
+      *reinterpret_cast<float2 *>(Ts + (32 * mJ + mr) * LDA + 32 * mJ + 16 + mc) =
+          make_float2(0.f, 0.f);
+    }
+    bar_sync_n(1, kPrepThreads);
+    {  // T21 = -T22 X16 within block J (T22 lower triangular)
+      const float *Tr = Ts + (32 * mJ + 16 + mr) * LDA + 32 * mJ + 16;
+      float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+      for (int s = 0; s < 16; s += 4) {
+        const float4 a = *reinterpret_cast<const float4 *>(Tr + s);
+        const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 t = *reinterpret_cast<const float2 *>(Xs + (16 * mJ + s + u) * LDX + mc);
+          x0 = fmaf(av[u], t.x, x0);
+          x1 = fmaf(av[u], t.y, x1);
+        }
+      }
+      *reinterpret_cast<float2 *>(Ts + (32 * mJ + 16 + mr) * LDA + 32 * mJ + mc) =
+          make_float2(-x0, -x1);
     }
     bar_sync_n(1, kPrepThreads);
     {  // X = A21 T11 (32 x 32): thread -> row r, columns c0..c0+3
