@@ -104,14 +104,15 @@ int64_t tr_tail_len(int64_t m, int64_t r_num, int64_t r_den);
  *   beta      [T, H] fp32.
  *   cu_seqlens      [N+1] int32 device offsets, cu[0] = 0, cu[N] = T, nondecreasing.
  *   cu_seqlens_host the same N+1 values in host memory (validation and the
- *                   longest-first schedule); must equal the device copy.
+ *                   workspace size); must equal the device copy.
  *   S0        [N, H, d_k, d_v] fp32 or NULL (zero start).
  *   o         [T, H, d_v] of `dtype`, or NULL to skip the readout.
  *   S_final   [N, H, d_k, d_v] fp32, required.  Must not alias S0.
  *   scale     readout scale (1.0 in every workload here).
  *   flags     TR_NORMALIZE_QK, TR_SCAN_RECURRENT.
- * Supported: d_k, d_v in {64, 128}; dtype TR_DTYPE_BF16 (chunked tensor-core
- * kernel) or TR_DTYPE_F32 (token-sequential fp32 FMA kernel, the test path);
+ * Supported: d_k, d_v in {64, 128}; dtype TR_DTYPE_BF16 (the chunked tensor-core
+ * scan when d_k = 128 and N <= 1024, else the token-sequential kernel) or
+ * TR_DTYPE_F32 (token-sequential fp32 FMA kernel, the test path);
  * 16-byte aligned q/k/v/o with strides that keep every row 16-byte aligned.
  * Workspace: tr_gdn_scan_workspace_size(args) bytes.
  */
