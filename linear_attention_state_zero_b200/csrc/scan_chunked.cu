@@ -11,19 +11,20 @@
 //   chunk transition:  M_C = gamma_C M_0 + A_c M_0 + B_c
 //       A_c = -K^T diag(gamma') W   (d_k x d_k),   B_c = K^T diag(gamma') U~
 //   chunk readout:     O = R M_0 + O0,   R = diag(gamma) Q - P W,   O0 = P U~
-// Nothing but the last two lines depends on M_0, so the work splits in two
-// launches:
+// Nothing but the transition and the readout depends on M_0, so the work splits in
+// three launches:
 //
-//   scan_prep_kernel  one CTA per (chunk, head), all chunks in parallel:
+//   scan_prep_kernel   persistent over all (chunk, head) items, in parallel:
 //     P1  [K; Q] K^T -> TMEM            (tcgen05, K-major operands)
-//     A, P on CUDA cores; T = (I + A)^{-1} by forward substitution in fp32
+//     A, P on CUDA cores; T = (I + A)^{-1} by blocked forward substitution in fp32
 //     P2  [-T''; T'] [V | K] -> -U~, W  (T' = T diag(beta gamma), T'' = T diag(beta))
 //     P3  P W, P U~, K^T (gamma' W), K^T (gamma' U~) in one batch
-//     -> workspace: A_c (bf16), R (bf16), B_c (fp32), O0 (fp32), gamma_C
-//   scan_chain_kernel one CTA per (sequence, head, 64-column slice of d_v):
-//     per chunk one tcgen05 round trip:  Z = A_c M_bf16,  O = R M_bf16  (TMEM),
-//     then M <- gamma_C M + Z + B_c in fp32 registers (thread d owns row d),
-//     o = O + O0.  Operands arrive by TMA, double-buffered one chunk ahead.
+//     -> workspace, by TMA stores: A_c (bf16), R (bf16), B_c (fp32), O0 (fp32), gamma_C
+//   scan_chain_kernel  one CTA per (sequence, head, 64-column slice of d_v), sequential
+//     over the chunks: one tcgen05 product Z = A_c M_bf16 per chunk, then
+//     M <- gamma_C M + Z + B_c in fp32 registers; the bf16 chunk-start states go to the
+//     workspace.  Operands arrive by TMA, double-buffered one chunk ahead.
+//   scan_out_kernel    one CTA per (chunk, head), in parallel: o = R M_c + O0.
 //
 // Every M-dependent product acts column by column on d_v, so d_v splits into
 // exact 64-column slices.  Tokens past the end of a sequence get beta = 0 and
