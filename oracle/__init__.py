@@ -35,4 +35,5 @@ from .tail_replay import (  # noqa: F401
     state_error,
     tail_len,
     tail_rows,
+    transition_product,
 )

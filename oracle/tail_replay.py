@@ -209,6 +209,33 @@ def gdn_scan(q, k, v, log_alpha, beta, cu_seqlens, S0=None, scale: float = 1.0,
     return o, S
 
 
+def transition_product(k, log_alpha, beta, cu_seqlens):
+    """P = T_t ... T_1 over each sequence's tokens, per head, T_i = alpha_i (I - beta_i k_i k_i^T).
+
+    RN section 2.3 writes the tail's error as E_m = (T_m ... T_{a+1}) S_a; HYPIC (abstract)
+    caches this product as the segment transition operator.  In the M = S^T layout a
+    state M_0 before the sequence becomes P M_0 + M_hat after it (M_hat: the zero-start
+    state of the scan).  Returns [N, H, d_k, d_k] fp64.  Each step applies T_i to the
+    running product as the rank-one update alpha_i (P - beta_i k_i (k_i^T P)), which is
+    T_i P without forming T_i.
+    """
+    k = _f64(k)
+    la = _f64(log_alpha)
+    b = _f64(beta)
+    cu = _f64(cu_seqlens).astype(np.int64)
+    T, H, dk = k.shape
+    N = cu.shape[0] - 1
+    out = np.zeros((N, H, dk, dk), dtype=np.float64)
+    for n in range(N):
+        P = np.broadcast_to(np.eye(dk), (H, dk, dk)).copy()
+        for t in range(int(cu[n]), int(cu[n + 1])):
+            kt = k[t]                                   # [H, dk]
+            kP = np.einsum('hd,hde->he', kt, P)         # k^T P, [H, dk]
+            P = np.exp(la[t])[:, None, None] * (P - b[t][:, None, None] * kt[:, :, None] * kP[:, None, :])
+        out[n] = P
+    return out
+
+
 # ------------------------------------------------------------------------- a6
 def out_projection_residual(x, o, W_o) -> np.ndarray:
     """x + o W_o^T with o flattened to [T, H d_v] and W_o [D, H d_v].

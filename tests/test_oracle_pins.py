@@ -366,3 +366,55 @@ def test_replay_cast_points_are_small():
     S_e, _ = oracle.replay_group(h, cu, layers, 2, 16, 16, emulate_casts=False)
     _, tot = oracle.state_error(S_e, S_c)
     assert 0 < tot < 2e-2
+
+
+# ---------------------------------------------------- transition product (HYPIC operator)
+def test_transition_product_explicit_matrices():
+    """Reading notes section 2.3: the tail's operator is the product T_t ... T_1 of the
+    explicit d_k x d_k matrices T_i = alpha_i (I - beta_i k_i k_i^T); varlen sequences are
+    independent and an empty one gives the identity."""
+    q, k, v, la, b = _rand_scan(17, 2, 6, 3, seed=31)
+    cu = [0, 9, 9, 17]
+    P = oracle.transition_product(k, la, b, cu)
+    for n in range(3):
+        for h in range(2):
+            want = np.eye(6)
+            for t in range(cu[n], cu[n + 1]):
+                want = _explicit_T(math.exp(la[t, h]), b[t, h], k[t, h]) @ want
+            np.testing.assert_allclose(P[n, h], want, atol=1e-14)
+
+
+def test_transition_product_is_the_scans_linear_part():
+    """Eq. (1) is affine in the state: scan(S0) - scan(0) = P S0 (in the M = S^T layout),
+    checked against the plain C recurrence, which never forms P."""
+    q, k, v, la, b = _rand_scan(40, 3, 8, 5, seed=32)
+    S0 = rng.standard_normal((2, 3, 8, 5))
+    cu = [0, 25, 40]
+    _, S1 = oracle.gdn_scan(q, k, v, la, b, cu, S0=S0, want_o=False)
+    _, Sz = oracle.gdn_scan(q, k, v, la, b, cu, want_o=False)
+    P = oracle.transition_product(k, la, b, cu)
+    np.testing.assert_allclose(S1 - Sz, np.einsum('nhij,nhjk->nhik', P, S0), atol=1e-12)
+
+
+def test_transition_product_identity_and_bound():
+    """alpha = 1, beta = 0 gives P = I; with unit keys and beta in (0, 1) every T_i is a
+    contraction times alpha_i, so ||P||_2 <= prod alpha_i (reading notes section 2.3)."""
+    q, k, v, la, b = _rand_scan(30, 2, 8, 4, seed=33)
+    P0 = oracle.transition_product(k, np.zeros_like(la), np.zeros_like(b), [0, 30])
+    np.testing.assert_allclose(P0[0], np.broadcast_to(np.eye(8), (2, 8, 8)), atol=0)
+    P = oracle.transition_product(k, la, b, [0, 30])
+    for h in range(2):
+        assert np.linalg.norm(P[0, h], 2) <= math.exp(la[:, h].sum()) * (1 + 1e-12)
+
+
+def test_transition_product_repairs_the_tail():
+    """The repair the operator makes possible: with an exact earlier state S_a, the full
+    state is S_m = P S_a + S_hat_m exactly (reading notes section 2.3, E_m = P S_a)."""
+    m, kk = 60, 22
+    q, k, v, la, b = _rand_scan(m, 2, 8, 6, seed=34)
+    a = m - kk
+    _, S_m = oracle.gdn_scan(q, k, v, la, b, [0, m], want_o=False)
+    _, S_a = oracle.gdn_scan(q[:a], k[:a], v[:a], la[:a], b[:a], [0, a], want_o=False)
+    _, S_hat = oracle.gdn_scan(q[a:], k[a:], v[a:], la[a:], b[a:], [0, kk], want_o=False)
+    P = oracle.transition_product(k[a:], la[a:], b[a:], [0, kk])
+    np.testing.assert_allclose(S_m, np.einsum('nhij,nhjk->nhik', P, S_a) + S_hat, atol=1e-12)
