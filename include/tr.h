@@ -135,6 +135,26 @@ typedef struct tr_scan_args {
 size_t tr_gdn_scan_workspace_size(const tr_scan_args *args);
 tr_status tr_gdn_scan(const tr_scan_args *args, void *ws, size_t ws_bytes, void *stream);
 
+/* Transition product of each (sequence, head) of a packed batch
+ * (Tail-Replay reading notes, section 2.3: the error identity E_m = (T_m ... T_{a+1}) S_a;
+ * HYPIC, abstract: the segment transition operator):
+ *   P = T_t ... T_1 over the sequence's tokens,  T_i = alpha_i (I - beta_i k_i k_i^T).
+ * In the M = S^T layout a state M_0 before the sequence becomes P M_0 + M_hat after it,
+ * M_hat being the zero-start state tr_gdn_scan returns.  So an earlier exact state M_a
+ * repairs a tail replay exactly, M_m = P M_a + M_hat_m, and ||P||_2 <= prod alpha_i
+ * bounds how much of M_a the zero start loses.
+ *   args  as for tr_gdn_scan; only n_seqs, n_heads, d_k, total_tokens, dtype, flags
+ *         (TR_NORMALIZE_QK), k, k_stride, log_alpha, beta, cu_seqlens and
+ *         cu_seqlens_host are read (v, q, S0, o, S_final and d_v are ignored).
+ *   P     [N, H, d_k, d_k] fp32 output (device).
+ * Computed by the scan itself, with v = 0 from S0 = I (the chunked kernels when dtype is
+ * bf16 and d_k = 128: bf16 operands, fp32 products, like the states).
+ * Workspace: tr_transition_product_workspace_size(args) bytes, 256-byte aligned.
+ */
+size_t tr_transition_product_workspace_size(const tr_scan_args *args);
+tr_status tr_transition_product(const tr_scan_args *args, float *P, void *ws, size_t ws_bytes,
+                                void *stream);
+
 /*
  * ---------------------------------------------------------- tr_replay_group
  * Replay of one group's LA layers over the packed k-token tails (RN section

@@ -59,6 +59,8 @@ _SIGNATURES = {
     "tr_tail_len": (c_i64, [c_i64, c_i64, c_i64]),
     "tr_gdn_scan_workspace_size": (c_sz, [ctypes.POINTER(ScanArgs)]),
     "tr_gdn_scan": (ctypes.c_int, [ctypes.POINTER(ScanArgs), c_vp, c_sz, c_vp]),
+    "tr_transition_product_workspace_size": (c_sz, [ctypes.POINTER(ScanArgs)]),
+    "tr_transition_product": (ctypes.c_int, [ctypes.POINTER(ScanArgs), c_vp, c_vp, c_sz, c_vp]),
     "tr_replay_group_workspace_size": (c_sz, [ctypes.POINTER(GroupArgs)]),
     "tr_replay_group": (ctypes.c_int, [ctypes.POINTER(GroupArgs), c_vp, c_sz, c_vp]),
     "tr_replay_group_kernel_count": (c_i32, [ctypes.POINTER(GroupArgs)]),
@@ -178,6 +180,31 @@ def gdn_scan(q, k, v, log_alpha, beta, cu_seqlens, *, S0=None, want_o=True, scal
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=k.device) if ws_bytes else None
     _ok(lib.tr_gdn_scan(ctypes.byref(a), _ptr(ws), ws_bytes, _stream(stream)), "tr_gdn_scan")
     return o, S_final
+
+
+def transition_product(k, log_alpha, beta, cu_seqlens, *, normalize_qk=False, recurrent=False,
+                       P=None, stream=None):
+    """P = T_t ... T_1 per (sequence, head): [N, H, d_k, d_k] fp32 (M = S^T convention:
+    a state M_0 before the sequence becomes P M_0 + the zero-start state after it)."""
+    _need_cuda(k, log_alpha, beta)
+    T, H, dk = k.shape
+    if k.stride(2) != 1 or k.stride(1) != dk:
+        raise ValueError("k must be [T, H, d] with contiguous heads")
+    la = log_alpha.contiguous()
+    be = beta.contiguous()
+    host, dev = _seqlens(cu_seqlens, k.device)
+    N = host.numel() - 1
+    if P is None:
+        P = torch.empty((N, H, dk, dk), dtype=torch.float32, device=k.device)
+    flags = (TR_NORMALIZE_QK if normalize_qk else 0) | (TR_SCAN_RECURRENT if recurrent else 0)
+    a = ScanArgs(N, H, dk, dk, T, _dtype_code(k), flags, 1.0, 0, k.stride(0), 0,
+                 None, _ptr(k), None, _ptr(la), _ptr(be), _ptr(dev), host.data_ptr(), None, None,
+                 None)
+    ws_bytes = lib.tr_transition_product_workspace_size(ctypes.byref(a))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=k.device) if ws_bytes else None
+    _ok(lib.tr_transition_product(ctypes.byref(a), _ptr(P), _ptr(ws), ws_bytes, _stream(stream)),
+        "tr_transition_product")
+    return P
 
 
 @dataclass

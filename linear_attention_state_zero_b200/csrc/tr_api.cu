@@ -452,6 +452,54 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
   return TR_OK;
 }
 
+// ------------------------------------------------------- transition product
+// The scan on v = 0 from S0 = I: its final state is the transition product P.
+__global__ void set_identity(float *M, int64_t n_mats, int d) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n_mats * d) M[(i / d) * d * d + (i % d) * (d + 1)] = 1.f;
+}
+
+struct TpLayout {
+  size_t v0 = 0, ident = 0, scan = 0, total = 0;
+  size_t v0_bytes = 0, ident_bytes = 0;
+};
+
+// Scan arguments of the product: d_v = d_k, v from the zero buffer, S0 the identities,
+// S_final = P, no readout.
+tr_scan_args tp_scan_args(const tr_scan_args *a, float *P, void *v0, float *ident) {
+  tr_scan_args b = *a;
+  b.d_v = a->d_k;
+  b.v = v0;
+  b.v_stride = 0;
+  b.q = nullptr;
+  b.q_stride = 0;
+  b.o = nullptr;
+  b.S0 = ident;
+  b.S_final = P;
+  return b;
+}
+
+tr_status tp_layout(const tr_scan_args *a, TpLayout *L, tr::ScanLaunch *p) {
+  if (!a) return fail(TR_ERR_INVALID_ARG, "args is NULL");
+  const size_t esz = a->dtype == TR_DTYPE_BF16 ? 2 : 4;
+  const size_t T = a->total_tokens > 0 ? (size_t)a->total_tokens : 0;
+  L->v0_bytes = T * (size_t)a->n_heads * (size_t)a->d_k * esz;
+  L->ident_bytes = (size_t)(a->n_seqs > 0 ? a->n_seqs : 0) * (size_t)a->n_heads * (size_t)a->d_k *
+                   (size_t)a->d_k * sizeof(float);
+  size_t off = 0;
+  L->v0 = off;    off = align256(off + L->v0_bytes);
+  L->ident = off; off = align256(off + L->ident_bytes);
+  L->scan = off;
+  // placeholders (aligned, non-NULL) to validate the derived scan arguments and size them
+  uint8_t *fake = reinterpret_cast<uint8_t *>(static_cast<uintptr_t>(1) << 12);
+  tr_scan_args b = tp_scan_args(a, reinterpret_cast<float *>(fake), fake,
+                                reinterpret_cast<float *>(fake + 256));
+  tr_status st = validate_scan(&b, p);
+  if (st != TR_OK) return st;
+  L->total = off + scan_ws_bytes(*p);
+  return TR_OK;
+}
+
 }  // namespace
 
 // ============================================================== extern "C"
@@ -496,6 +544,53 @@ tr_status tr_gdn_scan(const tr_scan_args *args, void *ws, size_t ws_bytes, void 
   if (!device_state(&dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
   p.err_word = errw;
   st = run_scan(p, static_cast<cudaStream_t>(stream));
+  return st == TR_OK ? ok() : st;
+}
+
+size_t tr_transition_product_workspace_size(const tr_scan_args *args) {
+  TpLayout L;
+  tr::ScanLaunch p;
+  if (tp_layout(args, &L, &p) != TR_OK) return 0;
+  return L.total;
+}
+
+tr_status tr_transition_product(const tr_scan_args *args, float *P, void *ws, size_t ws_bytes,
+                                void *stream) {
+  if (!P) return fail(TR_ERR_INVALID_ARG, "P is NULL");
+  if (!aligned16(P)) return fail(TR_ERR_ALIGNMENT, "P must be 16-byte aligned");
+  TpLayout L;
+  tr::ScanLaunch p;
+  tr_status st = tp_layout(args, &L, &p);
+  if (st != TR_OK) return st;
+  if (!ws || ws_bytes < L.total)
+    return fail(TR_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", ws_bytes, L.total);
+  if (reinterpret_cast<uintptr_t>(ws) & 255u)
+    return fail(TR_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  tr_scan_args b = tp_scan_args(args, P, base + L.v0, reinterpret_cast<float *>(base + L.ident));
+  st = validate_scan(&b, &p);
+  if (st != TR_OK) return st;
+  int dev;
+  unsigned *errw;
+  std::string err;
+  if (!device_state(&dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  if (L.v0_bytes) e = cudaMemsetAsync(base + L.v0, 0, L.v0_bytes, s);
+  if (e == cudaSuccess && L.ident_bytes) e = cudaMemsetAsync(base + L.ident, 0, L.ident_bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "transition product setup");
+  const int64_t n_mats = (int64_t)args->n_seqs * args->n_heads;
+  if (n_mats > 0) {
+    const int64_t n = n_mats * args->d_k;
+    set_identity<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(reinterpret_cast<float *>(base + L.ident),
+                                                              n_mats, args->d_k);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "transition product setup");
+  }
+  p.ws = base + L.scan;
+  p.ws_bytes = ws_bytes - L.scan;
+  p.err_word = errw;
+  st = run_scan(p, s);
   return st == TR_OK ? ok() : st;
 }
 
