@@ -539,6 +539,20 @@ def our_arm(args):
     upd = k5 * 32
     scan_bytes = upd * (3 * 256 + 8 + 256) + 32 * 128 * 128 * 4
     scan_gbs = scan_bytes / scan_t / 1e9
+    # the same tail's transition product P (32 heads of 128 x 128), the repair operator
+    cu5 = case.cu_seqlens
+    Pbuf = torch.empty(1, 32, 128, 128, dtype=torch.float32, device=dev)
+    for _ in range(3):
+        tr.transition_product(sk, sla, sb, cu5, P=Pbuf)
+    tp_ms = []
+    for _ in range(max(5, min(args.steps, 50))):
+        flush.zero_()
+        e0.record(stream)
+        tr.transition_product(sk, sla, sb, cu5, P=Pbuf)
+        e1.record(stream)
+        e1.synchronize()
+        tp_ms.append(e0.elapsed_time(e1))
+    tp_t = sum(tp_ms) / len(tp_ms) * 1e-3
     tr.check()
 
     if rank == 0:
@@ -573,6 +587,9 @@ def our_arm(args):
                      "roofline": {"bound": "hbm", "achieved": scan_gbs, "peak": peaks["hbm_gbs"],
                                   "unit": "GB/s", "frac": scan_gbs / peaks["hbm_gbs"],
                                   "traffic": None, "alg_bytes": scan_bytes}},
+            "transition_product": {
+                "workload": "P = T_t...T_1 of the scan cell's tail (32 heads, k=%d), fp32 out" % k5,
+                "us": tp_t * 1e6, "token_heads_per_s": upd / tp_t},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "replayed tokens/s",
                     "h2d_bytes_per_step": k * D * 2,
