@@ -234,6 +234,20 @@ tr_status tr_replay_groups(const tr_group_args *groups, int32_t n_groups, void *
                            size_t ws_bytes, void *stream);
 
 /*
+ * tr_replay_groups with the full-attention KV transfer overlapped (Tail-Replay reading
+ * notes, section 2.5: the KV of the matched prefix moves to the device on a separate
+ * stream while the linear-attention states are replayed, T ~ max(T_KV, T_replay)).
+ * `kv_bytes` are copied from `kv_host` (pinned host memory) to `kv_dev` on `copy_stream`,
+ * issued before the replay's kernels on `stream`; `stream` then waits for the copy, so
+ * work enqueued on it afterwards sees both the KV and the states.  One cudaMemcpyAsync;
+ * kv_bytes = 0 replays only.  The two streams must differ.  Same workspace as
+ * tr_replay_groups.
+ */
+tr_status tr_replay_groups_overlapped(const tr_group_args *groups, int32_t n_groups, void *ws,
+                                      size_t ws_bytes, const void *kv_host, void *kv_dev,
+                                      size_t kv_bytes, void *stream, void *copy_stream);
+
+/*
  * ---------------------------------------------------------- tr_state_error
  * Relative Frobenius error of a rebuilt state against the full-prefill state
  * (E_m = S_m - S_hat_m, RN section 2.3):

@@ -63,6 +63,8 @@ _SIGNATURES = {
     "tr_transition_product": (ctypes.c_int, [ctypes.POINTER(ScanArgs), c_vp, c_vp, c_sz, c_vp]),
     "tr_replay_group_workspace_size": (c_sz, [ctypes.POINTER(GroupArgs)]),
     "tr_replay_group": (ctypes.c_int, [ctypes.POINTER(GroupArgs), c_vp, c_sz, c_vp]),
+    "tr_replay_groups_overlapped": (ctypes.c_int, [ctypes.POINTER(GroupArgs), c_i32, c_vp, c_sz,
+                                                   c_vp, c_vp, c_sz, c_vp, c_vp]),
     "tr_replay_group_kernel_count": (c_i32, [ctypes.POINTER(GroupArgs)]),
     "tr_replay_group_profiled": (ctypes.c_int, [ctypes.POINTER(GroupArgs), c_vp, c_sz, c_vp,
                                                 ctypes.POINTER(c_vp), c_i32]),
@@ -298,6 +300,22 @@ class GroupsReplay:
     def run(self, stream=None):
         _ok(lib.tr_replay_groups(self._arr, len(self.groups), _ptr(self.workspace),
                                  self.ws_bytes, _stream(stream)), "tr_replay_groups")
+        return [(g.S_hat, g.x_out) for g in self.groups]
+
+    def run_overlapped(self, kv_host, kv_dev, stream=None, copy_stream=None):
+        """run() with kv_host (pinned) copied to kv_dev on copy_stream during the replay;
+        `stream` waits for the copy before anything enqueued after this call."""
+        if copy_stream is None:
+            raise ValueError("the KV copy needs a stream of its own (copy_stream)")
+        if kv_host.numel() * kv_host.element_size() != kv_dev.numel() * kv_dev.element_size():
+            raise ValueError("kv_host and kv_dev differ in size")
+        if not kv_host.is_pinned():
+            raise ValueError("kv_host must be pinned host memory")
+        nbytes = kv_host.numel() * kv_host.element_size()
+        _ok(lib.tr_replay_groups_overlapped(self._arr, len(self.groups), _ptr(self.workspace),
+                                            self.ws_bytes, kv_host.data_ptr(), _ptr(kv_dev),
+                                            nbytes, _stream(stream), _stream(copy_stream)),
+            "tr_replay_groups_overlapped")
         return [(g.S_hat, g.x_out) for g in self.groups]
 
 

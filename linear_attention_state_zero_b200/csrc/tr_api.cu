@@ -680,6 +680,34 @@ tr_status tr_replay_groups(const tr_group_args *groups, int32_t n_groups, void *
   return ok();
 }
 
+tr_status tr_replay_groups_overlapped(const tr_group_args *groups, int32_t n_groups, void *ws,
+                                      size_t ws_bytes, const void *kv_host, void *kv_dev,
+                                      size_t kv_bytes, void *stream, void *copy_stream) {
+  if (kv_bytes > 0 && (!kv_host || !kv_dev)) return fail(TR_ERR_INVALID_ARG, "KV pointer is NULL");
+  if (kv_bytes > 0 && stream == copy_stream)
+    return fail(TR_ERR_INVALID_ARG, "the copy needs a stream of its own");
+  cudaStream_t s = static_cast<cudaStream_t>(stream), cs = static_cast<cudaStream_t>(copy_stream);
+  cudaEvent_t done = nullptr;
+  if (kv_bytes > 0) {
+    cudaError_t e = cudaMemcpyAsync(kv_dev, kv_host, kv_bytes, cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&done, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventRecord(done, cs);
+    if (e != cudaSuccess) {
+      if (done) cudaEventDestroy(done);
+      return cuda_fail(e, "KV transfer");
+    }
+  }
+  tr_status st = tr_replay_groups(groups, n_groups, ws, ws_bytes, stream);
+  if (done) {
+    // the join is enqueued even when the replay failed, so the stream never runs ahead of
+    // the copy; the event is released once it has completed
+    cudaError_t e = cudaStreamWaitEvent(s, done, 0);
+    cudaEventDestroy(done);
+    if (st == TR_OK && e != cudaSuccess) return cuda_fail(e, "KV transfer join");
+  }
+  return st == TR_OK ? ok() : st;
+}
+
 size_t tr_state_error_workspace_size(int64_t n_mats) {
   // 2 doubles per matrix piece, up to 16 pieces per matrix
   return n_mats > 0 ? align256((size_t)n_mats * 16 * 2 * sizeof(double)) : 0;

@@ -107,3 +107,25 @@ def test_full_prefill_equals_tail_when_decay_is_strong(cuda_device):
                                d, skip_last_output=True)
     _, tot = tr.state_error(S_m.reshape(-1, d, d), S_hat.reshape(-1, d, d))
     assert float(tot.item()) < 1e-3
+
+
+def test_replay_with_overlapped_kv_transfer(cuda_device):
+    """Reading notes section 2.5: the FA KV moves to the device on its own stream while the
+    states are replayed.  The states equal the plain call's bitwise, the KV arrives intact,
+    and work after the call on the replay's stream sees both."""
+    D, H, d, L = 256, 2, 128, 2
+    gs = []
+    for g in range(2):
+        h, layers, cu = make_group([90, 33], D, H, d, L, seed=340 + g)
+        gs.append(tr.GroupReplay(h.to(cuda_device), cu, to_dev(layers, cuda_device), H, d, d))
+    plain = [(S.clone(), x.clone()) for S, x in tr.GroupsReplay(gs).run()]
+    kv_host = torch.randint(0, 255, (32 << 20,), dtype=torch.uint8).pin_memory()
+    kv_dev = torch.empty(kv_host.shape, dtype=torch.uint8, device=cuda_device)
+    side = torch.cuda.Stream(device=cuda_device)
+    outs = tr.GroupsReplay(gs).run_overlapped(kv_host, kv_dev, copy_stream=side)
+    chk = kv_dev[::4096].clone()  # enqueued after the call on the replay's stream
+    torch.cuda.synchronize()
+    assert torch.equal(chk.cpu(), kv_host[::4096])
+    assert torch.equal(kv_dev.cpu(), kv_host)
+    for (S, x), (S0, x0) in zip(outs, plain):
+        assert torch.equal(S, S0) and torch.equal(x, x0)
