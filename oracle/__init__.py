@@ -24,6 +24,7 @@ layer internals).
 """
 from .tail_replay import (  # noqa: F401
     bf16_round,
+    ffn_residual,
     gates,
     gdn_scan,
     in_projection,
@@ -32,6 +33,7 @@ from .tail_replay import (  # noqa: F401
     replay_group,
     replay_layer,
     rmsnorm,
+    silu,
     state_error,
     tail_len,
     tail_rows,

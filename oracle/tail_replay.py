@@ -12,11 +12,15 @@ RN section 2.3 says no model dimensions are to be made up from Eq. (1)):
     x_hat W_in^T = [q | k | v | a_alpha | a_beta] (no bias, no short
     convolution, no activation on v) -> q and k L2-normalised per head
     (x / sqrt(sum x^2 + 1e-6)) -> alpha = exp(-softplus(a_alpha)),
-    beta = sigmoid(a_beta) -> Eq. (1) scan -> x <- x + o W_o^T; the FFN sublayer
-    is left out, so the next LA layer reads the residual after the attention
-    sublayer;
+    beta = sigmoid(a_beta) -> Eq. (1) scan -> x <- x + o W_o^T;
+  * the FFN sublayer: where a layer carries FFN weights, a dense SwiGLU with its
+    own RMSNorm, x <- x + (silu(x_hat W_gate^T) * x_hat W_up^T) W_down^T, runs
+    after the LA sublayer, except after a group's last LA layer (RN section 2.5,
+    the tail-FFN skip); a layer without FFN weights passes the residual after its
+    LA sublayer straight to the next LA layer;
   * bf16 cast points of the boundary (``emulate_casts``): the projection
-    operands x_hat and o and the stored q, k, v are rounded to bf16
+    operands x_hat and o (and the FFN's pre-norm output and hidden activation)
+    and the stored q, k, v are rounded to bf16
     (round-to-nearest-even); everything else stays fp64 here.
 """
 from __future__ import annotations
@@ -249,11 +253,43 @@ def out_projection_residual(x, o, W_o) -> np.ndarray:
     return x + o.reshape(T, -1) @ _f64(W_o).T
 
 
+# ------------------------------------------------------------------------ a6b
+def silu(z) -> np.ndarray:
+    """z * sigmoid(z) = z / (1 + exp(-z)), elementwise (-0 where exp(-z) overflows)."""
+    z = _f64(z)
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def ffn_residual(x, W_gate, W_up, W_down, ffn_gain=None, rms_eps: float = 1e-6,
+                 emulate_casts: bool = True) -> np.ndarray:
+    """x + (silu(x_hat W_gate^T) * (x_hat W_up^T)) W_down^T, x_hat = RMSNorm(x) * ffn_gain.
+
+    RN section 2.5: inside a group, the FFN after each LA layer but the last still
+    runs, because it makes the next LA layer's input.  Reading (the pages never give
+    the FFN's form): a dense SwiGLU sublayer with its own pre-norm and a residual
+    add, W_gate and W_up [d_ff, D], W_down [D, d_ff], no biases.  Cast points: the
+    pre-norm output and the hidden activation are rounded to bf16 (the GEMM
+    operands); the two products and the residual stay fp64 here.
+    """
+    x = _f64(x)
+    cast = bf16_round if emulate_casts else (lambda a: a)
+    x_hat = cast(rmsnorm(x, ffn_gain, rms_eps))
+    g = x_hat @ _f64(W_gate).T
+    u = x_hat @ _f64(W_up).T
+    hmid = cast(silu(g) * u)
+    return x + hmid @ _f64(W_down).T
+
+
 # ---------------------------------------------------------------------- a2..a6
 def replay_layer(x, W_in, W_o, rms_gain, cu_seqlens, n_heads: int, d_k: int, d_v: int,
                  want_output: bool = True, emulate_casts: bool = True,
-                 rms_eps: float = 1e-6, norm_eps: float = 1e-6, n_threads=None):
-    """One LA layer of the replay from a zero state: returns (S_hat, x_next or None)."""
+                 rms_eps: float = 1e-6, norm_eps: float = 1e-6, n_threads=None, ffn=None):
+    """One LA layer of the replay from a zero state: returns (S_hat, x_next or None).
+
+    ``ffn`` = (W_gate, W_up, W_down, ffn_gain) runs the FFN sublayer on x_next
+    (``ffn_residual``); None leaves it out.
+    """
     x = _f64(x)
     cast = bf16_round if emulate_casts else (lambda a: a)
     x_hat = cast(rmsnorm(x, rms_gain, rms_eps))
@@ -267,31 +303,44 @@ def replay_layer(x, W_in, W_o, rms_gain, cu_seqlens, n_heads: int, d_k: int, d_v
     x_next = None
     if want_output:
         x_next = out_projection_residual(x, cast(o), W_o)
+        if ffn is not None:
+            W_gate, W_up, W_down, ffn_gain = ffn
+            x_next = ffn_residual(x_next, W_gate, W_up, W_down, ffn_gain, rms_eps, emulate_casts)
     return S_hat, x_next
 
 
 def replay_group(h_tail, cu_seqlens, layers: Sequence, n_heads: int, d_k: int, d_v: int,
                  emulate_casts: bool = True, skip_last_output: bool = False,
-                 rms_eps: float = 1e-6, norm_eps: float = 1e-6, n_threads=None):
+                 rms_eps: float = 1e-6, norm_eps: float = 1e-6, n_threads=None,
+                 skip_last_ffn: bool = True):
     """Replay one group's LA layers over the packed tails (RN section 2.2 steps 2-3).
 
     Every LA state of the group starts at zero at the tail start (step 2, GS
     "Key Mechanisms": initialise the replay state to zero); the tail hiddens
     h_{m-k+1..m} go through the group's LA layers in order (step 3), each layer
     feeding the next.  ``layers`` is a sequence of objects with W_in, W_o and
-    rms_gain.  Returns (S_hat [L, N, H, d_k, d_v], x_out [T, D] or None).
-    With ``skip_last_output`` the last layer's readout and output projection are
-    not computed (its output is not used to rebuild any state; RN section 2.5
-    makes the same argument for the tail FFN).
+    rms_gain, and W_gate, W_up, W_down, ffn_gain where the layer has an FFN
+    sublayer (W_gate None or absent: no FFN).  Returns (S_hat [L, N, H, d_k, d_v],
+    x_out [T, D] or None).
+    With ``skip_last_ffn`` the last layer's FFN is not run (RN section 2.5, the
+    tail-FFN skip: the next group starts from its own cached FA output, so that
+    FFN output rebuilds no state); x_out is then the residual after the last LA
+    sublayer.  With ``skip_last_output`` the last layer's readout and output
+    projection are not computed either (the same argument one sublayer earlier),
+    and x_out is None.
     """
     x = _f64(h_tail)
     S_all = []
     L = len(layers)
     for i, lw in enumerate(layers):
         want = not (skip_last_output and i == L - 1)
+        ffn = None
+        if getattr(lw, "W_gate", None) is not None and not (skip_last_ffn and i == L - 1):
+            ffn = (lw.W_gate, lw.W_up, lw.W_down, getattr(lw, "ffn_gain", None))
         S_hat, x_next = replay_layer(x, lw.W_in, lw.W_o, lw.rms_gain, cu_seqlens, n_heads, d_k, d_v,
                                      want_output=want, emulate_casts=emulate_casts,
-                                     rms_eps=rms_eps, norm_eps=norm_eps, n_threads=n_threads)
+                                     rms_eps=rms_eps, norm_eps=norm_eps, n_threads=n_threads,
+                                     ffn=ffn)
         S_all.append(S_hat)
         x = x_next
     return np.stack(S_all, 0), x

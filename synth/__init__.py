@@ -11,7 +11,8 @@ Distributions (all from ``torch.Generator`` on the CPU, or on the device for
 inputs too large to draw on the host; the same seed gives the same stream):
 
 * ``h``: N(0, 1), rounded to bf16 (hidden vectors leaving a full-attention layer).
-* projection weights: N(0, 0.02^2), rounded to bf16.
+* projection weights (the LA layer's and, where a layer has an FFN sublayer, its gate,
+  up and down weights): N(0, 0.02^2), rounded to bf16.
 * scan q, k: directions drawn uniformly on the unit sphere (a normalised Gaussian
   vector), then cast to the requested dtype.
 * scan v: N(0, 1).
@@ -33,6 +34,7 @@ SEED_BASE = 0x7A110001
 
 # tensor ids for sub-streams
 _T_H, _T_WIN, _T_WO, _T_GAIN = 1, 2, 3, 4
+_T_WGATE, _T_WUP, _T_WDOWN, _T_FGAIN = 5, 6, 7, 8
 _T_Q, _T_K, _T_V, _T_ALPHA, _T_BETA, _T_S0, _T_LENS = 11, 12, 13, 14, 15, 16, 17
 
 
@@ -118,6 +120,11 @@ class LALayerWeights:
     W_in: torch.Tensor            # bf16 [2H*d_k + H*d_v + 2H, D]  (out x in)
     W_o: torch.Tensor             # bf16 [D, H*d_v]
     rms_gain: Optional[torch.Tensor] = None  # fp32 [D] or None (= ones)
+    # FFN sublayer after the LA sublayer (all None: the layer has none)
+    W_gate: Optional[torch.Tensor] = None    # bf16 [d_ff, D]
+    W_up: Optional[torch.Tensor] = None      # bf16 [d_ff, D]
+    W_down: Optional[torch.Tensor] = None    # bf16 [D, d_ff]
+    ffn_gain: Optional[torch.Tensor] = None  # fp32 [D] or None (= ones)
 
 
 def in_features(n_heads: int, d_k: int, d_v: int) -> int:
@@ -125,7 +132,9 @@ def in_features(n_heads: int, d_k: int, d_v: int) -> int:
 
 
 def la_layers(n_layers: int, d_model: int, n_heads: int, d_k: int, d_v: int, seed: int,
-              std: float = 0.02, device: str = "cpu", with_gain: bool = False) -> List[LALayerWeights]:
+              std: float = 0.02, device: str = "cpu", with_gain: bool = False,
+              d_ff: int = 0) -> List[LALayerWeights]:
+    """Weights of ``n_layers`` LA layers; with ``d_ff > 0`` each also gets an FFN sublayer."""
     out = []
     n_in = in_features(n_heads, d_k, d_v)
     for l in range(n_layers):
@@ -135,7 +144,14 @@ def la_layers(n_layers: int, d_model: int, n_heads: int, d_k: int, d_v: int, see
         gain = None
         if with_gain:
             gain = 1.0 + normal((d_model,), s, _T_GAIN, 0.1, device)
-        out.append(LALayerWeights(W_in, W_o, gain))
+        lw = LALayerWeights(W_in, W_o, gain)
+        if d_ff > 0:
+            lw.W_gate = normal((d_ff, d_model), s, _T_WGATE, std, device).to(torch.bfloat16)
+            lw.W_up = normal((d_ff, d_model), s, _T_WUP, std, device).to(torch.bfloat16)
+            lw.W_down = normal((d_model, d_ff), s, _T_WDOWN, std, device).to(torch.bfloat16)
+            if with_gain:
+                lw.ffn_gain = 1.0 + normal((d_model,), s, _T_FGAIN, 0.1, device)
+        out.append(lw)
     return out
 
 

@@ -292,6 +292,68 @@ def test_out_projection_residual():
                                rtol=1e-15)
 
 
+# ------------------------------------------------------------ a6b FFN sublayer
+def test_silu_closed_forms():
+    """silu(z) = z sigmoid(z): library routine, odd-part identity, known values, limits."""
+    z = np.linspace(-30.0, 30.0, 241)
+    np.testing.assert_allclose(oracle.silu(z), torch.nn.functional.silu(torch.from_numpy(z)).numpy(),
+                               rtol=1e-14, atol=1e-300)
+    # silu(z) - silu(-z) = z (sigmoid(z) + sigmoid(-z) = 1)
+    np.testing.assert_allclose(oracle.silu(z) - oracle.silu(-z), z, rtol=1e-13, atol=1e-13)
+    assert oracle.silu([0.0])[0] == 0.0
+    assert abs(oracle.silu([1.0])[0] - math.e / (1.0 + math.e)) < 1e-15   # sigmoid(1)
+    big = oracle.silu([800.0, -800.0])
+    assert big[0] == 800.0 and big[1] == 0.0
+    # slope 1/2 at the origin
+    eps = 1e-6
+    assert abs((oracle.silu([eps])[0] - oracle.silu([-eps])[0]) / (2 * eps) - 0.5) < 1e-9
+
+
+def test_ffn_residual_worked_case():
+    """D = 2, d_ff = 1: x = [1, -1] has RMS 1, so x_hat = x; g = 1, u = 1, and the FFN adds
+    sigmoid(1) times the down column."""
+    x = np.array([[1.0, -1.0]])
+    Wg = np.array([[1.0, 0.0]])
+    Wu = np.array([[0.0, -1.0]])
+    Wd = np.array([[2.0], [3.0]])
+    y = oracle.ffn_residual(x, Wg, Wu, Wd, rms_eps=0.0, emulate_casts=False)
+    s1 = math.e / (1.0 + math.e)
+    np.testing.assert_allclose(y, [[1.0 + 2 * s1, -1.0 + 3 * s1]], rtol=1e-15)
+    # a gain scales x_hat: gain [2, 1] -> g = 2, u = 1
+    y2 = oracle.ffn_residual(x, Wg, Wu, Wd, ffn_gain=np.array([2.0, 1.0]), rms_eps=0.0,
+                             emulate_casts=False)
+    s2 = 2.0 * math.exp(2.0) / (1.0 + math.exp(2.0))
+    np.testing.assert_allclose(y2, [[1.0 + 2 * s2, -1.0 + 3 * s2]], rtol=1e-15)
+
+
+def test_ffn_residual_invariants():
+    """Zero down or up weights leave x; flipping the gate's sign changes the sublayer's output
+    by exactly (g * u) W_down^T, since silu(z) - silu(-z) = z; the sublayer depends on x only
+    through RMSNorm(x), so scaling x scales only the residual."""
+    T, D, F = 5, 12, 20
+    x = rng.standard_normal((T, D))
+    Wg = rng.standard_normal((F, D)) * 0.3
+    Wu = rng.standard_normal((F, D)) * 0.3
+    Wd = rng.standard_normal((D, F)) * 0.3
+    gain = 1.0 + 0.1 * rng.standard_normal(D)
+    np.testing.assert_array_equal(oracle.ffn_residual(x, Wg, Wu, np.zeros((D, F))), x)
+    np.testing.assert_array_equal(oracle.ffn_residual(x, Wg, np.zeros((F, D)), Wd), x)
+    f_pos = oracle.ffn_residual(x, Wg, Wu, Wd, gain, rms_eps=0.0, emulate_casts=False) - x
+    f_neg = oracle.ffn_residual(x, -Wg, Wu, Wd, gain, rms_eps=0.0, emulate_casts=False) - x
+    # x_hat by hand: x / RMS(x) * gain
+    xh = x / np.sqrt(np.mean(x * x, axis=1, keepdims=True)) * gain
+    np.testing.assert_allclose(f_pos - f_neg, ((xh @ Wg.T) * (xh @ Wu.T)) @ Wd.T,
+                               rtol=1e-11, atol=1e-12)
+    f_scaled = oracle.ffn_residual(3.5 * x, Wg, Wu, Wd, gain, rms_eps=0.0,
+                                   emulate_casts=False) - 3.5 * x
+    np.testing.assert_allclose(f_scaled, f_pos, rtol=1e-11, atol=1e-12)
+    # the bf16 cast points move the sublayer's output by about bf16 precision only
+    f_c = oracle.ffn_residual(x, Wg, Wu, Wd, gain) - x
+    f_e = oracle.ffn_residual(x, Wg, Wu, Wd, gain, emulate_casts=False) - x
+    rel = np.linalg.norm(f_c - f_e) / np.linalg.norm(f_e)
+    assert 0 < rel < 2e-2
+
+
 # ---------------------------------------------------------------- a8 state error
 def test_state_error_cases():
     S = rng.standard_normal((3, 4, 5))
@@ -366,6 +428,55 @@ def test_replay_cast_points_are_small():
     S_e, _ = oracle.replay_group(h, cu, layers, 2, 16, 16, emulate_casts=False)
     _, tot = oracle.state_error(S_e, S_c)
     assert 0 < tot < 2e-2
+
+
+def _tiny_ffn_group(lengths, D=48, H=2, dk=8, dv=8, L=3, F=64, seed=11):
+    layers = synth.la_layers(L, D, H, dk, dv, seed=seed, std=0.2, with_gain=True, d_ff=F)
+    h = torch.cat([synth.hidden_prefix(n, D, seed + i) for i, n in enumerate(lengths)])
+    return h, layers, synth.cu_seqlens_of(lengths)
+
+
+def _without_ffn(layers):
+    return [synth.LALayerWeights(lw.W_in, lw.W_o, lw.rms_gain) for lw in layers]
+
+
+def test_replay_group_ffn_placement_and_tail_skip():
+    """RN section 2.5: the FFNs between a group's LA layers feed the next LA layer; the last
+    layer's FFN feeds no state and is skipped.  So: the first layer's state sees no FFN; the
+    last layer's FFN changes no state; an FFN with zero down weights is no FFN; the skipped
+    FFN, applied to the skip's x_out, gives the unskipped x_out."""
+    lengths = [17, 0, 9]
+    H, dk = 2, 8
+    h, layers, cu = _tiny_ffn_group(lengths)
+    plain = _without_ffn(layers)
+    S_f, x_skip = oracle.replay_group(h, cu, layers, H, dk, dk)               # tail skip (default)
+    S_n, x_n = oracle.replay_group(h, cu, plain, H, dk, dk)
+    S_u, x_full = oracle.replay_group(h, cu, layers, H, dk, dk, skip_last_ffn=False)
+    np.testing.assert_array_equal(S_f[0], S_n[0])                # layer 0's state: no FFN before it
+    assert np.abs(S_f[1] - S_n[1]).max() > 1e-3                  # the layer-0 FFN feeds layer 1
+    np.testing.assert_array_equal(S_u, S_f)                      # the last FFN feeds no state
+    last = layers[-1]
+    np.testing.assert_allclose(x_full, oracle.ffn_residual(x_skip, last.W_gate, last.W_up,
+                                                           last.W_down, last.ffn_gain),
+                               rtol=1e-13, atol=1e-13)
+    S_o, _ = oracle.replay_group(h, cu, layers, H, dk, dk, skip_last_output=True)
+    np.testing.assert_array_equal(S_o, S_f)
+    # zero down weights: the FFN adds nothing
+    zeroed = [synth.LALayerWeights(lw.W_in, lw.W_o, lw.rms_gain, lw.W_gate, lw.W_up,
+                                   torch.zeros_like(lw.W_down), lw.ffn_gain) for lw in layers]
+    S_z, x_z = oracle.replay_group(h, cu, zeroed, H, dk, dk, skip_last_ffn=False)
+    np.testing.assert_array_equal(S_z, S_n)
+    np.testing.assert_array_equal(x_z, x_n)
+    # a one-layer group with the tail skip is the plain LA layer
+    S1, x1 = oracle.replay_group(h, cu, layers[:1], H, dk, dk)
+    S1n, x1n = oracle.replay_group(h, cu, plain[:1], H, dk, dk)
+    np.testing.assert_array_equal(S1, S1n)
+    np.testing.assert_array_equal(x1, x1n)
+    assert not S_f[:, 1].any()                                   # k = 0: zero state
+    # packed requests equal separate replays
+    Sa, xa = oracle.replay_group(h[:17], [0, 17], layers, H, dk, dk, skip_last_ffn=False)
+    np.testing.assert_allclose(S_u[:, 0], Sa[:, 0], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(x_full[:17], xa, rtol=1e-12, atol=1e-12)
 
 
 # ---------------------------------------------------- transition product (HYPIC operator)
