@@ -66,7 +66,12 @@ enum {
   TR_SKIP_LAST_OUTPUT = 2u,  /* tr_replay_group(s): skip the last LA layer's readout, q
                                 projection and output projection (its output rebuilds no
                                 state; RN section 2.5 makes the same point for the tail FFN) */
-  TR_SCAN_RECURRENT = 4u     /* force the token-sequential scan kernel (test path) */
+  TR_SCAN_RECURRENT = 4u,    /* force the token-sequential scan kernel (test path) */
+  TR_SKIP_LAST_FFN = 8u      /* tr_replay_group(s): do not run the last LA layer's FFN
+                                sublayer (RN section 2.5, tail-FFN skip: the next group
+                                starts from its own cached FA output, so that FFN output
+                                rebuilds no state); x_out is then the residual after the
+                                last LA sublayer */
 };
 
 /* Human-readable message for the last failing call on this host thread. */
@@ -171,7 +176,13 @@ tr_status tr_transition_product(const tr_scan_args *args, float *P, void *ws, si
  *   q, k <- bf16(x / sqrt(sum x^2 + norm_eps)) per head (norm_eps 0 -> 1e-6)
  *   v <- bf16(v); log alpha = -softplus(a_alpha), beta = sigmoid(a_beta) (fp32)
  *   o, S_hat[layer] = tr_gdn_scan(q, k, v, log alpha, beta), zero start
- *   x <- x + bf16(o) W_o^T                     fp32 residual; no FFN sublayer
+ *   x <- x + bf16(o) W_o^T                     fp32 residual
+ * and, where the layer has FFN weights (W_gate not NULL), the FFN sublayer that
+ * RN section 2.5 says still runs between a group's LA layers (the pages do not
+ * give its form; the reading is a dense SwiGLU with its own pre-norm):
+ *   x_hat = bf16(RMSNorm(x) * ffn_gain)        eps = rms_eps
+ *   h = bf16(silu(x_hat W_gate^T) * (x_hat W_up^T))   fp32 products, silu in fp32
+ *   x <- x + h W_down^T                        fp32 residual
  * x starts as h_tail.  The cast points above are part of this contract.
  *
  * Arguments (T = total_tokens, D = d_model, H = n_heads):
@@ -181,10 +192,15 @@ tr_status tr_transition_product(const tr_scan_args *args, float *P, void *ws, si
  *              W_in     [2 H d_k + H d_v + 2 H, D] bf16 (output x input features;
  *                       rows: q heads, k heads, v heads, a_alpha, a_beta)
  *              W_o      [D, H d_v] bf16
+ *              ffn_gain [D] fp32 or NULL (ones)
+ *              W_gate   [d_ff, D] bf16, or NULL: the layer has no FFN sublayer
+ *              W_up     [d_ff, D] bf16 (with W_gate)
+ *              W_down   [D, d_ff] bf16 (with W_gate)
+ *   d_ff     FFN width, a multiple of 128; 0 when no layer has an FFN.
  *   S_hat    [n_layers, N, H, d_k, d_v] fp32 output.
  *   x_out    [T, D] fp32 output of the last layer, or NULL (then the last
- *            layer's output projection is not run).  Must be NULL with
- *            TR_SKIP_LAST_OUTPUT.
+ *            layer's output projection and FFN are not run).  Must be NULL with
+ *            TR_SKIP_LAST_OUTPUT, which skips the last FFN as well.
  * Supported: d_k = d_v = 128 or 64; D a multiple of 64; 1 <= n_layers <= 64.
  * Workspace: tr_replay_group_workspace_size(args) bytes.
  */
@@ -192,6 +208,10 @@ typedef struct tr_la_layer {
   const float *rms_gain;
   const void *W_in;
   const void *W_o;
+  const float *ffn_gain;
+  const void *W_gate;
+  const void *W_up;
+  const void *W_down;
 } tr_la_layer;
 
 typedef struct tr_group_args {
@@ -199,6 +219,7 @@ typedef struct tr_group_args {
   int64_t total_tokens;
   uint32_t flags;
   float rms_eps, norm_eps;
+  int32_t d_ff;
   const void *h_tail;
   const int32_t *cu_seqlens;
   const int32_t *cu_seqlens_host;

@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libtr.so")
 
 TR_OK = 0
 TR_DTYPE_F32, TR_DTYPE_BF16 = 0, 1
-TR_NORMALIZE_QK, TR_SKIP_LAST_OUTPUT, TR_SCAN_RECURRENT = 1, 2, 4
+TR_NORMALIZE_QK, TR_SKIP_LAST_OUTPUT, TR_SCAN_RECURRENT, TR_SKIP_LAST_FFN = 1, 2, 4, 8
 
 STATUS_NAMES = {0: "TR_OK", 1: "TR_ERR_INVALID_ARG", 2: "TR_ERR_SHAPE", 3: "TR_ERR_DTYPE",
                 4: "TR_ERR_ALIGNMENT", 5: "TR_ERR_UNSUPPORTED", 6: "TR_ERR_WORKSPACE",
@@ -41,13 +41,14 @@ class ScanArgs(ctypes.Structure):
 
 
 class LALayer(ctypes.Structure):
-    _fields_ = [("rms_gain", c_vp), ("W_in", c_vp), ("W_o", c_vp)]
+    _fields_ = [("rms_gain", c_vp), ("W_in", c_vp), ("W_o", c_vp), ("ffn_gain", c_vp),
+                ("W_gate", c_vp), ("W_up", c_vp), ("W_down", c_vp)]
 
 
 class GroupArgs(ctypes.Structure):
     _fields_ = [("n_seqs", c_i32), ("n_heads", c_i32), ("d_k", c_i32), ("d_v", c_i32),
                 ("d_model", c_i32), ("n_layers", c_i32), ("total_tokens", c_i64),
-                ("flags", c_u32), ("rms_eps", c_f32), ("norm_eps", c_f32),
+                ("flags", c_u32), ("rms_eps", c_f32), ("norm_eps", c_f32), ("d_ff", c_i32),
                 ("h_tail", c_vp), ("cu_seqlens", c_vp), ("cu_seqlens_host", c_vp),
                 ("layers", ctypes.POINTER(LALayer)), ("S_hat", c_vp), ("x_out", c_vp)]
 
@@ -211,23 +212,31 @@ def transition_product(k, log_alpha, beta, cu_seqlens, *, normalize_qk=False, re
 
 @dataclass
 class Layer:
-    """One LA layer's weights, device tensors (W_in [2Hd_k + Hd_v + 2H, D], W_o [D, H d_v])."""
+    """One LA layer's weights, device tensors (W_in [2Hd_k + Hd_v + 2H, D], W_o [D, H d_v]),
+    and, if the layer has an FFN sublayer, W_gate and W_up [d_ff, D], W_down [D, d_ff]
+    (bf16) and ffn_gain [D] fp32 (None: ones)."""
     W_in: torch.Tensor
     W_o: torch.Tensor
     rms_gain: Optional[torch.Tensor] = None
+    W_gate: Optional[torch.Tensor] = None
+    W_up: Optional[torch.Tensor] = None
+    W_down: Optional[torch.Tensor] = None
+    ffn_gain: Optional[torch.Tensor] = None
 
 
 class GroupReplay:
     """A prepared tr_replay_group call: fixed buffers, so repeated calls cost one C call.
 
     ``h_tail`` [T, D] bf16 and ``cu_seqlens`` describe the packed tails of the
-    group's requests; ``layers`` the group's LA layers.  Outputs: ``S_hat``
+    group's requests; ``layers`` the group's LA layers (objects with the fields of
+    ``Layer``; FFN fields absent or None: no FFN sublayer).  Outputs: ``S_hat``
     [L, N, H, d_k, d_v] fp32 and, unless ``skip_last_output``, ``x_out`` [T, D].
+    ``skip_last_ffn`` (default on, the tail-FFN skip) leaves out the last layer's FFN.
     """
 
     def __init__(self, h_tail, cu_seqlens, layers: Sequence, n_heads: int, d_k: int, d_v: int,
                  *, skip_last_output=False, want_x_out=True, rms_eps=0.0, norm_eps=0.0,
-                 S_hat=None, x_out=None, workspace=None):
+                 skip_last_ffn=True, S_hat=None, x_out=None, workspace=None):
         _need_cuda(h_tail)
         if h_tail.dtype != torch.bfloat16 or not h_tail.is_contiguous():
             raise ValueError("h_tail must be contiguous bf16 [T, D]")
@@ -238,9 +247,18 @@ class GroupReplay:
         L = len(layers)
         self.layers = list(layers)
         self._layer_arr = (LALayer * L)()
+        d_ff = 0
         for i, lw in enumerate(self.layers):
             _need_cuda(lw.W_in, lw.W_o)
-            self._layer_arr[i] = LALayer(_ptr(lw.rms_gain), _ptr(lw.W_in), _ptr(lw.W_o))
+            Wg = getattr(lw, "W_gate", None)
+            Wu, Wd, fg = (getattr(lw, n, None) for n in ("W_up", "W_down", "ffn_gain"))
+            if Wg is not None:
+                _need_cuda(Wg, Wu, Wd)
+                if d_ff and Wg.shape[0] != d_ff:
+                    raise ValueError("all FFN sublayers of a group must have one width")
+                d_ff = Wg.shape[0]
+            self._layer_arr[i] = LALayer(_ptr(lw.rms_gain), _ptr(lw.W_in), _ptr(lw.W_o),
+                                         _ptr(fg), _ptr(Wg), _ptr(Wu), _ptr(Wd))
         self.S_hat = S_hat if S_hat is not None else torch.empty(
             (L, N, n_heads, d_k, d_v), dtype=torch.float32, device=dev)
         if skip_last_output:
@@ -249,10 +267,11 @@ class GroupReplay:
         if want_x_out:
             self.x_out = x_out if x_out is not None else torch.empty((T, D), dtype=torch.float32,
                                                                      device=dev)
-        flags = TR_SKIP_LAST_OUTPUT if skip_last_output else 0
+        flags = (TR_SKIP_LAST_OUTPUT if skip_last_output else 0) | \
+            (TR_SKIP_LAST_FFN if skip_last_ffn else 0)
         self.h_tail = h_tail
         self.args = GroupArgs(N, n_heads, d_k, d_v, D, L, T, flags, float(rms_eps),
-                              float(norm_eps), _ptr(h_tail), _ptr(self.dev_cu),
+                              float(norm_eps), d_ff, _ptr(h_tail), _ptr(self.dev_cu),
                               self.host.data_ptr(), self._layer_arr, _ptr(self.S_hat),
                               _ptr(self.x_out))
         self.ws_bytes = lib.tr_replay_group_workspace_size(ctypes.byref(self.args))

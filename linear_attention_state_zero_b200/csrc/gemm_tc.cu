@@ -4,6 +4,8 @@
 //   input projection  : [q|k|v|a_alpha|a_beta] = x_hat W_in^T, with the per-head
 //                       L2 norm of q and k, -softplus / sigmoid gates, bf16 q/k/v
 //   output projection : x <- x + o W_o^T (fp32 residual stream)
+//   FFN gate/up       : h = bf16(silu(x_hat W_gate^T) * (x_hat W_up^T)); a 256-column
+//                       tile holds 128 gate and the same 128 up columns (two B loads)
 //
 // C[M, N] = A[M, K] * B[N, K]^T, A and B bf16 with K contiguous (K-major).
 // One persistent CTA per SM walks the output tiles (128 x BN).  Warp roles:
@@ -30,7 +32,7 @@ constexpr int BK = 64;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 
-enum { EPI_INPROJ = 0, EPI_RESID = 1 };
+enum { EPI_INPROJ = 0, EPI_RESID = 1, EPI_SWIGLU = 2 };
 
 template <int BN>
 struct Cfg {
@@ -197,11 +199,30 @@ __device__ __forceinline__ void epi_resid(const ResidEpi &ep, uint32_t tbase, in
   }
 }
 
+// FFN epilogue for one tile of 128 gate (TMEM columns 0-127) and 128 up columns
+// (128-255): half `half` of the warps takes outputs 64 half .. +63.
+__device__ __forceinline__ void epi_swiglu(const SwigluEpi &ep, uint32_t tbase, int n0, int row,
+                                           int M, int half) {
+#pragma unroll 1
+  for (int j = 0; j < 2; ++j) {
+    const int c = 64 * half + 32 * j;  // output column within the tile
+    float g[32], u[32];
+    tmem_ld32(tbase + c, g);
+    tmem_ld32(tbase + 128 + c, u);
+    tc_wait_ld();
+    if (row >= M) continue;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) g[i] = g[i] / (1.f + exp_ftz(-g[i])) * u[i];
+    store_bf16x32(ep.h + (int64_t)row * ep.ld + n0 + c, g, 1.f);
+  }
+}
+
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, int M, int N, int K,
-                        InProjEpi ip, ResidEpi rs, unsigned *err_word) {
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmB2, int M, int N, int K,
+                        InProjEpi ip, ResidEpi rs, SwigluEpi sw, unsigned *err_word) {
   using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -228,6 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (EPI == EPI_SWIGLU) tma_prefetch_desc(&tmB2);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&ctl->tmem_base), C::TMEM_COLS);
@@ -255,7 +277,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t fb = smem_u32(&ctl->full[stage]);
           mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
           tma_load_2d(sa, &tmA, kb * BK, tm * BM, fb);
-          tma_load_2d(sa + C::A_BYTES, &tmB, kb * BK, tn * BN, fb);
+          if (EPI == EPI_SWIGLU) {  // gate rows, then the same up rows
+            tma_load_2d(sa + C::A_BYTES, &tmB, kb * BK, tn * (BN / 2), fb);
+            tma_load_2d(sa + C::A_BYTES + C::B_BYTES / 2, &tmB2, kb * BK, tn * (BN / 2), fb);
+          } else {
+            tma_load_2d(sa + C::A_BYTES, &tmB, kb * BK, tn * BN, fb);
+          }
           if (++stage == C::STAGES) {
             stage = 0;
             ph ^= 1u;
@@ -312,6 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tbase = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(b * BN);
       if (EPI == EPI_INPROJ)
         epi_inproj<BN>(ip, tbase, tn * BN, N, row, M, lo, hi);
+      else if (EPI == EPI_SWIGLU)
+        epi_swiglu(sw, tbase, tn * (BN / 2), row, M, half);
       else
         epi_resid<BN>(rs, tbase, tn * BN, N, row, M, lo, hi);
       tc_fence_before();
@@ -328,16 +357,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// N counts the tile's output columns; for the FFN gate/up product N = 2 d_ff, B = W_gate
+// and B2 = W_up ([d_ff, K] each).
 template <int BN, int EPI>
-cudaError_t launch(const void *A, int64_t lda, const void *B, int M, int N, int K,
-                   const InProjEpi &ip, const ResidEpi &rs, unsigned *err_word, cudaStream_t s,
-                   bool pdl, std::string *err) {
+cudaError_t launch(const void *A, int64_t lda, const void *B, const void *B2, int M, int N, int K,
+                   const InProjEpi &ip, const ResidEpi &rs, const SwigluEpi &sw,
+                   unsigned *err_word, cudaStream_t s, bool pdl, std::string *err) {
   using C = Cfg<BN>;
   if (M <= 0 || N <= 0) return cudaSuccess;
-  CUtensorMap ta, tb;
-  if (!make_tmap_bf16_2d(&ta, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 2, BK, BM, err) ||
-      !make_tmap_bf16_2d(&tb, B, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN, err))
-    return cudaErrorInvalidValue;
+  CUtensorMap ta, tb, tb2;
+  if (EPI == EPI_SWIGLU) {
+    if (!make_tmap_bf16_2d(&ta, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 2, BK, BM, err) ||
+        !make_tmap_bf16_2d(&tb, B, (uint64_t)K, (uint64_t)(N / 2), (uint64_t)K * 2, BK, BN / 2,
+                           err) ||
+        !make_tmap_bf16_2d(&tb2, B2, (uint64_t)K, (uint64_t)(N / 2), (uint64_t)K * 2, BK, BN / 2,
+                           err))
+      return cudaErrorInvalidValue;
+  } else {
+    if (!make_tmap_bf16_2d(&ta, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 2, BK, BM, err) ||
+        !make_tmap_bf16_2d(&tb, B, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN, err))
+      return cudaErrorInvalidValue;
+    tb2 = tb;
+  }
   auto kern = gemm_bf16_tn_kernel<BN, EPI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)C::SMEM);
@@ -345,8 +386,8 @@ cudaError_t launch(const void *A, int64_t lda, const void *B, int M, int N, int 
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   int grid = device_sm_count();
   if (grid > tiles) grid = tiles;
-  return launch_kernel(kern, dim3((unsigned)grid), dim3(kThreads), C::SMEM, s, pdl, ta, tb, M, N, K,
-                       ip, rs, err_word);
+  return launch_kernel(kern, dim3((unsigned)grid), dim3(kThreads), C::SMEM, s, pdl, ta, tb, tb2, M,
+                       N, K, ip, rs, sw, err_word);
 }
 
 }  // namespace
@@ -355,7 +396,8 @@ cudaError_t launch_gemm_inproj(const void *A, const void *B, int M, int N, int K
                                const InProjEpi &ep, unsigned *err_word, cudaStream_t s,
                                bool pdl, std::string *err) {
   ResidEpi none{};
-  return launch<256, EPI_INPROJ>(A, K, B, M, N, K, ep, none, err_word, s, pdl, err);
+  SwigluEpi no_sw{};
+  return launch<256, EPI_INPROJ>(A, K, B, nullptr, M, N, K, ep, none, no_sw, err_word, s, pdl, err);
 }
 
 cudaError_t launch_gemm_resid(const void *A, int64_t lda, const void *B, int M, int N, int K,
@@ -364,7 +406,17 @@ cudaError_t launch_gemm_resid(const void *A, int64_t lda, const void *B, int M, 
   InProjEpi none{};
   // 192-column tiles: the output is narrow (d_model), so 128 x 256 tiles would leave SMs
   // idle and N = 128 MMAs are issue-bound; d_model 2048 gives 11 x 13 = 143 tiles, one wave
-  return launch<192, EPI_RESID>(A, lda, B, M, N, K, none, ep, err_word, s, pdl, err);
+  SwigluEpi no_sw{};
+  return launch<192, EPI_RESID>(A, lda, B, nullptr, M, N, K, none, ep, no_sw, err_word, s, pdl, err);
+}
+
+cudaError_t launch_gemm_swiglu(const void *A, const void *W_gate, const void *W_up, int M, int d_ff,
+                               int K, const SwigluEpi &ep, unsigned *err_word, cudaStream_t s,
+                               bool pdl, std::string *err) {
+  InProjEpi no_ip{};
+  ResidEpi no_rs{};
+  return launch<256, EPI_SWIGLU>(A, K, W_gate, W_up, M, 2 * d_ff, K, no_ip, no_rs, ep, err_word, s,
+                                 pdl, err);
 }
 
 }  // namespace tr

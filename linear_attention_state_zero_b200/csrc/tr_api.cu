@@ -279,9 +279,11 @@ tr_status run_scan(const tr::ScanLaunch &p, cudaStream_t s,
 
 // ------------------------------------------------------------- replay group
 struct GroupLayout {
-  size_t x, xhat, qkv, la, beta, o, scan, total;
+  size_t x, xhat, qkv, la, beta, o, hmid, scan, total;
   int64_t ldq;
 };
+
+bool has_ffn(const tr_la_layer &w) { return w.W_gate != nullptr; }
 
 // The scan launch of one LA layer of a group (pointers filled in by the caller).
 tr::ScanLaunch group_scan_launch(const tr_group_args *a) {
@@ -309,6 +311,7 @@ GroupLayout group_layout(const tr_group_args *a) {
   L.la = off;   off = align256(off + T * H * 4);
   L.beta = off; off = align256(off + T * H * 4);
   L.o = off;    off = align256(off + T * H * (size_t)a->d_v * 2);
+  L.hmid = off; off = align256(off + T * (size_t)(a->d_ff > 0 ? a->d_ff : 0) * 2);
   L.scan = off; off = align256(off + scan_ws_bytes(group_scan_launch(a)));
   L.total = off;
   return L;
@@ -327,8 +330,10 @@ tr_status validate_group(const tr_group_args *a) {
                 a->d_v);
   if (a->d_model % 64) return fail(TR_ERR_UNSUPPORTED, "d_model = %d is not a multiple of 64",
                                    a->d_model);
-  if (a->flags & ~(unsigned)TR_SKIP_LAST_OUTPUT)
+  if (a->flags & ~(unsigned)(TR_SKIP_LAST_OUTPUT | TR_SKIP_LAST_FFN))
     return fail(TR_ERR_INVALID_ARG, "unknown replay flags 0x%x", a->flags);
+  if (a->d_ff < 0 || a->d_ff % 128)
+    return fail(TR_ERR_UNSUPPORTED, "d_ff = %d is not a non-negative multiple of 128", a->d_ff);
   if ((a->flags & TR_SKIP_LAST_OUTPUT) && a->x_out)
     return fail(TR_ERR_INVALID_ARG, "x_out must be NULL with TR_SKIP_LAST_OUTPUT");
   if (!a->cu_seqlens || !a->layers || !a->S_hat || (a->total_tokens > 0 && !a->h_tail))
@@ -340,6 +345,17 @@ tr_status validate_group(const tr_group_args *a) {
     if (!w.W_in || !w.W_o) return fail(TR_ERR_INVALID_ARG, "layer %d: W_in or W_o is NULL", l);
     if (!aligned16(w.W_in) || !aligned16(w.W_o) || (w.rms_gain && !aligned16(w.rms_gain)))
       return fail(TR_ERR_ALIGNMENT, "layer %d: weights must be 16-byte aligned", l);
+    if (has_ffn(w)) {
+      if (a->d_ff == 0)
+        return fail(TR_ERR_INVALID_ARG, "layer %d has FFN weights but d_ff = 0", l);
+      if (!w.W_up || !w.W_down)
+        return fail(TR_ERR_INVALID_ARG, "layer %d: W_gate without W_up or W_down", l);
+      if (!aligned16(w.W_gate) || !aligned16(w.W_up) || !aligned16(w.W_down) ||
+          (w.ffn_gain && !aligned16(w.ffn_gain)))
+        return fail(TR_ERR_ALIGNMENT, "layer %d: FFN weights must be 16-byte aligned", l);
+    } else if (w.W_up || w.W_down || w.ffn_gain) {
+      return fail(TR_ERR_INVALID_ARG, "layer %d: FFN weights without W_gate", l);
+    }
   }
   return check_cu_host(a->cu_seqlens_host, a->n_seqs, a->total_tokens);
 }
@@ -354,6 +370,15 @@ struct Marks {
   }
 };
 
+// Whether layer l runs its FFN sublayer: it has FFN weights, its LA output is computed,
+// and it is not the last layer under the tail-FFN skip.
+bool runs_ffn(const tr_group_args *a, int l) {
+  const bool last = l == a->n_layers - 1;
+  if (!has_ffn(a->layers[l])) return false;
+  if (last && ((a->flags & (TR_SKIP_LAST_OUTPUT | TR_SKIP_LAST_FFN)) || !a->x_out)) return false;
+  return true;
+}
+
 int group_kernel_count(const tr_group_args *a) {
   int n = 0;
   for (int l = 0; l < a->n_layers; ++l) {
@@ -361,6 +386,7 @@ int group_kernel_count(const tr_group_args *a) {
     const bool skip = last && (a->flags & TR_SKIP_LAST_OUTPUT);
     n += 2 + scan_kernel_count(group_scan_launch(a), !skip);
     if (!skip && (!last || a->x_out)) n += 1;
+    if (runs_ffn(a, l)) n += 3;
   }
   return n;
 }
@@ -381,6 +407,7 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
   float *la = reinterpret_cast<float *>(base + L.la);
   float *be = reinterpret_cast<float *>(base + L.beta);
   auto *obuf = reinterpret_cast<__nv_bfloat16 *>(base + L.o);
+  auto *hmid = reinterpret_cast<__nv_bfloat16 *>(base + L.hmid);
   const int T = (int)a->total_tokens, D = a->d_model, H = a->n_heads, dk = a->d_k, dv = a->d_v;
   const int n_in = 2 * H * dk + H * dv + 2 * H;
   const float rms_eps = a->rms_eps > 0.f ? a->rms_eps : 1e-6f;
@@ -447,6 +474,33 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
                              : fail(TR_ERR_CUDA, "%s", err.c_str());
         if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
       }
+    }
+    if (runs_ffn(a, l)) {
+      // FFN sublayer on the residual the LA sublayer just wrote, in place
+      float *xr = last ? a->x_out : x;
+      e = tr::launch_rmsnorm(xr, 0, w.ffn_gain, T, D, rms_eps, xhat, s, pdl);
+      if (e != cudaSuccess) return cuda_fail(e, "FFN rmsnorm");
+      if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
+      tr::SwigluEpi sw;
+      sw.h = hmid;
+      sw.ld = a->d_ff;
+      e = tr::launch_gemm_swiglu(xhat, w.W_gate, w.W_up, T, a->d_ff, D, sw, err_word, s, pdl,
+                                 &err);
+      if (e != cudaSuccess)
+        return err.empty() ? cuda_fail(e, "FFN gate/up projection")
+                           : fail(TR_ERR_CUDA, "%s", err.c_str());
+      if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
+      tr::ResidEpi rp;
+      rp.x_res = xr;
+      rp.res_is_bf16 = 0;
+      rp.x_out = xr;
+      rp.ld = D;
+      e = tr::launch_gemm_resid(hmid, a->d_ff, w.W_down, T, D, a->d_ff, rp, err_word, s, pdl,
+                                &err);
+      if (e != cudaSuccess)
+        return err.empty() ? cuda_fail(e, "FFN down projection")
+                           : fail(TR_ERR_CUDA, "%s", err.c_str());
+      if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
     }
   }
   return TR_OK;

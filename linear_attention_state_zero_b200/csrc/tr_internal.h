@@ -38,6 +38,12 @@ struct ResidEpi {
   int64_t ld;
 };
 
+// Epilogue of the FFN's gate/up projection: h = bf16(silu(gate) * up).
+struct SwigluEpi {
+  __nv_bfloat16 *h;    // [M, ld] bf16
+  int64_t ld;          // d_ff
+};
+
 struct ScanLaunch {
   int n_seqs, H, dk, dv;
   int64_t T;
@@ -97,6 +103,12 @@ cudaError_t launch_gemm_inproj(const void *A, const void *B, int M, int N, int K
 cudaError_t launch_gemm_resid(const void *A, int64_t lda, const void *B, int M, int N, int K,
                               const ResidEpi &ep, unsigned *err_word, cudaStream_t s, bool pdl,
                               std::string *err);
+
+// h[M, d_ff] = bf16(silu(A W_gate^T) * (A W_up^T)), W_gate and W_up [d_ff, K] (d_ff a
+// multiple of 128).
+cudaError_t launch_gemm_swiglu(const void *A, const void *W_gate, const void *W_up, int M, int d_ff,
+                               int K, const SwigluEpi &ep, unsigned *err_word, cudaStream_t s,
+                               bool pdl, std::string *err);
 
 cudaError_t launch_rmsnorm(const void *x, int x_is_bf16, const float *gain, int64_t rows, int D,
                            float eps, void *out, cudaStream_t s, bool pdl);

@@ -31,5 +31,8 @@ def per_matrix_rel_fro(got, want) -> np.ndarray:
 
 def to_dev(layers, device):
     import linear_attention_state_zero_b200 as tr
-    return [tr.Layer(l.W_in.to(device), l.W_o.to(device),
-                     None if l.rms_gain is None else l.rms_gain.to(device)) for l in layers]
+    def mv(t):
+        return None if t is None else t.to(device)
+    return [tr.Layer(mv(l.W_in), mv(l.W_o), mv(l.rms_gain), mv(getattr(l, "W_gate", None)),
+                     mv(getattr(l, "W_up", None)), mv(getattr(l, "W_down", None)),
+                     mv(getattr(l, "ffn_gain", None))) for l in layers]

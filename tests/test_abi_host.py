@@ -32,7 +32,9 @@ def test_struct_layouts_match_c():
     # offsets follow the C declaration order with natural alignment
     assert ctypes.sizeof(tr.ScanArgs) == 16 + 8 + 12 + 4 + 24 + 8 * 10
     assert tr.ScanArgs.q_stride.offset == 40
-    assert ctypes.sizeof(tr.LALayer) == 24
+    assert ctypes.sizeof(tr.LALayer) == 56
+    assert tr.LALayer.W_down.offset == 48
+    assert tr.GroupArgs.d_ff.offset == 44
     assert tr.GroupArgs.h_tail.offset == 48
     assert ctypes.sizeof(tr.GroupArgs) == 48 + 6 * 8
 
@@ -81,7 +83,7 @@ def test_scan_rejects_bad_cu_seqlens():
 def _group_args(**kw):
     cu = (ctypes.c_int32 * 2)(0, 16)
     layers = (tr.LALayer * 3)(*[tr.LALayer(None, FAKE, FAKE) for _ in range(3)])
-    a = tr.GroupArgs(1, 16, 128, 128, 2048, 3, 16, 0, 0.0, 0.0, FAKE, FAKE,
+    a = tr.GroupArgs(1, 16, 128, 128, 2048, 3, 16, 0, 0.0, 0.0, 0, FAKE, FAKE,
                      ctypes.addressof(cu), layers, FAKE, None)
     for k, v in kw.items():
         setattr(a, k, v)
@@ -90,7 +92,7 @@ def _group_args(**kw):
 
 @pytest.mark.parametrize("field,value,status", [
     ("n_layers", 0, 5), ("n_layers", 65, 5), ("d_model", 100, 5), ("d_k", 32, 5),
-    ("flags", 8, 1), ("h_tail", None, 1), ("S_hat", FAKE + 8, 4), ("total_tokens", 17, 2),
+    ("flags", 16, 1), ("d_ff", 100, 5), ("d_ff", -128, 5), ("h_tail", None, 1), ("S_hat", FAKE + 8, 4), ("total_tokens", 17, 2),
 ])
 def test_replay_rejects_bad_arguments(field, value, status):
     a, keep = _group_args(**{field: value})
@@ -100,6 +102,40 @@ def test_replay_rejects_bad_arguments(field, value, status):
 def test_replay_skip_flag_forbids_x_out():
     a, keep = _group_args(flags=tr.TR_SKIP_LAST_OUTPUT, x_out=FAKE)
     assert tr.lib.tr_replay_group(ctypes.byref(a), None, 0, None) == 1
+
+
+@pytest.mark.parametrize("ffn,d_ff,status", [   # ffn = (ffn_gain, W_gate, W_up, W_down)
+    ((None, None, FAKE, FAKE), 256, 1),         # W_gate NULL but W_up/W_down given
+    ((None, FAKE, None, FAKE), 256, 1),         # W_up NULL
+    ((None, FAKE, FAKE, None), 256, 1),         # W_down NULL
+    ((None, FAKE, FAKE, FAKE + 8), 256, 4),     # misaligned W_down
+    ((FAKE + 4, FAKE, FAKE, FAKE), 256, 4),     # misaligned ffn_gain
+    ((None, FAKE, FAKE, FAKE), 0, 1),           # FFN weights with d_ff = 0
+])
+def test_replay_rejects_bad_ffn(ffn, d_ff, status):
+    a, keep = _group_args(d_ff=d_ff)
+    lw = keep[1][1]
+    lw.ffn_gain, lw.W_gate, lw.W_up, lw.W_down = ffn
+    assert tr.lib.tr_replay_group(ctypes.byref(a), None, 0, None) == status, \
+        tr.lib.tr_last_error()
+
+
+def test_replay_ffn_workspace_and_kernel_count():
+    """The FFN's hidden activation [T, d_ff] bf16 is in the workspace; each FFN that runs adds
+    three kernels, and the tail-FFN skip drops the last one."""
+    a, keep = _group_args()
+    base_ws = tr.lib.tr_replay_group_workspace_size(ctypes.byref(a))
+    base_n = tr.lib.tr_replay_group_kernel_count(ctypes.byref(a))
+    a.d_ff = 1024
+    for lw in keep[1]:
+        lw.W_gate, lw.W_up, lw.W_down = FAKE, FAKE, FAKE
+    assert tr.lib.tr_replay_group_workspace_size(ctypes.byref(a)) >= base_ws + 16 * 1024 * 2
+    # x_out NULL: the last layer's output (and so its FFN) is not computed
+    assert tr.lib.tr_replay_group_kernel_count(ctypes.byref(a)) == base_n + 2 * 3
+    a.x_out = FAKE + 4096
+    with_out = tr.lib.tr_replay_group_kernel_count(ctypes.byref(a))
+    a.flags = tr.TR_SKIP_LAST_FFN
+    assert with_out == tr.lib.tr_replay_group_kernel_count(ctypes.byref(a)) + 3
 
 
 def test_replay_workspace_checks():

@@ -1,0 +1,129 @@
+"""GPU parity of the group replay with FFN sublayers between the LA layers, against the oracle.
+
+Tail-Replay reading notes section 2.5: inside a group the FFN after every LA layer but the
+last still runs (it makes the next LA layer's input); the last layer's FFN rebuilds no state
+and is skipped.  The FFN is a dense SwiGLU with its own pre-norm (the reading used on both
+sides); the oracle restates its cast points (bf16 pre-norm output and hidden activation).
+Tolerance: relative Frobenius error 5e-3 per output tensor, as for the LA layers; at the
+full-size group, layers behind an FFN are held to 5e-3 layer by layer (teacher-forced) and to
+DRIFT_TOL end to end (the derivation is in that test)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import linear_attention_state_zero_b200 as tr
+from gpu_util import f64, per_matrix_rel_fro, rel_fro, to_dev
+
+pytestmark = pytest.mark.gpu
+
+TOL = 5e-3
+DRIFT_TOL = 1e-2   # end-to-end bar for layers after an FFN (see the paper-shape test)
+
+
+def _tails(lengths, D, seed):
+    return torch.cat([synth.hidden_prefix(max(n, 1), D, seed * 10 + i)[:n]
+                      for i, n in enumerate(lengths)])
+
+
+@pytest.mark.parametrize("skip_last_ffn", [False, True])
+def test_small_group_with_ffn_varlen(cuda_device, skip_last_ffn):
+    """Ragged requests (several 128-row tiles, a ragged tail, an empty request), d_ff = 384
+    (three 128-column gate/up tiles), RMSNorm gains on both sublayers."""
+    D, H, d, L, F = 256, 2, 128, 3, 384
+    lengths = [37, 130, 0, 201, 64]
+    layers = synth.la_layers(L, D, H, d, d, seed=311, with_gain=True, d_ff=F)
+    h = _tails(lengths, D, 311)
+    cu = synth.cu_seqlens_of(lengths)
+    S, x = tr.replay_group(h.to(cuda_device), cu, to_dev(layers, cuda_device), H, d, d,
+                           skip_last_ffn=skip_last_ffn)
+    torch.cuda.synchronize()
+    tr.check()
+    wS, wx = oracle.replay_group(h, cu, layers, H, d, d, skip_last_ffn=skip_last_ffn)
+    for l in range(L):
+        assert rel_fro(S[l], wS[l]) < TOL, l
+    nz = [0, 1, 3, 4]
+    assert np.all(per_matrix_rel_fro(S[:, nz], wS[:, nz]) < 2 * TOL)
+    assert not f64(S[:, 2]).any()
+    assert rel_fro(x, wx) < TOL
+
+
+def test_tail_ffn_skip_changes_no_state(cuda_device):
+    """The last FFN feeds no state: with and without the skip the states are bitwise equal,
+    and the skip's x_out is the residual after the last LA sublayer (oracle); zero down
+    weights make every FFN a no-op, bitwise (x + 0 = x)."""
+    D, H, d, L, F = 512, 4, 128, 3, 1024
+    lengths = [300, 77]
+    layers = synth.la_layers(L, D, H, d, d, seed=313, d_ff=F)
+    h = _tails(lengths, D, 313).to(cuda_device)
+    cu = synth.cu_seqlens_of(lengths)
+    dl = to_dev(layers, cuda_device)
+    S_run, x_run = tr.replay_group(h, cu, dl, H, d, d, skip_last_ffn=False)
+    S_skip, x_skip = tr.replay_group(h, cu, dl, H, d, d, skip_last_ffn=True)
+    S_none, _ = tr.replay_group(h, cu, dl, H, d, d, skip_last_output=True)
+    torch.cuda.synchronize()
+    tr.check()
+    assert torch.equal(S_run, S_skip) and torch.equal(S_run, S_none)
+    assert not torch.equal(x_run, x_skip)
+    _, wx = oracle.replay_group(h.cpu(), cu, layers, H, d, d, skip_last_ffn=True)
+    assert rel_fro(x_skip, wx) < TOL
+    # zero down weights
+    zl = [tr.Layer(l.W_in, l.W_o, l.rms_gain, l.W_gate, l.W_up, torch.zeros_like(l.W_down),
+                   l.ffn_gain) for l in dl]
+    plain = [tr.Layer(l.W_in, l.W_o, l.rms_gain) for l in dl]
+    S_z, x_z = tr.replay_group(h, cu, zl, H, d, d, skip_last_ffn=False)
+    S_p, x_p = tr.replay_group(h, cu, plain, H, d, d)
+    torch.cuda.synchronize()
+    assert torch.equal(S_z, S_p) and torch.equal(x_z, x_p)
+
+
+def test_group_with_ffn_paper_shape(cuda_device):
+    """One group of 3 LA layers with SwiGLU FFNs between them, d_model 2048, 16 heads of 128,
+    d_ff 5632, matched prefix m = 32768, r = 5%: the last 1639 cached hiddens replayed from a
+    zero state, the last FFN run as well (so x_out is checked too).
+
+    Two checks per layer:
+    - teacher-forced, bar 5e-3: the oracle replays layer l from the GPU's own fp32 input to
+      that layer (the x_out of the GPU replay of layers 0..l-1, which is bitwise the group's
+      intermediate: same kernels, same inputs), so only layer l's arithmetic is compared;
+    - end to end, bar 5e-3 for layer 0 and DRIFT_TOL beyond: each bf16 cast point rounds
+      slightly different values on the two sides, and the next layers amplify the flipped
+      roundings; the oracle alone, fed inputs perturbed at fp32 level (1e-6 relative),
+      drifts by 3.1e-3 and 4.5e-3 at layers 1 and 2 of this group, so twice that is the bar.
+    """
+    D, H, d, L, F, m = 2048, 16, 128, 3, 5632, 32768
+    k = tr.tail_len(m, 5, 100)
+    seed = synth.SEED_BASE + 9
+    h = synth.hidden_prefix(m, D, seed)[m - k:].contiguous()
+    layers = synth.la_layers(L, D, H, d, d, seed=seed, d_ff=F)
+    cu = synth.cu_seqlens_of([k])
+    dl = to_dev(layers, cuda_device)
+    hd = h.to(cuda_device)
+    S, x = tr.replay_group(hd, cu, dl, H, d, d, skip_last_ffn=False)
+    torch.cuda.synchronize()
+    tr.check()
+    # teacher-forced: layer l from the GPU's input to it
+    for l in range(L):
+        if l == 0:
+            x_in = h
+        else:
+            S_pre, x_in = tr.replay_group(hd, cu, dl[:l], H, d, d, skip_last_ffn=False)
+            assert torch.equal(S_pre, S[:l])                    # the prefix is the same work
+        lw = layers[l]
+        ffn = (lw.W_gate, lw.W_up, lw.W_down, lw.ffn_gain)
+        wS_l, wx_l = oracle.replay_layer(f64(x_in), lw.W_in, lw.W_o, lw.rms_gain, cu, H, d, d,
+                                         ffn=ffn)
+        assert rel_fro(S[l], wS_l) < TOL, l
+        if l == L - 1:
+            assert rel_fro(x, wx_l) < TOL
+    # end to end
+    wS, wx = oracle.replay_group(h, cu, layers, H, d, d, skip_last_ffn=False)
+    assert rel_fro(S[0], wS[0]) < TOL
+    for l in range(1, L):
+        assert rel_fro(S[l], wS[l]) < DRIFT_TOL, l
+    assert rel_fro(x, wx) < DRIFT_TOL
+    # the FFN moves the later layers' states (it is not a no-op at this size)
+    wS0, _ = oracle.replay_group(h, cu, [synth.LALayerWeights(l.W_in, l.W_o) for l in layers],
+                                 H, d, d, skip_last_output=True)
+    assert rel_fro(wS[1], wS0[1]) > 20 * TOL
