@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "replayed tokens/s & GDN scan state-updates/s on 1 B200; % of HBM/TC roofline"
 D, H, DH, L, M_PREFIX, R_NUM, R_DEN = 2048, 16, 128, 3, 32768, 5, 100
+D_FF = 5632   # FFN width of the FFN cell (2.75 d_model, a multiple of 128)
 WORKLOAD = ("one group = 1 FA + 3 LA (Gated DeltaNet) layers, d_model 2048, 16 heads "
             "d_k=d_v=128, bf16 cached h ~N(0,1), weights N(0,0.02), alpha=exp(-softplus), "
             "m=32768, r=0.05 (k=1639), batch 1")
@@ -589,6 +590,43 @@ def our_arm(args):
     tp_t = sum(tp_ms) / len(tp_ms) * 1e-3
     tr.check()
 
+    # FFN cell: the same group and tail with a dense SwiGLU FFN (d_ff = D_FF) after each LA
+    # layer but the last (the tail-FFN skip), weights drawn on the device
+    fl_dev = synth.la_layers(L, D, H, DH, DH, seed=seed + 7, device=str(dev), d_ff=D_FF)
+    frep = tr.GroupReplay(h_tail, [0, k], [tr.Layer(l.W_in, l.W_o, None, l.W_gate, l.W_up,
+                                                    l.W_down) for l in fl_dev],
+                          H, DH, DH, skip_last_output=True)
+    n_f = frep.kernel_count()
+    fev = [torch.cuda.Event(enable_timing=True) for _ in range(n_f + 1)]
+    for e in fev:
+        e.record(stream)
+    fh = [e.cuda_event for e in fev]
+    for _ in range(3):
+        frep.run(stream)
+    f_t = timed(lambda: frep.run(stream), n_ov)
+    f_kern = [0.0] * n_f
+    for _ in range(n_ov):
+        flush.zero_()
+        frep.run_profiled(fh, stream)
+        torch.cuda.synchronize()
+        for i in range(n_f):
+            f_kern[i] += fev[i].elapsed_time(fev[i + 1]) / n_ov
+    tr.check()
+    # launch order of a non-last layer: rmsnorm, in_proj, 3 scan kernels, out_proj, then the
+    # FFN's rmsnorm, gate/up (SwiGLU) and down projections
+    ffn_pos = [(9 * l + 6, 9 * l + 7, 9 * l + 8) for l in range(L - 1)] if chunked else []
+    if ffn_pos and n_f == 9 * (L - 1) + 4:
+        sw_us = sum(f_kern[b] for _, b, _ in ffn_pos) * 1e3
+        dn_us = sum(f_kern[c] for _, _, c in ffn_pos) * 1e3
+        fn_us = sum(f_kern[a] for a, _, _ in ffn_pos) * 1e3
+    else:
+        sw_us = dn_us = fn_us = float("nan")
+    sw_flops = 2.0 * k * D * 2 * D_FF          # per launch
+    dn_flops = 2.0 * k * D_FF * D
+    sw_tf = sw_flops * (L - 1) / (sw_us * 1e-6) / 1e12
+    dn_tf = dn_flops * (L - 1) / (dn_us * 1e-6) / 1e12
+    del frep, fl_dev
+
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
@@ -629,6 +667,20 @@ def our_arm(args):
             "transition_product": {
                 "workload": "P = T_t...T_1 of the scan cell's tail (32 heads, k=%d), fp32 out" % k5,
                 "us": tp_t * 1e6, "token_heads_per_s": upd / tp_t},
+            "ffn_group": {
+                "workload": "the headline group and tail with a dense SwiGLU FFN (d_ff=%d) after "
+                            "each LA layer but the last (tail-FFN skip)" % D_FF,
+                "us": f_t * 1e3, "replayed_tokens_per_s": k / (f_t * 1e-3),
+                "kernels_per_step": n_f,
+                "ffn_us_per_step": {"rmsnorm": fn_us, "gate_up_swiglu": sw_us, "down": dn_us},
+                "gate_up_roofline": {"bound": "tensor", "achieved": sw_tf,
+                                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                     "frac": sw_tf / peaks["bf16_tflops"],
+                                     "flops_per_launch": sw_flops},
+                "down_roofline": {"bound": "tensor", "achieved": dn_tf,
+                                  "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                  "frac": dn_tf / peaks["bf16_tflops"],
+                                  "flops_per_launch": dn_flops}},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "replayed tokens/s",
                     "h2d_bytes_per_step": k * D * 2,
