@@ -24,7 +24,9 @@ layer internals).
 """
 from .tail_replay import (  # noqa: F401
     bf16_round,
+    conv_state,
     ffn_residual,
+    gated_rmsnorm,
     gates,
     gdn_scan,
     in_projection,
@@ -33,6 +35,7 @@ from .tail_replay import (  # noqa: F401
     replay_group,
     replay_layer,
     rmsnorm,
+    short_conv,
     silu,
     state_error,
     tail_len,

@@ -13,6 +13,10 @@ RN section 2.3 says no model dimensions are to be made up from Eq. (1)):
     convolution, no activation on v) -> q and k L2-normalised per head
     (x / sqrt(sum x^2 + 1e-6)) -> alpha = exp(-softplus(a_alpha)),
     beta = sigmoid(a_beta) -> Eq. (1) scan -> x <- x + o W_o^T;
+  * the Gated DeltaNet details the pages leave out, each optional: a short causal
+    depthwise convolution + silu over the bf16 q, k, v projections (zero
+    history at the tail start), per-head gate parameters A_log and dt_bias,
+    and a gated RMSNorm of the readout (z rows appended to W_in after v);
   * the FFN sublayer: where a layer carries FFN weights, a dense SwiGLU with its
     own RMSNorm, x <- x + (silu(x_hat W_gate^T) * x_hat W_up^T) W_down^T, runs
     after the LA sublayer, except after a group's last LA layer (RN section 2.5,
@@ -119,11 +123,13 @@ def rmsnorm(x, gain=None, eps: float = 1e-6) -> np.ndarray:
 
 
 # ------------------------------------------------------------------------- a3
-def in_projection(x_hat, W_in, n_heads: int, d_k: int, d_v: int):
+def in_projection(x_hat, W_in, n_heads: int, d_k: int, d_v: int, output_gate: bool = False):
     """[q | k | v | a_alpha | a_beta] = x_hat W_in^T, split per head.
 
     W_in is [2 H d_k + H d_v + 2 H, D] (output features x input features).
-    Reading (pages silent): one bias-free projection, no short convolution.
+    Reading (pages silent): one bias-free projection.  With ``output_gate`` W_in
+    has H d_v more rows, [q | k | v | z | a_alpha | a_beta], and z [T, H, d_v]
+    (the output gate's input) is returned after v.
     """
     x_hat = _f64(x_hat)
     W = _f64(W_in)
@@ -134,10 +140,69 @@ def in_projection(x_hat, W_in, n_heads: int, d_k: int, d_v: int):
     q = y[:, o:o + H * d_k].reshape(T, H, d_k); o += H * d_k
     k = y[:, o:o + H * d_k].reshape(T, H, d_k); o += H * d_k
     v = y[:, o:o + H * d_v].reshape(T, H, d_v); o += H * d_v
+    z = None
+    if output_gate:
+        z = y[:, o:o + H * d_v].reshape(T, H, d_v); o += H * d_v
     a_alpha = y[:, o:o + H]; o += H
     a_beta = y[:, o:o + H]; o += H
     assert o == W.shape[0]
+    if output_gate:
+        return q, k, v, z, a_alpha, a_beta
     return q, k, v, a_alpha, a_beta
+
+
+# ----------------------------------------------------------- a3b short convolution
+def short_conv(x, w, cu_seqlens) -> np.ndarray:
+    """y_t[c] = silu(sum_j w[c, j] x_{t-W+1+j}[c]) per packed sequence, zero history.
+
+    Reading (the pages give no layer internals; this is the Gated DeltaNet layer's
+    short causal depthwise convolution): ``w`` [C, W], tap W-1 weighs the current
+    token; rows before a sequence's first token are zero (the replay starts every
+    state at zero, RN section 2.2 step 2, the convolution's included).
+    """
+    x = _f64(x)
+    w = _f64(w)
+    cu = [int(c) for c in cu_seqlens]
+    W = w.shape[1]
+    y = np.zeros_like(x)
+    for s in range(len(cu) - 1):
+        a, b = cu[s], cu[s + 1]
+        xp = np.concatenate([np.zeros((W - 1, x.shape[1])), x[a:b]], 0)
+        acc = np.zeros((b - a, x.shape[1]))
+        for j in range(W):
+            acc += w[:, j][None, :] * xp[j:j + b - a]
+        y[a:b] = acc
+    return silu(y)
+
+
+def conv_state(x, width: int, cu_seqlens) -> np.ndarray:
+    """[N, W-1, C]: each sequence's last W-1 convolution inputs, oldest first, zero where
+    the sequence is shorter (the state the convolution carries to the next token)."""
+    x = _f64(x)
+    cu = [int(c) for c in cu_seqlens]
+    out = np.zeros((len(cu) - 1, width - 1, x.shape[1]))
+    for s in range(len(cu) - 1):
+        a, b = cu[s], cu[s + 1]
+        for i in range(width - 1):
+            t = b - (width - 1) + i
+            if t >= a:
+                out[s, i] = x[t]
+    return out
+
+
+def gated_rmsnorm(o, z, gain=None, eps: float = 1e-6) -> np.ndarray:
+    """o / sqrt(mean_{d_v} o^2 + eps) * gain * silu(z), per token and head.
+
+    Reading (pages silent; the Gated DeltaNet layer's output gate and norm): the
+    readout of each head is RMS-normalised over d_v, scaled by a gain shared by the
+    heads ([d_v], ones when None) and gated by silu of a projection z of x_hat.
+    """
+    o = _f64(o)
+    z = _f64(z)
+    r = o / np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + eps)
+    if gain is not None:
+        r = r * _f64(gain)
+    return r * silu(z)
 
 
 # ------------------------------------------------------------------------- a4
@@ -151,18 +216,23 @@ def l2_normalize(x, eps: float = 1e-6) -> np.ndarray:
     return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps)
 
 
-def gates(a_alpha, a_beta):
-    """log alpha = -softplus(a_alpha), beta = sigmoid(a_beta).
+def gates(a_alpha, a_beta, A_log=None, dt_bias=None):
+    """log alpha = -exp(A_log) softplus(a_alpha + dt_bias), beta = sigmoid(a_beta).
 
     RN section 2.3 only fixes alpha in (0, 1]; the exp(-softplus) form gives
     alpha in (0, 1) and beta in (0, 1), inside the [0, 2] range of the
     non-expansive condition.  softplus(a) = max(a, 0) + log1p(exp(-|a|)) is the
-    overflow-free form of log(1 + e^a).
+    overflow-free form of log(1 + e^a).  The per-head A_log and dt_bias [H] of the
+    Gated DeltaNet layer are optional (None: A_log = 0, dt_bias = 0).
     """
     a = _f64(a_alpha)
     b = _f64(a_beta)
+    if dt_bias is not None:
+        a = a + _f64(dt_bias)[None, :]
     softplus = np.maximum(a, 0.0) + np.log1p(np.exp(-np.abs(a)))
     log_alpha = -softplus
+    if A_log is not None:
+        log_alpha = log_alpha * np.exp(_f64(A_log))[None, :]
     beta = np.where(b >= 0, 1.0 / (1.0 + np.exp(-np.abs(b))),
                     np.exp(-np.abs(b)) / (1.0 + np.exp(-np.abs(b))))
     return log_alpha, beta
@@ -284,25 +354,50 @@ def ffn_residual(x, W_gate, W_up, W_down, ffn_gain=None, rms_eps: float = 1e-6,
 # ---------------------------------------------------------------------- a2..a6
 def replay_layer(x, W_in, W_o, rms_gain, cu_seqlens, n_heads: int, d_k: int, d_v: int,
                  want_output: bool = True, emulate_casts: bool = True,
-                 rms_eps: float = 1e-6, norm_eps: float = 1e-6, n_threads=None, ffn=None):
+                 rms_eps: float = 1e-6, norm_eps: float = 1e-6, n_threads=None, ffn=None,
+                 conv_w=None, A_log=None, dt_bias=None, output_gate: bool = False,
+                 o_norm_gain=None, conv_states: Optional[list] = None):
     """One LA layer of the replay from a zero state: returns (S_hat, x_next or None).
 
     ``ffn`` = (W_gate, W_up, W_down, ffn_gain) runs the FFN sublayer on x_next
-    (``ffn_residual``); None leaves it out.
+    (``ffn_residual``); None leaves it out.  The Gated DeltaNet details the pages
+    leave out are options: ``conv_w`` [2 H d_k + H d_v, W] the short convolution
+    over the bf16 q, k, v projections (``short_conv``, zero history; its state
+    is appended to ``conv_states`` when a list is given), ``A_log``/``dt_bias``
+    the gate parameters (``gates``), ``output_gate`` the gated RMSNorm of the
+    bf16 readout (``gated_rmsnorm`` with gain ``o_norm_gain``, eps = rms_eps,
+    rounded to bf16 again).
     """
     x = _f64(x)
     cast = bf16_round if emulate_casts else (lambda a: a)
     x_hat = cast(rmsnorm(x, rms_gain, rms_eps))
-    q, k, v, a_alpha, a_beta = in_projection(x_hat, W_in, n_heads, d_k, d_v)
+    proj = in_projection(x_hat, W_in, n_heads, d_k, d_v, output_gate)
+    if output_gate:
+        q, k, v, z, a_alpha, a_beta = proj
+    else:
+        q, k, v, a_alpha, a_beta = proj
+    if conv_w is not None:
+        T = q.shape[0]
+        nq, nk = n_heads * d_k, 2 * n_heads * d_k
+        pre = cast(np.concatenate([q.reshape(T, -1), k.reshape(T, -1), v.reshape(T, -1)], 1))
+        if conv_states is not None:
+            conv_states.append(conv_state(pre, _f64(conv_w).shape[1], cu_seqlens))
+        y = short_conv(pre, conv_w, cu_seqlens)
+        q = y[:, :nq].reshape(q.shape)
+        k = y[:, nq:nk].reshape(k.shape)
+        v = y[:, nk:].reshape(v.shape)
     q = cast(l2_normalize(q, norm_eps))
     k = cast(l2_normalize(k, norm_eps))
     v = cast(v)
-    log_alpha, beta = gates(a_alpha, a_beta)
+    log_alpha, beta = gates(a_alpha, a_beta, A_log, dt_bias)
     o, S_hat = gdn_scan(q, k, v, log_alpha, beta, cu_seqlens, None, 1.0, want_o=want_output,
                         n_threads=n_threads)
     x_next = None
     if want_output:
-        x_next = out_projection_residual(x, cast(o), W_o)
+        o = cast(o)
+        if output_gate:
+            o = cast(gated_rmsnorm(o, cast(z), o_norm_gain, rms_eps))
+        x_next = out_projection_residual(x, o, W_o)
         if ffn is not None:
             W_gate, W_up, W_down, ffn_gain = ffn
             x_next = ffn_residual(x_next, W_gate, W_up, W_down, ffn_gain, rms_eps, emulate_casts)
@@ -312,7 +407,8 @@ def replay_layer(x, W_in, W_o, rms_gain, cu_seqlens, n_heads: int, d_k: int, d_v
 def replay_group(h_tail, cu_seqlens, layers: Sequence, n_heads: int, d_k: int, d_v: int,
                  emulate_casts: bool = True, skip_last_output: bool = False,
                  rms_eps: float = 1e-6, norm_eps: float = 1e-6, n_threads=None,
-                 skip_last_ffn: bool = True):
+                 skip_last_ffn: bool = True, output_gate: bool = False,
+                 conv_states: Optional[list] = None):
     """Replay one group's LA layers over the packed tails (RN section 2.2 steps 2-3).
 
     Every LA state of the group starts at zero at the tail start (step 2, GS
@@ -328,6 +424,10 @@ def replay_group(h_tail, cu_seqlens, layers: Sequence, n_heads: int, d_k: int, d
     sublayer.  With ``skip_last_output`` the last layer's readout and output
     projection are not computed either (the same argument one sublayer earlier),
     and x_out is None.
+    The optional Gated DeltaNet details (``replay_layer``) come from the layer
+    objects' conv_w, A_log, dt_bias and o_norm_gain (absent or None: not used) and
+    ``output_gate`` (every layer's W_in then carries the z rows); a list passed as
+    ``conv_states`` receives each layer's convolution state [N, W-1, C].
     """
     x = _f64(h_tail)
     S_all = []
@@ -340,7 +440,12 @@ def replay_group(h_tail, cu_seqlens, layers: Sequence, n_heads: int, d_k: int, d
         S_hat, x_next = replay_layer(x, lw.W_in, lw.W_o, lw.rms_gain, cu_seqlens, n_heads, d_k, d_v,
                                      want_output=want, emulate_casts=emulate_casts,
                                      rms_eps=rms_eps, norm_eps=norm_eps, n_threads=n_threads,
-                                     ffn=ffn)
+                                     ffn=ffn, conv_w=getattr(lw, "conv_w", None),
+                                     A_log=getattr(lw, "A_log", None),
+                                     dt_bias=getattr(lw, "dt_bias", None),
+                                     output_gate=output_gate,
+                                     o_norm_gain=getattr(lw, "o_norm_gain", None),
+                                     conv_states=conv_states)
         S_all.append(S_hat)
         x = x_next
     return np.stack(S_all, 0), x

@@ -13,6 +13,9 @@ inputs too large to draw on the host; the same seed gives the same stream):
 * ``h``: N(0, 1), rounded to bf16 (hidden vectors leaving a full-attention layer).
 * projection weights (the LA layer's and, where a layer has an FFN sublayer, its gate,
   up and down weights): N(0, 0.02^2), rounded to bf16.
+* optional Gated DeltaNet layer parameters: short-convolution taps U[-0.5, 0.5] (fp32,
+  [channels, width]); per-head A_log U[0, log 16] and dt_bias U[-7, -2] (fp32); the
+  output-gate norm gain 1 + N(0, 0.1^2).
 * scan q, k: directions drawn uniformly on the unit sphere (a normalised Gaussian
   vector), then cast to the requested dtype.
 * scan v: N(0, 1).
@@ -35,6 +38,7 @@ SEED_BASE = 0x7A110001
 # tensor ids for sub-streams
 _T_H, _T_WIN, _T_WO, _T_GAIN = 1, 2, 3, 4
 _T_WGATE, _T_WUP, _T_WDOWN, _T_FGAIN = 5, 6, 7, 8
+_T_CONV, _T_ALOG, _T_DTB, _T_OGAIN = 9, 10, 18, 19
 _T_Q, _T_K, _T_V, _T_ALPHA, _T_BETA, _T_S0, _T_LENS = 11, 12, 13, 14, 15, 16, 17
 
 
@@ -125,18 +129,26 @@ class LALayerWeights:
     W_up: Optional[torch.Tensor] = None      # bf16 [d_ff, D]
     W_down: Optional[torch.Tensor] = None    # bf16 [D, d_ff]
     ffn_gain: Optional[torch.Tensor] = None  # fp32 [D] or None (= ones)
+    # optional Gated DeltaNet layer parameters (None: not used)
+    conv_w: Optional[torch.Tensor] = None       # fp32 [2H*d_k + H*d_v, width]
+    A_log: Optional[torch.Tensor] = None        # fp32 [H]
+    dt_bias: Optional[torch.Tensor] = None      # fp32 [H]
+    o_norm_gain: Optional[torch.Tensor] = None  # fp32 [d_v]
 
 
-def in_features(n_heads: int, d_k: int, d_v: int) -> int:
-    return 2 * n_heads * d_k + n_heads * d_v + 2 * n_heads
+def in_features(n_heads: int, d_k: int, d_v: int, output_gate: bool = False) -> int:
+    return 2 * n_heads * d_k + n_heads * d_v * (2 if output_gate else 1) + 2 * n_heads
 
 
 def la_layers(n_layers: int, d_model: int, n_heads: int, d_k: int, d_v: int, seed: int,
               std: float = 0.02, device: str = "cpu", with_gain: bool = False,
-              d_ff: int = 0) -> List[LALayerWeights]:
-    """Weights of ``n_layers`` LA layers; with ``d_ff > 0`` each also gets an FFN sublayer."""
+              d_ff: int = 0, conv_width: int = 0, gate_params: bool = False,
+              output_gate: bool = False) -> List[LALayerWeights]:
+    """Weights of ``n_layers`` LA layers; with ``d_ff > 0`` each also gets an FFN sublayer,
+    with ``conv_width > 0`` short-convolution taps, with ``gate_params`` A_log and dt_bias,
+    with ``output_gate`` the z rows of W_in (after v) and the output norm's gain."""
     out = []
-    n_in = in_features(n_heads, d_k, d_v)
+    n_in = in_features(n_heads, d_k, d_v, output_gate)
     for l in range(n_layers):
         s = seed * 64 + l
         W_in = normal((n_in, d_model), s, _T_WIN, std, device).to(torch.bfloat16)
@@ -151,6 +163,14 @@ def la_layers(n_layers: int, d_model: int, n_heads: int, d_k: int, d_v: int, see
             lw.W_down = normal((d_model, d_ff), s, _T_WDOWN, std, device).to(torch.bfloat16)
             if with_gain:
                 lw.ffn_gain = 1.0 + normal((d_model,), s, _T_FGAIN, 0.1, device)
+        if conv_width > 0:
+            lw.conv_w = uniform((2 * n_heads * d_k + n_heads * d_v, conv_width), s, _T_CONV,
+                                -0.5, 0.5, device)
+        if gate_params:
+            lw.A_log = uniform((n_heads,), s, _T_ALOG, 0.0, math.log(16.0), device)
+            lw.dt_bias = uniform((n_heads,), s, _T_DTB, -7.0, -2.0, device)
+        if output_gate:
+            lw.o_norm_gain = 1.0 + normal((d_v,), s, _T_OGAIN, 0.1, device)
         out.append(lw)
     return out
 

@@ -354,6 +354,168 @@ def test_ffn_residual_invariants():
     assert 0 < rel < 2e-2
 
 
+# ------------------------------------------- Gated DeltaNet details (optional)
+def test_short_conv_against_library_convolution():
+    """Per sequence and channel, the causal convolution is numpy's full convolution with the
+    taps reversed, cut to the sequence (zero history), then silu."""
+    lengths = [7, 0, 1, 12]
+    C, W = 5, 4
+    x = rng.standard_normal((sum(lengths), C))
+    w = rng.standard_normal((C, W))
+    cu = np.cumsum([0] + lengths)
+    y = oracle.short_conv(x, w, cu)
+    for s_ in range(len(lengths)):
+        a, b = cu[s_], cu[s_ + 1]
+        if a == b:
+            continue
+        for c in range(C):
+            ref = np.convolve(x[a:b, c], w[c, ::-1])[:b - a]
+            np.testing.assert_allclose(y[a:b, c], torch.nn.functional.silu(
+                torch.from_numpy(ref)).numpy(), rtol=1e-13, atol=1e-15)
+
+
+def test_short_conv_taps_and_state():
+    """The current-token tap alone is pointwise; the oldest tap alone shifts by W-1 with zeros
+    at each sequence start; continuing a sequence from its convolution state gives the same
+    outputs as convolving it whole (the state holds the last W-1 inputs, oldest first)."""
+    lengths = [9, 2, 6]
+    C, W = 3, 4
+    x = rng.standard_normal((sum(lengths), C))
+    cu = np.cumsum([0] + lengths)
+    cur = np.zeros((C, W)); cur[:, W - 1] = 1.5
+    np.testing.assert_allclose(oracle.short_conv(x, cur, cu), oracle.silu(1.5 * x), rtol=1e-15)
+    old = np.zeros((C, W)); old[:, 0] = 1.0
+    y = oracle.short_conv(x, old, cu)
+    for s_ in range(3):
+        a, b = cu[s_], cu[s_ + 1]
+        want = np.zeros((b - a, C))
+        want[W - 1:] = x[a:b - (W - 1)] if b - a > W - 1 else want[W - 1:]
+        np.testing.assert_allclose(y[a:b], oracle.silu(want), rtol=1e-15, atol=0)
+    st = oracle.conv_state(x, W, cu)
+    assert st.shape == (3, W - 1, C)
+    np.testing.assert_array_equal(st[0], x[6:9])
+    np.testing.assert_array_equal(st[1, 0], 0.0)           # length 2 < W - 1: zero-padded
+    np.testing.assert_array_equal(st[1, 1:], x[9:11])
+    # continuation: [x_0 .. x_8] split at 5; state of the head + tail == whole
+    w = rng.standard_normal((C, W))
+    whole = oracle.short_conv(x[:9], w, [0, 9])
+    head_state = oracle.conv_state(x[:5], W, [0, 5])[0]
+    cont = oracle.short_conv(np.concatenate([head_state, x[5:9]]), w, [0, W - 1 + 4])
+    np.testing.assert_allclose(cont[W - 1:], whole[5:], rtol=1e-14)
+    assert not oracle.conv_state(np.zeros((0, C)), W, [0, 0]).any()
+
+
+def test_gated_rmsnorm_library_and_identities():
+    T, H, dv = 4, 3, 8
+    o = rng.standard_normal((T, H, dv))
+    z = rng.standard_normal((T, H, dv))
+    g = 1.0 + 0.1 * rng.standard_normal(dv)
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(o), (dv,), torch.from_numpy(g), eps=1e-6)
+    ref = ref * torch.nn.functional.silu(torch.from_numpy(z))
+    np.testing.assert_allclose(oracle.gated_rmsnorm(o, z, g, 1e-6), ref.numpy(), rtol=1e-12)
+    assert not oracle.gated_rmsnorm(o, np.zeros_like(z), g).any()           # silu(0) = 0
+    np.testing.assert_allclose(oracle.gated_rmsnorm(4.0 * o, z, g, 0.0),
+                               oracle.gated_rmsnorm(o, z, g, 0.0), rtol=1e-14)
+    c = np.full((1, 1, dv), -2.5)                                          # RMS = 2.5
+    np.testing.assert_allclose(oracle.gated_rmsnorm(c, np.ones_like(c), None, 0.0),
+                               -np.full_like(c, math.e / (1 + math.e)), rtol=1e-15)
+
+
+def test_gate_parameters():
+    """dt_bias shifts the softplus argument, exp(A_log) scales log alpha, zeros change nothing."""
+    T, H = 6, 4
+    a, b = rng.standard_normal((T, H)) * 3, rng.standard_normal((T, H))
+    la0, b0 = oracle.gates(a, b)
+    la1, b1 = oracle.gates(a, b, np.zeros(H), np.zeros(H))
+    np.testing.assert_array_equal(la0, la1)
+    np.testing.assert_array_equal(b0, b1)
+    bias = np.array([-3.0, 0.5, 2.0, -7.0])
+    np.testing.assert_allclose(oracle.gates(a, b, None, bias)[0], oracle.gates(a + bias, b)[0],
+                               rtol=1e-15)
+    A_log = np.log(np.array([1.0, 2.0, 3.0, 16.0]))
+    np.testing.assert_allclose(oracle.gates(a, b, A_log)[0], la0 * np.exp(A_log), rtol=1e-15)
+    assert np.all(oracle.gates(a, b, A_log, bias)[0] < 0)                   # alpha in (0, 1)
+
+
+def _tiny_gdn_group(lengths, D=48, H=2, dk=8, dv=8, L=2, seed=17, **kw):
+    layers = synth.la_layers(L, D, H, dk, dv, seed=seed, std=0.2, with_gain=True, **kw)
+    h = torch.cat([synth.hidden_prefix(n, D, seed + i) for i, n in enumerate(lengths)])
+    return h, layers, synth.cu_seqlens_of(lengths)
+
+
+def test_replay_short_conv_zero_history_and_state():
+    """With the convolution the tail replay gives layer 0 the same keys as the full replay
+    except for the first W-1 tail tokens, whose history the zero start drops; with the
+    current-token tap alone it drops nothing and the first layer's error identity of the
+    reading notes (section 2.3) holds again.  Each layer's returned convolution state is the
+    last W-1 rows of its bf16 pre-convolution projection."""
+    m, H, dk, W = 30, 2, 8, 4
+    kk = oracle.tail_len(m, 30, 100)                   # 9
+    a = m - kk
+    h, layers, _ = _tiny_gdn_group([m], conv_width=W)
+    lw = layers[0]
+    x_hat = oracle.bf16_round(oracle.rmsnorm(h, lw.rms_gain))
+    q, k, v, _, _ = oracle.in_projection(x_hat, lw.W_in, H, dk, dk)
+    pre = oracle.bf16_round(np.concatenate([q.reshape(m, -1), k.reshape(m, -1),
+                                            v.reshape(m, -1)], 1))
+    y_full = oracle.short_conv(pre, lw.conv_w, [0, m])
+    y_tail = oracle.short_conv(pre[a:], lw.conv_w, [0, kk])
+    np.testing.assert_array_equal(y_tail[W - 1:], y_full[a + W - 1:])
+    assert np.abs(y_tail[:W - 1] - y_full[a:a + W - 1]).max() > 1e-3
+    states = []
+    oracle.replay_group(h[a:], [0, kk], layers, H, dk, dk, conv_states=states)
+    assert len(states) == 2
+    np.testing.assert_array_equal(states[0][0], pre[m - (W - 1):])
+    # current-token tap only: the first layer's error identity holds
+    cur = [synth.LALayerWeights(l.W_in, l.W_o, l.rms_gain, conv_w=torch.zeros_like(l.conv_w))
+           for l in layers]
+    for l in cur:
+        l.conv_w[:, W - 1] = 0.8
+    S_full, _ = oracle.replay_group(h, [0, m], cur, H, dk, dk)
+    S_tail, _ = oracle.replay_group(h[a:], [0, kk], cur, H, dk, dk)
+    S_a, _ = oracle.replay_group(h[:a], [0, a], cur, H, dk, dk)
+    k0 = oracle.bf16_round(oracle.l2_normalize(oracle.silu(0.8 * pre[:, H * dk:2 * H * dk])
+                                               .reshape(m, H, dk)))
+    _, _, _, aa, ab = oracle.in_projection(x_hat, lw.W_in, H, dk, dk)
+    la, b = oracle.gates(aa, ab)
+    for hh in range(H):
+        P = np.eye(dk)
+        for i in range(a, m):
+            P = _explicit_T(math.exp(la[i, hh]), b[i, hh], k0[i, hh]) @ P
+        np.testing.assert_allclose(S_full[0, 0, hh] - S_tail[0, 0, hh], P @ S_a[0, 0, hh],
+                                   rtol=1e-9, atol=1e-12)
+
+
+def test_replay_output_gate_and_gate_parameters():
+    """The output gate acts after the scan: layer 0's states do not see it, layer 1's do; a
+    zero output-norm gain silences the attention sublayer (x passes unchanged); the gate
+    parameters change the first layer's states through alpha only."""
+    lengths = [11, 0, 6]
+    H, dk = 2, 8
+    h, layers, cu = _tiny_gdn_group(lengths, output_gate=True, gate_params=True)
+    S, x = oracle.replay_group(h, cu, layers, H, dk, dk, output_gate=True)
+    no_gp = [synth.LALayerWeights(l.W_in, l.W_o, l.rms_gain, o_norm_gain=l.o_norm_gain)
+             for l in layers]
+    S_ng, _ = oracle.replay_group(h, cu, no_gp, H, dk, dk, output_gate=True)
+    assert np.abs(S[0] - S_ng[0]).max() > 1e-6
+    # the z rows removed: the same layers without the output gate
+    n_plain = synth.in_features(H, dk, dk)
+    plain = []
+    for l in layers:
+        W = l.W_in
+        W_no_z = torch.cat([W[:2 * H * dk + H * dk], W[2 * H * dk + 2 * H * dk:]])
+        assert W_no_z.shape[0] == n_plain
+        plain.append(synth.LALayerWeights(W_no_z, l.W_o, l.rms_gain, A_log=l.A_log,
+                                          dt_bias=l.dt_bias))
+    S_p, _ = oracle.replay_group(h, cu, plain, H, dk, dk)
+    np.testing.assert_array_equal(S[0], S_p[0])
+    assert np.abs(S[1] - S_p[1]).max() > 1e-6
+    silent = [synth.LALayerWeights(l.W_in, l.W_o, l.rms_gain, A_log=l.A_log, dt_bias=l.dt_bias,
+                                   o_norm_gain=torch.zeros_like(l.o_norm_gain)) for l in layers]
+    _, x_s = oracle.replay_group(h[:11], [0, 11], silent[:1], H, dk, dk, output_gate=True)
+    np.testing.assert_array_equal(x_s, h[:11].double().numpy())
+
+
 # ---------------------------------------------------------------- a8 state error
 def test_state_error_cases():
     S = rng.standard_normal((3, 4, 5))
