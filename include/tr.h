@@ -71,7 +71,10 @@ enum {
                                 sublayer (RN section 2.5, tail-FFN skip: the next group
                                 starts from its own cached FA output, so that FFN output
                                 rebuilds no state); x_out is then the residual after the
-                                last LA sublayer */
+                                last LA sublayer */,
+  TR_OUTPUT_GATE = 16u       /* tr_replay_group(s): every layer's W_in carries H d_v more
+                                rows (z, after v) and the readout goes through the gated
+                                RMSNorm before the output projection (see below) */
 };
 
 /* Human-readable message for the last failing call on this host thread. */
@@ -177,6 +180,18 @@ tr_status tr_transition_product(const tr_scan_args *args, float *P, void *ws, si
  *   v <- bf16(v); log alpha = -softplus(a_alpha), beta = sigmoid(a_beta) (fp32)
  *   o, S_hat[layer] = tr_gdn_scan(q, k, v, log alpha, beta), zero start
  *   x <- x + bf16(o) W_o^T                     fp32 residual
+ * Optional Gated DeltaNet details (the pages omit them; these are the public Gated
+ * DeltaNet layer's, off unless asked for):
+ *   conv_width > 0: the bf16 q|k|v projections (stored without the L2 norm) go through
+ *     a causal depthwise convolution of that width and silu, with zero history at each
+ *     tail start, before the L2 norm of q and k:
+ *       y_t[c] = silu(sum_j conv_w[c][j] * x_{t-W+1+j}[c]) (fp32), q, k, v <- bf16(...)
+ *     conv_state (optional) receives each layer's convolution state: the last W-1
+ *     projected rows of every sequence, oldest first, zero-padded.
+ *   A_log, dt_bias [H] (per layer, optional):
+ *       log alpha = -exp(A_log) * softplus(a_alpha + dt_bias)
+ *   TR_OUTPUT_GATE: z = x_hat W_z^T from the extra W_in rows (bf16), and per head
+ *       o <- bf16(o / sqrt(mean_{d_v} o^2 + rms_eps) * o_norm_gain * silu(z))
  * and, where the layer has FFN weights (W_gate not NULL), the FFN sublayer that
  * RN section 2.5 says still runs between a group's LA layers (the pages do not
  * give its form; the reading is a dense SwiGLU with its own pre-norm):
@@ -190,13 +205,23 @@ tr_status tr_transition_product(const tr_scan_args *args, float *P, void *ws, si
  *   layers   HOST array of n_layers tr_la_layer:
  *              rms_gain [D] fp32 or NULL (ones)
  *              W_in     [2 H d_k + H d_v + 2 H, D] bf16 (output x input features;
- *                       rows: q heads, k heads, v heads, a_alpha, a_beta)
+ *                       rows: q heads, k heads, v heads, a_alpha, a_beta); with
+ *                       TR_OUTPUT_GATE [2 H d_k + 2 H d_v + 2 H, D], rows q, k, v,
+ *                       z heads, a_alpha, a_beta
  *              W_o      [D, H d_v] bf16
  *              ffn_gain [D] fp32 or NULL (ones)
  *              W_gate   [d_ff, D] bf16, or NULL: the layer has no FFN sublayer
  *              W_up     [d_ff, D] bf16 (with W_gate)
  *              W_down   [D, d_ff] bf16 (with W_gate)
+ *              conv_w   [2 H d_k + H d_v, conv_width] fp32, given exactly when
+ *                       conv_width > 0 (tap conv_width-1 weighs the current token)
+ *              A_log, dt_bias  [H] fp32 or NULL (0)
+ *              o_norm_gain     [d_v] fp32 or NULL (ones); only with TR_OUTPUT_GATE
  *   d_ff     FFN width, a multiple of 128; 0 when no layer has an FFN.
+ *   conv_width   0 (no convolution) or 2..4; needs d_k = d_v.
+ *   conv_state   [n_layers, N, conv_width - 1, 2 H d_k + H d_v] bf16 output, or NULL.
+ *                With it, the last layer's q projection is computed even under
+ *                TR_SKIP_LAST_OUTPUT (the state holds the q channels too).
  *   S_hat    [n_layers, N, H, d_k, d_v] fp32 output.
  *   x_out    [T, D] fp32 output of the last layer, or NULL (then the last
  *            layer's output projection and FFN are not run).  Must be NULL with
@@ -212,6 +237,10 @@ typedef struct tr_la_layer {
   const void *W_gate;
   const void *W_up;
   const void *W_down;
+  const float *conv_w;
+  const float *A_log;
+  const float *dt_bias;
+  const float *o_norm_gain;
 } tr_la_layer;
 
 typedef struct tr_group_args {
@@ -226,6 +255,8 @@ typedef struct tr_group_args {
   const tr_la_layer *layers;
   float *S_hat;
   float *x_out;
+  int32_t conv_width;
+  void *conv_state;
 } tr_group_args;
 
 size_t tr_replay_group_workspace_size(const tr_group_args *args);

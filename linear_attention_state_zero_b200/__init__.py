@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libtr.so")
 TR_OK = 0
 TR_DTYPE_F32, TR_DTYPE_BF16 = 0, 1
 TR_NORMALIZE_QK, TR_SKIP_LAST_OUTPUT, TR_SCAN_RECURRENT, TR_SKIP_LAST_FFN = 1, 2, 4, 8
+TR_OUTPUT_GATE = 16
 
 STATUS_NAMES = {0: "TR_OK", 1: "TR_ERR_INVALID_ARG", 2: "TR_ERR_SHAPE", 3: "TR_ERR_DTYPE",
                 4: "TR_ERR_ALIGNMENT", 5: "TR_ERR_UNSUPPORTED", 6: "TR_ERR_WORKSPACE",
@@ -42,7 +43,8 @@ class ScanArgs(ctypes.Structure):
 
 class LALayer(ctypes.Structure):
     _fields_ = [("rms_gain", c_vp), ("W_in", c_vp), ("W_o", c_vp), ("ffn_gain", c_vp),
-                ("W_gate", c_vp), ("W_up", c_vp), ("W_down", c_vp)]
+                ("W_gate", c_vp), ("W_up", c_vp), ("W_down", c_vp), ("conv_w", c_vp),
+                ("A_log", c_vp), ("dt_bias", c_vp), ("o_norm_gain", c_vp)]
 
 
 class GroupArgs(ctypes.Structure):
@@ -50,7 +52,8 @@ class GroupArgs(ctypes.Structure):
                 ("d_model", c_i32), ("n_layers", c_i32), ("total_tokens", c_i64),
                 ("flags", c_u32), ("rms_eps", c_f32), ("norm_eps", c_f32), ("d_ff", c_i32),
                 ("h_tail", c_vp), ("cu_seqlens", c_vp), ("cu_seqlens_host", c_vp),
-                ("layers", ctypes.POINTER(LALayer)), ("S_hat", c_vp), ("x_out", c_vp)]
+                ("layers", ctypes.POINTER(LALayer)), ("S_hat", c_vp), ("x_out", c_vp),
+                ("conv_width", c_i32), ("conv_state", c_vp)]
 
 
 # exported symbol -> (restype, argtypes)
@@ -135,6 +138,17 @@ def _need_cuda(*ts):
             raise ValueError("tensors must live on a CUDA device")
 
 
+def _need_layout(name, t, dtype, shape=None):
+    """A weight or parameter tensor must be contiguous, of the dtype the kernels read, and
+    (where given) of the expected shape; None passes."""
+    if t is None:
+        return
+    if t.dtype != dtype or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous %s tensor, got %s" % (name, dtype, t.dtype))
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+
+
 def _seqlens(cu_seqlens, device):
     """(host int32 tensor, device int32 tensor) for a cu_seqlens given either way."""
     cu = torch.as_tensor(cu_seqlens, dtype=torch.int32)
@@ -214,7 +228,9 @@ def transition_product(k, log_alpha, beta, cu_seqlens, *, normalize_qk=False, re
 class Layer:
     """One LA layer's weights, device tensors (W_in [2Hd_k + Hd_v + 2H, D], W_o [D, H d_v]),
     and, if the layer has an FFN sublayer, W_gate and W_up [d_ff, D], W_down [D, d_ff]
-    (bf16) and ffn_gain [D] fp32 (None: ones)."""
+    (bf16) and ffn_gain [D] fp32 (None: ones).  Optional Gated DeltaNet details (fp32):
+    conv_w [2Hd_k + Hd_v, width] (the short convolution), A_log and dt_bias [H] (gate
+    parameters), o_norm_gain [d_v] (the output gate's norm; W_in then has the z rows)."""
     W_in: torch.Tensor
     W_o: torch.Tensor
     rms_gain: Optional[torch.Tensor] = None
@@ -222,6 +238,10 @@ class Layer:
     W_up: Optional[torch.Tensor] = None
     W_down: Optional[torch.Tensor] = None
     ffn_gain: Optional[torch.Tensor] = None
+    conv_w: Optional[torch.Tensor] = None
+    A_log: Optional[torch.Tensor] = None
+    dt_bias: Optional[torch.Tensor] = None
+    o_norm_gain: Optional[torch.Tensor] = None
 
 
 class GroupReplay:
@@ -232,11 +252,15 @@ class GroupReplay:
     ``Layer``; FFN fields absent or None: no FFN sublayer).  Outputs: ``S_hat``
     [L, N, H, d_k, d_v] fp32 and, unless ``skip_last_output``, ``x_out`` [T, D].
     ``skip_last_ffn`` (default on, the tail-FFN skip) leaves out the last layer's FFN.
+    ``output_gate`` turns on the gated output norm (W_in with the z rows); the layers'
+    conv_w turn on the short convolution, and ``want_conv_state`` returns its state
+    ``conv_state`` [L, N, width - 1, 2Hd_k + Hd_v] bf16.
     """
 
     def __init__(self, h_tail, cu_seqlens, layers: Sequence, n_heads: int, d_k: int, d_v: int,
                  *, skip_last_output=False, want_x_out=True, rms_eps=0.0, norm_eps=0.0,
-                 skip_last_ffn=True, S_hat=None, x_out=None, workspace=None):
+                 skip_last_ffn=True, output_gate=False, want_conv_state=False,
+                 S_hat=None, x_out=None, workspace=None):
         _need_cuda(h_tail)
         if h_tail.dtype != torch.bfloat16 or not h_tail.is_contiguous():
             raise ValueError("h_tail must be contiguous bf16 [T, D]")
@@ -248,8 +272,12 @@ class GroupReplay:
         self.layers = list(layers)
         self._layer_arr = (LALayer * L)()
         d_ff = 0
+        n_in = 2 * n_heads * d_k + n_heads * d_v * (2 if output_gate else 1) + 2 * n_heads
         for i, lw in enumerate(self.layers):
             _need_cuda(lw.W_in, lw.W_o)
+            _need_layout("W_in", lw.W_in, torch.bfloat16, (n_in, D))
+            _need_layout("W_o", lw.W_o, torch.bfloat16, (D, n_heads * d_v))
+            _need_layout("rms_gain", lw.rms_gain, torch.float32, (D,))
             Wg = getattr(lw, "W_gate", None)
             Wu, Wd, fg = (getattr(lw, n, None) for n in ("W_up", "W_down", "ffn_gain"))
             if Wg is not None:
@@ -257,8 +285,27 @@ class GroupReplay:
                 if d_ff and Wg.shape[0] != d_ff:
                     raise ValueError("all FFN sublayers of a group must have one width")
                 d_ff = Wg.shape[0]
+                _need_layout("W_gate", Wg, torch.bfloat16, (d_ff, D))
+                _need_layout("W_up", Wu, torch.bfloat16, (d_ff, D))
+                _need_layout("W_down", Wd, torch.bfloat16, (D, d_ff))
+                _need_layout("ffn_gain", fg, torch.float32, (D,))
+            cw, al, db, og = (getattr(lw, n, None) for n in ("conv_w", "A_log", "dt_bias",
+                                                                 "o_norm_gain"))
+            _need_cuda(cw, al, db, og)
+            _need_layout("conv_w", cw, torch.float32)
+            if cw is not None and cw.shape[0] != 2 * n_heads * d_k + n_heads * d_v:
+                raise ValueError("conv_w must be [2 H d_k + H d_v, width]")
+            _need_layout("A_log", al, torch.float32, (n_heads,))
+            _need_layout("dt_bias", db, torch.float32, (n_heads,))
+            _need_layout("o_norm_gain", og, torch.float32, (d_v,))
+            widths = {cw.shape[1]} if cw is not None else {0}
+            if i == 0:
+                conv_width = widths.pop()
+            elif widths.pop() != conv_width:
+                raise ValueError("every layer of a group has the same convolution width")
             self._layer_arr[i] = LALayer(_ptr(lw.rms_gain), _ptr(lw.W_in), _ptr(lw.W_o),
-                                         _ptr(fg), _ptr(Wg), _ptr(Wu), _ptr(Wd))
+                                         _ptr(fg), _ptr(Wg), _ptr(Wu), _ptr(Wd), _ptr(cw),
+                                         _ptr(al), _ptr(db), _ptr(og))
         self.S_hat = S_hat if S_hat is not None else torch.empty(
             (L, N, n_heads, d_k, d_v), dtype=torch.float32, device=dev)
         if skip_last_output:
@@ -268,12 +315,17 @@ class GroupReplay:
             self.x_out = x_out if x_out is not None else torch.empty((T, D), dtype=torch.float32,
                                                                      device=dev)
         flags = (TR_SKIP_LAST_OUTPUT if skip_last_output else 0) | \
-            (TR_SKIP_LAST_FFN if skip_last_ffn else 0)
+            (TR_SKIP_LAST_FFN if skip_last_ffn else 0) | (TR_OUTPUT_GATE if output_gate else 0)
+        self.conv_state = None
+        if want_conv_state and conv_width > 0:
+            self.conv_state = torch.empty(
+                (L, N, conv_width - 1, (2 * d_k + d_v) * n_heads), dtype=torch.bfloat16,
+                device=dev)
         self.h_tail = h_tail
         self.args = GroupArgs(N, n_heads, d_k, d_v, D, L, T, flags, float(rms_eps),
                               float(norm_eps), d_ff, _ptr(h_tail), _ptr(self.dev_cu),
                               self.host.data_ptr(), self._layer_arr, _ptr(self.S_hat),
-                              _ptr(self.x_out))
+                              _ptr(self.x_out), conv_width, _ptr(self.conv_state))
         self.ws_bytes = lib.tr_replay_group_workspace_size(ctypes.byref(self.args))
         if workspace is None and self.ws_bytes:
             workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev)

@@ -79,22 +79,27 @@ __device__ __forceinline__ void epi_inproj(const InProjEpi &ep, uint32_t tbase, 
   const int dk = ep.dk;
   const int nq = 2 * ep.H * dk;          // q and k features
   const int nv = nq + ep.H * ep.dv;      // end of the v features
+  const int nz = nv + (ep.z ? ep.H * ep.dv : 0);  // end of the z features
   for (int blk = lo / dk; blk < hi / dk; ++blk) {
     const int c0 = n0 + blk * dk;  // GEMM column
     if (c0 >= N) break;
     const int g0 = c0 + ep.col_offset;  // feature index in W_in
     const uint32_t tb = tbase + (uint32_t)(c0 - n0);
     if (g0 < nq) {
-      // one q or k head: L2 norm over its d_k features (two passes over TMEM)
-      float ssq = 0.f;
-      for (int j = 0; j < dk / 32; ++j) {
-        float v[32];
-        tmem_ld32(tb + 32 * j, v);
-        tc_wait_ld();
+      // one q or k head: L2 norm over its d_k features (two passes over TMEM); raw when
+      // a convolution comes first
+      float inv = 1.f;
+      if (!ep.raw_qk) {
+        float ssq = 0.f;
+        for (int j = 0; j < dk / 32; ++j) {
+          float v[32];
+          tmem_ld32(tb + 32 * j, v);
+          tc_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) ssq = fmaf(v[i], v[i], ssq);
+          for (int i = 0; i < 32; ++i) ssq = fmaf(v[i], v[i], ssq);
+        }
+        inv = rsqrtf(ssq + ep.norm_eps);
       }
-      const float inv = rsqrtf(ssq + ep.norm_eps);
       for (int j = 0; j < dk / 32; ++j) {
         float v[32];
         tmem_ld32(tb + 32 * j, v);
@@ -112,14 +117,18 @@ __device__ __forceinline__ void epi_inproj(const InProjEpi &ep, uint32_t tbase, 
         if (row >= M) continue;
         if (g + 32 <= nv) {
           store_bf16x32(ep.qkv + (int64_t)row * ep.ldq + g, v, 1.f);
+        } else if (g + 32 <= nz) {
+          store_bf16x32(ep.z + (int64_t)row * ep.H * ep.dv + (g - nv), v, 1.f);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const int gi = g + i - nv;
+            const int gi = g + i - nz;
             if (c + i >= N) break;
-            if (gi < ep.H)
-              ep.log_alpha[(int64_t)row * ep.H + gi] = -softplus_f(v[i]);
-            else if (gi < 2 * ep.H)
+            if (gi < ep.H) {
+              const float a = v[i] + (ep.dt_bias ? ep.dt_bias[gi] : 0.f);
+              const float A = ep.A_log ? exp_ftz(ep.A_log[gi]) : 1.f;
+              ep.log_alpha[(int64_t)row * ep.H + gi] = -A * softplus_f(a);
+            } else if (gi < 2 * ep.H)
               ep.beta[(int64_t)row * ep.H + (gi - ep.H)] = sigmoid_f(v[i]);
           }
         }

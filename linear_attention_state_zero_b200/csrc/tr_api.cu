@@ -40,6 +40,7 @@ tr_status cuda_fail(cudaError_t e, const char *what) {
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // The library's device error word; kernels OR their ERRBIT_* into it.
@@ -279,11 +280,18 @@ tr_status run_scan(const tr::ScanLaunch &p, cudaStream_t s,
 
 // ------------------------------------------------------------- replay group
 struct GroupLayout {
-  size_t x, xhat, qkv, la, beta, o, hmid, scan, total;
+  size_t x, xhat, qkv, post, zbuf, la, beta, o, hmid, scan, total;
   int64_t ldq;
 };
 
 bool has_ffn(const tr_la_layer &w) { return w.W_gate != nullptr; }
+bool output_gate(const tr_group_args *a) { return (a->flags & TR_OUTPUT_GATE) != 0; }
+
+// W_in rows: [q | k | v | z (with the output gate) | a_alpha | a_beta]
+int in_rows(const tr_group_args *a) {
+  return 2 * a->n_heads * a->d_k + a->n_heads * a->d_v * (output_gate(a) ? 2 : 1) +
+         2 * a->n_heads;
+}
 
 // The scan launch of one LA layer of a group (pointers filled in by the caller).
 tr::ScanLaunch group_scan_launch(const tr_group_args *a) {
@@ -308,6 +316,8 @@ GroupLayout group_layout(const tr_group_args *a) {
   L.x = off;    off = align256(off + T * D * 4);
   L.xhat = off; off = align256(off + T * D * 2);
   L.qkv = off;  off = align256(off + T * (size_t)L.ldq * 2);
+  L.post = off; off = align256(off + (a->conv_width > 0 ? T * (size_t)L.ldq * 2 : 0));
+  L.zbuf = off; off = align256(off + (output_gate(a) ? T * H * (size_t)a->d_v * 2 : 0));
   L.la = off;   off = align256(off + T * H * 4);
   L.beta = off; off = align256(off + T * H * 4);
   L.o = off;    off = align256(off + T * H * (size_t)a->d_v * 2);
@@ -330,8 +340,16 @@ tr_status validate_group(const tr_group_args *a) {
                 a->d_v);
   if (a->d_model % 64) return fail(TR_ERR_UNSUPPORTED, "d_model = %d is not a multiple of 64",
                                    a->d_model);
-  if (a->flags & ~(unsigned)(TR_SKIP_LAST_OUTPUT | TR_SKIP_LAST_FFN))
+  if (a->flags & ~(unsigned)(TR_SKIP_LAST_OUTPUT | TR_SKIP_LAST_FFN | TR_OUTPUT_GATE))
     return fail(TR_ERR_INVALID_ARG, "unknown replay flags 0x%x", a->flags);
+  if (a->conv_width != 0 && (a->conv_width < 2 || a->conv_width > 4))
+    return fail(TR_ERR_UNSUPPORTED, "conv_width = %d (0 or 2..4 supported)", a->conv_width);
+  if (a->conv_width > 0 && a->d_k != a->d_v)
+    return fail(TR_ERR_UNSUPPORTED, "the short convolution needs d_k = d_v");
+  if (a->conv_state && a->conv_width == 0)
+    return fail(TR_ERR_INVALID_ARG, "conv_state given without a convolution");
+  if (a->conv_state && !aligned16(a->conv_state))
+    return fail(TR_ERR_ALIGNMENT, "conv_state must be 16-byte aligned");
   if (a->d_ff < 0 || a->d_ff % 128)
     return fail(TR_ERR_UNSUPPORTED, "d_ff = %d is not a non-negative multiple of 128", a->d_ff);
   if ((a->flags & TR_SKIP_LAST_OUTPUT) && a->x_out)
@@ -356,6 +374,14 @@ tr_status validate_group(const tr_group_args *a) {
     } else if (w.W_up || w.W_down || w.ffn_gain) {
       return fail(TR_ERR_INVALID_ARG, "layer %d: FFN weights without W_gate", l);
     }
+    if ((a->conv_width > 0) != (w.conv_w != nullptr))
+      return fail(TR_ERR_INVALID_ARG, "layer %d: conv_w must be given exactly when conv_width > 0",
+                  l);
+    if (w.o_norm_gain && !output_gate(a))
+      return fail(TR_ERR_INVALID_ARG, "layer %d: o_norm_gain without TR_OUTPUT_GATE", l);
+    if (!aligned4(w.conv_w) || !aligned4(w.A_log) || !aligned4(w.dt_bias) ||
+        !aligned4(w.o_norm_gain))
+      return fail(TR_ERR_ALIGNMENT, "layer %d: GDN parameters must be 4-byte aligned", l);
   }
   return check_cu_host(a->cu_seqlens_host, a->n_seqs, a->total_tokens);
 }
@@ -385,7 +411,8 @@ int group_kernel_count(const tr_group_args *a) {
     const bool last = l == a->n_layers - 1;
     const bool skip = last && (a->flags & TR_SKIP_LAST_OUTPUT);
     n += 2 + scan_kernel_count(group_scan_launch(a), !skip);
-    if (!skip && (!last || a->x_out)) n += 1;
+    if (a->conv_width > 0) n += 1;
+    if (!skip && (!last || a->x_out)) n += 1 + (output_gate(a) ? 1 : 0);
     if (runs_ffn(a, l)) n += 3;
   }
   return n;
@@ -408,8 +435,13 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
   float *be = reinterpret_cast<float *>(base + L.beta);
   auto *obuf = reinterpret_cast<__nv_bfloat16 *>(base + L.o);
   auto *hmid = reinterpret_cast<__nv_bfloat16 *>(base + L.hmid);
+  auto *post = reinterpret_cast<__nv_bfloat16 *>(base + L.post);
+  auto *zbuf = reinterpret_cast<__nv_bfloat16 *>(base + L.zbuf);
   const int T = (int)a->total_tokens, D = a->d_model, H = a->n_heads, dk = a->d_k, dv = a->d_v;
-  const int n_in = 2 * H * dk + H * dv + 2 * H;
+  const int n_in = in_rows(a);
+  const bool conv = a->conv_width > 0;
+  // q and k after the convolution (or straight from the projection)
+  const __nv_bfloat16 *qkv_s = conv ? post : qkv;
   const float rms_eps = a->rms_eps > 0.f ? a->rms_eps : 1e-6f;
   const float norm_eps = a->norm_eps > 0.f ? a->norm_eps : 1e-6f;
   const size_t state_elems = (size_t)a->n_seqs * H * dk * dv;
@@ -419,12 +451,14 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
     const tr_la_layer &w = a->layers[l];
     const bool last = l == a->n_layers - 1;
     const bool skip = last && (a->flags & TR_SKIP_LAST_OUTPUT);
+    // the q columns are still projected when the convolution state (which holds them) is kept
+    const bool skip_q = skip && !a->conv_state;
     const void *x_in = l == 0 ? a->h_tail : static_cast<const void *>(x);
     const int in_bf16 = l == 0 ? 1 : 0;
     e = tr::launch_rmsnorm(x_in, in_bf16, w.rms_gain, T, D, rms_eps, xhat, s, pdl);
     if (e != cudaSuccess) return cuda_fail(e, "rmsnorm");
     if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
-    tr::InProjEpi ep;
+    tr::InProjEpi ep{};
     ep.qkv = qkv;
     ep.ldq = L.ldq;
     ep.log_alpha = la;
@@ -432,21 +466,48 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
     ep.H = H;
     ep.dk = dk;
     ep.dv = dv;
-    ep.col_offset = skip ? H * dk : 0;
+    ep.col_offset = skip_q ? H * dk : 0;
     ep.norm_eps = norm_eps;
+    ep.raw_qk = conv ? 1 : 0;
+    ep.z = output_gate(a) ? zbuf : nullptr;
+    ep.A_log = w.A_log;
+    ep.dt_bias = w.dt_bias;
     const void *Wb = static_cast<const __nv_bfloat16 *>(w.W_in) + (size_t)ep.col_offset * D;
     e = tr::launch_gemm_inproj(xhat, Wb, T, n_in - ep.col_offset, D, ep, err_word, s, pdl, &err);
     if (e != cudaSuccess)
       return err.empty() ? cuda_fail(e, "input projection") : fail(TR_ERR_CUDA, "%s", err.c_str());
     if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
+    if (conv) {
+      tr::ShortConvLaunch cp{};
+      cp.pre = qkv;
+      cp.post = post;
+      cp.ld = L.ldq;
+      cp.w = w.conv_w;
+      cp.width = a->conv_width;
+      cp.cu_seqlens = a->cu_seqlens;
+      cp.n_seqs = a->n_seqs;
+      cp.T = T;
+      cp.H = H;
+      cp.dk = dk;
+      cp.dv = dv;
+      cp.skip_q = skip_q ? 1 : 0;
+      cp.norm_eps = norm_eps;
+      cp.state = a->conv_state
+                     ? static_cast<__nv_bfloat16 *>(a->conv_state) +
+                           (size_t)l * a->n_seqs * (a->conv_width - 1) * L.ldq
+                     : nullptr;
+      e = tr::launch_short_conv(cp, s, pdl);
+      if (e != cudaSuccess) return cuda_fail(e, "short convolution");
+      if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
+    }
     tr::ScanLaunch sp = group_scan_launch(a);
     sp.ws = base + L.scan;
     sp.ws_bytes = L.total - L.scan;
     sp.q_stride = sp.k_stride = sp.v_stride = L.ldq;
     sp.o_stride = (int64_t)H * dv;
-    sp.q = skip ? nullptr : qkv;
-    sp.k = qkv + (size_t)H * dk;
-    sp.v = qkv + (size_t)2 * H * dk;
+    sp.q = skip ? nullptr : qkv_s;
+    sp.k = qkv_s + (size_t)H * dk;
+    sp.v = qkv_s + (size_t)2 * H * dk;
     sp.log_alpha = la;
     sp.beta = be;
     sp.cu_seqlens = a->cu_seqlens;
@@ -461,6 +522,11 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
     if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
     if (!skip) {
       float *out = last ? a->x_out : x;
+      if (out && output_gate(a)) {
+        e = tr::launch_gated_norm(obuf, zbuf, w.o_norm_gain, T, H, dv, rms_eps, s, pdl);
+        if (e != cudaSuccess) return cuda_fail(e, "output gate");
+        if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
+      }
       if (out) {
         tr::ResidEpi rp;
         rp.x_res = x_in;
@@ -823,7 +889,7 @@ tr_status tr_in_projection(const void *x_hat, const void *W_in, int64_t n_tokens
   std::string err;
   if (!device_state(&dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
   const int n_in = 2 * n_heads * d_k + n_heads * d_v + 2 * n_heads;
-  tr::InProjEpi ep;
+  tr::InProjEpi ep{};
   ep.qkv = static_cast<__nv_bfloat16 *>(qkv);
   ep.ldq = 2 * (int64_t)n_heads * d_k + (int64_t)n_heads * d_v;
   ep.log_alpha = log_alpha;

@@ -28,6 +28,28 @@ struct InProjEpi {
   int H, dk, dv;
   int col_offset;      // W_in row that is GEMM column 0 (H d_k when q is skipped)
   float norm_eps;
+  // optional Gated DeltaNet details (all zero / NULL: not used)
+  int raw_qk;             // q, k stored without the L2 norm (a convolution follows)
+  __nv_bfloat16 *z;       // [M, H d_v] bf16: the output gate's input, W_in rows after v
+  const float *A_log;     // [H]: log alpha = -exp(A_log) softplus(a + dt_bias)
+  const float *dt_bias;   // [H]
+};
+
+// Short causal depthwise convolution + silu over the bf16 q/k/v projections (zero history
+// per sequence), then the per-head L2 norm of q and k, written as bf16 to `post`.
+struct ShortConvLaunch {
+  const __nv_bfloat16 *pre;  // [T, ld] bf16 (channels from col0 are read)
+  __nv_bfloat16 *post;       // [T, ld] bf16
+  int64_t ld;                // 2 H d_k + H d_v
+  const float *w;            // [2 H d_k + H d_v, width] fp32
+  int width;                 // 2..4
+  const int32_t *cu_seqlens; // device [n_seqs + 1]
+  int n_seqs;
+  int64_t T;
+  int H, dk, dv;
+  int skip_q;                // q channels neither read nor written
+  float norm_eps;
+  __nv_bfloat16 *state;      // [n_seqs, width - 1, 2 H d_k + H d_v] bf16, or NULL
 };
 
 // Epilogue of the output projection: x_out = x_res + acc (fp32 out).
@@ -109,6 +131,12 @@ cudaError_t launch_gemm_resid(const void *A, int64_t lda, const void *B, int M, 
 cudaError_t launch_gemm_swiglu(const void *A, const void *W_gate, const void *W_up, int M, int d_ff,
                                int K, const SwigluEpi &ep, unsigned *err_word, cudaStream_t s,
                                bool pdl, std::string *err);
+
+cudaError_t launch_short_conv(const ShortConvLaunch &p, cudaStream_t s, bool pdl);
+
+// o <- bf16(o / sqrt(mean_{d_v} o^2 + eps) * gain * silu(z)) per token and head, in place.
+cudaError_t launch_gated_norm(__nv_bfloat16 *o, const __nv_bfloat16 *z, const float *gain,
+                              int64_t T, int H, int dv, float eps, cudaStream_t s, bool pdl);
 
 cudaError_t launch_rmsnorm(const void *x, int x_is_bf16, const float *gain, int64_t rows, int D,
                            float eps, void *out, cudaStream_t s, bool pdl);

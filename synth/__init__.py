@@ -165,10 +165,10 @@ def la_layers(n_layers: int, d_model: int, n_heads: int, d_k: int, d_v: int, see
                 lw.ffn_gain = 1.0 + normal((d_model,), s, _T_FGAIN, 0.1, device)
         if conv_width > 0:
             lw.conv_w = uniform((2 * n_heads * d_k + n_heads * d_v, conv_width), s, _T_CONV,
-                                -0.5, 0.5, device)
+                                -0.5, 0.5, device).float()
         if gate_params:
-            lw.A_log = uniform((n_heads,), s, _T_ALOG, 0.0, math.log(16.0), device)
-            lw.dt_bias = uniform((n_heads,), s, _T_DTB, -7.0, -2.0, device)
+            lw.A_log = uniform((n_heads,), s, _T_ALOG, 0.0, math.log(16.0), device).float()
+            lw.dt_bias = uniform((n_heads,), s, _T_DTB, -7.0, -2.0, device).float()
         if output_gate:
             lw.o_norm_gain = 1.0 + normal((d_v,), s, _T_OGAIN, 0.1, device)
         out.append(lw)

@@ -31,8 +31,9 @@ def per_matrix_rel_fro(got, want) -> np.ndarray:
 
 def to_dev(layers, device):
     import linear_attention_state_zero_b200 as tr
+    import dataclasses
+
     def mv(t):
         return None if t is None else t.to(device)
-    return [tr.Layer(mv(l.W_in), mv(l.W_o), mv(l.rms_gain), mv(getattr(l, "W_gate", None)),
-                     mv(getattr(l, "W_up", None)), mv(getattr(l, "W_down", None)),
-                     mv(getattr(l, "ffn_gain", None))) for l in layers]
+    names = [f.name for f in dataclasses.fields(tr.Layer)]
+    return [tr.Layer(**{n: mv(getattr(l, n, None)) for n in names}) for l in layers]

@@ -32,11 +32,12 @@ def test_struct_layouts_match_c():
     # offsets follow the C declaration order with natural alignment
     assert ctypes.sizeof(tr.ScanArgs) == 16 + 8 + 12 + 4 + 24 + 8 * 10
     assert tr.ScanArgs.q_stride.offset == 40
-    assert ctypes.sizeof(tr.LALayer) == 56
-    assert tr.LALayer.W_down.offset == 48
+    assert ctypes.sizeof(tr.LALayer) == 88
+    assert tr.LALayer.W_down.offset == 48 and tr.LALayer.o_norm_gain.offset == 80
     assert tr.GroupArgs.d_ff.offset == 44
     assert tr.GroupArgs.h_tail.offset == 48
-    assert ctypes.sizeof(tr.GroupArgs) == 48 + 6 * 8
+    assert tr.GroupArgs.conv_width.offset == 96 and tr.GroupArgs.conv_state.offset == 104
+    assert ctypes.sizeof(tr.GroupArgs) == 112
 
 
 def test_tail_len_matches_oracle():
@@ -92,7 +93,8 @@ def _group_args(**kw):
 
 @pytest.mark.parametrize("field,value,status", [
     ("n_layers", 0, 5), ("n_layers", 65, 5), ("d_model", 100, 5), ("d_k", 32, 5),
-    ("flags", 16, 1), ("d_ff", 100, 5), ("d_ff", -128, 5), ("h_tail", None, 1), ("S_hat", FAKE + 8, 4), ("total_tokens", 17, 2),
+    ("flags", 32, 1), ("d_ff", 100, 5), ("conv_width", 5, 5), ("conv_width", 1, 5),
+    ("conv_width", 4, 1), ("conv_state", FAKE, 1), ("d_ff", -128, 5), ("h_tail", None, 1), ("S_hat", FAKE + 8, 4), ("total_tokens", 17, 2),
 ])
 def test_replay_rejects_bad_arguments(field, value, status):
     a, keep = _group_args(**{field: value})
@@ -136,6 +138,48 @@ def test_replay_ffn_workspace_and_kernel_count():
     with_out = tr.lib.tr_replay_group_kernel_count(ctypes.byref(a))
     a.flags = tr.TR_SKIP_LAST_FFN
     assert with_out == tr.lib.tr_replay_group_kernel_count(ctypes.byref(a)) + 3
+
+
+def test_replay_rejects_bad_gdn_options():
+    # d_k != d_v with the convolution
+    a, keep = _group_args(conv_width=4, d_v=64)
+    for lw in keep[1]:
+        lw.conv_w = FAKE
+    assert tr.lib.tr_replay_group(ctypes.byref(a), None, 0, None) == 5
+    # conv_w on a layer without conv_width
+    a, keep = _group_args()
+    keep[1][2].conv_w = FAKE
+    assert tr.lib.tr_replay_group(ctypes.byref(a), None, 0, None) == 1
+    # o_norm_gain without the output gate; misaligned gate parameters
+    a, keep = _group_args()
+    keep[1][0].o_norm_gain = FAKE
+    assert tr.lib.tr_replay_group(ctypes.byref(a), None, 0, None) == 1
+    a, keep = _group_args()
+    keep[1][1].A_log = FAKE + 2
+    assert tr.lib.tr_replay_group(ctypes.byref(a), None, 0, None) == 4
+    # misaligned convolution state
+    a, keep = _group_args(conv_width=4, conv_state=FAKE + 8)
+    for lw in keep[1]:
+        lw.conv_w = FAKE
+    assert tr.lib.tr_replay_group(ctypes.byref(a), None, 0, None) == 4
+
+
+def test_replay_gdn_workspace_and_kernel_count():
+    """The convolution adds one kernel per layer and a [T, 2Hd_k + Hd_v] bf16 buffer; the output
+    gate adds one kernel per computed output and a [T, H d_v] bf16 buffer."""
+    a, keep = _group_args()
+    ws0 = tr.lib.tr_replay_group_workspace_size(ctypes.byref(a))
+    n0 = tr.lib.tr_replay_group_kernel_count(ctypes.byref(a))
+    T, H, d = 16, 16, 128
+    a.conv_width = 4
+    for lw in keep[1]:
+        lw.conv_w = FAKE
+    assert tr.lib.tr_replay_group_kernel_count(ctypes.byref(a)) == n0 + 3
+    assert tr.lib.tr_replay_group_workspace_size(ctypes.byref(a)) >= ws0 + T * 3 * H * d * 2
+    a.flags = tr.TR_OUTPUT_GATE
+    # x_out NULL: outputs of layers 0 and 1 only
+    assert tr.lib.tr_replay_group_kernel_count(ctypes.byref(a)) == n0 + 3 + 2
+    assert tr.lib.tr_replay_group_workspace_size(ctypes.byref(a)) >= ws0 + T * 4 * H * d * 2
 
 
 def test_replay_workspace_checks():
