@@ -627,6 +627,43 @@ def our_arm(args):
     dn_tf = dn_flops * (L - 1) / (dn_us * 1e-6) / 1e12
     del frep, fl_dev
 
+    # GDN-options cell: the same group and tail with the short convolution (width 4), the
+    # per-head gate parameters and the gated output norm
+    gl_dev = synth.la_layers(L, D, H, DH, DH, seed=seed + 11, device=str(dev), conv_width=4,
+                             gate_params=True, output_gate=True)
+    grep_ = tr.GroupReplay(h_tail, [0, k], [tr.Layer(l.W_in, l.W_o, conv_w=l.conv_w, A_log=l.A_log,
+                                                     dt_bias=l.dt_bias, o_norm_gain=l.o_norm_gain)
+                                            for l in gl_dev],
+                           H, DH, DH, skip_last_output=True, output_gate=True)
+    n_g = grep_.kernel_count()
+    gev = [torch.cuda.Event(enable_timing=True) for _ in range(n_g + 1)]
+    for e in gev:
+        e.record(stream)
+    gh = [e.cuda_event for e in gev]
+    for _ in range(3):
+        grep_.run(stream)
+    g_t = timed(lambda: grep_.run(stream), n_ov)
+    g_kern = [0.0] * n_g
+    for _ in range(n_ov):
+        flush.zero_()
+        grep_.run_profiled(gh, stream)
+        torch.cuda.synchronize()
+        for i in range(n_g):
+            g_kern[i] += gev[i].elapsed_time(gev[i + 1]) / n_ov
+    tr.check()
+    # launch order: per non-last layer rmsnorm, in_proj, conv, 3 scan kernels, gated norm,
+    # out_proj; the last layer rmsnorm, in_proj, conv, prep, chain
+    conv_us = gn_us = float("nan")
+    if chunked and n_g == 8 * (L - 1) + 5:
+        conv_us = sum(g_kern[8 * l + 2] for l in range(L)) * 1e3
+        gn_us = sum(g_kern[8 * l + 6] for l in range(L - 1)) * 1e3
+    C_conv = 3 * H * DH
+    conv_bytes = (L - 1) * k * C_conv * 4 + k * (2 * H * DH) * 4   # bf16 in + out per channel
+    gn_bytes = (L - 1) * k * H * DH * 6                            # o, z in; o out (bf16)
+    conv_gbs = conv_bytes / (conv_us * 1e-6) / 1e9
+    gn_gbs = gn_bytes / (gn_us * 1e-6) / 1e9
+    del grep_, gl_dev
+
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
@@ -681,6 +718,17 @@ def our_arm(args):
                                   "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                                   "frac": dn_tf / peaks["bf16_tflops"],
                                   "flops_per_launch": dn_flops}},
+            "gdn_options": {
+                "workload": "the headline group and tail with the short convolution (width 4), "
+                            "per-head A_log/dt_bias and the gated output norm",
+                "us": g_t * 1e3, "replayed_tokens_per_s": k / (g_t * 1e-3),
+                "kernels_per_step": n_g,
+                "conv": {"us_per_step": conv_us, "bound": "hbm", "achieved": conv_gbs,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": conv_gbs / peaks["hbm_gbs"], "bytes_per_step": conv_bytes},
+                "gated_norm": {"us_per_step": gn_us, "bound": "hbm", "achieved": gn_gbs,
+                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                               "frac": gn_gbs / peaks["hbm_gbs"], "bytes_per_step": gn_bytes}},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "replayed tokens/s",
                     "h2d_bytes_per_step": k * D * 2,
