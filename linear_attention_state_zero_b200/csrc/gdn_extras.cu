@@ -6,8 +6,8 @@
 //                       then the per-head L2 norm of q and k; also writes each sequence's
 //                       convolution state (its last width-1 inputs)
 //   gated_norm_kernel : o <- bf16(RMSNorm_{d_v}(o) * gain * silu(z)) per token and head
-// Both are HBM-bound elementwise passes: one warp per (token, head) row segment, 16-byte
-// or 8-byte loads, fp32 arithmetic.
+// Both are HBM-bound streaming passes (each input row read once, each output row written
+// once), 8-byte or 4-byte loads per lane, fp32 arithmetic.
 #include <math.h>
 
 #include "tr_internal.h"
@@ -64,9 +64,14 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 // Segments: H q heads (d_k wide), H k heads (d_k), H v heads (d_v); all one width D here
-// (d_k = d_v = D, 64 or 128).  Items 0 .. T*n_seg-1 are (segment, token) with the token
-// fastest, so a block's warps read overlapping rows; items after that are (sequence,
-// segment) pairs that write the convolution state.
+// (d_k = d_v = D, 64 or 128).  Work units 0 .. n_chunks*n_seg-1 are (32-token chunk,
+// segment) pairs, segment fastest, so a block's warps read the same rows: the warp loads
+// its taps once, keeps the last W-1 inputs in registers and streams the chunk's rows with
+// kBatch loads in flight.  Units after that are (sequence, segment) pairs that write the
+// convolution state.
+constexpr int kTokChunk = 32;
+constexpr int kBatch = 8;
+
 template <int D, int W>
 __global__ void __launch_bounds__(kThreads)
     short_conv_kernel(ShortConvLaunch p) {
@@ -76,48 +81,82 @@ __global__ void __launch_bounds__(kThreads)
   const int lane = threadIdx.x & 31;
   const int seg0 = p.skip_q ? p.H : 0;
   const int n_seg = 3 * p.H - seg0;
-  const int64_t n_conv = p.T * n_seg;
-  const int64_t n_items = n_conv + (p.state ? (int64_t)p.n_seqs * n_seg : 0);
+  const int64_t n_chunks = (p.T + kTokChunk - 1) / kTokChunk;
+  const int64_t n_conv = n_chunks * n_seg;
+  const int64_t n_units = n_conv + (p.state ? (int64_t)p.n_seqs * n_seg : 0);
   const int64_t C = (int64_t)3 * p.H * D;
   const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
-  for (int64_t it = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); it < n_items;
-       it += warps) {
-    if (it < n_conv) {
-      const int seg = seg0 + (int)(it / p.T);
-      const int64_t t = it % p.T;
-      const int s = seq_of(p.cu_seqlens, p.n_seqs, t);
-      const int64_t start = p.cu_seqlens[s];
+  for (int64_t u = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); u < n_units;
+       u += warps) {
+    if (u < n_conv) {
+      const int seg = seg0 + (int)(u % n_seg);
+      const int64_t t0 = (u / n_seg) * kTokChunk;
+      const int64_t t1 = t0 + kTokChunk < p.T ? t0 + kTokChunk : p.T;
       const int c0 = seg * D + lane * VPL;  // first channel of this lane
+      const bool qk = seg < 2 * p.H;
       float wv[VPL][W];
 #pragma unroll
       for (int i = 0; i < VPL; ++i)
 #pragma unroll
-        for (int j = 0; j < W; ++j) wv[i][j] = p.w[(int64_t)(c0 + i) * p.width + j];
-      float y[VPL];
+        for (int j = 0; j < W; ++j) wv[i][j] = p.w[(int64_t)(c0 + i) * W + j];
+      int s = seq_of(p.cu_seqlens, p.n_seqs, t0);
+      int64_t next = p.cu_seqlens[s + 1];  // first token after this sequence
+      // history of t0: the W-1 inputs before it inside its sequence, oldest first
+      const int64_t start = p.cu_seqlens[s];
+      float hist[W - 1][VPL];
 #pragma unroll
-      for (int i = 0; i < VPL; ++i) y[i] = 0.f;
+      for (int j = 0; j < W - 1; ++j) {
+        const int64_t src = t0 - (W - 1) + j;
+        if (src >= start) {
+          load_bf16<VPL>(p.pre + src * p.ld + c0, hist[j]);
+        } else {
 #pragma unroll
-      for (int j = 0; j < W; ++j) {
-        const int64_t src = t - (W - 1) + j;
-        if (src < start) continue;
-        float x[VPL];
-        load_bf16<VPL>(p.pre + src * p.ld + c0, x);
-#pragma unroll
-        for (int i = 0; i < VPL; ++i) y[i] = fmaf(wv[i][j], x[i], y[i]);
+          for (int i = 0; i < VPL; ++i) hist[j][i] = 0.f;
+        }
       }
+      for (int64_t tb = t0; tb < t1; tb += kBatch) {
+        float xb[kBatch][VPL];
 #pragma unroll
-      for (int i = 0; i < VPL; ++i) y[i] = silu_f(y[i]);
-      if (seg < 2 * p.H) {  // q or k head: L2 norm over its D channels
-        float ssq = 0.f;
+        for (int b = 0; b < kBatch; ++b)
+          if (tb + b < t1) load_bf16<VPL>(p.pre + (tb + b) * p.ld + c0, xb[b]);
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) ssq = fmaf(y[i], y[i], ssq);
-        const float inv = rsqrtf(warp_sum(ssq) + p.norm_eps);
+        for (int b = 0; b < kBatch; ++b) {
+          const int64_t t = tb + b;
+          if (t >= t1) break;
+          if (t >= next) {  // a new sequence starts here (skipping empty ones): zero history
+            while (t >= next) next = p.cu_seqlens[++s + 1];
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) y[i] *= inv;
+            for (int j = 0; j < W - 1; ++j)
+#pragma unroll
+              for (int i = 0; i < VPL; ++i) hist[j][i] = 0.f;
+          }
+          float y[VPL];
+#pragma unroll
+          for (int i = 0; i < VPL; ++i) {
+            float acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < W - 1; ++j) acc = fmaf(wv[i][j], hist[j][i], acc);
+            y[i] = silu_f(fmaf(wv[i][W - 1], xb[b][i], acc));
+          }
+          if (qk) {  // q or k head: L2 norm over its D channels
+            float ssq = 0.f;
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) ssq = fmaf(y[i], y[i], ssq);
+            const float inv = rsqrtf(warp_sum(ssq) + p.norm_eps);
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) y[i] *= inv;
+          }
+          store_bf16<VPL>(p.post + t * p.ld + c0, y);
+#pragma unroll
+          for (int j = 0; j + 1 < W - 1; ++j)
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) hist[j][i] = hist[j + 1][i];
+#pragma unroll
+          for (int i = 0; i < VPL; ++i) hist[W - 2][i] = xb[b][i];
+        }
       }
-      store_bf16<VPL>(p.post + t * p.ld + c0, y);
     } else {
-      const int64_t r = it - n_conv;
+      const int64_t r = u - n_conv;
       const int s = (int)(r / n_seg);
       const int seg = seg0 + (int)(r % n_seg);
       const int64_t start = p.cu_seqlens[s], end = p.cu_seqlens[s + 1];
@@ -130,13 +169,16 @@ __global__ void __launch_bounds__(kThreads)
           load_bf16<VPL>(p.pre + t * p.ld + c0, x);
         } else {
 #pragma unroll
-          for (int u = 0; u < VPL; ++u) x[u] = 0.f;
+          for (int u2 = 0; u2 < VPL; ++u2) x[u2] = 0.f;
         }
         store_bf16<VPL>(p.state + ((int64_t)s * (W - 1) + i) * C + c0, x);
       }
     }
   }
 }
+
+// Rows of (token, head) with kRows rows per warp in flight.
+constexpr int kRows = 4;
 
 template <int D>
 __global__ void __launch_bounds__(kThreads)
@@ -150,18 +192,27 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
   for (int i = 0; i < VPL; ++i) g[i] = gain ? gain[lane * VPL + i] : 1.f;
   const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
-  for (int64_t r = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); r < n_rows;
-       r += warps) {
-    float v[VPL], zz[VPL];
-    load_bf16<VPL>(o + r * D + lane * VPL, v);
-    load_bf16<VPL>(z + r * D + lane * VPL, zz);
-    float ssq = 0.f;
+  for (int64_t r0 = ((int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5)) * kRows;
+       r0 < n_rows; r0 += warps * kRows) {
+    float v[kRows][VPL], zz[kRows][VPL];
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) ssq = fmaf(v[i], v[i], ssq);
-    const float inv = rsqrtf(warp_sum(ssq) * (1.f / D) + eps);
+    for (int b = 0; b < kRows; ++b) {
+      if (r0 + b < n_rows) {
+        load_bf16<VPL>(o + (r0 + b) * D + lane * VPL, v[b]);
+        load_bf16<VPL>(z + (r0 + b) * D + lane * VPL, zz[b]);
+      }
+    }
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) v[i] = v[i] * inv * g[i] * silu_f(zz[i]);
-    store_bf16<VPL>(o + r * D + lane * VPL, v);
+    for (int b = 0; b < kRows; ++b) {
+      if (r0 + b >= n_rows) break;
+      float ssq = 0.f;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) ssq = fmaf(v[b][i], v[b][i], ssq);
+      const float inv = rsqrtf(warp_sum(ssq) * (1.f / D) + eps);
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) v[b][i] = v[b][i] * inv * g[i] * silu_f(zz[b][i]);
+      store_bf16<VPL>(o + (r0 + b) * D + lane * VPL, v[b]);
+    }
   }
 }
 
@@ -187,9 +238,10 @@ cudaError_t conv_dispatch_w(const ShortConvLaunch &p, int grid, cudaStream_t s, 
 cudaError_t launch_short_conv(const ShortConvLaunch &p, cudaStream_t s, bool pdl) {
   if (p.dk != p.dv || (p.dk != 64 && p.dk != 128)) return cudaErrorInvalidValue;
   const int n_seg = 3 * p.H - (p.skip_q ? p.H : 0);
-  const int64_t items = p.T * n_seg + (p.state ? (int64_t)p.n_seqs * n_seg : 0);
-  if (items == 0) return cudaSuccess;
-  const int grid = grid_for(items);
+  const int64_t units = (p.T + kTokChunk - 1) / kTokChunk * n_seg +
+                        (p.state ? (int64_t)p.n_seqs * n_seg : 0);
+  if (units == 0) return cudaSuccess;
+  const int grid = grid_for(units);
   return p.dk == 128 ? conv_dispatch_w<128>(p, grid, s, pdl) : conv_dispatch_w<64>(p, grid, s, pdl);
 }
 
@@ -197,7 +249,7 @@ cudaError_t launch_gated_norm(__nv_bfloat16 *o, const __nv_bfloat16 *z, const fl
                               int64_t T, int H, int dv, float eps, cudaStream_t s, bool pdl) {
   const int64_t rows = T * H;
   if (rows == 0) return cudaSuccess;
-  const int grid = grid_for(rows);
+  const int grid = grid_for((rows + kRows - 1) / kRows);
   if (dv == 128)
     return launch_kernel(gated_norm_kernel<128>, dim3(grid), dim3(kThreads), 0, s, pdl, o, z, gain,
                          rows, eps);
