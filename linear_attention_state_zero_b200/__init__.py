@@ -272,6 +272,7 @@ class GroupReplay:
         self.layers = list(layers)
         self._layer_arr = (LALayer * L)()
         d_ff = 0
+        conv_width = 0
         n_in = 2 * n_heads * d_k + n_heads * d_v * (2 if output_gate else 1) + 2 * n_heads
         for i, lw in enumerate(self.layers):
             _need_cuda(lw.W_in, lw.W_o)
