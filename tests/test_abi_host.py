@@ -74,6 +74,24 @@ def test_scan_rejects_bad_arguments(field, value, status):
     assert tr.lib.tr_last_error()
 
 
+def test_transition_product_checks():
+    """tr_transition_product sizes its workspace (the zero v and the identities, then the
+    scan's) and rejects bad arguments before any device work."""
+    a, cu = _scan_args()
+    need = tr.lib.tr_transition_product_workspace_size(ctypes.byref(a))
+    T, H, d, N = 9, 4, 128, 2
+    assert need >= T * H * d * 2 + N * H * d * d * 4
+    tp = tr.lib.tr_transition_product
+    assert tp(ctypes.byref(a), None, FAKE, need, None) == 1          # P NULL
+    assert tp(ctypes.byref(a), FAKE + 4, FAKE, need, None) == 4      # P misaligned
+    assert tp(ctypes.byref(a), FAKE, None, need, None) == 6          # no workspace
+    assert tp(ctypes.byref(a), FAKE, FAKE, need - 1, None) == 6      # too small
+    assert tp(ctypes.byref(a), FAKE, FAKE + 16, need, None) == 4     # not 256-byte aligned
+    b, cu_b = _scan_args(d_k=96)
+    assert tr.lib.tr_transition_product_workspace_size(ctypes.byref(b)) == 0
+    assert tp(ctypes.byref(b), FAKE, FAKE, 1 << 30, None) == 5
+
+
 def test_scan_rejects_bad_cu_seqlens():
     a, _ = _scan_args()
     bad = (ctypes.c_int32 * 3)(0, 6, 5)

@@ -680,6 +680,21 @@ def test_transition_product_identity_and_bound():
         assert np.linalg.norm(P[0, h], 2) <= math.exp(la[:, h].sum()) * (1 + 1e-12)
 
 
+def test_transition_product_composes():
+    """The operator of a span is the later part's times the earlier part's, for any split
+    (T_m ... T_1 = (T_m ... T_{c+1})(T_c ... T_1)), and a packed batch of two spans gives
+    each span's operator."""
+    q, k, v, la, b = _rand_scan(30, 2, 8, 4, seed=35)
+    P_all = oracle.transition_product(k, la, b, [0, 30])[0]
+    for c in (1, 12, 29):
+        P_pair = oracle.transition_product(k, la, b, [0, c, 30])
+        for h in range(2):
+            np.testing.assert_allclose(P_pair[1, h] @ P_pair[0, h], P_all[h], rtol=1e-12,
+                                       atol=1e-15)
+        np.testing.assert_allclose(P_pair[0], oracle.transition_product(
+            k[:c], la[:c], b[:c], [0, c])[0], rtol=1e-15, atol=0)
+
+
 def test_transition_product_repairs_the_tail():
     """The repair the operator makes possible: with an exact earlier state S_a, the full
     state is S_m = P S_a + S_hat_m exactly (reading notes section 2.3, E_m = P S_a)."""
