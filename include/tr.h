@@ -293,7 +293,8 @@ tr_status tr_replay_groups(const tr_group_args *groups, int32_t n_groups, void *
  * issued before the replay's kernels on `stream`; `stream` then waits for the copy, so
  * work enqueued on it afterwards sees both the KV and the states.  One cudaMemcpyAsync;
  * kv_bytes = 0 replays only.  The two streams must differ.  Same workspace as
- * tr_replay_groups.
+ * tr_replay_groups.  Every argument (the KV pointers and streams, each group, the
+ * workspace) is checked before the copy is issued: a rejected call moves no bytes.
  */
 tr_status tr_replay_groups_overlapped(const tr_group_args *groups, int32_t n_groups, void *ws,
                                       size_t ws_bytes, const void *kv_host, void *kv_dev,

@@ -620,6 +620,27 @@ tr_status tp_layout(const tr_scan_args *a, TpLayout *L, tr::ScanLaunch *p) {
   return TR_OK;
 }
 
+// The group array, every group and the shared workspace of tr_replay_groups.
+tr_status validate_groups(const tr_group_args *groups, int32_t n_groups, const void *ws,
+                          size_t ws_bytes) {
+  if (n_groups < 0 || (n_groups > 0 && !groups))
+    return fail(TR_ERR_INVALID_ARG, "bad group array");
+  size_t need = 0;
+  for (int32_t g = 0; g < n_groups; ++g) {
+    tr_status st = validate_group(&groups[g]);
+    if (st != TR_OK) {
+      std::string m = g_last_error;
+      return fail(st, "group %d: %s", g, m.c_str());
+    }
+    need = std::max(need, group_layout(&groups[g]).total);
+  }
+  if (need > 0 && (!ws || ws_bytes < need))
+    return fail(TR_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", ws_bytes, need);
+  if (need > 0 && (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(TR_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  return TR_OK;
+}
+
 }  // namespace
 
 // ============================================================== extern "C"
@@ -774,21 +795,8 @@ size_t tr_replay_groups_workspace_size(const tr_group_args *groups, int32_t n_gr
 
 tr_status tr_replay_groups(const tr_group_args *groups, int32_t n_groups, void *ws,
                            size_t ws_bytes, void *stream) {
-  if (n_groups < 0 || (n_groups > 0 && !groups))
-    return fail(TR_ERR_INVALID_ARG, "bad group array");
-  size_t need = 0;
-  for (int32_t g = 0; g < n_groups; ++g) {
-    tr_status st = validate_group(&groups[g]);
-    if (st != TR_OK) {
-      std::string m = g_last_error;
-      return fail(st, "group %d: %s", g, m.c_str());
-    }
-    need = std::max(need, group_layout(&groups[g]).total);
-  }
-  if (need > 0 && (!ws || ws_bytes < need))
-    return fail(TR_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", ws_bytes, need);
-  if (need > 0 && (reinterpret_cast<uintptr_t>(ws) & 255u))
-    return fail(TR_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  tr_status vst = validate_groups(groups, n_groups, ws, ws_bytes);
+  if (vst != TR_OK) return vst;
   int dev;
   unsigned *errw;
   std::string err;
@@ -806,6 +814,9 @@ tr_status tr_replay_groups_overlapped(const tr_group_args *groups, int32_t n_gro
   if (kv_bytes > 0 && (!kv_host || !kv_dev)) return fail(TR_ERR_INVALID_ARG, "KV pointer is NULL");
   if (kv_bytes > 0 && stream == copy_stream)
     return fail(TR_ERR_INVALID_ARG, "the copy needs a stream of its own");
+  // every argument is checked before the copy starts, so a rejected call moves no bytes
+  tr_status vst = validate_groups(groups, n_groups, ws, ws_bytes);
+  if (vst != TR_OK) return vst;
   cudaStream_t s = static_cast<cudaStream_t>(stream), cs = static_cast<cudaStream_t>(copy_stream);
   cudaEvent_t done = nullptr;
   if (kv_bytes > 0) {

@@ -200,6 +200,24 @@ def test_replay_gdn_workspace_and_kernel_count():
     assert tr.lib.tr_replay_group_workspace_size(ctypes.byref(a)) >= ws0 + T * 4 * H * d * 2
 
 
+def test_overlapped_replay_checks_everything_before_the_copy():
+    """tr_replay_groups_overlapped rejects its KV arguments and every group argument before
+    it issues the copy (a rejected call moves no bytes and needs no device)."""
+    a, keep = _group_args()
+    arr = (tr.GroupArgs * 1)(a)
+    need = tr.lib.tr_replay_groups_workspace_size(arr, 1)
+    ov = tr.lib.tr_replay_groups_overlapped
+    S1, S2 = FAKE, FAKE + 64          # two distinct stream handles (never used)
+    assert ov(arr, 1, FAKE, need, FAKE, FAKE, 4096, S1, S1) == 1      # one stream for both
+    assert ov(arr, 1, FAKE, need, None, FAKE, 4096, S1, S2) == 1      # KV source NULL
+    assert ov(arr, 1, FAKE, need - 1, FAKE, FAKE, 4096, S1, S2) == 6  # workspace too small
+    bad = (tr.GroupArgs * 2)(a, a)
+    bad[1].n_layers = 0
+    assert ov(bad, 2, FAKE, need, FAKE, FAKE, 4096, S1, S2) == 5      # group 1 invalid
+    assert "group 1" in tr.lib.tr_last_error().decode()
+    assert ov(arr, -1, FAKE, need, FAKE, FAKE, 4096, S1, S2) == 1
+
+
 def test_replay_workspace_checks():
     a, keep = _group_args()
     need = tr.lib.tr_replay_group_workspace_size(ctypes.byref(a))
