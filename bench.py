@@ -268,8 +268,15 @@ class ClockSampler:
             self.proc.kill()
         self.tmp.flush()
         self.tmp.seek(0)
-        rows = [r for r in csv.reader(io.StringIO(self.tmp.read())) if len(r) >= 9]
+        text = self.tmp.read()
         os.unlink(self.tmp.name)
+        return self.summarize(text)
+
+    @staticmethod
+    def summarize(text):
+        """Median SM clock, the largest max clock and every throttle reason seen active, from
+        `nvidia-smi --query-gpu=FIELDS --format=csv,noheader,nounits` lines."""
+        rows = [r for r in csv.reader(io.StringIO(text)) if len(r) >= 9]
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:

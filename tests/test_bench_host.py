@@ -89,3 +89,22 @@ def test_kernel_rooflines_aggregate_one_step():
 
 def test_job_throughput_is_all_ranks_over_the_slowest():
     assert bench.job_throughput(K, 4, 2.0) == pytest.approx(4 * K / 2e-3)
+
+
+def test_clock_summary_from_nvidia_smi_lines():
+    """The clocks key: median SM clock under load, the max clock, and every throttle reason
+    that was active in any sample (a run that saw a hardware or thermal slowdown is rejected
+    by the driver, so none may be lost); malformed lines are skipped."""
+    lines = [
+        "0, 1965, 1965, 812.3, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1950, 1965, 990.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1800, 1965, 1001.0, 0x0000000000000008, Active, Not Active, Not Active, Active",
+        "0, [N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "garbage",
+    ]
+    r = bench.ClockSampler.summarize("\n".join(lines) + "\n")
+    assert r["samples"] == 3
+    assert r["sm_mhz"] == 1950.0 and r["sm_max_mhz"] == 1965.0
+    assert r["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    empty = bench.ClockSampler.summarize("")
+    assert empty["sm_mhz"] is None and empty["samples"] == 0 and empty["reasons"] == []
