@@ -516,6 +516,30 @@ def test_replay_output_gate_and_gate_parameters():
     np.testing.assert_array_equal(x_s, h[:11].double().numpy())
 
 
+def test_replay_ffn_with_gdn_options():
+    """With the FFN and every Gated DeltaNet option in one group: layer 0's states see no
+    FFN, the last FFN changes no state, and zero down weights give the FFN-free group."""
+    lengths = [14, 5]
+    H, dk = 2, 8
+    h, layers, cu = _tiny_gdn_group(lengths, L=3, conv_width=3, gate_params=True,
+                                    output_gate=True, d_ff=32)
+    S_f, x_f = oracle.replay_group(h, cu, layers, H, dk, dk, output_gate=True,
+                                   skip_last_ffn=False)
+    S_s, _ = oracle.replay_group(h, cu, layers, H, dk, dk, output_gate=True)
+    no_ffn = [synth.LALayerWeights(l.W_in, l.W_o, l.rms_gain, conv_w=l.conv_w, A_log=l.A_log,
+                                   dt_bias=l.dt_bias, o_norm_gain=l.o_norm_gain) for l in layers]
+    S_n, x_n = oracle.replay_group(h, cu, no_ffn, H, dk, dk, output_gate=True)
+    np.testing.assert_array_equal(S_f, S_s)
+    np.testing.assert_array_equal(S_f[0], S_n[0])
+    assert np.abs(S_f[1] - S_n[1]).max() > 1e-6
+    zero = [synth.LALayerWeights(l.W_in, l.W_o, l.rms_gain, l.W_gate, l.W_up,
+                                 torch.zeros_like(l.W_down), None, l.conv_w, l.A_log, l.dt_bias,
+                                 l.o_norm_gain) for l in layers]
+    S_z, x_z = oracle.replay_group(h, cu, zero, H, dk, dk, output_gate=True, skip_last_ffn=False)
+    np.testing.assert_array_equal(S_z, S_n)
+    np.testing.assert_array_equal(x_z, x_n)
+
+
 # ---------------------------------------------------------------- a8 state error
 def test_state_error_cases():
     S = rng.standard_normal((3, 4, 5))
