@@ -50,6 +50,8 @@ def parse():
                    help="reference arm: tail tokens per timed step (a bounded sample)")
     p.add_argument("--profile", choices=["scan", "group"], default=None,
                    help="run only one workload a few times (for ncu captures), no JSON line")
+    p.add_argument("--no-configs", action="store_true",
+                   help="skip the other workload configurations (1, 3, 4 and the sweep)")
     return p.parse_args()
 
 
@@ -160,7 +162,7 @@ KERNEL_DESC = {
     "scan_chain": "chunked scan, chunk-to-chunk state chain (bytes: final state out)",
     "scan_out": "chunked scan, readout (bytes: o out)",
     "out_proj": "out-proj tcgen05 GEMM + residual (flops)",
-    "scan": "token-recurrent scan (bytes: q, k, v, gates in, o out)",
+    "scan_recurrent": "token-recurrent scan (bytes: q, k, v, gates in, o out)",
 }
 
 
@@ -174,25 +176,30 @@ def kernel_work(name, layer, k):
     if name == "scan_prep":
         return "hbm", k * H * ((2 if last else 3) * DH * 2 + 8)
     if name == "scan_chain":
-        return "hbm", H * DH * DH * 4
+        # the final state out, plus o when the readout is fused into the chain
+        return "hbm", H * DH * DH * 4 + (0 if last or "scan_out" in KERNELS_SEEN else k * H * DH * 2)
     if name == "scan_out":
         return "hbm", k * H * DH * 2
     if name == "out_proj":
         return "tensor", flops_outproj(k)
-    if name == "scan":
+    if name == "scan_recurrent":
         return "hbm", k * H * ((2 if last else 3) * DH * 2 + 8 + (0 if last else DH * 2))
     raise KeyError(name)
+
+
+KERNELS_SEEN = set()
 
 
 def kernel_rooflines(names, avg_ms, k, peaks):
     """Per kernel (summed over the layers): achieved algorithmic rate / measured peak."""
     out = {}
-    layer, seen = 0, set()
+    layer = -1
     work, ms, launches, bound = {}, {}, {}, {}
+    KERNELS_SEEN.clear()
+    KERNELS_SEEN.update(names)
     for n, t in zip(names, avg_ms):
-        if n in seen and n == "rmsnorm":
+        if n == "rmsnorm":
             layer += 1
-        seen.add(n)
         b, w = kernel_work(n, layer, k)
         bound[n] = b
         work[n] = work.get(n, 0.0) + w
@@ -291,6 +298,244 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+# ------------------------------------------------------- the other configurations
+SWEEP_M = [4096, 8192, 16384, 32768, 65536, 131072]
+SWEEP_R = [1, 2, 5, 10, 20, 100]   # percent
+
+
+def _timer(stream, flush):
+    """fn, n -> mean ms of n device-timed calls, L2 flushed before each (outside the timing)."""
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(fn, n):
+        ts = []
+        for _ in range(n):
+            flush.zero_()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return sum(ts) / len(ts)
+    return timed
+
+
+def _group_flops_bytes(T, Dm, Hh, d, n_layers, n_groups, d_in_bytes=2):
+    """Algorithmic FLOPs and bytes of replaying n_groups groups of n_layers LA layers over T
+    tail tokens (last layer's readout skipped): projections + chunked scan; weights once per
+    group, the h tails in, the states out."""
+    F = Bw = 0.0
+    for l in range(n_layers):
+        last = l == n_layers - 1
+        n_in = 3 * Hh * d + 2 * Hh - (Hh * d if last else 0)
+        F += 2.0 * T * Dm * n_in + (0 if last else 2.0 * T * Hh * d * Dm)
+        Bw += n_in * Dm * 2 + (0 if last else Dm * Hh * d * 2)
+    F += n_layers * T * Hh * scan_flops_per_token_head(dk=d, dv=d)
+    F *= n_groups
+    B = n_groups * (Bw + T * Dm * d_in_bytes) + 0.0
+    return F, B
+
+
+def config_cells(dev, peaks, stream, flush, n_rep, cpu):
+    """Configurations 1, 3, 4 and the scan sweep: throughput, roofline fraction, state errors
+    and (with cpu) the oracle's rate on a bounded sample of each."""
+    import torch
+    import synth
+    import linear_attention_state_zero_b200 as tr
+    timed = _timer(stream, flush)
+    out = {}
+
+    # ---- 1: single head, fp32, d = 64, m = 4096, r = 5% (k = 205): the fp32 test path
+    m1 = 4096
+    k1 = tr.tail_len(m1, 5, 100)
+    full, tail = synth.scan_case_from_prefix(m1, k1, 1, 64, 64, torch.float32, 0.90, 1.00,
+                                             seed=synth.SEED_BASE + 0)
+    fd = [x.to(dev) for x in (full.q, full.k, full.v, full.log_alpha, full.beta)]
+    td = [x.to(dev) for x in (tail.q, tail.k, tail.v, tail.log_alpha, tail.beta)]
+    o1 = torch.empty_like(td[2])
+    S1m = torch.empty(1, 1, 64, 64, device=dev)
+    S1h = torch.empty_like(S1m)
+    cu_t, cu_f = tr.seqlens(tail.cu_seqlens, dev), tr.seqlens(full.cu_seqlens, dev)
+    run_tail = lambda: tr.gdn_scan(*td, cu_t, o=o1, S_final=S1h)
+    run_full = lambda: tr.gdn_scan(*fd, cu_f, want_o=False, S_final=S1m)
+    for _ in range(3):
+        run_tail(); run_full()
+    t_tail = timed(run_tail, n_rep) * 1e-3
+    t_full = timed(run_full, n_rep) * 1e-3
+    _, tot1 = tr.state_error(S1m.reshape(-1, 64, 64), S1h.reshape(-1, 64, 64), per_mat=False)
+    by1 = k1 * (3 * 64 * 4 + 8 + 64 * 4) + 64 * 64 * 4
+    c1 = {"workload": "single-head Gated DeltaNet scan, fp32, d_k=d_v=64, m=4096, r=0.05 "
+                      "(k=205), alpha~U[0.90,1]",
+          "tail_us": t_tail * 1e6, "state_updates_per_s": k1 / t_tail,
+          "full_prefill_us": t_full * 1e6, "full_prefill_state_updates_per_s": m1 / t_full,
+          "state_error": float(tot1.item()),
+          "roofline": {"bound": "latency", "achieved": by1 / t_tail / 1e9, "unit": "GB/s",
+                       "peak": peaks["hbm_gbs"], "frac": by1 / t_tail / 1e9 / peaks["hbm_gbs"],
+                       "note": "one head of 205 tokens: a chain of 205 dependent updates; "
+                               "reported for information"}}
+    if cpu:
+        import oracle
+        t0 = time.perf_counter()
+        reps = 0
+        while reps < 3 or time.perf_counter() - t0 < 1.0:
+            oracle.gdn_scan(tail.q, tail.k, tail.v, tail.log_alpha, tail.beta, tail.cu_seqlens)
+            reps += 1
+        c1["cpu_baseline"] = {"value": k1 * reps / (time.perf_counter() - t0),
+                              "unit": "state-updates/s", "cores": os.cpu_count(),
+                              "kind": "oracle", "sample": "the whole k=205 tail, %d runs" % reps}
+    out["config1_fp32_single_head"] = c1
+    del fd, td
+
+    # ---- 3: 8 concurrent hits x 8 groups x 3 LA layers, d_model 2048, 16 heads, m = 32768
+    Dm, Hh, d, Lg, G, N, m3 = 2048, 16, 128, 3, 8, 8, 32768
+    base = synth.SEED_BASE + 2
+    layers3 = [synth.la_layers(Lg, Dm, Hh, d, d, seed=base * 16 + g, device=str(dev))
+               for g in range(G)]
+    for r_num in (5, 10):
+        k3 = tr.tail_len(m3, r_num, 100)
+        cu3 = synth.cu_seqlens_of([k3] * N)
+        hs = [synth.hidden_prefix(N * k3, Dm, base * 1024 + 8 * g + r_num, device=str(dev))
+              for g in range(G)]
+        reps = [tr.GroupReplay(hs[g], cu3, [tr.Layer(l.W_in, l.W_o) for l in layers3[g]],
+                               Hh, d, d, skip_last_output=True) for g in range(G)]
+        grp = tr.GroupsReplay(reps)
+        for _ in range(2):
+            grp.run(stream)
+        t3 = timed(lambda: grp.run(stream), max(3, n_rep // 4)) * 1e-3
+        tr.check()
+        F3, B3 = _group_flops_bytes(N * k3, Dm, Hh, d, Lg, G)
+        t_roof = max(F3 / (peaks["bf16_tflops"] * 1e12), B3 / (peaks["hbm_gbs"] * 1e9))
+        c3 = {"workload": "8 concurrent hits x 8 groups x 3 LA layers, d_model 2048, 16 heads "
+                          "d=128, m=32768, r=%.2f (k=%d), one tr_replay_groups call" % (r_num / 100, k3),
+              "us": t3 * 1e6, "replayed_tokens_per_s": N * k3 / t3,
+              "token_layers_per_s": N * k3 * G * Lg / t3,
+              "state_updates_per_s": N * k3 * G * Lg * Hh / t3,
+              "roofline": {"bound": "tensor", "t_roof_us": t_roof * 1e6, "alg_flops": F3,
+                           "alg_bytes": B3, "achieved": F3 / t3 / 1e12, "unit": "TFLOP/s",
+                           "peak": peaks["bf16_tflops"], "frac": t_roof / t3}}
+        out["config3_8hits_8groups_r%02d" % r_num] = c3
+        del grp, reps, hs
+    if cpu:
+        import oracle
+        lc = synth.la_layers(Lg, Dm, Hh, d, d, seed=base * 16)
+        hcpu = synth.hidden_prefix(128, Dm, base)
+        t0 = time.perf_counter()
+        oracle.replay_group(hcpu, [0, 128], lc, Hh, d, d, skip_last_output=True)
+        dt = time.perf_counter() - t0
+        for r_num in (5, 10):
+            out["config3_8hits_8groups_r%02d" % r_num]["cpu_baseline"] = {
+                "value": 128 / dt / G, "unit": "replayed tokens/s", "cores": os.cpu_count(),
+                "kind": "oracle",
+                "sample": "128 tail tokens through one group's 3 LA layers (%.1f s), "
+                          "extrapolated to 8 groups" % dt}
+    del layers3
+
+    # ---- 4: 64 requests, m ~ U[1024, 131072], r = 10%, d_model 4096, 32 heads, 8 groups x 3
+    Dm, Hh, G, n = 4096, 32, 8, 64
+    seed = synth.SEED_BASE + 3
+    ms = synth.varlen_prefix_lengths(n, 1024, 131072, seed)
+    ks = [tr.tail_len(mi, 10, 100) for mi in ms]
+    cu4 = synth.cu_seqlens_of(ks)
+    T4 = int(cu4[-1])
+    # the packed tails (about 3.5 GB), drawn on the device and shared by the 8 groups: the
+    # groups' cost does not depend on the values
+    h4 = synth.hidden_prefix(T4, Dm, seed, device=str(dev))
+    layers4 = [synth.la_layers(Lg, Dm, Hh, d, d, seed=seed * 16 + g, device=str(dev))
+               for g in range(G)]
+    reps = [tr.GroupReplay(h4, cu4, [tr.Layer(l.W_in, l.W_o) for l in layers4[g]], Hh, d, d,
+                           skip_last_output=True) for g in range(G)]
+    grp = tr.GroupsReplay(reps)
+    grp.run(stream)
+    torch.cuda.synchronize()
+    t4 = timed(lambda: grp.run(stream), 2) * 1e-3
+    tr.check()
+    F4, B4 = _group_flops_bytes(T4, Dm, Hh, d, Lg, G)
+    t_roof = max(F4 / (peaks["bf16_tflops"] * 1e12), B4 / (peaks["hbm_gbs"] * 1e9))
+    c4 = {"workload": "varlen batch of 64 requests, m~U[1024,131072] packed via cu_seqlens, "
+                      "r=0.10 (sum k=%d), d_model 4096, 32 heads d=128, 8 groups x 3 LA layers, "
+                      "one tr_replay_groups call (the 8 groups share one packed h buffer)" % T4,
+          "us": t4 * 1e6, "replayed_tokens_per_s": T4 / t4,
+          "token_layers_per_s": T4 * G * Lg / t4, "state_updates_per_s": T4 * G * Lg * Hh / t4,
+          "max_k": max(ks), "min_k": min(ks),
+          "roofline": {"bound": "tensor", "t_roof_us": t_roof * 1e6, "alg_flops": F4,
+                       "alg_bytes": B4, "achieved": F4 / t4 / 1e12, "unit": "TFLOP/s",
+                       "peak": peaks["bf16_tflops"], "frac": t_roof / t4}}
+    if cpu:
+        import oracle
+        lc = synth.la_layers(Lg, Dm, Hh, d, d, seed=seed * 16)
+        hcpu = synth.hidden_prefix(64, Dm, seed)
+        t0 = time.perf_counter()
+        oracle.replay_group(hcpu, [0, 64], lc, Hh, d, d, skip_last_output=True)
+        dt = time.perf_counter() - t0
+        c4["cpu_baseline"] = {"value": 64 / dt / G, "unit": "replayed tokens/s",
+                              "cores": os.cpu_count(), "kind": "oracle",
+                              "sample": "64 tail tokens through one group's 3 LA layers (%.1f s),"
+                                        " extrapolated to 8 groups" % dt}
+    out["config4_varlen_64req_d4096"] = c4
+    del grp, reps, h4, layers4
+    torch.cuda.empty_cache()
+
+    # ---- 5: the scan sweep, 32 heads d = 128, bf16, alpha ~ U[0.80, 1] and U[0.97, 1]
+    Hh = 32
+    cells = []
+    gen = torch.Generator(device=dev)
+    for alpha_lo in (0.80, 0.97):
+        for mi, m in enumerate(SWEEP_M):
+            gen.manual_seed(synth.SEED_BASE + 4 + 16 * mi + (0 if alpha_lo == 0.80 else 8))
+            # inputs drawn on the device with the sweep's distributions (unit q, k; N(0,1) v;
+            # alpha ~ U[alpha_lo, 1]; beta = sigmoid(N(0,1)))
+            def unit(shape):
+                x = torch.randn(*shape, generator=gen, device=dev)
+                return (x / x.norm(dim=-1, keepdim=True)).to(torch.bfloat16)
+            q, kk = unit((m, Hh, d)), unit((m, Hh, d))
+            v = torch.randn(m, Hh, d, generator=gen, device=dev).to(torch.bfloat16)
+            la = torch.log(alpha_lo + (1 - alpha_lo) * torch.rand(m, Hh, generator=gen, device=dev))
+            be = torch.sigmoid(torch.randn(m, Hh, generator=gen, device=dev))
+            S_m = torch.empty(1, Hh, d, d, device=dev)
+            tr.gdn_scan(q, kk, v, la, be, [0, m], want_o=False, S_final=S_m)
+            for r in SWEEP_R:
+                k5 = tr.tail_len(m, r, 100)
+                a = m - k5
+                o5 = torch.empty(k5, Hh, d, dtype=torch.bfloat16, device=dev)
+                Sh = torch.empty_like(S_m)
+                args5 = (q[a:], kk[a:], v[a:], la[a:].contiguous(), be[a:].contiguous())
+                cu5 = tr.seqlens([0, k5], dev)
+                fn = lambda: tr.gdn_scan(*args5, cu5, o=o5, S_final=Sh)
+                fn()
+                t5 = timed(fn, max(3, min(n_rep, 10))) * 1e-3
+                _, tot = tr.state_error(S_m.reshape(-1, d, d), Sh.reshape(-1, d, d),
+                                        per_mat=False)
+                upd = k5 * Hh
+                by = upd * (3 * 256 + 8 + 256) + Hh * d * d * 4
+                cells.append({"m": m, "r": r / 100, "k": k5, "alpha": [alpha_lo, 1.0],
+                              "us": t5 * 1e6, "state_updates_per_s": upd / t5,
+                              "achieved_gbs": by / t5 / 1e9,
+                              "frac": by / t5 / 1e9 / peaks["hbm_gbs"],
+                              "rel_state_error": float(tot.item())})
+            del q, kk, v, la, be
+    tr.check()
+    c5 = {"workload": "scan sweep m in {4K..128K} x r in {1,2,5,10,20,100}%, 32 heads d=128, "
+                      "bf16 q/k/v, alpha~U[0.80,1] and U[0.97,1]; per cell the tail replay "
+                      "(readout included) timed, ||S_m - S_hat_m||/||S_m|| against the full "
+                      "prefill",
+          "roofline_basis": "HBM: 1032 B per token-head + 64 KB state out per head, of the "
+                            "measured copy bandwidth",
+          "cells": cells}
+    if cpu:
+        import oracle
+        case = synth.scan_case([512], Hh, d, d, torch.bfloat16, 0.97, 1.0, seed=synth.SEED_BASE + 4)
+        t0 = time.perf_counter()
+        oracle.gdn_scan(case.q, case.k, case.v, case.log_alpha, case.beta, case.cu_seqlens)
+        dt = time.perf_counter() - t0
+        c5["cpu_baseline"] = {"value": 512 * Hh / dt, "unit": "state-updates/s",
+                              "cores": os.cpu_count(), "kind": "oracle",
+                              "sample": "512 tokens x 32 heads with readout (%.1f s); the same "
+                                        "rate applies to every cell (extrapolated)" % dt}
+    out["config5_scan_sweep"] = c5
+    return out
 
 
 # ------------------------------------------------------------------ reference
@@ -448,20 +693,9 @@ def our_arm(args):
             kern_ms[i].append(events[i].elapsed_time(events[i + 1]))
     tr.check()
 
-    # per-kernel breakdown (launch order: per layer rmsnorm, in-proj, scan[, out-proj])
-    # launch order per layer: rmsnorm, in_proj, scan kernels, out_proj (not after the last
-    # layer, whose readout and output projection are skipped)
-    # the chunked scan is prep + chain + readout (the last layer has no readout)
-    chunked = n_k == L * 4 + (L - 1) * 2
-    names = []
-    for l in range(L):
-        last = l == L - 1
-        if chunked:
-            scan_names = ["scan_prep", "scan_chain"] + ([] if last else ["scan_out"])
-        else:
-            scan_names = ["scan"]
-        names += ["rmsnorm", "in_proj"] + scan_names + ([] if last else ["out_proj"])
-    assert len(names) == n_k, (len(names), n_k)
+    # per-kernel breakdown, in launch order (the library names its launches)
+    names = rep.kernel_names()
+    assert len(names) == n_k, (names, n_k)
     avg = [sum(x) / len(x) for x in kern_ms]
     brk = {}
     for n, a in zip(names, avg):
@@ -546,10 +780,8 @@ def our_arm(args):
         return sum(ts) / len(ts)
 
     def copy_only():
-        side.wait_stream(stream)
-        with torch.cuda.stream(side):
-            kv_dev.copy_(kv_host, non_blocking=True)
-        stream.wait_stream(side)
+        # the same entry point with no groups: one cudaMemcpyAsync on the copy stream
+        tr.kv_transfer(kv_host, kv_dev, stream=stream, copy_stream=side)
 
     n_ov = max(5, min(args.steps, 30))
     for _ in range(3):
@@ -567,13 +799,14 @@ def our_arm(args):
     sla, sb = case.log_alpha.to(dev), case.beta.to(dev)
     so = torch.empty_like(sv)
     sS = torch.empty(1, 32, 128, 128, dtype=torch.float32, device=dev)
+    cu_s = tr.seqlens(case.cu_seqlens, dev)
     for _ in range(3):
-        tr.gdn_scan(sq, sk, sv, sla, sb, case.cu_seqlens, o=so, S_final=sS)
+        tr.gdn_scan(sq, sk, sv, sla, sb, cu_s, o=so, S_final=sS)
     scan_ms = []
     for _ in range(max(5, min(args.steps, 50))):
         flush.zero_()
         e0.record(stream)
-        tr.gdn_scan(sq, sk, sv, sla, sb, case.cu_seqlens, o=so, S_final=sS)
+        tr.gdn_scan(sq, sk, sv, sla, sb, cu_s, o=so, S_final=sS)
         e1.record(stream)
         e1.synchronize()
         scan_ms.append(e0.elapsed_time(e1))
@@ -582,7 +815,7 @@ def our_arm(args):
     scan_bytes = upd * (3 * 256 + 8 + 256) + 32 * 128 * 128 * 4
     scan_gbs = scan_bytes / scan_t / 1e9
     # the same tail's transition product P (32 heads of 128 x 128), the repair operator
-    cu5 = case.cu_seqlens
+    cu5 = cu_s
     Pbuf = torch.empty(1, 32, 128, 128, dtype=torch.float32, device=dev)
     for _ in range(3):
         tr.transition_product(sk, sla, sb, cu5, P=Pbuf)
@@ -619,15 +852,12 @@ def our_arm(args):
         for i in range(n_f):
             f_kern[i] += fev[i].elapsed_time(fev[i + 1]) / n_ov
     tr.check()
-    # launch order of a non-last layer: rmsnorm, in_proj, 3 scan kernels, out_proj, then the
-    # FFN's rmsnorm, gate/up (SwiGLU) and down projections
-    ffn_pos = [(9 * l + 6, 9 * l + 7, 9 * l + 8) for l in range(L - 1)] if chunked else []
-    if ffn_pos and n_f == 9 * (L - 1) + 4:
-        sw_us = sum(f_kern[b] for _, b, _ in ffn_pos) * 1e3
-        dn_us = sum(f_kern[c] for _, _, c in ffn_pos) * 1e3
-        fn_us = sum(f_kern[a] for a, _, _ in ffn_pos) * 1e3
-    else:
-        sw_us = dn_us = fn_us = float("nan")
+    # the FFN's launches by name (rmsnorm, gate/up with the SwiGLU epilogue, down)
+    f_names = frep.kernel_names()
+    def f_sum(name):
+        v = [t for n, t in zip(f_names, f_kern) if n == name]
+        return sum(v) * 1e3 if v else float("nan")
+    sw_us, dn_us, fn_us = f_sum("ffn_gate_up"), f_sum("ffn_down"), f_sum("ffn_rmsnorm")
     sw_flops = 2.0 * k * D * 2 * D_FF          # per launch
     dn_flops = 2.0 * k * D_FF * D
     sw_tf = sw_flops * (L - 1) / (sw_us * 1e-6) / 1e12
@@ -658,18 +888,22 @@ def our_arm(args):
         for i in range(n_g):
             g_kern[i] += gev[i].elapsed_time(gev[i + 1]) / n_ov
     tr.check()
-    # launch order: per non-last layer rmsnorm, in_proj, conv, 3 scan kernels, gated norm,
-    # out_proj; the last layer rmsnorm, in_proj, conv, prep, chain
-    conv_us = gn_us = float("nan")
-    if chunked and n_g == 8 * (L - 1) + 5:
-        conv_us = sum(g_kern[8 * l + 2] for l in range(L)) * 1e3
-        gn_us = sum(g_kern[8 * l + 6] for l in range(L - 1)) * 1e3
+    g_names = grep_.kernel_names()
+    def g_sum(name):
+        v = [t for n, t in zip(g_names, g_kern) if n == name]
+        return sum(v) * 1e3 if v else float("nan")
+    conv_us, gn_us = g_sum("short_conv"), g_sum("gated_norm")
     C_conv = 3 * H * DH
     conv_bytes = (L - 1) * k * C_conv * 4 + k * (2 * H * DH) * 4   # bf16 in + out per channel
     gn_bytes = (L - 1) * k * H * DH * 6                            # o, z in; o out (bf16)
     conv_gbs = conv_bytes / (conv_us * 1e-6) / 1e9
     gn_gbs = gn_bytes / (gn_us * 1e-6) / 1e9
     del grep_, gl_dev
+
+    configs = None
+    if world == 1 and not args.no_configs:
+        configs = config_cells(dev, peaks, stream, flush, args.steps,
+                               cpu=not args.no_cpu_baseline)
 
     if rank == 0:
         cpu = None
@@ -687,10 +921,13 @@ def our_arm(args):
             "token_layers_per_s": value * L,
             "state_updates_per_s": value * L * H,
             "state_error_vs_full_prefill": float(err_tot.item()),
+            # the dominant kernel's figure (the contract), with the whole step's fraction of
+            # its own roofline beside it (group_step_frac = t_roof / t_step)
             "roofline": dict(kernels[dominant], kernel=dominant,
                              traffic=traffic.get(dominant),
                              peak_source=peak_src + (" (burst bf16)" if kernels[dominant]["bound"] ==
-                                                     "tensor" else " (HBM copy)")),
+                                                     "tensor" else " (HBM copy)"),
+                             group_step_frac=t_roof / (ms_per_step * 1e-3)),
             "kernel_rooflines": {n: dict(r, traffic=traffic.get(n)) for n, r in kernels.items()},
             "profiled_ms_per_step": sum(prof_ms) / len(prof_ms),
             "group_roofline": {"t_roof_us": t_roof * 1e6, "t_step_us": ms_per_step * 1e3,
@@ -736,6 +973,7 @@ def our_arm(args):
                 "gated_norm": {"us_per_step": gn_us, "bound": "hbm", "achieved": gn_gbs,
                                "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                "frac": gn_gbs / peaks["hbm_gbs"], "bytes_per_step": gn_bytes}},
+            "configs": configs,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "replayed tokens/s",
                     "h2d_bytes_per_step": k * D * 2,

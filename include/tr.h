@@ -271,6 +271,9 @@ tr_status tr_replay_group(const tr_group_args *args, void *ws, size_t ws_bytes, 
  * 1 + tr_replay_group_kernel_count(args); the rest are left alone.
  */
 int32_t tr_replay_group_kernel_count(const tr_group_args *args);
+/* The names of those kernels, comma-separated, in launch order (a thread-local string,
+ * valid until the next call from the same thread; "" for invalid args).  Host-only. */
+const char *tr_replay_group_kernel_names(const tr_group_args *args);
 tr_status tr_replay_group_profiled(const tr_group_args *args, void *ws, size_t ws_bytes,
                                    void *stream, void *const *events, int32_t n_events);
 
@@ -290,8 +293,10 @@ tr_status tr_replay_groups(const tr_group_args *groups, int32_t n_groups, void *
  * notes, section 2.5: the KV of the matched prefix moves to the device on a separate
  * stream while the linear-attention states are replayed, T ~ max(T_KV, T_replay)).
  * `kv_bytes` are copied from `kv_host` (pinned host memory) to `kv_dev` on `copy_stream`,
- * issued before the replay's kernels on `stream`; `stream` then waits for the copy, so
- * work enqueued on it afterwards sees both the KV and the states.  One cudaMemcpyAsync;
+ * issued before the replay's kernels on `stream`.  The copy waits for everything enqueued
+ * on `stream` before the call (an event recorded at entry), so earlier work that still
+ * reads kv_dev finishes first; `stream` then waits for the copy, so work enqueued on it
+ * afterwards sees both the KV and the states.  One cudaMemcpyAsync;
  * kv_bytes = 0 replays only.  The two streams must differ.  Same workspace as
  * tr_replay_groups.  Every argument (the KV pointers and streams, each group, the
  * workspace) is checked before the copy is issued: a rejected call moves no bytes.
@@ -326,8 +331,12 @@ tr_status tr_state_error(const float *S, const float *S_hat, int64_t n_mats, int
  *   - Scratch space is a fixed array inside the library (2 x 65536 doubles, 1 MiB
  *     per GPU that loads the library, held until the process exits); n_mats above
  *     65536 is rejected with TR_ERR_UNSUPPORTED.  Nothing is allocated.
- *   - The first call on a device looks up the array's device address for that
- *     device (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call made outside stream capture looks up the array's device address in
+ *     the current context (cudaGetSymbolAddress), so a context created again after
+ *     cudaDeviceReset is served correctly.  A call made while its stream captures
+ *     reuses the address of the last uncaptured call on that device: make one
+ *     uncaptured call on a device (in the current context) before capturing one;
+ *     without it the captured call returns TR_ERR_INVALID_ARG.
  *   - All calls share the array: calls whose kernels may overlap on the GPU race.
  *     Each call writes every scratch entry it reads, so nothing needs clearing.
  */

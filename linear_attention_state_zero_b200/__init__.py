@@ -70,6 +70,7 @@ _SIGNATURES = {
     "tr_replay_groups_overlapped": (ctypes.c_int, [ctypes.POINTER(GroupArgs), c_i32, c_vp, c_sz,
                                                    c_vp, c_vp, c_sz, c_vp, c_vp]),
     "tr_replay_group_kernel_count": (c_i32, [ctypes.POINTER(GroupArgs)]),
+    "tr_replay_group_kernel_names": (ctypes.c_char_p, [ctypes.POINTER(GroupArgs)]),
     "tr_replay_group_profiled": (ctypes.c_int, [ctypes.POINTER(GroupArgs), c_vp, c_sz, c_vp,
                                                 ctypes.POINTER(c_vp), c_i32]),
     "tr_replay_groups_workspace_size": (c_sz, [ctypes.POINTER(GroupArgs), c_i32]),
@@ -118,9 +119,10 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
-def _stream(stream) -> Optional[int]:
+def _stream(stream, device=None) -> Optional[int]:
+    """The raw handle of `stream`, or of the current stream of `device` when None."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
     return stream.cuda_stream
 
 
@@ -133,9 +135,21 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def _need_cuda(*ts):
+    """Every given tensor lives on one CUDA device; returns that device (None if no tensor).
+
+    The library launches on the current device, so each call below runs with this device
+    made current (``torch.cuda.device``) and on its current stream unless one is given."""
+    dev = None
     for t in ts:
-        if t is not None and not t.is_cuda:
+        if t is None:
+            continue
+        if not t.is_cuda:
             raise ValueError("tensors must live on a CUDA device")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError("tensors must live on one device (%s and %s)" % (dev, t.device))
+    return dev
 
 
 def _need_layout(name, t, dtype, shape=None):
@@ -149,8 +163,20 @@ def _need_layout(name, t, dtype, shape=None):
         raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
 
 
+def seqlens(cu_seqlens, device):
+    """cu_seqlens prepared once as (host int32 tensor, device int32 tensor); the calls below
+    accept this pair in place of cu_seqlens and then copy nothing."""
+    return _seqlens(cu_seqlens, device)
+
+
 def _seqlens(cu_seqlens, device):
     """(host int32 tensor, device int32 tensor) for a cu_seqlens given either way."""
+    if isinstance(cu_seqlens, tuple) and len(cu_seqlens) == 2:
+        host, dev = cu_seqlens
+        if host.device.type != "cpu" or dev.device != torch.device(device) or \
+                host.dtype != torch.int32 or dev.dtype != torch.int32:
+            raise ValueError("a (host, device) cu_seqlens pair must hold int32 tensors")
+        return host, dev
     cu = torch.as_tensor(cu_seqlens, dtype=torch.int32)
     host = cu.cpu().contiguous()
     dev = cu.to(device).contiguous() if not (cu.is_cuda and cu.is_contiguous()) else cu
@@ -172,7 +198,7 @@ def tail_len(m: int, r_num: int, r_den: int) -> int:
 def gdn_scan(q, k, v, log_alpha, beta, cu_seqlens, *, S0=None, want_o=True, scale=1.0,
              normalize_qk=False, recurrent=False, o=None, S_final=None, stream=None):
     """Eq. (1) scan over a packed batch: returns (o or None, S_final [N, H, d_k, d_v] fp32)."""
-    _need_cuda(k, v, log_alpha, beta)
+    dev_ = _need_cuda(q, k, v, log_alpha, beta, S0, o, S_final)
     T, H, dk = k.shape
     dv = v.shape[2]
     for t in (q, k, v):
@@ -195,7 +221,9 @@ def gdn_scan(q, k, v, log_alpha, beta, cu_seqlens, *, S0=None, want_o=True, scal
                  _ptr(dev), host.data_ptr(), _ptr(S0), _ptr(o), _ptr(S_final))
     ws_bytes = lib.tr_gdn_scan_workspace_size(ctypes.byref(a))
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=k.device) if ws_bytes else None
-    _ok(lib.tr_gdn_scan(ctypes.byref(a), _ptr(ws), ws_bytes, _stream(stream)), "tr_gdn_scan")
+    with torch.cuda.device(dev_):
+        _ok(lib.tr_gdn_scan(ctypes.byref(a), _ptr(ws), ws_bytes, _stream(stream, dev_)),
+            "tr_gdn_scan")
     return o, S_final
 
 
@@ -203,7 +231,7 @@ def transition_product(k, log_alpha, beta, cu_seqlens, *, normalize_qk=False, re
                        P=None, stream=None):
     """P = T_t ... T_1 per (sequence, head): [N, H, d_k, d_k] fp32 (M = S^T convention:
     a state M_0 before the sequence becomes P M_0 + the zero-start state after it)."""
-    _need_cuda(k, log_alpha, beta)
+    dev_ = _need_cuda(k, log_alpha, beta, P)
     T, H, dk = k.shape
     if k.stride(2) != 1 or k.stride(1) != dk:
         raise ValueError("k must be [T, H, d] with contiguous heads")
@@ -219,8 +247,9 @@ def transition_product(k, log_alpha, beta, cu_seqlens, *, normalize_qk=False, re
                  None)
     ws_bytes = lib.tr_transition_product_workspace_size(ctypes.byref(a))
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=k.device) if ws_bytes else None
-    _ok(lib.tr_transition_product(ctypes.byref(a), _ptr(P), _ptr(ws), ws_bytes, _stream(stream)),
-        "tr_transition_product")
+    with torch.cuda.device(dev_):
+        _ok(lib.tr_transition_product(ctypes.byref(a), _ptr(P), _ptr(ws), ws_bytes,
+                                      _stream(stream, dev_)), "tr_transition_product")
     return P
 
 
@@ -275,14 +304,14 @@ class GroupReplay:
         conv_width = 0
         n_in = 2 * n_heads * d_k + n_heads * d_v * (2 if output_gate else 1) + 2 * n_heads
         for i, lw in enumerate(self.layers):
-            _need_cuda(lw.W_in, lw.W_o)
+            _need_cuda(h_tail, lw.W_in, lw.W_o, lw.rms_gain)
             _need_layout("W_in", lw.W_in, torch.bfloat16, (n_in, D))
             _need_layout("W_o", lw.W_o, torch.bfloat16, (D, n_heads * d_v))
             _need_layout("rms_gain", lw.rms_gain, torch.float32, (D,))
             Wg = getattr(lw, "W_gate", None)
             Wu, Wd, fg = (getattr(lw, n, None) for n in ("W_up", "W_down", "ffn_gain"))
             if Wg is not None:
-                _need_cuda(Wg, Wu, Wd)
+                _need_cuda(h_tail, Wg, Wu, Wd, fg)
                 if d_ff and Wg.shape[0] != d_ff:
                     raise ValueError("all FFN sublayers of a group must have one width")
                 d_ff = Wg.shape[0]
@@ -292,7 +321,7 @@ class GroupReplay:
                 _need_layout("ffn_gain", fg, torch.float32, (D,))
             cw, al, db, og = (getattr(lw, n, None) for n in ("conv_w", "A_log", "dt_bias",
                                                                  "o_norm_gain"))
-            _need_cuda(cw, al, db, og)
+            _need_cuda(h_tail, cw, al, db, og)
             _need_layout("conv_w", cw, torch.float32)
             if cw is not None and cw.shape[0] != 2 * n_heads * d_k + n_heads * d_v:
                 raise ValueError("conv_w must be [2 H d_k + H d_v, width]")
@@ -307,6 +336,7 @@ class GroupReplay:
             self._layer_arr[i] = LALayer(_ptr(lw.rms_gain), _ptr(lw.W_in), _ptr(lw.W_o),
                                          _ptr(fg), _ptr(Wg), _ptr(Wu), _ptr(Wd), _ptr(cw),
                                          _ptr(al), _ptr(db), _ptr(og))
+        _need_cuda(h_tail, S_hat, x_out, workspace)
         self.S_hat = S_hat if S_hat is not None else torch.empty(
             (L, N, n_heads, d_k, d_v), dtype=torch.float32, device=dev)
         if skip_last_output:
@@ -333,19 +363,28 @@ class GroupReplay:
         self.workspace = workspace
 
     def run(self, stream=None):
-        _ok(lib.tr_replay_group(ctypes.byref(self.args), _ptr(self.workspace), self.ws_bytes,
-                                _stream(stream)), "tr_replay_group")
+        dev = self.h_tail.device
+        with torch.cuda.device(dev):
+            _ok(lib.tr_replay_group(ctypes.byref(self.args), _ptr(self.workspace), self.ws_bytes,
+                                    _stream(stream, dev)), "tr_replay_group")
         return self.S_hat, self.x_out
 
     def kernel_count(self) -> int:
         return int(lib.tr_replay_group_kernel_count(ctypes.byref(self.args)))
 
+    def kernel_names(self) -> list:
+        """The kernels one run() launches, in order (the events of run_profiled bracket them)."""
+        names = lib.tr_replay_group_kernel_names(ctypes.byref(self.args)).decode()
+        return names.split(",") if names else []
+
     def run_profiled(self, event_handles, stream=None):
         """Same as run(), recording the given raw cudaEvent_t handles between kernel launches."""
         arr = (c_vp * len(event_handles))(*event_handles)
-        _ok(lib.tr_replay_group_profiled(ctypes.byref(self.args), _ptr(self.workspace),
-                                         self.ws_bytes, _stream(stream), arr, len(event_handles)),
-            "tr_replay_group_profiled")
+        dev = self.h_tail.device
+        with torch.cuda.device(dev):
+            _ok(lib.tr_replay_group_profiled(ctypes.byref(self.args), _ptr(self.workspace),
+                                             self.ws_bytes, _stream(stream, dev), arr,
+                                             len(event_handles)), "tr_replay_group_profiled")
         return self.S_hat, self.x_out
 
 
@@ -370,8 +409,10 @@ class GroupsReplay:
             if self.ws_bytes else None
 
     def run(self, stream=None):
-        _ok(lib.tr_replay_groups(self._arr, len(self.groups), _ptr(self.workspace),
-                                 self.ws_bytes, _stream(stream)), "tr_replay_groups")
+        dev = self.groups[0].h_tail.device
+        with torch.cuda.device(dev):
+            _ok(lib.tr_replay_groups(self._arr, len(self.groups), _ptr(self.workspace),
+                                     self.ws_bytes, _stream(stream, dev)), "tr_replay_groups")
         return [(g.S_hat, g.x_out) for g in self.groups]
 
     def run_overlapped(self, kv_host, kv_dev, stream=None, copy_stream=None):
@@ -384,83 +425,113 @@ class GroupsReplay:
         if not kv_host.is_pinned():
             raise ValueError("kv_host must be pinned host memory")
         nbytes = kv_host.numel() * kv_host.element_size()
-        _ok(lib.tr_replay_groups_overlapped(self._arr, len(self.groups), _ptr(self.workspace),
-                                            self.ws_bytes, kv_host.data_ptr(), _ptr(kv_dev),
-                                            nbytes, _stream(stream), _stream(copy_stream)),
-            "tr_replay_groups_overlapped")
+        dev = self.groups[0].h_tail.device
+        if _need_cuda(kv_dev) != dev:
+            raise ValueError("kv_dev must live on the groups' device")
+        with torch.cuda.device(dev):
+            _ok(lib.tr_replay_groups_overlapped(self._arr, len(self.groups),
+                                                _ptr(self.workspace), self.ws_bytes,
+                                                kv_host.data_ptr(), _ptr(kv_dev), nbytes,
+                                                _stream(stream, dev), _stream(copy_stream, dev)),
+                "tr_replay_groups_overlapped")
         return [(g.S_hat, g.x_out) for g in self.groups]
+
+
+def kv_transfer(kv_host, kv_dev, stream=None, copy_stream=None):
+    """The FA KV copy of tr_replay_groups_overlapped alone (no groups): kv_host (pinned) to
+    kv_dev on copy_stream, after the work already on `stream`, which then waits for it."""
+    dev = _need_cuda(kv_dev)
+    if copy_stream is None:
+        raise ValueError("the KV copy needs a stream of its own (copy_stream)")
+    if kv_host.numel() * kv_host.element_size() != kv_dev.numel() * kv_dev.element_size():
+        raise ValueError("kv_host and kv_dev differ in size")
+    if not kv_host.is_pinned():
+        raise ValueError("kv_host must be pinned host memory")
+    nbytes = kv_host.numel() * kv_host.element_size()
+    with torch.cuda.device(dev):
+        _ok(lib.tr_replay_groups_overlapped(None, 0, None, 0, kv_host.data_ptr(), _ptr(kv_dev),
+                                            nbytes, _stream(stream, dev),
+                                            _stream(copy_stream, dev)),
+            "tr_replay_groups_overlapped")
 
 
 def state_error(S, S_hat, *, per_mat=True, stream=None):
     """(err_per_mat [n_mats] fp64 or None, err_total [1] fp64), device tensors."""
-    _need_cuda(S, S_hat)
+    dev = _need_cuda(S, S_hat)
     if S.shape != S_hat.shape or S.dtype != torch.float32 or S_hat.dtype != torch.float32:
         raise ValueError("S and S_hat must be fp32 tensors of one shape")
     dk, dv = S.shape[-2:]
     S, S_hat = S.contiguous(), S_hat.contiguous()
     n = S.numel() // (dk * dv)
-    per = torch.empty(n, dtype=torch.float64, device=S.device) if per_mat else None
-    tot = torch.empty(1, dtype=torch.float64, device=S.device)
+    per = torch.empty(n, dtype=torch.float64, device=dev) if per_mat else None
+    tot = torch.empty(1, dtype=torch.float64, device=dev)
     ws_bytes = lib.tr_state_error_workspace_size(n)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=S.device) if ws_bytes else None
-    _ok(lib.tr_state_error(_ptr(S), _ptr(S_hat), n, dk, dv, _ptr(per), _ptr(tot), _ptr(ws),
-                           ws_bytes, _stream(stream)), "tr_state_error")
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
+    with torch.cuda.device(dev):
+        _ok(lib.tr_state_error(_ptr(S), _ptr(S_hat), n, dk, dv, _ptr(per), _ptr(tot), _ptr(ws),
+                               ws_bytes, _stream(stream, dev)), "tr_state_error")
     return per, tot
 
 
 def state_error_noalloc(S, S_hat, *, per_mat=True, stream=None):
     """Same as state_error, through the entry point that allocates no scratch
     (for callers that cannot allocate device memory at the call; see include/tr.h)."""
-    _need_cuda(S, S_hat)
+    dev = _need_cuda(S, S_hat)
     if S.shape != S_hat.shape or S.dtype != torch.float32 or S_hat.dtype != torch.float32:
         raise ValueError("S and S_hat must be fp32 tensors of one shape")
     dk, dv = S.shape[-2:]
     S, S_hat = S.contiguous(), S_hat.contiguous()
     n = S.numel() // (dk * dv)
-    per = torch.empty(n, dtype=torch.float64, device=S.device) if per_mat else None
-    tot = torch.empty(1, dtype=torch.float64, device=S.device)
-    _ok(lib.tr_state_error_noalloc(_ptr(S), _ptr(S_hat), n, dk, dv, _ptr(per), _ptr(tot),
-                                   _stream(stream)), "tr_state_error_noalloc")
+    per = torch.empty(n, dtype=torch.float64, device=dev) if per_mat else None
+    tot = torch.empty(1, dtype=torch.float64, device=dev)
+    # the library's fixed scratch and the kernel belong to the current device: make the
+    # tensors' device current for the call
+    with torch.cuda.device(dev):
+        _ok(lib.tr_state_error_noalloc(_ptr(S), _ptr(S_hat), n, dk, dv, _ptr(per), _ptr(tot),
+                                       _stream(stream, dev)), "tr_state_error_noalloc")
     return per, tot
 
 
 def rmsnorm(x, gain=None, eps=0.0, stream=None):
-    _need_cuda(x, gain)
+    dev = _need_cuda(x, gain)
     x = x.contiguous()
     T, D = x.shape
-    out = torch.empty((T, D), dtype=torch.bfloat16, device=x.device)
-    _ok(lib.tr_rmsnorm(_ptr(x), _dtype_code(x), _ptr(gain), T, D, float(eps), _ptr(out),
-                       _stream(stream)), "tr_rmsnorm")
+    out = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.device(dev):
+        _ok(lib.tr_rmsnorm(_ptr(x), _dtype_code(x), _ptr(gain), T, D, float(eps), _ptr(out),
+                           _stream(stream, dev)), "tr_rmsnorm")
     return out
 
 
 def in_projection(x_hat, W_in, n_heads, d_k, d_v, *, skip_q=False, norm_eps=0.0, stream=None):
     """(qkv [T, 2Hd_k + Hd_v] bf16, log_alpha [T, H], beta [T, H])."""
-    _need_cuda(x_hat, W_in)
+    dev = _need_cuda(x_hat, W_in)
     T, D = x_hat.shape
-    dev = x_hat.device
     x_hat = x_hat.contiguous()
     W_in = W_in.contiguous()
     qkv = torch.zeros((T, 2 * n_heads * d_k + n_heads * d_v), dtype=torch.bfloat16, device=dev)
     la = torch.empty((T, n_heads), dtype=torch.float32, device=dev)
     be = torch.empty((T, n_heads), dtype=torch.float32, device=dev)
-    _ok(lib.tr_in_projection(_ptr(x_hat), _ptr(W_in), T, D, n_heads,
-                             d_k, d_v, TR_SKIP_LAST_OUTPUT if skip_q else 0, float(norm_eps),
-                             _ptr(qkv), _ptr(la), _ptr(be), _stream(stream)), "tr_in_projection")
+    with torch.cuda.device(dev):
+        _ok(lib.tr_in_projection(_ptr(x_hat), _ptr(W_in), T, D, n_heads,
+                                 d_k, d_v, TR_SKIP_LAST_OUTPUT if skip_q else 0, float(norm_eps),
+                                 _ptr(qkv), _ptr(la), _ptr(be), _stream(stream, dev)),
+            "tr_in_projection")
     return qkv, la, be
 
 
 def out_projection(o, W_o, x_res, stream=None):
     """x_res + o W_o^T in fp32; o [T, H d_v] bf16 (rows may be strided)."""
-    _need_cuda(o, W_o, x_res)
+    dev = _need_cuda(o, W_o, x_res)
     T, hv = o.shape
     D = W_o.shape[0]
     W_o = W_o.contiguous()
     x_res = x_res.contiguous()
-    out = torch.empty((T, D), dtype=torch.float32, device=o.device)
-    _ok(lib.tr_out_projection(_ptr(o), o.stride(0), _ptr(W_o),
-                              _ptr(x_res), _dtype_code(x_res), T, D, hv, _ptr(out),
-                              _stream(stream)), "tr_out_projection")
+    out = torch.empty((T, D), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _ok(lib.tr_out_projection(_ptr(o), o.stride(0), _ptr(W_o),
+                                  _ptr(x_res), _dtype_code(x_res), T, D, hv, _ptr(out),
+                                  _stream(stream, dev)), "tr_out_projection")
     return out
 
 

@@ -31,16 +31,23 @@ constexpr int kMaxDevices = 64;
 double *g_scratch_ptr[kMaxDevices];
 std::mutex g_scratch_mu;
 
-// Device address of the scratch array for the current device, looked up once per
-// device (with that device current).  Host code must not use the array's name as a
-// device address: in host code it names a host-side stand-in.
-cudaError_t scratch_for_current_device(double **out) {
+// Device address of the scratch array in the current device's context.  Host code must
+// not use the array's name as a device address: in host code it names a host-side
+// stand-in.  The address is looked up again on every call made outside stream capture
+// (so a context created anew after cudaDeviceReset gets its own module's address); a
+// call made while `s` is capturing reuses the address the last uncaptured call on this
+// device found, because lookups that may load a module do not belong in a capture.
+cudaError_t scratch_for_current_device(cudaStream_t s, double **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(s, &cap);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone || !g_scratch_ptr[dev]) {
+    if (cap != cudaStreamCaptureStatusNone) return cudaErrorStreamCaptureUnsupported;
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
@@ -68,9 +75,12 @@ extern "C" tr_status tr_state_error_noalloc(const float *S, const float *S_hat, 
   if (!aligned16(S) || !aligned16(S_hat)) return tr::record_error(TR_ERR_ALIGNMENT, "S/S_hat alignment");
   if (!err_per_mat && !err_total) return tr::record_error(TR_OK, "");
   double *scratch = nullptr;
-  cudaError_t e = scratch_for_current_device(&scratch);
+  cudaError_t e = scratch_for_current_device(static_cast<cudaStream_t>(stream), &scratch);
+  if (e == cudaErrorStreamCaptureUnsupported)
+    return tr::record_error(TR_ERR_INVALID_ARG,
+                            "the first call on a device must come before any stream capture");
   if (e != cudaSuccess)
-    return tr::record_error(TR_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    return tr::record_error(TR_ERR_CUDA, "scratch address: %s", cudaGetErrorString(e));
   const int64_t elems = (int64_t)d_k * d_v;
   e = tr::launch_state_error(S, S_hat, n_mats, elems, tr::state_error_splits(n_mats, elems, kStaticMats),
                              scratch, err_per_mat, err_total, static_cast<cudaStream_t>(stream),

@@ -1149,9 +1149,10 @@ size_t scan_chunked_workspace(const ScanLaunch &p) {
   return total;
 }
 
-int scan_chunked_kernels(const ScanLaunch &p, bool with_readout) {
+std::vector<const char *> scan_chunked_kernel_names(const ScanLaunch &p, bool with_readout) {
   (void)p;
-  return with_readout ? 3 : 2;
+  if (with_readout) return {"scan_prep", "scan_chain", "scan_out"};
+  return {"scan_prep", "scan_chain"};
 }
 
 cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string *err,

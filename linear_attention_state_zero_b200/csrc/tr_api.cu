@@ -51,15 +51,29 @@ unsigned *g_err_ptr[kMaxDevices];
 int g_sms[kMaxDevices];
 std::mutex g_dev_mu;
 
-bool device_state(int *dev_out, unsigned **err_out, std::string *err) {
+// The device's SM count and the address of the library's error word in the current
+// context.  The address is looked up again on every call made outside stream capture (a
+// context created anew after cudaDeviceReset has its own copy of the word); a call made
+// while `s` captures reuses what the last uncaptured call on this device found.
+bool device_state(cudaStream_t s, int *dev_out, unsigned **err_out, std::string *err) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     if (err) *err = std::string("cudaGetDevice: ") + cudaGetErrorString(e);
     return false;
   }
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(s, &cap);
+  if (e != cudaSuccess) {
+    if (err) *err = std::string("cudaStreamIsCapturing: ") + cudaGetErrorString(e);
+    return false;
+  }
   std::lock_guard<std::mutex> lk(g_dev_mu);
-  if (!g_err_ptr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone || !g_err_ptr[dev]) {
+    if (cap != cudaStreamCaptureStatusNone) {
+      if (err) *err = "the first call on a device must come before any stream capture";
+      return false;
+    }
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_err_word);
     if (e != cudaSuccess) {
@@ -259,8 +273,10 @@ size_t scan_ws_bytes(const tr::ScanLaunch &p) {
   return use_chunked(p) ? tr::scan_chunked_workspace(p) : 0;
 }
 
-int scan_kernel_count(const tr::ScanLaunch &p, bool with_readout) {
-  return use_chunked(p) ? tr::scan_chunked_kernels(p, with_readout) : 1;
+// Names of the kernels one scan call launches, in launch order.
+std::vector<const char *> scan_kernel_names(const tr::ScanLaunch &p, bool with_readout) {
+  if (use_chunked(p)) return tr::scan_chunked_kernel_names(p, with_readout);
+  return {"scan_recurrent"};
 }
 
 tr_status run_scan(const tr::ScanLaunch &p, cudaStream_t s,
@@ -405,18 +421,33 @@ bool runs_ffn(const tr_group_args *a, int l) {
   return true;
 }
 
-int group_kernel_count(const tr_group_args *a) {
-  int n = 0;
+// Names of the kernels tr_replay_group launches for `a`, in launch order (the order in
+// which replay_group_enqueue records its events).
+std::vector<const char *> group_kernel_names(const tr_group_args *a) {
+  std::vector<const char *> n;
   for (int l = 0; l < a->n_layers; ++l) {
     const bool last = l == a->n_layers - 1;
     const bool skip = last && (a->flags & TR_SKIP_LAST_OUTPUT);
-    n += 2 + scan_kernel_count(group_scan_launch(a), !skip);
-    if (a->conv_width > 0) n += 1;
-    if (!skip && (!last || a->x_out)) n += 1 + (output_gate(a) ? 1 : 0);
-    if (runs_ffn(a, l)) n += 3;
+    n.push_back("rmsnorm");
+    n.push_back("in_proj");
+    if (a->conv_width > 0) n.push_back("short_conv");
+    for (const char *k : scan_kernel_names(group_scan_launch(a), !skip)) n.push_back(k);
+    if (!skip && (!last || a->x_out)) {
+      if (output_gate(a)) n.push_back("gated_norm");
+      n.push_back("out_proj");
+    }
+    if (runs_ffn(a, l)) {
+      n.push_back("ffn_rmsnorm");
+      n.push_back("ffn_gate_up");
+      n.push_back("ffn_down");
+    }
   }
   return n;
 }
+
+int group_kernel_count(const tr_group_args *a) { return (int)group_kernel_names(a).size(); }
+
+thread_local std::string g_names;
 
 tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_word,
                                cudaStream_t s, Marks *mk = nullptr) {
@@ -682,7 +713,7 @@ tr_status tr_gdn_scan(const tr_scan_args *args, void *ws, size_t ws_bytes, void 
   int dev;
   unsigned *errw;
   std::string err;
-  if (!device_state(&dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
+  if (!device_state(static_cast<cudaStream_t>(stream), &dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
   p.err_word = errw;
   st = run_scan(p, static_cast<cudaStream_t>(stream));
   return st == TR_OK ? ok() : st;
@@ -714,7 +745,7 @@ tr_status tr_transition_product(const tr_scan_args *args, float *P, void *ws, si
   int dev;
   unsigned *errw;
   std::string err;
-  if (!device_state(&dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
+  if (!device_state(static_cast<cudaStream_t>(stream), &dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaSuccess;
   if (L.v0_bytes) e = cudaMemsetAsync(base + L.v0, 0, L.v0_bytes, s);
@@ -751,7 +782,7 @@ tr_status tr_replay_group(const tr_group_args *args, void *ws, size_t ws_bytes, 
   int dev;
   unsigned *errw;
   std::string err;
-  if (!device_state(&dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
+  if (!device_state(static_cast<cudaStream_t>(stream), &dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
   st = replay_group_enqueue(args, ws, errw, static_cast<cudaStream_t>(stream));
   return st == TR_OK ? ok() : st;
 }
@@ -759,6 +790,16 @@ tr_status tr_replay_group(const tr_group_args *args, void *ws, size_t ws_bytes, 
 int32_t tr_replay_group_kernel_count(const tr_group_args *args) {
   if (!args || args->n_layers < 1 || args->n_layers > 64) return 0;
   return group_kernel_count(args);
+}
+
+const char *tr_replay_group_kernel_names(const tr_group_args *args) {
+  g_names.clear();
+  if (!args || args->n_layers < 1 || args->n_layers > 64 || !args->layers) return g_names.c_str();
+  for (const char *k : group_kernel_names(args)) {
+    if (!g_names.empty()) g_names += ',';
+    g_names += k;
+  }
+  return g_names.c_str();
 }
 
 tr_status tr_replay_group_profiled(const tr_group_args *args, void *ws, size_t ws_bytes,
@@ -778,7 +819,7 @@ tr_status tr_replay_group_profiled(const tr_group_args *args, void *ws, size_t w
   int dev;
   unsigned *errw;
   std::string err;
-  if (!device_state(&dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
+  if (!device_state(static_cast<cudaStream_t>(stream), &dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
   Marks mk;
   mk.ev = events;
   mk.n = n_events;
@@ -800,7 +841,7 @@ tr_status tr_replay_groups(const tr_group_args *groups, int32_t n_groups, void *
   int dev;
   unsigned *errw;
   std::string err;
-  if (!device_state(&dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
+  if (!device_state(static_cast<cudaStream_t>(stream), &dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
   for (int32_t g = 0; g < n_groups; ++g) {
     tr_status st = replay_group_enqueue(&groups[g], ws, errw, static_cast<cudaStream_t>(stream));
     if (st != TR_OK) return st;
@@ -818,11 +859,18 @@ tr_status tr_replay_groups_overlapped(const tr_group_args *groups, int32_t n_gro
   tr_status vst = validate_groups(groups, n_groups, ws, ws_bytes);
   if (vst != TR_OK) return vst;
   cudaStream_t s = static_cast<cudaStream_t>(stream), cs = static_cast<cudaStream_t>(copy_stream);
-  cudaEvent_t done = nullptr;
+  cudaEvent_t done = nullptr, entry = nullptr;
   if (kv_bytes > 0) {
-    cudaError_t e = cudaMemcpyAsync(kv_dev, kv_host, kv_bytes, cudaMemcpyHostToDevice, cs);
+    // the copy starts after everything already enqueued on `stream` (earlier readers of
+    // kv_dev, such as the previous step's attention, finish before it overwrites them)
+    cudaError_t e = cudaEventCreateWithFlags(&entry, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventRecord(entry, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, entry, 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(kv_dev, kv_host, kv_bytes, cudaMemcpyHostToDevice, cs);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&done, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventRecord(done, cs);
+    if (entry) cudaEventDestroy(entry);
     if (e != cudaSuccess) {
       if (done) cudaEventDestroy(done);
       return cuda_fail(e, "KV transfer");
@@ -857,7 +905,7 @@ tr_status tr_state_error(const float *S, const float *S_hat, int64_t n_mats, int
   int dev;
   unsigned *errw;
   std::string err;
-  if (!device_state(&dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
+  if (!device_state(static_cast<cudaStream_t>(stream), &dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
   const int64_t elems = (int64_t)d_k * d_v;
   const int splits = tr::state_error_splits(n_mats, elems, (int64_t)(ws_bytes / (2 * sizeof(double))));
   cudaError_t e = tr::launch_state_error(S, S_hat, n_mats, elems, splits,
@@ -898,7 +946,7 @@ tr_status tr_in_projection(const void *x_hat, const void *W_in, int64_t n_tokens
   int dev;
   unsigned *errw;
   std::string err;
-  if (!device_state(&dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
+  if (!device_state(static_cast<cudaStream_t>(stream), &dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
   const int n_in = 2 * n_heads * d_k + n_heads * d_v + 2 * n_heads;
   tr::InProjEpi ep{};
   ep.qkv = static_cast<__nv_bfloat16 *>(qkv);
@@ -934,7 +982,7 @@ tr_status tr_out_projection(const void *o, int64_t o_stride, const void *W_o, co
   int dev;
   unsigned *errw;
   std::string err;
-  if (!device_state(&dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
+  if (!device_state(static_cast<cudaStream_t>(stream), &dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
   tr::ResidEpi rp;
   rp.x_res = x_res;
   rp.res_is_bf16 = x_res_dtype == TR_DTYPE_BF16;

@@ -9,6 +9,7 @@
 
 #include <functional>
 #include <string>
+#include <vector>
 
 namespace tr {
 
@@ -153,7 +154,8 @@ cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string
                                 const std::function<cudaError_t()> &between);
 bool scan_chunked_supported(const ScanLaunch &p);
 size_t scan_chunked_workspace(const ScanLaunch &p);  // needs p.cu_seqlens_host, H, dv
-int scan_chunked_kernels(const ScanLaunch &p, bool with_readout);  // launches of one call
+// the kernels one call launches, in order
+std::vector<const char *> scan_chunked_kernel_names(const ScanLaunch &p, bool with_readout);
 
 // Pieces per matrix of the state error's first pass (partials holds 2 doubles per piece;
 // at most max_pieces pieces in all).

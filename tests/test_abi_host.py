@@ -234,3 +234,25 @@ def test_state_error_workspace_and_args():
     assert tr.lib.tr_state_error(FAKE, FAKE, 100, 128, 128, FAKE, FAKE, None, 0, None) == 6
     assert tr.lib.tr_state_error(FAKE, FAKE + 4, 1, 8, 8, None, FAKE, FAKE, 4096, None) == 4
     assert tr.lib.tr_state_error(FAKE, FAKE, -1, 8, 8, None, FAKE, FAKE, 4096, None) == 1
+
+
+def test_replay_kernel_names_match_the_count():
+    """tr_replay_group_kernel_names lists exactly the launches tr_replay_group_kernel_count
+    counts, in launch order: per layer the RMSNorm, the input projection, the scan's kernels
+    and the output projection (not after the last layer without x_out), plus the options'."""
+    a, keep = _group_args()
+    names = tr.lib.tr_replay_group_kernel_names(ctypes.byref(a)).decode().split(",")
+    assert len(names) == tr.lib.tr_replay_group_kernel_count(ctypes.byref(a))
+    assert names[:2] == ["rmsnorm", "in_proj"] and names[-1] != "out_proj"
+    assert names.count("rmsnorm") == 3 and names.count("out_proj") == 2
+    assert all(n.startswith("scan") for n in names if n not in ("rmsnorm", "in_proj", "out_proj"))
+    a.d_ff = 1024
+    a.conv_width = 4
+    a.flags = tr.TR_OUTPUT_GATE
+    for lw in keep[1]:
+        lw.W_gate, lw.W_up, lw.W_down, lw.conv_w = FAKE, FAKE, FAKE, FAKE
+    names = tr.lib.tr_replay_group_kernel_names(ctypes.byref(a)).decode().split(",")
+    assert len(names) == tr.lib.tr_replay_group_kernel_count(ctypes.byref(a))
+    assert names.count("short_conv") == 3 and names.count("gated_norm") == 2
+    assert names.count("ffn_gate_up") == 2 and names.count("ffn_down") == 2
+    assert tr.lib.tr_replay_group_kernel_names(None) == b""

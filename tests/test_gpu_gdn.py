@@ -147,3 +147,37 @@ def test_binding_rejects_wrong_parameter_dtype(cuda_device):
     bad = [tr.Layer(**{**l.__dict__, "W_in": l.W_in[:-1]}) for l in dl]
     with pytest.raises(ValueError, match="W_in"):
         tr.GroupReplay(h, [0, 8], bad, H, d, d)
+
+
+@pytest.mark.parametrize("skip_last_ffn", [False, True])
+def test_small_group_ffn_and_all_options_varlen(cuda_device, skip_last_ffn):
+    """The FFN sublayer and every Gated DeltaNet option in one group (they share the
+    workspace's normalised-input buffer and run in one launch sequence): ragged requests
+    with sequences shorter than the convolution's history and an empty one, gains on all
+    norms; states, x_out and the convolution state against the oracle."""
+    D, H, d, L, F, width = 256, 2, 128, 3, 384, 4
+    lengths = [37, 2, 0, 130, 1, 64]
+    layers = synth.la_layers(L, D, H, d, d, seed=341, with_gain=True, d_ff=F, conv_width=width,
+                             gate_params=True, output_gate=True)
+    h = _tails(lengths, D, 341)
+    cu = synth.cu_seqlens_of(lengths)
+    g = tr.GroupReplay(h.to(cuda_device), cu, to_dev(layers, cuda_device), H, d, d,
+                       output_gate=True, want_conv_state=True, skip_last_ffn=skip_last_ffn)
+    S, x = g.run()
+    torch.cuda.synchronize()
+    tr.check()
+    states = []
+    wS, wx = oracle.replay_group(h, cu, layers, H, d, d, output_gate=True, conv_states=states,
+                                 skip_last_ffn=skip_last_ffn)
+    for l in range(L):
+        assert rel_fro(S[l], wS[l]) < TOL, l
+        assert rel_fro(g.conv_state[l], states[l]) < TOL, l
+    nz = [0, 1, 3, 4, 5]
+    assert np.all(per_matrix_rel_fro(S[:, nz], wS[:, nz]) < 2 * TOL)
+    assert not f64(S[:, 2]).any() and not f64(g.conv_state[:, 2]).any()
+    assert rel_fro(x, wx) < TOL
+    # the FFNs are not no-ops here: without them the later layers' states move
+    plain = [synth.LALayerWeights(l.W_in, l.W_o, l.rms_gain, conv_w=l.conv_w, A_log=l.A_log,
+                                  dt_bias=l.dt_bias, o_norm_gain=l.o_norm_gain) for l in layers]
+    wS0, _ = oracle.replay_group(h, cu, plain, H, d, d, output_gate=True)
+    assert rel_fro(wS[1], wS0[1]) > 4 * TOL

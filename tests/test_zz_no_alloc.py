@@ -12,6 +12,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 import linear_attention_state_zero_b200 as tr
 from gpu_util import f64
@@ -35,6 +36,11 @@ def test_matches_workspace_entry_point_on_consecutive_calls(cuda_device):
         torch.cuda.synchronize()
         np.testing.assert_allclose(f64(per_a), f64(per_b), rtol=1e-12, atol=0)
         np.testing.assert_allclose(f64(tot_a), f64(tot_b), rtol=1e-12, atol=0)
+        # and directly against the oracle's fp64 definition (both sides sum fp32 inputs in
+        # fp64; only the summation order differs)
+        wper, wtot = oracle.state_error(S.cpu(), Sh.cpu())
+        np.testing.assert_allclose(f64(per_a), wper, rtol=1e-9, atol=0)
+        np.testing.assert_allclose(f64(tot_a)[0], wtot, rtol=1e-9, atol=0)
 
 
 def test_rejects_more_matrices_than_the_fixed_scratch(cuda_device):
