@@ -163,6 +163,9 @@ KERNEL_DESC = {
     "scan_out": "chunked scan, readout (bytes: o out)",
     "out_proj": "out-proj tcgen05 GEMM + residual (flops)",
     "scan_recurrent": "token-recurrent scan (bytes: q, k, v, gates in, o out)",
+    "scan_fused": "chunked scan, prep and chain in one launch (bytes: q, k, v, gates in, o and "
+                  "final state out)",
+    "scan_plan": "chunked scan plan (chunk offsets, longest-first order; bytes: none counted)",
 }
 
 
@@ -182,6 +185,11 @@ def kernel_work(name, layer, k):
         return "hbm", k * H * DH * 2
     if name == "out_proj":
         return "tensor", flops_outproj(k)
+    if name == "scan_fused":
+        return "hbm", k * H * ((2 if last else 3) * DH * 2 + 8 + (0 if last else DH * 2)) + \
+            H * DH * DH * 4
+    if name == "scan_plan":
+        return "hbm", 0.0
     if name == "scan_recurrent":
         return "hbm", k * H * ((2 if last else 3) * DH * 2 + 8 + (0 if last else DH * 2))
     raise KeyError(name)

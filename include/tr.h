@@ -72,9 +72,13 @@ enum {
                                 starts from its own cached FA output, so that FFN output
                                 rebuilds no state); x_out is then the residual after the
                                 last LA sublayer */,
-  TR_OUTPUT_GATE = 16u       /* tr_replay_group(s): every layer's W_in carries H d_v more
+  TR_OUTPUT_GATE = 16u,      /* tr_replay_group(s): every layer's W_in carries H d_v more
                                 rows (z, after v) and the readout goes through the gated
                                 RMSNorm before the output projection (see below) */
+  TR_SCAN_STALL_TEST = 256u  /* tr_gdn_scan, test hook: the chunked chain kernel never
+                                announces its first state, so its bounded waits run out
+                                (after tr_set_wait_limit_ns) and the call ends with
+                                TR_ERR_TIMEOUT at tr_check; outputs undefined */
 };
 
 /* Human-readable message for the last failing call on this host thread. */
@@ -117,7 +121,7 @@ int64_t tr_tail_len(int64_t m, int64_t r_num, int64_t r_den);
  *   o         [T, H, d_v] of `dtype`, or NULL to skip the readout.
  *   S_final   [N, H, d_k, d_v] fp32, required.  Must not alias S0.
  *   scale     readout scale (1.0 in every workload here).
- *   flags     TR_NORMALIZE_QK, TR_SCAN_RECURRENT.
+ *   flags     TR_NORMALIZE_QK, TR_SCAN_RECURRENT, TR_SCAN_STALL_TEST (test hook).
  * Supported: d_k, d_v in {64, 128}; dtype TR_DTYPE_BF16 (the chunked tensor-core
  * scan when d_k = 128 and N <= 1024, else the token-sequential kernel) or
  * TR_DTYPE_F32 (token-sequential fp32 FMA kernel, the test path);
@@ -378,6 +382,18 @@ tr_status tr_in_projection(const void *x_hat, const void *W_in, int64_t n_tokens
 tr_status tr_out_projection(const void *o, int64_t o_stride, const void *W_o, const void *x_res,
                             int32_t x_res_dtype, int64_t n_tokens, int32_t d_model,
                             int32_t hv, float *x_out, void *stream);
+
+/*
+ * tr_set_wait_limit_ns: the wall-clock limit of every bounded wait in the chunked scan's
+ * kernels (their mbarrier waits on copies, products and the other roles of a CTA), for
+ * calls made after it; 0 restores the default of 4 s, above 60 s is rejected.  A wait that
+ * runs out makes its CTA stop: it lets the copies and products it already issued finish
+ * (a drain bounded separately, at 0.2 s), writes no further output, and sets the device
+ * error word that tr_check reports as TR_ERR_TIMEOUT; the outputs of that call are then
+ * undefined, and later calls work normally.  Process-wide (not per thread or device).
+ * Every legitimate wait ends within microseconds; a short limit serves to test this path.
+ */
+tr_status tr_set_wait_limit_ns(uint64_t ns);
 
 /*
  * tr_check: waits for `stream`, then reads and clears the library's device error

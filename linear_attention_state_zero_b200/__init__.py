@@ -23,6 +23,7 @@ TR_OK = 0
 TR_DTYPE_F32, TR_DTYPE_BF16 = 0, 1
 TR_NORMALIZE_QK, TR_SKIP_LAST_OUTPUT, TR_SCAN_RECURRENT, TR_SKIP_LAST_FFN = 1, 2, 4, 8
 TR_OUTPUT_GATE = 16
+TR_SCAN_STALL_TEST = 256
 
 STATUS_NAMES = {0: "TR_OK", 1: "TR_ERR_INVALID_ARG", 2: "TR_ERR_SHAPE", 3: "TR_ERR_DTYPE",
                 4: "TR_ERR_ALIGNMENT", 5: "TR_ERR_UNSUPPORTED", 6: "TR_ERR_WORKSPACE",
@@ -85,6 +86,7 @@ _SIGNATURES = {
     "tr_out_projection": (ctypes.c_int, [c_vp, c_i64, c_vp, c_vp, c_i32, c_i64, c_i32, c_i32,
                                          c_vp, c_vp]),
     "tr_check": (ctypes.c_int, [c_vp]),
+    "tr_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64]),
 }
 
 
@@ -196,7 +198,8 @@ def tail_len(m: int, r_num: int, r_den: int) -> int:
 
 
 def gdn_scan(q, k, v, log_alpha, beta, cu_seqlens, *, S0=None, want_o=True, scale=1.0,
-             normalize_qk=False, recurrent=False, o=None, S_final=None, stream=None):
+             normalize_qk=False, recurrent=False, o=None, S_final=None, stream=None,
+             stall_test=False):
     """Eq. (1) scan over a packed batch: returns (o or None, S_final [N, H, d_k, d_v] fp32)."""
     dev_ = _need_cuda(q, k, v, log_alpha, beta, S0, o, S_final)
     T, H, dk = k.shape
@@ -214,7 +217,8 @@ def gdn_scan(q, k, v, log_alpha, beta, cu_seqlens, *, S0=None, want_o=True, scal
         o = None
     if S_final is None:
         S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=k.device)
-    flags = (TR_NORMALIZE_QK if normalize_qk else 0) | (TR_SCAN_RECURRENT if recurrent else 0)
+    flags = (TR_NORMALIZE_QK if normalize_qk else 0) | (TR_SCAN_RECURRENT if recurrent else 0) | \
+        (TR_SCAN_STALL_TEST if stall_test else 0)
     a = ScanArgs(N, H, dk, dv, T, _dtype_code(k), flags, float(scale),
                  q.stride(0) if q is not None else 0, k.stride(0), v.stride(0),
                  _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(be),
@@ -358,11 +362,18 @@ class GroupReplay:
                               self.host.data_ptr(), self._layer_arr, _ptr(self.S_hat),
                               _ptr(self.x_out), conv_width, _ptr(self.conv_state))
         self.ws_bytes = lib.tr_replay_group_workspace_size(ctypes.byref(self.args))
-        if workspace is None and self.ws_bytes:
-            workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev)
+        # allocated at the first run(): a description used only inside GroupsReplay (which
+        # has a workspace of its own) never holds one
         self.workspace = workspace
 
+    def _ws(self):
+        if self.workspace is None and self.ws_bytes:
+            self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8,
+                                         device=self.h_tail.device)
+        return self.workspace
+
     def run(self, stream=None):
+        self._ws()
         dev = self.h_tail.device
         with torch.cuda.device(dev):
             _ok(lib.tr_replay_group(ctypes.byref(self.args), _ptr(self.workspace), self.ws_bytes,
@@ -380,6 +391,7 @@ class GroupReplay:
     def run_profiled(self, event_handles, stream=None):
         """Same as run(), recording the given raw cudaEvent_t handles between kernel launches."""
         arr = (c_vp * len(event_handles))(*event_handles)
+        self._ws()
         dev = self.h_tail.device
         with torch.cuda.device(dev):
             _ok(lib.tr_replay_group_profiled(ctypes.byref(self.args), _ptr(self.workspace),
@@ -405,6 +417,9 @@ class GroupsReplay:
             self._arr[i] = g.args
         self.ws_bytes = lib.tr_replay_groups_workspace_size(self._arr, n)
         dev = self.groups[0].h_tail.device
+        for g in self.groups:
+            if g.h_tail.device != dev:
+                raise ValueError("every group must live on one device")
         self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev) \
             if self.ws_bytes else None
 
@@ -533,6 +548,11 @@ def out_projection(o, W_o, x_res, stream=None):
                                   _ptr(x_res), _dtype_code(x_res), T, D, hv, _ptr(out),
                                   _stream(stream, dev)), "tr_out_projection")
     return out
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Wall-clock limit of the scan kernels' bounded waits for later calls (0: the default 4 s)."""
+    _ok(lib.tr_set_wait_limit_ns(int(ns)), "tr_set_wait_limit_ns")
 
 
 def check(stream=None) -> None:

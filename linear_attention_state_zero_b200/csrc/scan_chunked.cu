@@ -2,34 +2,46 @@
 //
 // Eq. (1) (Tail-Replay reading notes, section 2.3) in the M = S^T layout,
 //   M_t = alpha_t (M_{t-1} - beta_t k_t (k_t^T M_{t-1})) + beta_t k_t v_t^T,
-// regrouped over chunks of C = 64 tokens (the WY / UT form of the delta rule,
-// derived here from Eq. (1)).  Inside a chunk, with g_t = sum_{s<=t} log alpha_s,
-// gamma_t = e^{g_t}, gamma'_t = e^{g_C - g_t} and the incoming state M_0:
-//   A_ts = beta_t e^{g_t - g_s} k_t.k_s  (s < t),   T = (I + A)^{-1}
-//   W = T diag(beta gamma) K,   U~ = T diag(beta) V
-//   P_ts = e^{g_t - g_s} q_t.k_s  (s <= t)
-//   chunk transition:  M_C = gamma_C M_0 + A_c M_0 + B_c
-//       A_c = -K^T diag(gamma') W   (d_k x d_k),   B_c = K^T diag(gamma') U~
-//   chunk readout:     O = R M_0 + O0,   R = diag(gamma) Q - P W,   O0 = P U~
-// Nothing but the transition and the readout depends on M_0, so the work splits in
-// three launches:
+// regrouped over chunks of C = 64 tokens (the WY / UT form of the delta rule, derived
+// here from Eq. (1)).  Inside chunk c, with g_t = sum_{s<=t} log alpha_s, gamma_t = e^{g_t},
+// gamma'_t = e^{g_C - g_t}, gamma_C = e^{g_C} and the state M_c at the chunk start:
+//   A_ts = beta_t e^{g_t - g_s} k_t.k_s (s < t),  T = (I + A)^{-1}
+//   W = T diag(beta gamma) K,  U~ = T diag(beta) V,  U_c = U~ - W M_c
+//   P_ts = e^{g_t - g_s} q_t.k_s (s <= t)
+//   output   O_c = diag(gamma) Q M_c + P U_c
+//   state    M_{c+1} = gamma_C M_c + K^T diag(gamma') U_c
+// Substituting M_{c+1} into U_{c+1} gives the look-ahead form the chain uses:
+//   U_{c+1} = U~_{c+1} - gamma_C W_{c+1} M_c - Y_{c+1} U_c,   Y_{c+1} = W_{c+1} (diag(gamma'_c) K_c)^T
+// so U_{c+1} needs M_c and U_c (not M_{c+1}): per chunk, one product of M_c and one of U_c
+// give both the chunk's output and the next chunk's U, and the state update runs beside
+// them.  Everything that does not depend on the state is computed first, for all chunks in
+// parallel:
 //
-//   scan_prep_kernel   persistent over all (chunk, head) items, in parallel:
-//     P1  [K; Q] K^T -> TMEM            (tcgen05, K-major operands)
-//     A, P on CUDA cores; T = (I + A)^{-1} by blocked forward substitution in fp32
-//     P2  [-T''; T'] [V | K] -> -U~, W  (T' = T diag(beta gamma), T'' = T diag(beta))
-//     P3  P W, P U~, K^T (gamma' W), K^T (gamma' U~) in one batch
-//     -> workspace, by TMA stores: A_c (bf16), R (bf16), B_c (fp32), O0 (fp32), gamma_C
-//   scan_chain_kernel  one CTA per (sequence, head, 64-column slice of d_v), sequential
-//     over the chunks: one tcgen05 product Z = A_c M_bf16 per chunk, then
-//     M <- gamma_C M + Z + B_c in fp32 registers; the bf16 chunk-start states go to the
-//     workspace.  Operands arrive by TMA, double-buffered one chunk ahead.
-//   scan_out_kernel    one CTA per (chunk, head), in parallel: o = R M_c + O0.
+//   scan_prep_kernel   persistent over all (chunk, head) items (256 threads):
+//     [Q; K] [K; K_prev]^T -> TMEM (tcgen05): P, A and Z = K_c (diag(gamma'_{c-1}) K_{c-1})^T
+//     T = (I + A)^{-1} on CUDA cores (blocked forward substitution, fp32)
+//     [T'; T''] [K | V | Z] -> W, U~, Y (T' = T diag(beta gamma), T'' = T diag(beta); T as a
+//        bf16 hi + lo pair for U~)
+//     -> workspace, by TMA stores: gamma Q, -gamma_C(prev) W, P, -Y, K (bf16), U~ (fp32),
+//        gamma' and gamma_C
+//   scan_chain_kernel  one CTA per (sequence, head, 64-column slice of d_v), sequential over
+//     the sequence's chunks, longest sequences first:
+//       D = [gamma Q_c; -gamma_C W_{c+1}] M_c + [P_c; -Y_{c+1}] U_c   (rows 0-63: O_c,
+//                                                   rows 64-127: U_{c+1} - U~_{c+1})
+//       dM = K_c^T (gamma' U_c),  M_{c+1} = gamma_C M_c + dM  (fp32 registers; gamma' U_c
+//       as a bf16 hi + lo pair, so the state's update keeps fp32-level accuracy)
+//     warp-specialised: a TMA producer, an MMA issuer, four state warps, four output warps.
+//   scan_plan_kernel   (only for more than kParamSeqs sequences) chunk offsets per sequence
+//     and the longest-first order; fewer sequences get both from the host in the launch.
 //
-// Every M-dependent product acts column by column on d_v, so d_v splits into
-// exact 64-column slices.  Tokens past the end of a sequence get beta = 0 and
-// log alpha = 0: their rows of T are the identity and their W, U~ rows vanish.
+// Every M-dependent product acts column by column on d_v, so d_v splits into exact
+// 64-column slices.  Tokens past the end of a sequence get beta = 0 and log alpha = 0: their
+// rows of T are the identity, their W, U~ and Y rows vanish, and so do their U rows.
 #include <cuda_bf16.h>
+
+#include <algorithm>
+#include <atomic>
+#include <numeric>
 
 #include "../../include/tr.h"
 #include "tr_internal.h"
@@ -41,10 +53,11 @@ namespace {
 constexpr int C = 64;      // chunk length
 constexpr int DK = 128;    // key dimension handled here
 constexpr int DVS = 64;    // d_v columns per chain CTA
+constexpr int kParamSeqs = 64;   // up to this many sequences, the plan travels in the launch
 
 // --------------------------------------------------------------- helpers
-// Shared-memory descriptors are built once per operand (sw128_desc) and advanced
-// per K step by adding to the 16-byte start-address field only.
+// Shared-memory descriptors are built once per operand (sw128_desc) and advanced per K
+// step by adding to the 16-byte start-address field only.
 //   K-major operand: 128-byte rows, 64-column halves `half_stride` bytes apart; K step kk
 //   (16 elements) starts 32 bytes further inside the 128-byte swizzle atom.
 //   MN-major operand: rows are the K dimension, 128-byte rows hold 64 M/N elements
@@ -82,6 +95,16 @@ __device__ __forceinline__ void store_row32_f32(uint8_t *tile, int row, const fl
                  __float_as_uint(v[4 * ch + 2] * s), __float_as_uint(v[4 * ch + 3] * s));
 }
 
+// One row (32 floats = 128 B) of a 128-byte-swizzled fp32 tile.
+__device__ __forceinline__ void load_row32_f32(const uint8_t *tile, int row, float *f) {
+#pragma unroll
+  for (int ch = 0; ch < 8; ++ch) {
+    const float4 u = *reinterpret_cast<const float4 *>(
+        tile + sw128_offset((uint32_t)row, (uint32_t)ch * 16u));
+    f[4 * ch] = u.x; f[4 * ch + 1] = u.y; f[4 * ch + 2] = u.z; f[4 * ch + 3] = u.w;
+  }
+}
+
 // 8 consecutive bf16 of row `row` starting at column col0 (multiple of 8).
 __device__ __forceinline__ void load_row8_bf16(const uint8_t *tile, int row, int col0, float *f) {
   const uint4 u = *reinterpret_cast<const uint4 *>(
@@ -94,121 +117,6 @@ __device__ __forceinline__ void load_row8_bf16(const uint8_t *tile, int row, int
     f[2 * i + 1] = t.y;
   }
 }
-
-
-// sum over sequences i < seq of ceil(len_i / C); every thread of the CTA gets the value
-__device__ int chunk_base(const int32_t *cu, int seq, int *red) {
-  int s = 0;
-  for (int i = threadIdx.x; i < seq; i += blockDim.x) s += (cu[i + 1] - cu[i] + C - 1) / C;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
-  __syncthreads();
-  int t = 0;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
-  __syncthreads();
-  return t;
-}
-
-// L2-normalise one 128-element bf16 row of a KQ tile in place (TR_NORMALIZE_QK).
-__device__ __forceinline__ void normalize_row(uint8_t *kq, int row) {
-  float ss = 0.f;
-  for (int c0 = 0; c0 < DK; c0 += 8) {
-    float f[8];
-    load_row8_bf16(kq + (c0 >> 6) * 16384, row, c0 & 63, f);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) ss = fmaf(f[i], f[i], ss);
-  }
-  const float inv = rsqrtf(ss + 1e-6f);
-  for (int c0 = 0; c0 < DK; c0 += 8) {
-    float f[8];
-    uint8_t *h = kq + (c0 >> 6) * 16384;
-    load_row8_bf16(h, row, c0 & 63, f);
-    const uint32_t off = sw128_offset((uint32_t)row, (uint32_t)(c0 & 63) * 2u);
-    st_shared_v4(smem_u32(h + off), pack_bf16x2(f[0] * inv, f[1] * inv),
-                 pack_bf16x2(f[2] * inv, f[3] * inv), pack_bf16x2(f[4] * inv, f[5] * inv),
-                 pack_bf16x2(f[6] * inv, f[7] * inv));
-  }
-}
-
-// workspace arrays (slot = (first chunk of the sequence + chunk) * H + head)
-struct ScanWs {
-  __nv_bfloat16 *A;  // [slots][128][128]  A_c = -K^T diag(gamma') W
-  __nv_bfloat16 *R;  // [slots][64][128]   R = diag(gamma) Q - P W
-  float *B;          // [slots][128][dv]   B_c = K^T diag(gamma') U~
-  float *O;          // [slots][64][dv]    O0 = P U~
-  float *G;          // [slots]            gamma_C
-  __nv_bfloat16 *M;  // [slots][128][dv]   bf16 state at the chunk start (chain -> readout)
-  int64_t slots;
-};
-
-size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
-
-int64_t count_slots(const ScanLaunch &p, int *max_chunks) {
-  int64_t n = 0;
-  int mx = 0;
-  for (int i = 0; i < p.n_seqs; ++i) {
-    const int c = (p.cu_seqlens_host[i + 1] - p.cu_seqlens_host[i] + C - 1) / C;
-    n += c;
-    mx = c > mx ? c : mx;
-  }
-  if (max_chunks) *max_chunks = mx;
-  return n * p.H;
-}
-
-ScanWs ws_layout(const ScanLaunch &p, void *base, size_t *total) {
-  ScanWs w{};
-  w.slots = count_slots(p, nullptr);
-  const size_t S = (size_t)w.slots;
-  size_t off = 0;
-  const size_t oA = off; off = align256(off + S * 128 * 128 * 2);
-  const size_t oR = off; off = align256(off + S * 64 * 128 * 2);
-  const size_t oB = off; off = align256(off + S * 128 * (size_t)p.dv * 4);
-  const size_t oO = off; off = align256(off + S * 64 * (size_t)p.dv * 4);
-  const size_t oG = off; off = align256(off + S * 4);
-  const size_t oM = off; off = align256(off + S * 128 * (size_t)p.dv * 2);
-  if (total) *total = off;
-  uint8_t *b = static_cast<uint8_t *>(base);
-  if (b) {
-    w.A = reinterpret_cast<__nv_bfloat16 *>(b + oA);
-    w.R = reinterpret_cast<__nv_bfloat16 *>(b + oR);
-    w.B = reinterpret_cast<float *>(b + oB);
-    w.O = reinterpret_cast<float *>(b + oO);
-    w.G = reinterpret_cast<float *>(b + oG);
-    w.M = reinterpret_cast<__nv_bfloat16 *>(b + oM);
-  }
-  return w;
-}
-
-// ============================================================ prep kernel
-// 256 threads, persistent over work items (slot order: chunk-major, head-minor), with
-// the next items' K/Q/V tiles prefetched by TMA into a second buffer.
-// shared memory (bytes from a 1024-aligned base):
-constexpr uint32_t P_IN = 0;          // 2 x 48 KB: [KQ 32 KB: half x (K rows 0-63 | Q rows 64-127)][V 16 KB]
-constexpr uint32_t P_IN_BYTES = 49152;
-constexpr uint32_t P_AP = 98304;      // 128 x 64 bf16: rows 0-63 zero, 64-127 = P
-constexpr uint32_t P_TSH = 114688;    // [-T''; T'] high bf16 parts   (after P2: gamma' U~ high)
-constexpr uint32_t P_TSL = 131072;    // [-T''; T'] low bf16 parts    (after P2: gamma' U~ low)
-constexpr uint32_t P_AW = 147456;     // A fp32 [64][68] during the inverse; then W (16 KB) + gamma' W
-constexpr uint32_t P_TU = 180224;     // T fp32 [64][68] + X fp32 [32][36]; then U~ high + U~ low
-constexpr uint32_t P_END = 212992;
-constexpr int LDA = 68;               // fp32 row stride of A and T (16-byte aligned rows)
-constexpr int LDX = 36;
-constexpr size_t PREP_SMEM = P_END + 1024 + 1024;
-constexpr int kPrepThreads = 256;
-constexpr int kMaxSeqsChunked = 1024;
-
-struct PrepCtl {
-  uint64_t tma_bar[2];
-  uint64_t mma_bar;
-  uint32_t tmem;
-  int abort;
-  float g[C];      // inclusive cumsum of log alpha over the chunk
-  float beta[C];
-  float bg[C];     // beta * gamma
-  int cu_chunks[kMaxSeqsChunked + 1];
-  int cu_tok[kMaxSeqsChunked + 1];  // the sequence offsets (cu_seqlens)
-};
 
 // hi + lo bf16 split of 32 values (v[i] * s) into two 128-byte-row swizzled tiles.
 __device__ __forceinline__ void store_row_split(uint8_t *hi, uint8_t *lo, int row, int col0,
@@ -231,53 +139,302 @@ __device__ __forceinline__ void store_row_split(uint8_t *hi, uint8_t *lo, int ro
   }
 }
 
-// Output staging after the last product of an item (every region below is free by then;
-// each tile is 128-byte swizzled, one TMA box):
-//   A_c  [2 halves][128 rows][64 bf16]  at P_TU
-//   B_c  [DV/32 boxes][128 rows][32 fp32] at P_TSH (spans TSH, TSL, AW)
-//   R    [2 halves][64 rows][64 bf16]   at P_AP
-//   O0   [DV/32 boxes][64 rows][32 fp32] in the item's input buffer, over the K rows and V
-//        (the Q rows stay intact: R reads them)
-__device__ __forceinline__ uint32_t o0_box_offset(int b) {
-  return b < 2 ? (uint32_t)b * 16384u : 32768u + (uint32_t)(b - 2) * 8192u;
+// Scale 32 bf16 of row `row`, columns col0..col0+31, of a swizzled tile in place.
+__device__ __forceinline__ void scale_row32_bf16(uint8_t *tile, int row, int col0, float s) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    float f[8];
+    load_row8_bf16(tile, row, col0 + 8 * w, f);
+    const uint32_t off = sw128_offset((uint32_t)row, (uint32_t)(col0 + 8 * w) * 2u);
+    st_shared_v4(smem_u32(tile + off), pack_bf16x2(f[0] * s, f[1] * s),
+                 pack_bf16x2(f[2] * s, f[3] * s), pack_bf16x2(f[4] * s, f[5] * s),
+                 pack_bf16x2(f[6] * s, f[7] * s));
+  }
 }
 
-// The prep work of one CTA: items first, then second, second + stride, ... (256 threads;
-// every barrier is the named barrier 1 over those threads).
+// ------------------------------------------------------------------ plan
+// cu_chunks[i] = sum_{j < i} ceil(len_j / C) (i = 0..n), and the sequences ordered by
+// chunk count, longest first (ties by index).
+struct ScanPlan {
+  int32_t cu_chunks[kParamSeqs + 1];
+  int32_t order[kParamSeqs];
+  int in_params;     // 1: the arrays above hold the plan; 0: it is in the workspace
+};
+
+// workspace arrays (slot = (cu_chunks[seq] + chunk) * H + head)
+struct ScanWs {
+  __nv_bfloat16 *QW;  // [slots][128][128]: rows 0-63 gamma Q, rows 64-127 -gamma_C(prev) W
+  __nv_bfloat16 *PY;  // [slots][128][64]:  rows 0-63 P, rows 64-127 -Y
+  __nv_bfloat16 *KT;  // [slots][64][128]:  K (L2-normalised in place with TR_NORMALIZE_QK)
+  float *UT;          // [slots][64][dv]:   U~
+  float *GP;          // [slots][64]:       gamma'
+  float *G;           // [slots][4]:        gamma_C (16 bytes per slot, for one bulk copy)
+  int32_t *cu_chunks; // [n_seqs + 1]       (plan kernel output; unused with a launch plan)
+  int32_t *order;     // [n_seqs]
+  unsigned long long *flags;  // [slots]: the call's epoch once the slot is stored (fused launch)
+  int64_t slots;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int64_t count_chunks(const ScanLaunch &p) {
+  int64_t n = 0;
+  for (int i = 0; i < p.n_seqs; ++i)
+    n += (p.cu_seqlens_host[i + 1] - p.cu_seqlens_host[i] + C - 1) / C;
+  return n;
+}
+
+ScanWs ws_layout(const ScanLaunch &p, void *base, size_t *total) {
+  ScanWs w{};
+  w.slots = count_chunks(p) * p.H;
+  const size_t S = (size_t)w.slots;
+  size_t off = 0;
+  const size_t oQW = off; off = align256(off + S * 128 * 128 * 2);
+  const size_t oPY = off; off = align256(off + S * 128 * 64 * 2);
+  const size_t oKT = off; off = align256(off + S * 64 * 128 * 2);
+  const size_t oUT = off; off = align256(off + S * 64 * (size_t)p.dv * 4);
+  const size_t oGP = off; off = align256(off + S * 64 * 4);
+  const size_t oG = off;  off = align256(off + S * 16);
+  const size_t oCU = off; off = align256(off + (size_t)(p.n_seqs + 1) * 4);
+  const size_t oOR = off; off = align256(off + (size_t)(p.n_seqs + 1) * 4);
+  const size_t oFL = off; off = align256(off + S * 8);
+  if (total) *total = off;
+  uint8_t *b = static_cast<uint8_t *>(base);
+  if (b) {
+    w.QW = reinterpret_cast<__nv_bfloat16 *>(b + oQW);
+    w.PY = reinterpret_cast<__nv_bfloat16 *>(b + oPY);
+    w.KT = reinterpret_cast<__nv_bfloat16 *>(b + oKT);
+    w.UT = reinterpret_cast<float *>(b + oUT);
+    w.GP = reinterpret_cast<float *>(b + oGP);
+    w.G = reinterpret_cast<float *>(b + oG);
+    w.cu_chunks = reinterpret_cast<int32_t *>(b + oCU);
+    w.order = reinterpret_cast<int32_t *>(b + oOR);
+    w.flags = reinterpret_cast<unsigned long long *>(b + oFL);
+  }
+  return w;
+}
+
+constexpr int kPlanThreads = 1024;
+constexpr int kSortMax = 4096;   // longest-first order for up to this many sequences
+
+// One block: chunk offsets by a block-wide scan, then the longest-first order by a bitonic
+// sort of (chunk count, index) keys in shared memory (the identity order beyond kSortMax).
+__global__ void __launch_bounds__(kPlanThreads)
+    scan_plan_kernel(const int32_t *cu_seqlens, int n_seqs, int32_t *cu_chunks, int32_t *order) {
+  __shared__ unsigned long long keys[kSortMax];
+  __shared__ int warp_sum[kPlanThreads / 32];
+  __shared__ int carry_s;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_trigger();
+  pdl_wait();
+  if (tid == 0) carry_s = 0;
+  __syncthreads();
+  for (int base = 0; base < n_seqs; base += kPlanThreads) {
+    const int i = base + tid;
+    const int nch = i < n_seqs ? (cu_seqlens[i + 1] - cu_seqlens[i] + C - 1) / C : 0;
+    int x = nch;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sum[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int w = warp_sum[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      warp_sum[lane] = w;   // inclusive over warps
+    }
+    __syncthreads();
+    const int carry = carry_s;
+    const int excl = carry + (warp > 0 ? warp_sum[warp - 1] : 0) + x - nch;
+    if (i < n_seqs) {
+      cu_chunks[i] = excl;
+      if (n_seqs <= kSortMax)
+        keys[i] = ((unsigned long long)(0x7fffffff - nch) << 32) | (unsigned)i;
+    }
+    __syncthreads();
+    if (tid == 0) carry_s = carry + warp_sum[kPlanThreads / 32 - 1];
+    __syncthreads();
+  }
+  if (tid == 0) cu_chunks[n_seqs] = carry_s;
+  if (n_seqs > kSortMax) {
+    for (int i = tid; i < n_seqs; i += kPlanThreads) order[i] = i;
+    return;
+  }
+  int n2 = 1;
+  while (n2 < n_seqs) n2 <<= 1;
+  for (int i = n_seqs + tid; i < n2; i += kPlanThreads) keys[i] = ~0ull;
+  __syncthreads();
+  for (int k = 2; k <= n2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < n2; i += kPlanThreads) {
+        const int l = i ^ j;
+        if (l > i) {
+          const unsigned long long a = keys[i], b = keys[l];
+          const bool up = (i & k) == 0;
+          if ((a > b) == up) {
+            keys[i] = b;
+            keys[l] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = tid; i < n_seqs; i += kPlanThreads) order[i] = (int32_t)(keys[i] & 0xffffffffu);
+}
+
+__device__ __forceinline__ const int32_t *plan_cu_chunks(const ScanPlan &pl, const ScanWs &ws) {
+  return pl.in_params ? pl.cu_chunks : ws.cu_chunks;
+}
+__device__ __forceinline__ const int32_t *plan_order(const ScanPlan &pl, const ScanWs &ws) {
+  return pl.in_params ? pl.order : ws.order;
+}
+
+// ============================================================ prep kernel
+// 256 threads, persistent over work items (item = chunk_global * H + head, CTA b takes
+// items b, b + grid, ...); the next item's tiles are prefetched by TMA into the other
+// input stage.  Shared memory (bytes from a 1024-aligned base):
+//   stage s (64 KB at s * 64 KB): half h (d_k columns 64h..64h+63) at + 32 KB h, bands of
+//   64 rows x 128 B at + 8 KB b: b = 0 Q, 1 K, 2 K of the previous chunk, 3 V (d_v
+//   columns 64h..).  After the item's products the Q band holds gamma Q and the
+//   previous-K band -gamma_C(prev) W: they are stored from there, with the K band.
+constexpr uint32_t P_STAGE = 65536;
+constexpr uint32_t P_AF = 131072;         // A fp32 [64][68]
+constexpr uint32_t P_TF = P_AF + 17408;   // T fp32 [64][68], then X fp32 [32][36]
+constexpr uint32_t P_THI = 171008;        // [T'; T''] high bf16 parts [128][64] (then U~ staging)
+constexpr uint32_t P_TLO = P_THI + 16384; // low parts
+constexpr uint32_t P_P = P_TLO + 16384;   // P bf16 [64][64]
+constexpr uint32_t P_Z = P_P + 8192;      // Z bf16 [64][64] (then -Y staging)
+constexpr uint32_t P_END = P_Z + 8192;
+constexpr int LDA = 68;                   // fp32 row stride of A and T (16-byte aligned rows)
+constexpr int LDX = 36;
+constexpr size_t PREP_SMEM = P_END + 1024;
+constexpr int kPrepThreads = 256;
+static_assert(P_TF + 17408 + 4608 <= P_THI, "prep shared-memory layout");
+static_assert(P_THI % 1024 == 0 && P_P % 1024 == 0 && P_Z % 1024 == 0,
+              "swizzled tiles are 1024-byte aligned");
+static_assert(PREP_SMEM <= 232448, "prep shared memory");
+
+struct PrepItem {
+  int seq, c, head, t0, nv, has_prev;
+  int64_t slot;
+};
+
+struct PrepCtl {
+  uint64_t tma_bar[2];
+  uint64_t mma_bar;
+  uint64_t drain_bar;
+  uint32_t tmem;
+  int abort;
+  PrepItem cur, nxt;
+  float g[C];      // inclusive cumsum of log alpha over the chunk
+  float beta[C];
+  float bg[C];     // beta * gamma
+  float gp[C];     // gamma' = e^{g_C - g_t}
+  float gpp[C];    // the previous chunk's gamma'
+  float gq[C];     // gamma
+  float gpv[C];    // the previous chunk's cumsum
+  float gc_prev;   // the previous chunk's gamma_C (1 without one)
+};
+
+// The item's location given its sequence (cu_chunks[seq] <= chunk < cu_chunks[seq + 1]).
+__device__ __forceinline__ PrepItem item_at(int64_t item, int seq, const ScanLaunch &p,
+                                            const int32_t *cu_chunks) {
+  PrepItem it;
+  const int chunk = (int)(item / p.H);
+  it.seq = seq;
+  it.c = chunk - cu_chunks[seq];
+  it.head = (int)(item % p.H);
+  it.t0 = p.cu_seqlens[seq] + it.c * C;
+  it.nv = min(C, p.cu_seqlens[seq + 1] - it.t0);
+  it.has_prev = it.c > 0;
+  it.slot = item;
+  return it;
+}
+// First item of a CTA: binary search for the last sequence whose first chunk is <= chunk
+// and that owns chunks (sequences without tokens own none).
+__device__ int seq_of_chunk(int chunk, int n_seqs, const int32_t *cu_chunks) {
+  int lo = 0, hi = n_seqs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (cu_chunks[mid] <= chunk) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+// Later items: chunks only grow, so the sequence index only moves forward.
+__device__ __forceinline__ int advance_seq(int seq, int chunk, const int32_t *cu_chunks) {
+  while (cu_chunks[seq + 1] <= chunk) ++seq;
+  return seq;
+}
+
+// L2-normalise one 128-element bf16 row of band `band` (row r) in place (TR_NORMALIZE_QK).
+__device__ __forceinline__ void normalize_band_row(uint8_t *stage, int band, int r) {
+  float ss = 0.f;
+  for (int c0 = 0; c0 < DK; c0 += 8) {
+    float f[8];
+    load_row8_bf16(stage + (c0 >> 6) * 32768 + band * 8192, r, c0 & 63, f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss = fmaf(f[i], f[i], ss);
+  }
+  const float inv = rsqrtf(ss + 1e-6f);
+  for (int c0 = 0; c0 < DK; c0 += 32)
+    scale_row32_bf16(stage + (c0 >> 6) * 32768 + band * 8192, r, c0 & 63, inv);
+}
+
+// The maps both kernels' bodies read (prep: q, k, v in; workspace out; chain: workspace in,
+// o out).
+struct ScanMaps {
+  CUtensorMap q, k, v, QW, PY, KT, UT, o;
+};
+
+// Publish item `slot` as complete for the chain running beside the prep (fused launch):
+// its output stores have completed; the release store orders them before the flag.
+__device__ __forceinline__ void publish_slot(const ScanWs &ws, int64_t slot, unsigned long long epoch) {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(ws.flags + slot), "l"(epoch) : "memory");
+}
+
+// The prep work of CTA `vb` of `vg` (256 threads: warps 0-7).  With `publish`, each item's
+// flag is set once its stores have completed (one item later, so thread 0 never waits).
 template <int DV>
-__device__ __forceinline__ void prep_body(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
-                                          const CUtensorMap &tm_v, const CUtensorMap &tm_A,
-                                          const CUtensorMap &tm_B, const CUtensorMap &tm_R,
-                                          const CUtensorMap &tm_O, const ScanLaunch &p,
-                                          const ScanWs &ws, int total_chunks, int64_t first,
-                                          int64_t second, int64_t stride) {
+__device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &p, const ScanWs &ws,
+                                          const ScanPlan &plan, int vb, int vg, bool publish) {
+  const CUtensorMap &tm_q = mp.q, &tm_k = mp.k, &tm_v = mp.v, &tm_QW = mp.QW, &tm_PY = mp.PY,
+                    &tm_KT = mp.KT, &tm_UT = mp.UT;
   extern __shared__ uint8_t smem_raw[];
   __shared__ PrepCtl ctl_s;
   PrepCtl *ctl = &ctl_s;
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
-  float *As = reinterpret_cast<float *>(sm + P_AW);
-  float *Ts = reinterpret_cast<float *>(sm + P_TU);
+  float *As = reinterpret_cast<float *>(sm + P_AF);
+  float *Ts = reinterpret_cast<float *>(sm + P_TF);
   float *Xs = Ts + C * LDA;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, hsel = warp >> 2;   // TMEM lane quarter, column half
   const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-  const int row = q4 * 32 + lane;              // TMEM lane = row of a 128-row result
-  const int H = p.H;
   const bool want_o = p.o != nullptr;
-  const int64_t n_items = (int64_t)total_chunks * H;
+  const int64_t n_items = ws.slots;
+  const int64_t stride = vg;
+  const int32_t *cu_chunks = plan_cu_chunks(plan, ws);
 
   if (tid == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
-    tma_prefetch_desc(&tm_A);
-    tma_prefetch_desc(&tm_B);
-    tma_prefetch_desc(&tm_R);
-    tma_prefetch_desc(&tm_O);
+    tma_prefetch_desc(&tm_QW);
+    tma_prefetch_desc(&tm_PY);
+    tma_prefetch_desc(&tm_KT);
+    tma_prefetch_desc(&tm_UT);
     mbar_init(smem_u32(&ctl->tma_bar[0]), 1);
     mbar_init(smem_u32(&ctl->tma_bar[1]), 1);
     mbar_init(smem_u32(&ctl->mma_bar), 1);
+    mbar_init(smem_u32(&ctl->drain_bar), 1);
     ctl->abort = 0;
     fence_mbar_init();
   }
@@ -285,178 +442,197 @@ __device__ __forceinline__ void prep_body(const CUtensorMap &tm_q, const CUtenso
     tmem_alloc(smem_u32(&ctl->tmem), 512);
     tmem_relinquish();
   }
-  for (int i = tid; i < 8192 / 16; i += kPrepThreads) st_shared_v4(smem_u32(sm + P_AP) + 16 * i, 0, 0, 0, 0);
-  if (!want_o)
-    for (int i = tid; i < 4 * 8192 / 16; i += kPrepThreads) {
-      const int blk = i >> 9;  // (buffer, half)
-      st_shared_v4(smem_u32(sm + P_IN + (blk >> 1) * P_IN_BYTES + (blk & 1) * 16384 + 8192) +
-                       16 * (i & 511), 0, 0, 0, 0);
-    }
   tc_fence_before();
   bar_sync_n(1, kPrepThreads);
   tc_fence_after();
   const uint32_t tmem = ctl->tmem;
-  const AbortFlag ab{&ctl->abort, p.err_word, ERRBIT_SCAN_TIMEOUT};
+  const AbortFlag ab{&ctl->abort, p.err_word, ERRBIT_SCAN_TIMEOUT, p.wait_ns};
   // TMEM is held: let the next kernel launch; then wait for the previous one's outputs
   pdl_trigger();
   pdl_wait();
-  // first chunk of every sequence
-  if (tid == 0) {
-    int acc = 0;
-    for (int i = 0; i < p.n_seqs; ++i) {
-      ctl->cu_chunks[i] = acc;
-      acc += (p.cu_seqlens[i + 1] - p.cu_seqlens[i] + C - 1) / C;
-    }
-    ctl->cu_chunks[p.n_seqs] = acc;
-  }
-  for (int i = tid; i <= p.n_seqs; i += kPrepThreads) ctl->cu_tok[i] = p.cu_seqlens[i];
-  bar_sync_n(1, kPrepThreads);
 
-  // (sequence, chunk) of an item
-  auto locate = [&](int64_t item, int &seq, int &cc) {
-    const int chunk = (int)(item / H);
-    int lo = 0, hi = p.n_seqs - 1;
-    while (lo < hi) {  // last sequence whose first chunk is <= chunk
-      const int mid = (lo + hi + 1) >> 1;
-      if (ctl->cu_chunks[mid] <= chunk) lo = mid; else hi = mid - 1;
-    }
-    seq = lo;
-    cc = chunk - ctl->cu_chunks[lo];
-  };
-  auto issue = [&](int64_t item, int buf) {
-    int seq, cc;
-    locate(item, seq, cc);
-    const int head = (int)(item % H);
-    const int t0 = ctl->cu_tok[seq] + cc * C;
+  int fills[2] = {0, 0};   // TMA fills issued per stage (thread 0)
+  int64_t prev_slot = -1;  // thread 0: the last item whose flag is not yet published
+  auto issue = [&](const PrepItem &it, int buf) {
     const uint32_t bar = smem_u32(&ctl->tma_bar[buf]);
-    const uint32_t kq = smem_u32(sm + P_IN + buf * P_IN_BYTES);
-    mbar_arrive_expect_tx(bar, 16384u + (want_o ? 16384u : 0u) + (uint32_t)DV * 128u);
-    tma_load_2d(kq, &tm_k, head * DK, t0, bar);
-    tma_load_2d(kq + 16384, &tm_k, head * DK + 64, t0, bar);
-    if (want_o) {
-      tma_load_2d(kq + 8192, &tm_q, head * DK, t0, bar);
-      tma_load_2d(kq + 16384 + 8192, &tm_q, head * DK + 64, t0, bar);
+    const uint32_t st = smem_u32(sm + buf * P_STAGE);
+    const uint32_t bytes = 16384u + (want_o ? 16384u : 0u) + (it.has_prev ? 16384u : 0u) +
+                           (uint32_t)DV * 128u;
+    mbar_arrive_expect_tx(bar, bytes);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int x = it.head * DK + 64 * h;
+      if (want_o) tma_load_2d(st + h * 32768, &tm_q, x, it.t0, bar);
+      tma_load_2d(st + h * 32768 + 8192, &tm_k, x, it.t0, bar);
+      if (it.has_prev) tma_load_2d(st + h * 32768 + 16384, &tm_k, x, it.t0 - C, bar);
     }
 #pragma unroll
-    for (int b = 0; b < DV / 64; ++b)
-      tma_load_2d(kq + 32768 + 8192 * b, &tm_v, head * DV + 64 * b, t0, bar);
+    for (int h = 0; h < DV / 64; ++h)
+      tma_load_2d(st + h * 32768 + 24576, &tm_v, it.head * DV + 64 * h, it.t0, bar);
+    ++fills[buf];
   };
-  if (tid == 0) {
-    fence_proxy_async_smem();
-    if (first < n_items) issue(first, 0);
-    if (second < n_items) issue(second, 1);
-  }
-  // log alpha and beta of an item's 64 tokens (thread tid < C: token tid; 0 past the end)
-  auto load_gates = [&](int64_t it, float &la, float &b) {
-    int sq, cq;
-    locate(it, sq, cq);
-    const int hd = (int)(it % H);
-    const int tt = ctl->cu_tok[sq] + cq * C;
+  // an item's gates, loaded into registers one item ahead: token tid (< 64) of the chunk,
+  // and (threads 64..127) token tid - 64 of the previous chunk
+  auto load_gates = [&](const PrepItem &it, float &la, float &b) {
     la = 0.f;
     b = 0.f;
-    if (tid < min(C, ctl->cu_tok[sq + 1] - tt)) {
-      la = p.log_alpha[(size_t)(tt + tid) * H + hd];
-      b = p.beta[(size_t)(tt + tid) * H + hd];
+    if (tid < C) {
+      if (tid < it.nv) {
+        la = p.log_alpha[(size_t)(it.t0 + tid) * p.H + it.head];
+        b = p.beta[(size_t)(it.t0 + tid) * p.H + it.head];
+      }
+    } else if (tid < 2 * C && it.has_prev) {
+      la = p.log_alpha[(size_t)(it.t0 - C + (tid - C)) * p.H + it.head];
     }
   };
-  // the next item's gates are loaded during the current item
+
+  int64_t item = vb;
+  int seq_cur = 0;   // thread 0: the sequence of the current item
   float la_next = 0.f, b_next = 0.f;
-  if (tid < C && first < n_items) load_gates(first, la_next, b_next);
-  auto next_item = [&](int64_t it) -> int64_t { return it == first ? second : it + stride; };
+  if (tid == 0 && item < n_items) {
+    seq_cur = seq_of_chunk((int)(item / p.H), p.n_seqs, cu_chunks);
+    seq_cur = advance_seq(seq_cur, (int)(item / p.H), cu_chunks);
+    ctl->cur = item_at(item, seq_cur, p, cu_chunks);
+    fence_proxy_async_smem();
+    issue(ctl->cur, 0);
+  }
+  bar_sync_n(1, kPrepThreads);
+  if (item < n_items) load_gates(ctl->cur, la_next, b_next);
+
   const uint32_t mma_bar = smem_u32(&ctl->mma_bar);
   uint32_t mma_phase = 0;
+  bool mma_pending = false;   // thread 0: products issued whose completion was not seen
   auto mma_wait = [&]() -> bool {
     const bool ok = mbar_wait(mma_bar, mma_phase, ab);
     mma_phase ^= 1u;
+    if (tid == 0 && ok) mma_pending = false;
     if (bar_or_n(1, kPrepThreads, !ok)) return false;
     tc_fence_after();
     return true;
   };
 
   int n = 0;
-  for (int64_t item = first; item < n_items; item = next_item(item), ++n) {
+  for (; item < n_items; item += stride, ++n) {
     const int buf = n & 1;
-    uint8_t *KQ = sm + P_IN + buf * P_IN_BYTES;
-    const uint32_t kq_u = smem_u32(KQ);
-    const uint32_t v_u = kq_u + 32768;
+    uint8_t *ST = sm + buf * P_STAGE;
+    const uint32_t st_u = smem_u32(ST);
+    const PrepItem it = ctl->cur;
+    const bool has_next = item + stride < n_items;
 
-    // gates: g = inclusive cumsum of log alpha (0 past the end), beta, beta * gamma
-    if (tid < C) {
+    // gates: g = inclusive cumsum of log alpha (0 past the end), and the previous chunk's
+    if (tid < 2 * C) {
       const float la = la_next, b = b_next;
-      if (next_item(item) < n_items) load_gates(next_item(item), la_next, b_next);
       float s = la;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const float y = __shfl_up_sync(0xffffffffu, s, o);
         if (lane >= o) s += y;
       }
-      ctl->g[tid] = s;
-      ctl->beta[tid] = b;
+      if (tid < C) {
+        ctl->g[tid] = s;
+        ctl->beta[tid] = b;
+      } else {
+        ctl->gpv[tid - C] = s;
+      }
     }
     bar_sync_n(1, kPrepThreads);
     if (tid >= 32 && tid < C) ctl->g[tid] += ctl->g[31];
+    if (tid >= C + 32 && tid < 2 * C) ctl->gpv[tid - C] += ctl->gpv[31];
     bar_sync_n(1, kPrepThreads);
-    if (tid < C) ctl->bg[tid] = ctl->beta[tid] * exp_ftz(ctl->g[tid]);
+    if (tid < C) {
+      const float gt = ctl->g[tid];
+      ctl->gq[tid] = exp_ftz(gt);
+      ctl->bg[tid] = ctl->beta[tid] * ctl->gq[tid];
+      ctl->gp[tid] = exp_ftz(ctl->g[C - 1] - gt);
+    } else if (tid < 2 * C) {
+      ctl->gpp[tid - C] = it.has_prev ? exp_ftz(ctl->gpv[C - 1] - ctl->gpv[tid - C]) : 0.f;
+    } else if (tid == 2 * C) {
+      ctl->gc_prev = it.has_prev ? exp_ftz(ctl->gpv[C - 1]) : 1.f;
+    }
     const bool ok_tma = mbar_wait(smem_u32(&ctl->tma_bar[buf]), (uint32_t)(n >> 1) & 1u, ab);
     if (bar_or_n(1, kPrepThreads, !ok_tma)) break;
     if (p.flags & TR_NORMALIZE_QK) {
-      if (tid < C || (tid < 2 * C && want_o)) normalize_row(KQ, tid);
+      if (tid < C) normalize_band_row(ST, 1, tid);
+      else if (tid < 2 * C && want_o) normalize_band_row(ST, 0, tid - C);
+      else if (tid >= 2 * C && tid < 3 * C && it.has_prev) normalize_band_row(ST, 2, tid - 2 * C);
       fence_proxy_async_smem();
       bar_sync_n(1, kPrepThreads);
     }
 
-    // P1: [K; Q] K^T -> TMEM cols [0, 64)
+    // group 1: [Q; K] [K; K_prev]^T -> TMEM cols [0, 128)
     if (tid == 0) {
       tc_fence_after();
-      const uint64_t dkq = kmaj(kq_u);
+      const uint64_t da = kmaj(st_u), db = kmaj(st_u + 8192);
 #pragma unroll
       for (int kk = 0; kk < DK / 16; ++kk)
-        tc_mma_bf16(tmem, desc_k(dkq, kk, 16384), desc_k(dkq, kk, 16384),
-                    idesc_bf16(128, 64, 0, 0), kk > 0);
+        tc_mma_bf16(tmem, desc_k(da, kk, 32768), desc_k(db, kk, 32768),
+                    idesc_bf16(128, 128, 0, 0), kk > 0);
       tc_commit(mma_bar);
-      // the previous item's output stores of R and B_c boxes 2, 3 must have read their
-      // staging before the A/P phase overwrites it (all threads pass the barrier in
-      // mma_wait after this); A_c and B_c boxes 0, 1 are waited for before the inverse
-      bulk_wait_read<1>();
+      mma_pending = true;
+      // the next item's location (its gates are loaded under the inverse)
+      if (has_next) {
+        seq_cur = advance_seq(seq_cur, (int)((item + stride) / p.H), cu_chunks);
+        ctl->nxt = item_at(item + stride, seq_cur, p, cu_chunks);
+      }
+      // the previous item's first store group (P, -Y) has read its staging: P and Z are
+      // written below
+      bulk_wait_read<2>();
     }
     if (!mma_wait()) break;
 
-    // A (strictly lower, fp32) and P (lower incl. diagonal, bf16); columns split by hsel
+    // P (rows 0-63, bf16), A (rows 64-127, fp32) and Z = K K~_prev^T (rows 64-127, bf16)
     {
       float v[32];
-      tmem_ld32(tmem + lane_base + 32 * hsel, v);
-      tc_wait_ld();
-      const int t = row & 63;
-      const float gt = ctl->g[t];
-      if (row < C) {
-        const float bt = ctl->beta[t];
+      // warps whose 32 columns all lie right of the diagonal (hsel 1, rows 0-31) write zeros
+      const bool upper = hsel == 1 && (q4 & 1) == 0;
+      if (q4 < 2) {
+        if (want_o) {
+          const int t = q4 * 32 + lane;
+          if (upper) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int s = 32 * hsel + i;
-          v[i] = (s < t) ? bt * exp_ftz(gt - ctl->g[s]) * v[i] : 0.f;
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+          } else {
+            tmem_ld32(tmem + lane_base + 32 * hsel, v);
+            tc_wait_ld();
+            const float gt = ctl->g[t];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int s = 32 * hsel + i;
+              v[i] = (s <= t) ? exp_ftz(gt - ctl->g[s]) * v[i] : 0.f;
+            }
+          }
+          store_row_bf16(sm + P_P, t, 32 * hsel, v, 1.f);
+        }
+      } else {
+        const int t = (q4 - 2) * 32 + lane;
+        if (upper) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        } else {
+          tmem_ld32(tmem + lane_base + 32 * hsel, v);
+          tc_wait_ld();
+          const float gt = ctl->g[t], bt = ctl->beta[t];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int s = 32 * hsel + i;
+            v[i] = (s < t) ? bt * exp_ftz(gt - ctl->g[s]) * v[i] : 0.f;
+          }
         }
         float4 *dst = reinterpret_cast<float4 *>(As + t * LDA + 32 * hsel);
 #pragma unroll
         for (int w = 0; w < 8; ++w) dst[w] = make_float4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]);
-      } else if (want_o) {
+        if (it.has_prev) {
+          tmem_ld32(tmem + lane_base + 64 + 32 * hsel, v);
+          tc_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int s = 32 * hsel + i;
-          v[i] = (s <= t) ? exp_ftz(gt - ctl->g[s]) * v[i] : 0.f;
+          for (int i = 0; i < 32; ++i) v[i] *= ctl->gpp[32 * hsel + i];
+          store_row_bf16(sm + P_Z, t, 32 * hsel, v, 1.f);
         }
-        store_row_bf16(sm + P_AP, row, 32 * hsel, v, 1.f);
-      }
-    }
-    if (tid == 0) {
-      bulk_wait_read<0>();  // the staging of A_c, B_c boxes 0, 1 is free
-      // the previous item's input buffer (its K/Q/V, then its O0 staging) is free now:
-      // prefetch the next item into it (items 0 and 1 were loaded before the loop)
-      if (n >= 1 && next_item(item) < n_items) {
-        fence_proxy_async_smem();
-        issue(next_item(item), buf ^ 1);
       }
     }
     bar_sync_n(1, kPrepThreads);
+    // the next item's gates: their loads run under the inverse
+    if (has_next) load_gates(ctl->nxt, la_next, b_next);
 
     // T = (I + A)^{-1}, blocked.  (a) the four 16 x 16 diagonal blocks by forward
     // substitution (thread = column, fp32 registers); (b) each 32 x 32 diagonal block from
@@ -467,8 +643,6 @@ __device__ __forceinline__ void prep_body(const CUtensorMap &tm_q, const CUtenso
       float Tc[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        // row i of the block's A (16-byte aligned), 4 at a time; entries at columns >= i
-        // are zeros of the strictly lower A and are skipped
         const float4 *Ar4 = reinterpret_cast<const float4 *>(As + (base + i) * LDA + base);
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
@@ -488,9 +662,8 @@ __device__ __forceinline__ void prep_body(const CUtensorMap &tm_q, const CUtenso
       for (int i = 0; i < 16; ++i) Ts[(base + i) * LDA + base + c] = Tc[i];
     }
     bar_sync_n(1, kPrepThreads);
-    // (b) thread -> 32-block J, row r of its lower 16 x 16 block, columns c0, c0 + 1
     const int mJ = tid >> 7, mr = (tid >> 3) & 15, mc = (tid & 7) * 2;
-    {  // X16 = A21 T11 within block J
+    {  // X16 = A21 T11 within 32-block J
       const float *Ar = As + (32 * mJ + 16 + mr) * LDA + 32 * mJ;
       float x0 = 0.f, x1 = 0.f;
 #pragma unroll
@@ -505,8 +678,7 @@ __device__ __forceinline__ void prep_body(const CUtensorMap &tm_q, const CUtenso
         }
       }
       *reinterpret_cast<float2 *>(Xs + (16 * mJ + mr) * LDX + mc) = make_float2(x0, x1);
-      // the upper-right 16 x 16 of the 32-block is zero (T is lower triangular); nothing
-      // in this step reads it
+      // the upper-right 16 x 16 of the 32-block is zero (T is lower triangular)
       *reinterpret_cast<float2 *>(Ts + (32 * mJ + mr) * LDA + 32 * mJ + 16 + mc) =
           make_float2(0.f, 0.f);
     }
@@ -564,9 +736,11 @@ __device__ __forceinline__ void prep_body(const CUtensorMap &tm_q, const CUtenso
       }
       *reinterpret_cast<float4 *>(Ts + (32 + r) * LDA + c0) = make_float4(-x0, -x1, -x2, -x3);
     }
+    // the previous item's second store group (U~) has read the T tiles written below
+    if (tid == 0) bulk_wait_read<1>();
     bar_sync_n(1, kPrepThreads);
-    {  // [-T diag(beta); T diag(beta gamma)] as high + low bf16 parts; consecutive lanes
-       // take consecutive rows (conflict-free reads of T and swizzled stores)
+    {  // [T diag(beta gamma); T diag(beta)] as high + low bf16 parts; consecutive lanes take
+       // consecutive rows (conflict-free reads of T and swizzled stores)
       const int rr = tid & 127, half = tid >> 7, t = rr & 63;
       const bool zero = t < 32 && half == 1;  // T is lower triangular: T12 = 0
       float v[32];
@@ -578,175 +752,131 @@ __device__ __forceinline__ void prep_body(const CUtensorMap &tm_q, const CUtenso
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int s = 32 * half + 4 * w + u;
-          v[4 * w + u] = (rr < C) ? -te[u] * ctl->beta[s] : te[u] * ctl->bg[s];
+          v[4 * w + u] = te[u] * (rr < C ? ctl->bg[s] : ctl->beta[s]);
         }
       }
-      store_row_split(sm + P_TSH, sm + P_TSL, rr, 32 * half, v, 1.f);
+      store_row_split(sm + P_THI, sm + P_TLO, rr, 32 * half, v, 1.f);
     }
     fence_proxy_async_smem();
     bar_sync_n(1, kPrepThreads);
 
-    // P2: [-T''; T'] V -> cols [64, 64+DV) (lanes 0-63: -U~); [-T''; T'] K -> [192, 320) (lanes 64-127: W)
+    // group 2: [T'; T''] K -> cols [128, 256) (rows 0-63: W); [T'; T''] V (hi + lo) ->
+    // [256, 256 + DV) (rows 64-127: U~); [T'; T''] Z -> [384, 448) (rows 0-63: Y)
     if (tid == 0) {
       tc_fence_after();
-      const uint64_t th = kmaj(smem_u32(sm + P_TSH)), tl = kmaj(smem_u32(sm + P_TSL));
-      const uint64_t dv_ = mnmaj(v_u, 8192), dk_ = mnmaj(kq_u, 16384);
+      const uint64_t th = kmaj(smem_u32(sm + P_THI)), tl = kmaj(smem_u32(sm + P_TLO));
+      const uint64_t dk_ = mnmaj(st_u + 8192, 32768), dv_ = mnmaj(st_u + 24576, 32768);
+      const uint64_t dz = mnmaj(smem_u32(sm + P_Z), 8192);
 #pragma unroll
       for (int kk = 0; kk < C / 16; ++kk)
-        tc_mma_bf16(tmem + 64, desc_k(th, kk, 0), desc_mn(dv_, kk), idesc_bf16(128, DV, 0, 1), kk > 0);
+        tc_mma_bf16(tmem + 128, desc_k(th, kk, 0), desc_mn(dk_, kk), idesc_bf16(128, 128, 0, 1), kk > 0);
 #pragma unroll
       for (int kk = 0; kk < C / 16; ++kk)
-        tc_mma_bf16(tmem + 64, desc_k(tl, kk, 0), desc_mn(dv_, kk), idesc_bf16(128, DV, 0, 1), 1u);
+        tc_mma_bf16(tmem + 256, desc_k(th, kk, 0), desc_mn(dv_, kk), idesc_bf16(128, DV, 0, 1), kk > 0);
 #pragma unroll
       for (int kk = 0; kk < C / 16; ++kk)
-        tc_mma_bf16(tmem + 192, desc_k(th, kk, 0), desc_mn(dk_, kk), idesc_bf16(128, 128, 0, 1), kk > 0);
+        tc_mma_bf16(tmem + 256, desc_k(tl, kk, 0), desc_mn(dv_, kk), idesc_bf16(128, DV, 0, 1), 1u);
+      if (it.has_prev) {
 #pragma unroll
-      for (int kk = 0; kk < C / 16; ++kk)
-        tc_mma_bf16(tmem + 192, desc_k(tl, kk, 0), desc_mn(dk_, kk), idesc_bf16(128, 128, 0, 1), 1u);
+        for (int kk = 0; kk < C / 16; ++kk)
+          tc_mma_bf16(tmem + 384, desc_k(th, kk, 0), desc_mn(dz, kk), idesc_bf16(128, 64, 0, 1), kk > 0);
+      }
       tc_commit(mma_bar);
+      mma_pending = true;
+      // prefetch the next item into the other stage once the previous item's output stores
+      // have finished reading their staging there (issued an item ago: usually done)
+      bulk_wait_read<0>();
+      if (has_next) {
+        fence_proxy_async_smem();
+        issue(ctl->nxt, buf ^ 1);
+      }
     }
     if (!mma_wait()) break;
 
-    const float gC = ctl->g[C - 1];
     {
       float v[32];
-      const int t = row & 63;
-      const float gp = exp_ftz(gC - ctl->g[t]);
-      if (row >= C) {  // W row t, columns 64*hsel..+63 -> W and gamma' W ([t][d], 8 KB halves)
+      if (q4 < 2) {
+        const int t = q4 * 32 + lane;
+        // -gamma_C(prev) W -> the previous-K band of half hsel (row t)
+        const float s = -ctl->gc_prev;
 #pragma unroll 1
         for (int j = 0; j < 2; ++j) {
-          tmem_ld32(tmem + 192 + lane_base + 64 * hsel + 32 * j, v);
+          tmem_ld32(tmem + 128 + lane_base + 64 * hsel + 32 * j, v);
           tc_wait_ld();
-          store_row_bf16(sm + P_AW + hsel * 8192, t, 32 * j, v, 1.f);
-          store_row_bf16(sm + P_AW + 16384 + hsel * 8192, t, 32 * j, v, gp);
+          store_row_bf16(ST + hsel * 32768 + 16384, t, 32 * j, v, s);
         }
-      } else {  // -U~ row t, columns (DV/2)*hsel.. -> U~ (hi, lo) and gamma' U~ (hi, lo)
+        if (it.has_prev) {  // -Y -> the Z tile (consumed)
+          tmem_ld32(tmem + 384 + lane_base + 32 * hsel, v);
+          tc_wait_ld();
+          store_row_bf16(sm + P_Z, t, 32 * hsel, v, -1.f);
+        }
+      } else {
+        const int t = (q4 - 2) * 32 + lane;
+        // U~ row t (fp32), columns (DV/2) hsel.. -> 32-column boxes over the T tiles
 #pragma unroll 1
         for (int j = 0; j < DV / 64; ++j) {
           const int col = (DV / 2) * hsel + 32 * j;
-          tmem_ld32(tmem + 64 + lane_base + col, v);
+          tmem_ld32(tmem + 256 + lane_base + col, v);
           tc_wait_ld();
-          const int blkoff = (col >> 6) * 8192, c0 = col & 63;
-          store_row_split(sm + P_TU + blkoff, sm + P_TU + 16384 + blkoff, t, c0, v, -1.f);
-          store_row_split(sm + P_TSH + blkoff, sm + P_TSL + blkoff, t, c0, v, -gp);
+          store_row32_f32(sm + P_THI + 8192 * (col >> 5), t, v, 1.f);
         }
       }
+      // gamma Q in place (thread -> row, 32-column piece)
+      const int r = tid & 63, pc = tid >> 6, h = pc >> 1, c0 = 32 * (pc & 1);
+      if (want_o) scale_row32_bf16(ST + h * 32768, r, c0, ctl->gq[r]);
     }
     fence_proxy_async_smem();
     tc_fence_before();
     bar_sync_n(1, kPrepThreads);
-
-    // batch: P W -> [0,128), P U~ -> [128,128+DV), A_c -> [256,384), B_c -> [384,384+DV)
     if (tid == 0) {
-      tc_fence_after();
-      const uint64_t ap = kmaj(smem_u32(sm + P_AP));
-      const uint32_t w_u = smem_u32(sm + P_AW), uh_u = smem_u32(sm + P_TU);
-      const uint64_t w_d = mnmaj(w_u, 8192), wg_d = mnmaj(w_u + 16384, 8192);
-      const uint64_t uh = mnmaj(uh_u, 8192), ul = mnmaj(uh_u + 16384, 8192);
-      const uint64_t gh = mnmaj(smem_u32(sm + P_TSH), 8192), gl = mnmaj(smem_u32(sm + P_TSL), 8192);
-      const uint64_t kt = mnmaj(kq_u, 16384);
-      if (want_o) {
+      const int64_t slot = it.slot;
+      const int32_t y128 = (int32_t)(slot * 128), y64 = (int32_t)(slot * 64);
+      // three bulk groups, in the order their staging is written again by the next item:
+      // P and -Y (p1), U~ (over the T tiles: p3), the stage's bands (the prefetch after it)
+      if (want_o) tma_store_2d(&tm_PY, smem_u32(sm + P_P), 0, y128);
+      if (it.has_prev) tma_store_2d(&tm_PY, smem_u32(sm + P_Z), 0, y128 + 64);
+      bulk_commit();
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk)
-          tc_mma_bf16(tmem + 0, desc_k(ap, kk, 0), desc_mn(w_d, kk), idesc_bf16(128, 128, 0, 1), kk > 0);
+      for (int b = 0; b < DV / 32; ++b)
+        tma_store_2d(&tm_UT, smem_u32(sm + P_THI + 8192 * b), 32 * b, y64);
+      bulk_commit();
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk)
-          tc_mma_bf16(tmem + 128, desc_k(ap, kk, 0), desc_mn(uh, kk), idesc_bf16(128, DV, 0, 1), kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk)
-          tc_mma_bf16(tmem + 128, desc_k(ap, kk, 0), desc_mn(ul, kk), idesc_bf16(128, DV, 0, 1), 1u);
+      for (int h = 0; h < 2; ++h) {
+        if (want_o) tma_store_2d(&tm_QW, st_u + h * 32768, 64 * h, y128);
+        tma_store_2d(&tm_QW, st_u + h * 32768 + 16384, 64 * h, y128 + 64);
+        tma_store_2d(&tm_KT, st_u + h * 32768 + 8192, 64 * h, y64);
       }
-#pragma unroll
-      for (int kk = 0; kk < C / 16; ++kk)
-        tc_mma_bf16(tmem + 256, desc_mn(kt, kk), desc_mn(wg_d, kk), idesc_bf16(128, 128, 1, 1), kk > 0);
-#pragma unroll
-      for (int kk = 0; kk < C / 16; ++kk)
-        tc_mma_bf16(tmem + 384, desc_mn(kt, kk), desc_mn(gh, kk), idesc_bf16(128, DV, 1, 1), kk > 0);
-#pragma unroll
-      for (int kk = 0; kk < C / 16; ++kk)
-        tc_mma_bf16(tmem + 384, desc_mn(kt, kk), desc_mn(gl, kk), idesc_bf16(128, DV, 1, 1), 1u);
-      tc_commit(mma_bar);
-    }
-    if (!mma_wait()) break;
-
-    {
-      float v[32];
-      // A_c row d = -(K^T gamma' W)[d] (bf16), columns 64*hsel..+63
-#pragma unroll 1
-      for (int j = 0; j < 2; ++j) {
-        tmem_ld32(tmem + 256 + lane_base + 64 * hsel + 32 * j, v);
-        tc_wait_ld();
-        store_row_bf16(sm + P_TU + hsel * 16384, row, 32 * j, v, -1.f);
-      }
-      // B_c row d (fp32), columns (DV/2)*hsel.. (one 32-column box per 32 columns)
-#pragma unroll 1
-      for (int j = 0; j < DV / 64; ++j) {
-        tmem_ld32(tmem + 384 + lane_base + (DV / 2) * hsel + 32 * j, v);
-        tc_wait_ld();
-        store_row32_f32(sm + P_TSH + 16384 * (((DV / 2) * hsel + 32 * j) >> 5), row, v, 1.f);
-      }
-      if (want_o && row >= C) {
-        const int t = row - C;
-        const float gam = exp_ftz(ctl->g[t]);
-        // R row t = gamma_t q_t - (P W)_t (bf16), columns 64*hsel..+63
-#pragma unroll 1
-        for (int j = 0; j < 2; ++j) {
-          tmem_ld32(tmem + 0 + lane_base + 64 * hsel + 32 * j, v);
-          tc_wait_ld();
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            float f[8];
-            load_row8_bf16(KQ + hsel * 16384, 64 + t, 32 * j + 8 * w, f);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v[8 * w + i] = gam * f[i] - v[8 * w + i];
-          }
-          store_row_bf16(sm + P_AP + hsel * 8192, t, 32 * j, v, 1.f);
+      bulk_commit();
+      ws.G[slot * 4] = exp_ftz(ctl->g[C - 1]);
+      if (has_next) ctl->cur = ctl->nxt;
+      if (publish) {
+        // the previous item's three store groups have completed (this item's three may not)
+        if (prev_slot >= 0) {
+          bulk_wait<3>();
+          publish_slot(ws, prev_slot, p.epoch);
         }
-        // O0 row t (fp32), columns (DV/2)*hsel..
-#pragma unroll 1
-        for (int j = 0; j < DV / 64; ++j) {
-          tmem_ld32(tmem + 128 + lane_base + (DV / 2) * hsel + 32 * j, v);
-          tc_wait_ld();
-          store_row32_f32(KQ + o0_box_offset(((DV / 2) * hsel + 32 * j) >> 5), t, v, 1.f);
-        }
+        prev_slot = slot;
       }
-      fence_proxy_async_smem();
     }
-    tc_fence_before();
+    if (tid < C) ws.GP[it.slot * C + tid] = ctl->gp[tid];
     bar_sync_n(1, kPrepThreads);
-    if (tid == 0) {
-      const int64_t slot = item;
-      // three bulk groups, in the order the staging tiles are needed again:
-      //   1. O0 (this item's input buffer: the prefetch below refills it)
-      //   2. R (P_AP) and B_c boxes 2, 3 (P_AW): the next item's A/P phase writes there
-      //   3. A_c (P_TU) and B_c boxes 0, 1 (P_TSH, P_TSL): its inverse and split write there
-      if (want_o) {
-#pragma unroll
-        for (int b = 0; b < DV / 32; ++b)
-          tma_store_2d(&tm_O, smem_u32(KQ + o0_box_offset(b)), 32 * b, (int32_t)(slot * 64));
-      }
-      bulk_commit();
-      if (want_o) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-          tma_store_2d(&tm_R, smem_u32(sm + P_AP + h * 8192), 64 * h, (int32_t)(slot * 64));
-      }
-#pragma unroll
-      for (int b = 2; b < DV / 32; ++b)
-        tma_store_2d(&tm_B, smem_u32(sm + P_TSH + 16384 * b), 32 * b, (int32_t)(slot * 128));
-      bulk_commit();
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-        tma_store_2d(&tm_A, smem_u32(sm + P_TU + h * 16384), 64 * h, (int32_t)(slot * 128));
-#pragma unroll
-      for (int b = 0; b < 2; ++b)
-        tma_store_2d(&tm_B, smem_u32(sm + P_TSH + 16384 * b), 32 * b, (int32_t)(slot * 128));
-      bulk_commit();
-      ws.G[slot] = exp_ftz(gC);
-    }
   }
 
-  if (tid == 0) bulk_wait<0>();
+  if (tid == 0) {
+    // every output store has completed before the grid does (the chain reads them)
+    bulk_wait<0>();
+    if (publish && prev_slot >= 0 && item >= n_items) publish_slot(ws, prev_slot, p.epoch);
+    if (item < n_items) {
+      // left the loop at a wait that gave up: nothing issued may still be in flight when
+      // the CTA releases its shared memory and TMEM
+      for (int b = 0; b < 2; ++b)
+        if (fills[b] > 0) mbar_wait_drain(smem_u32(&ctl->tma_bar[b]), (uint32_t)(fills[b] - 1) & 1u);
+      if (mma_pending) {
+        tc_commit(smem_u32(&ctl->drain_bar));
+        mbar_wait_drain(smem_u32(&ctl->drain_bar), 0);
+      }
+    }
+  }
   tc_fence_before();
   bar_sync_n(1, kPrepThreads);
   if (warp == 0) {
@@ -757,379 +887,511 @@ __device__ __forceinline__ void prep_body(const CUtensorMap &tm_q, const CUtenso
 
 template <int DV>
 __global__ void __launch_bounds__(kPrepThreads, 1)
-    scan_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_A,
-                     const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_R,
-                     const __grid_constant__ CUtensorMap tm_O, const __grid_constant__ ScanLaunch p,
-                     const __grid_constant__ ScanWs ws, int total_chunks) {
-  prep_body<DV>(tm_q, tm_k, tm_v, tm_A, tm_B, tm_R, tm_O, p, ws, total_chunks, blockIdx.x,
-                (int64_t)blockIdx.x + gridDim.x, gridDim.x);
+    scan_prep_kernel(const __grid_constant__ ScanMaps mp, const __grid_constant__ ScanLaunch p,
+                     const __grid_constant__ ScanWs ws, const __grid_constant__ ScanPlan plan) {
+  prep_body<DV>(mp, p, ws, plan, blockIdx.x, gridDim.x, false);
 }
 
 // =========================================================== chain kernel
-// One CTA per (sequence, head, 64-column slice of d_v), 288 threads.  Warps 0-7:
-// thread (quarter q4 = warp % 4, column group cg = warp / 4) owns row d = 32 q4 + lane
-// of the fp32 state slice and its columns kCols cg .. +kCols-1 (the per-chunk update is
-// latency-bound: 16 state warps with half the columns each measured no faster).  Warp 8
-// only refills the TMA ring (a tensor load can stall its issuing thread while many are in flight, so the
-// state-owning threads never issue them).  Per chunk: one tcgen05 product
-// Z = A_c M (M in bf16 in shared memory, 8 MMAs of K = 16), then
-// M <- gamma_C M + Z + B_c in registers.  A_c and the B_c slice arrive through a
-// 2-stage TMA ring; all gamma_C of the sequence are read into shared memory at the
-// start.  The bf16 state at the start of every chunk (double buffered by chunk
-// parity) is the operand of the next product and goes to the workspace, for the
-// readout kernel, by a TMA store.
-constexpr int kStages = 2;
-constexpr uint32_t H_STAGE = 65536;             // A_c [half][128 rows][128 B] + B_c [box][128][32 fp32]
-constexpr uint32_t H_MB = kStages * H_STAGE;    // 2 x bf16 state slice [128 d][128 B]
+// One CTA per (sequence, head, 64-column slice of d_v), in longest-first order of the
+// sequences; 320 threads:
+//   warp 0      TMA producer: stage k (k = 0..n) holds chunk k-1's gamma Q, P, K~ and
+//               gamma_C and chunk k's -gamma_C W, -Y and U~ slice (2 stages)
+//   warp 1      MMA issuer (one thread)
+//   warps 2-5   state warps: thread (quarter q = warp % 4) owns row d = 32 q + lane of the
+//               fp32 state slice M (64 columns in registers); M_{c+1} = gamma_C M_c + dM
+//   warps 6, 7  U warps (TMEM lanes 64-127): U_{c+1} = U~_{c+1} + D rows 64-127, written as
+//               bf16 and gamma' U_{c+1} as a bf16 hi + lo pair (shared memory)
+//   warps 8, 9  O warps (TMEM lanes 0-63): the chunk's output rows, bf16, stored by TMA
+//               (off the chain's critical path)
+// Per chunk c the issuer waits for M_c and U_c and issues
+//   D[c % 2] = A1 M_c (8 MMAs; 16 with the state as a hi + lo pair) once M_c is ready, then,
+//   once U_c is, dM = K^T [gamma' U_c hi | lo] (4 MMAs of N = 128), commit S;
+//   D[c % 2] += A2 U_c (4), commit D (and the buffer's output barrier).  TMEM: D[2] at
+//   columns 0 and 64, dM at 128 (hi) and 192 (lo).
+constexpr uint32_t C_A1 = 0;        // [2 halves][128 rows][128 B]
+constexpr uint32_t C_A2 = 32768;    // [128 rows][128 B]
+constexpr uint32_t C_KT = 49152;    // [2 halves][64 rows][128 B]
+constexpr uint32_t C_UT = 65536;    // [2 boxes][64 rows][32 fp32]
+constexpr uint32_t C_GP = 81920;    // gamma' [64] fp32
+constexpr uint32_t C_G = 82176;     // gamma_C (16 bytes)
+constexpr uint32_t C_STAGE = 82944;
+constexpr uint32_t C_MT = 2 * C_STAGE;          // M bf16 [128 d][64 cols] (high parts)
+constexpr uint32_t C_MTL = C_MT + 16384;        // low parts (precise_state)
+constexpr uint32_t C_UTL = C_MTL + 16384;       // U bf16 [64 t][64 cols]
+constexpr uint32_t C_GUH = C_UTL + 8192;        // gamma' U, high bf16 parts
+constexpr uint32_t C_GUL = C_GUH + 8192;        // low parts
+constexpr size_t CHAIN_SMEM = C_GUL + 8192 + 1024;
+static_assert(C_MT % 1024 == 0, "swizzled tiles are 1024-byte aligned");
+constexpr int kChainThreads = 320;
+static_assert(CHAIN_SMEM <= 232448, "chain shared memory");
 
 struct ChainCtl {
-  alignas(16) float g4[kStages][4];  // the 16-byte aligned group of G holding the stage's gamma_C
-  uint64_t tma_bar[kStages];
-  uint64_t empty_bar[kStages];  // stage consumed (arrived by thread 0 after the barrier)
-  uint64_t bar_z;
+  uint64_t full[2], empty[2];
+  uint64_t bar_s, bar_d, bar_m, bar_u, drain;
+  uint64_t bar_dO[2];   // D[b] holds a finished chunk output (for the O warps)
+  uint64_t bar_o[2];    // the O warps have read D[b]
   uint32_t tmem;
   int abort;
 };
-constexpr uint32_t H_CTL = H_MB + 2 * 16384;    // the control block, in dynamic shared memory
-constexpr size_t CHAIN_SMEM = H_CTL + sizeof(ChainCtl) + 1024;
 
-__device__ __forceinline__ void load_row32_f32(const uint8_t *tile, int row, float *f) {
-  // one row (32 floats = 128 B) of a 128-byte-swizzled fp32 tile
-#pragma unroll
-  for (int ch = 0; ch < 8; ++ch) {
-    const float4 u = *reinterpret_cast<const float4 *>(
-        tile + sw128_offset((uint32_t)row, (uint32_t)ch * 16u));
-    f[4 * ch] = u.x; f[4 * ch + 1] = u.y; f[4 * ch + 2] = u.z; f[4 * ch + 3] = u.w;
+// Wait until the prep running beside this chain (fused launch) has published `slot`: an
+// acquire load of its flag, bounded like every other wait; then order the flag before this
+// thread's TMA loads of the slot's data.
+__device__ bool wait_slot(const ScanWs &ws, int64_t slot, unsigned long long epoch,
+                          const AbortFlag &ab) {
+  const unsigned long long *f = ws.flags + slot;
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
+  if (v != epoch) {
+    const unsigned long long t0 = globaltimer_ns();
+    for (int i = 0;; ++i) {
+      __nanosleep(64);
+      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
+      if (v == epoch) break;
+      if ((i & 15) == 15) {
+        if (*ab.flag) return false;
+        if (globaltimer_ns() - t0 > ab.limit_ns) {
+          *ab.flag = 1;
+          if (ab.err_word) atomicOr(ab.err_word, ab.err_bit);
+          return false;
+        }
+      }
+    }
   }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return true;
 }
 
-constexpr int kStateWarps = 8;
-constexpr int kChainThreads = 32 * (kStateWarps + 1);
-constexpr int kCols = DVS * 4 / kStateWarps;  // state columns per thread
-static_assert(kCols == 32, "state columns per thread");
-
-
-
-// The chain of one (sequence * H + head, slice) task (kChainThreads threads).  The
-// loads of chunk c (A_c, the B_c slice and gamma_C, into stage c % kStages) are issued
-// by the producer warp.
-__device__ __forceinline__ void chain_body(const CUtensorMap &tm_A, const CUtensorMap &tm_B,
-                                           const CUtensorMap &tm_M, const ScanLaunch &p,
-                                           const ScanWs &ws, int seqhead, int slice) {
+// The chain of CTA `cta` (320 threads); with `wait_flags` each stage's slots are awaited
+// first (their prep runs in the same launch).
+__device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch &p,
+                                           const ScanWs &ws, const ScanPlan &plan, int cta,
+                                           bool wait_flags) {
+  const CUtensorMap &tm_QW = mp.QW, &tm_PY = mp.PY, &tm_KT = mp.KT, &tm_UT = mp.UT, &tm_o = mp.o;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ int red[32];  // one entry per warp (chunk_base)
+  __shared__ ChainCtl ctl_s;
+  ChainCtl *ctl = &ctl_s;
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
-  ChainCtl *ctl = reinterpret_cast<ChainCtl *>(sm + H_CTL);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int q4 = warp & 3, cg = warp >> 2;
-  const int d = q4 * 32 + lane;
-  const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-  const int H = p.H, DV = p.dv;
-  const int seq = seqhead / H, head = seqhead % H;
-  const int col = slice * DVS + kCols * cg;   // this thread's first d_v column
+  const int NS = p.dv / DVS;
+  const int H = p.H;
+  const int pos = cta / (H * NS);
+  const int head = (cta / NS) % H, slice = cta % NS;
+  const bool want_o = p.o != nullptr;
 
   if (tid == 0) {
-    tma_prefetch_desc(&tm_A);
-    tma_prefetch_desc(&tm_B);
-    tma_prefetch_desc(&tm_M);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&ctl->tma_bar[s]), 1);
-      mbar_init(smem_u32(&ctl->empty_bar[s]), 1);
+    tma_prefetch_desc(&tm_QW);
+    tma_prefetch_desc(&tm_PY);
+    tma_prefetch_desc(&tm_KT);
+    tma_prefetch_desc(&tm_UT);
+    if (want_o) tma_prefetch_desc(&tm_o);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&ctl->full[s]), 1);
+      mbar_init(smem_u32(&ctl->empty[s]), 2);   // the state warps and the output warps
     }
-    mbar_init(smem_u32(&ctl->bar_z), 1);
+    mbar_init(smem_u32(&ctl->bar_s), 1);
+    mbar_init(smem_u32(&ctl->bar_d), 1);
+    mbar_init(smem_u32(&ctl->bar_m), 1);
+    mbar_init(smem_u32(&ctl->bar_u), 1);
+    mbar_init(smem_u32(&ctl->drain), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&ctl->bar_dO[b]), 1);
+      mbar_init(smem_u32(&ctl->bar_o[b]), 1);
+    }
     ctl->abort = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(&ctl->tmem), 64);
+    tmem_alloc(smem_u32(&ctl->tmem), 256);
     tmem_relinquish();
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  // TMEM is held: let the next kernel launch; then wait for the previous one's outputs
-  pdl_trigger();
-  pdl_wait();
-  const int t_begin = p.cu_seqlens[seq], t_end = p.cu_seqlens[seq + 1];
-  const int nch = (t_end - t_begin + C - 1) / C;
-  const int cb = chunk_base(p.cu_seqlens, seq, red);
-  auto slot_of = [&](int c) -> int64_t { return ((int64_t)cb + c) * H + head; };
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem;
-  const AbortFlag ab{&ctl->abort, p.err_word, ERRBIT_SCAN_TIMEOUT};
-  // bf16 state copy par (chunk parity) -> workspace slot of chunk c, by one TMA store
-  auto store_mc = [&](int c, int par) {
-    tma_store_2d(&tm_M, smem_u32(sm + H_MB + 16384 * par), slice * DVS, (int32_t)(slot_of(c) * 128));
-    bulk_commit();
-  };
+  const AbortFlag ab{&ctl->abort, p.err_word, ERRBIT_SCAN_TIMEOUT, p.wait_ns};
+  // TMEM is held: let the next kernel launch; then wait for the previous one's outputs
+  pdl_trigger();
+  pdl_wait();
 
-  float Mr[kCols];
-  const bool m_zero = p.S0 == nullptr;
-  const bool producer = warp == kStateWarps;
-  const size_t s_off = ((size_t)seq * H + head) * DK * DV + (size_t)d * DV + col;
-  if (!m_zero && !producer) {
-#pragma unroll
-    for (int j = 0; j < kCols; j += 4) {
-      const float4 a = *reinterpret_cast<const float4 *>(p.S0 + s_off + j);
-      Mr[j] = a.x; Mr[j + 1] = a.y; Mr[j + 2] = a.z; Mr[j + 3] = a.w;
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < kCols; ++j) Mr[j] = 0.f;
-  }
-  auto store_state = [&](uint8_t *tile) { store_row_bf16(tile, d, kCols * cg, Mr, 1.f); };
-  if (nch > 0 && !producer) store_state(sm + H_MB);
+  const int seq = plan_order(plan, ws)[pos];
+  const int cb = plan_cu_chunks(plan, ws)[seq];
+  const int t_begin = p.cu_seqlens[seq], t_end = p.cu_seqlens[seq + 1];
+  const int n = (t_end - t_begin + C - 1) / C;
+  auto slot_of = [&](int c) -> int64_t { return ((int64_t)cb + c) * H + head; };
+  const bool s0 = p.S0 != nullptr;
+  const uint32_t mt_u = smem_u32(sm + C_MT), utl_u = smem_u32(sm + C_UTL);
+  int last_k[2] = {-1, -1};   // producer: the last stage loaded into each buffer
+  bool mma_pending = false;   // issuer: products issued whose completion was not seen
 
-  auto issue_tma = [&](int c) {
-    const int st = c % kStages;
-    const int64_t slot = slot_of(c);
-    const uint32_t bar = smem_u32(&ctl->tma_bar[st]);
-    const uint32_t a_u = smem_u32(sm + st * H_STAGE);
-    mbar_arrive_expect_tx(bar, 65536u + 16u);
-    tma_load_2d(a_u, &tm_A, 0, (int32_t)(slot * 128), bar);
-    tma_load_2d(a_u + 16384, &tm_A, 64, (int32_t)(slot * 128), bar);
-    tma_load_2d(a_u + 32768, &tm_B, slice * DVS, (int32_t)(slot * 128), bar);
-    tma_load_2d(a_u + 49152, &tm_B, slice * DVS + 32, (int32_t)(slot * 128), bar);
-    // gamma_C: the 16-byte group of G that holds it (G is padded to 256 bytes)
-    bulk_load(smem_u32(&ctl->g4[st][0]), ws.G + (slot & ~(int64_t)3), 16u, bar);
-  };
-
-  auto issue_mma = [&](int c) -> bool {
-    const int st = c % kStages;
-    if (!mbar_wait(smem_u32(&ctl->tma_bar[st]), (uint32_t)(c / kStages) & 1u, ab)) return false;
-    tc_fence_after();
-    const uint64_t ad = kmaj(smem_u32(sm + st * H_STAGE));
-    const uint64_t md = mnmaj(smem_u32(sm + H_MB + 16384 * (c & 1)), 16384);
-#pragma unroll
-    for (int kk = 0; kk < DK / 16; ++kk)
-      tc_mma_bf16(tmem, desc_k(ad, kk, 16384), desc_mn(md, kk), idesc_bf16(128, DVS, 0, 1), kk > 0);
-    tc_commit(smem_u32(&ctl->bar_z));
-    return true;
-  };
-
-  bool failed = false;
-  fence_proxy_async_smem();
-  __syncthreads();
-  if (tid == 0 && nch > 0) store_mc(0, 0);
-
-  if (producer) {
-    // fill stage c % kStages with chunk c once chunk c - kStages has consumed it
+  if (warp == 0) {
+    // ------------------------------------------------------------- producer
     if (lane == 0) {
-      for (int c = 0; c < nch; ++c) {
-        const int st = c % kStages;
-        if (c >= kStages &&
-            !mbar_wait(smem_u32(&ctl->empty_bar[st]), (uint32_t)((c - kStages) / kStages) & 1u, ab))
+      for (int k = 0; k <= n; ++k) {
+        const int st = k & 1;
+        if (k >= 2 && !mbar_wait(smem_u32(&ctl->empty[st]), (uint32_t)((k - 2) >> 1) & 1u, ab)) break;
+        const bool cur = k >= 1, nxt = k <= n - 1;
+        const uint32_t bytes = (cur ? (want_o ? 16384u + 8192u : 0u) + 16384u + 16u : 0u) +
+                               (nxt ? 16384u + (k >= 1 ? 8192u : 0u) + 16384u + 256u : 0u);
+        const int64_t sc = cur ? slot_of(k - 1) : 0, sn = nxt ? slot_of(k) : 0;
+        if (wait_flags && ((cur && !wait_slot(ws, sc, p.epoch, ab)) ||
+                           (nxt && !wait_slot(ws, sn, p.epoch, ab))))
           break;
-        issue_tma(c);
+        const uint32_t bar = smem_u32(&ctl->full[st]);
+        const uint32_t base = smem_u32(sm + st * C_STAGE);
+        mbar_arrive_expect_tx(bar, bytes);
+        if (cur) {
+          if (want_o) {
+            tma_load_2d(base + C_A1, &tm_QW, 0, (int32_t)(sc * 128), bar);
+            tma_load_2d(base + C_A1 + 16384, &tm_QW, 64, (int32_t)(sc * 128), bar);
+            tma_load_2d(base + C_A2, &tm_PY, 0, (int32_t)(sc * 128), bar);
+          }
+          tma_load_2d(base + C_KT, &tm_KT, 0, (int32_t)(sc * 64), bar);
+          tma_load_2d(base + C_KT + 8192, &tm_KT, 64, (int32_t)(sc * 64), bar);
+          bulk_load(base + C_G, ws.G + sc * 4, 16u, bar);
+        }
+        if (nxt) {
+          tma_load_2d(base + C_A1 + 8192, &tm_QW, 0, (int32_t)(sn * 128 + 64), bar);
+          tma_load_2d(base + C_A1 + 16384 + 8192, &tm_QW, 64, (int32_t)(sn * 128 + 64), bar);
+          if (k >= 1) tma_load_2d(base + C_A2 + 8192, &tm_PY, 0, (int32_t)(sn * 128 + 64), bar);
+          tma_load_2d(base + C_UT, &tm_UT, slice * DVS, (int32_t)(sn * 64), bar);
+          tma_load_2d(base + C_UT + 8192, &tm_UT, slice * DVS + 32, (int32_t)(sn * 64), bar);
+          bulk_load(base + C_GP, ws.GP + sn * C, 256u, bar);
+        }
+        last_k[st] = k;
       }
     }
-  } else {
-    if (tid == 0 && !m_zero && nch > 0 && !issue_mma(0)) failed = true;
-    bool mma_for_c = !m_zero;
-    uint32_t z_phase = 0;
-    for (int c = 0; c < nch; ++c) {
-      const int st = c % kStages;
-      float v[kCols], b[kCols];
-      if (mma_for_c) {
-        if (!mbar_wait(smem_u32(&ctl->bar_z), z_phase, ab)) failed = true;
-        z_phase ^= 1u;
-        tc_fence_after();
-        tmem_ld32(tmem + lane_base + kCols * cg, v);
-      } else {
-#pragma unroll
-        for (int j = 0; j < kCols; ++j) v[j] = 0.f;
-      }
-      // the stage's B_c has landed (its A_c did, for the product); read this thread's
-      // columns of row d from the 32-column box that holds them
-      if (!mbar_wait(smem_u32(&ctl->tma_bar[st]), (uint32_t)(c / kStages) & 1u, ab)) failed = true;
-      {
-        const int c0 = kCols * cg;
-        const uint8_t *bt = sm + st * H_STAGE + 32768 + (c0 >> 5) * 16384;
-#pragma unroll
-        for (int ch = 0; ch < kCols / 4; ++ch) {
-          const float4 u = *reinterpret_cast<const float4 *>(
-              bt + sw128_offset((uint32_t)d, (uint32_t)(((c0 & 31) >> 2) + ch) * 16u));
-          b[4 * ch] = u.x; b[4 * ch + 1] = u.y; b[4 * ch + 2] = u.z; b[4 * ch + 3] = u.w;
-        }
-      }
-      if (mma_for_c) tc_wait_ld();
-      const float gC = ctl->g4[st][slot_of(c) & 3];
-      // M <- gamma_C M + A_c M + B_c (fp32); bf16 copy for the next product and the readout
-#pragma unroll
-      for (int j = 0; j < kCols; ++j) Mr[j] = fmaf(gC, Mr[j], v[j] + b[j]);
-      if (c + 1 < nch) store_state(sm + H_MB + 16384 * ((c + 1) & 1));
-      fence_proxy_async_smem();
-      tc_fence_before();
-      // copy (c + 1) & 1 was last stored to global two chunks ago: that store must have
-      // finished reading it before anyone rewrites it (after the barrier below)
-      if (tid == 0) bulk_wait_read<0>();
-      // named barrier over the state-owning threads, voting on `failed` so that all of
-      // them leave the loop together
-      uint32_t any_failed;
-      asm volatile(
-          "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
-          "bar.red.or.pred p, 1, %2, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-          : "=r"(any_failed)
-          : "r"((uint32_t)(failed || *ab.flag)), "n"(32 * kStateWarps)
-          : "memory");
-      if (any_failed) { failed = true; break; }
-      if (tid == 0) {
-        // chunk c's stage is consumed: its product completed and its B_c rows were read
-        mbar_arrive(smem_u32(&ctl->empty_bar[st]));
-        if (c + 1 < nch) {
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0 && n > 0) {
+      const uint32_t bar_s = smem_u32(&ctl->bar_s), bar_d = smem_u32(&ctl->bar_d);
+      const uint64_t md = mnmaj(mt_u, 16384), ud = mnmaj(utl_u, 8192);
+      const uint64_t mdl = mnmaj(smem_u32(sm + C_MTL), 16384);
+      const bool lo2 = p.precise_state;
+      const uint64_t gu = mnmaj(smem_u32(sm + C_GUH), 8192);   // [hi | lo] blocks, 8 KB apart
+      const uint32_t id_s = idesc_bf16(128, 2 * DVS, 1, 1);
+      const uint32_t id_mn = idesc_bf16(128, DVS, 0, 1);
+      bool ok = mbar_wait(smem_u32(&ctl->full[0]), 0, ab);
+      if (ok && s0) {
+        // U_0 = U~_0 - W_0 M_0: D[1] rows 64-127 = -W_0 M_0
+        ok = mbar_wait(smem_u32(&ctl->bar_m), 0, ab);
+        if (ok) {
           tc_fence_after();
-          if (!issue_mma(c + 1)) failed = true;
-          store_mc(c + 1, (c + 1) & 1);
+          const uint64_t a1 = kmaj(smem_u32(sm + C_A1));
+#pragma unroll
+          for (int kk = 0; kk < DK / 16; ++kk)
+            tc_mma_bf16(tmem + 64, desc_k(a1, kk, 16384), desc_mn(md, kk), id_mn, kk > 0);
+          if (lo2) {
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk)
+              tc_mma_bf16(tmem + 64, desc_k(a1, kk, 16384), desc_mn(mdl, kk), id_mn, 1u);
+          }
+          tc_commit(bar_d);
+          mma_pending = true;
         }
       }
-      mma_for_c = true;
+      for (int j = 0; ok && j < n; ++j) {
+        const int k = j + 1, st = k & 1;
+        const uint32_t base = smem_u32(sm + st * C_STAGE);
+        const uint32_t dcol = tmem + 64 * (j & 1);
+        const uint64_t a1 = kmaj(base + C_A1), a2 = kmaj(base + C_A2);
+        const uint64_t kt = mnmaj(base + C_KT, 8192);
+        // D = A1 M_j as soon as M_j is ready (it does not need U_j), once the O warps have
+        // read D[j % 2]'s previous chunk
+        if (!mbar_wait(smem_u32(&ctl->full[st]), (uint32_t)(k >> 1) & 1u, ab)) break;
+        if (!mbar_wait(smem_u32(&ctl->bar_m), (uint32_t)j & 1u, ab)) break;
+        if (want_o && j >= 2 &&
+            !mbar_wait(smem_u32(&ctl->bar_o[j & 1]), (uint32_t)((j >> 1) - 1) & 1u, ab))
+          break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk)
+          tc_mma_bf16(dcol, desc_k(a1, kk, 16384), desc_mn(md, kk), id_mn, kk > 0);
+        if (lo2) {
+#pragma unroll
+          for (int kk = 0; kk < DK / 16; ++kk)
+            tc_mma_bf16(dcol, desc_k(a1, kk, 16384), desc_mn(mdl, kk), id_mn, 1u);
+        }
+        mma_pending = true;
+        if (!mbar_wait(smem_u32(&ctl->bar_u), (uint32_t)j & 1u, ab)) break;
+        tc_fence_after();
+        // dM = K^T [gamma' U_hi | gamma' U_lo]: one N = 128 product, two 64-column results
+        // the state warps add; then D += A2 U_j
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk)
+          tc_mma_bf16(tmem + 128, desc_mn(kt, kk), desc_mn(gu, kk), id_s, kk > 0);
+        tc_commit(bar_s);
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk)
+          tc_mma_bf16(dcol, desc_k(a2, kk, 0), desc_mn(ud, kk), id_mn, 1u);
+        tc_commit(bar_d);
+        if (want_o) tc_commit(smem_u32(&ctl->bar_dO[j & 1]));
+      }
+      // the last step's products complete before the final barrier either way: the state
+      // and output warps wait for them, or, after an abort, the drain below does
     }
+  } else if (warp < 6) {
+    // ---------------------------------------------------------- state warps
+    const int q = warp & 3, d = 32 * q + lane;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    float M[DVS];
+    const size_t s_off = ((size_t)(seq * H + head) * DK + d) * p.dv + (size_t)slice * DVS;
+    if (s0) {
+#pragma unroll
+      for (int j = 0; j < DVS; j += 4) {
+        const float4 a = *reinterpret_cast<const float4 *>(p.S0 + s_off + j);
+        M[j] = a.x; M[j + 1] = a.y; M[j + 2] = a.z; M[j + 3] = a.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < DVS; ++j) M[j] = 0.f;
+    }
+    bool failed = false;
+    const bool lo2 = p.precise_state;
+    auto store_state = [&]() {
+      if (lo2) {
+        store_row_split(sm + C_MT, sm + C_MTL, d, 0, M, 1.f);
+        store_row_split(sm + C_MT, sm + C_MTL, d, 32, M + 32, 1.f);
+      } else {
+        store_row_bf16(sm + C_MT, d, 0, M, 1.f);
+        store_row_bf16(sm + C_MT, d, 32, M + 32, 1.f);
+      }
+    };
+    if (n > 0) {
+      store_state();
+      fence_proxy_async_smem();
+      bar_sync_n(2, 128);
+      // (the test hook withholds this signal: every role's bounded wait then runs out)
+      if (warp == 2 && lane == 0 && !(p.flags & TR_SCAN_STALL_TEST))
+        mbar_arrive(smem_u32(&ctl->bar_m));
+    }
+    for (int j = 0; j < n; ++j) {
+      const int k = j + 1, st = k & 1;
+      const bool got = mbar_wait(smem_u32(&ctl->bar_s), (uint32_t)j & 1u, ab) &&
+                       mbar_wait(smem_u32(&ctl->full[st]), (uint32_t)(k >> 1) & 1u, ab);
+      // all four state warps leave together (the named barrier below counts them)
+      if (bar_or_n(2, 128, !got)) {
+        failed = true;
+        break;
+      }
+      tc_fence_after();
+      const float gC = *reinterpret_cast<const float *>(sm + st * C_STAGE + C_G);
+      float v0[32], v1[32];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        tmem_ld32(tmem + 128 + lane_base + 32 * h, v0);   // K^T (gamma' U_hi)
+        tmem_ld32(tmem + 192 + lane_base + 32 * h, v1);   // K^T (gamma' U_lo)
+        tc_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) M[32 * h + i] = fmaf(gC, M[32 * h + i], v0[i] + v1[i]);
+      }
+      if (j + 1 < n) {
+        store_state();
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      bar_sync_n(2, 128);
+      if (warp == 2 && lane == 0) {
+        if (j + 1 < n) mbar_arrive(smem_u32(&ctl->bar_m));
+        mbar_arrive(smem_u32(&ctl->empty[st]));   // gamma_C read
+      }
+    }
+    if (!failed) {
+      float *dst = p.S_final + s_off;
+#pragma unroll
+      for (int j = 0; j < DVS; j += 4)
+        *reinterpret_cast<float4 *>(dst + j) = make_float4(M[j], M[j + 1], M[j + 2], M[j + 3]);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------- U warps
+    // warps 6, 7 (TMEM lanes 64-127): U_{c+1} = U~_{c+1} + D rows 64-127, written as bf16
+    // (for A2 U) and gamma' U as a bf16 hi + lo pair (for dM); then U is announced
+    const int q = warp & 3, t = 32 * (q - 2) + lane;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    uint32_t d_phase = 0;
+    if (n > 0) {
+      bool ok = mbar_wait(smem_u32(&ctl->full[0]), 0, ab);
+      if (ok && s0) {
+        ok = mbar_wait(smem_u32(&ctl->bar_d), d_phase, ab);
+        d_phase ^= 1u;
+      }
+      if (!bar_or_n(3, 64, !ok)) {
+        tc_fence_after();
+        const float gp = reinterpret_cast<const float *>(sm + C_GP)[t];
+        float u0[32], u1[32], v0[32], v1[32];
+        if (s0) {
+          tmem_ld32(tmem + 64 + lane_base, v0);
+          tmem_ld32(tmem + 64 + lane_base + 32, v1);
+        }
+        load_row32_f32(sm + C_UT, t, u0);
+        load_row32_f32(sm + C_UT + 8192, t, u1);
+        if (s0) {
+          tc_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) { u0[i] += v0[i]; u1[i] += v1[i]; }
+        }
+        store_row_bf16(sm + C_UTL, t, 0, u0, 1.f);
+        store_row_bf16(sm + C_UTL, t, 32, u1, 1.f);
+        store_row_split(sm + C_GUH, sm + C_GUL, t, 0, u0, gp);
+        store_row_split(sm + C_GUH, sm + C_GUL, t, 32, u1, gp);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        bar_sync_n(3, 64);
+        if (warp == 6 && lane == 0) {
+          mbar_arrive(smem_u32(&ctl->bar_u));
+          mbar_arrive(smem_u32(&ctl->empty[0]));
+          mbar_arrive(smem_u32(&ctl->empty[0]));   // stage 0 holds no gamma_C
+        }
+        for (int j = 0; j < n; ++j) {
+          const int k = j + 1, st = k & 1;
+          const bool got = mbar_wait(smem_u32(&ctl->bar_d), d_phase, ab) &&
+                           mbar_wait(smem_u32(&ctl->full[st]), (uint32_t)(k >> 1) & 1u, ab);
+          if (bar_or_n(3, 64, !got)) break;
+          d_phase ^= 1u;
+          tc_fence_after();
+          if (j + 1 < n) {
+            const uint32_t dcol = tmem + 64 * (j & 1) + lane_base;
+            const uint8_t *ut = sm + st * C_STAGE + C_UT;
+            const float gq = reinterpret_cast<const float *>(sm + st * C_STAGE + C_GP)[t];
+            tmem_ld32(dcol, v0);
+            tmem_ld32(dcol + 32, v1);
+            load_row32_f32(ut, t, u0);
+            load_row32_f32(ut + 8192, t, u1);
+            tc_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) { u0[i] += v0[i]; u1[i] += v1[i]; }
+            store_row_bf16(sm + C_UTL, t, 0, u0, 1.f);
+            store_row_bf16(sm + C_UTL, t, 32, u1, 1.f);
+            store_row_split(sm + C_GUH, sm + C_GUL, t, 0, u0, gq);
+            store_row_split(sm + C_GUH, sm + C_GUL, t, 32, u1, gq);
+            fence_proxy_async_smem();
+          }
+          tc_fence_before();
+          bar_sync_n(3, 64);
+          if (warp == 6 && lane == 0) {
+            if (j + 1 < n) mbar_arrive(smem_u32(&ctl->bar_u));
+            mbar_arrive(smem_u32(&ctl->empty[st]));
+          }
+        }
+      }
+    }
+  } else if (want_o) {
+    // ------------------------------------------------------------- O warps
+    // warps 8, 9 (TMEM lanes 0-63): O_c = D rows 0-63 (scaled, bf16).  Full chunks go out
+    // by one TMA store from a double-buffered staging tile; the ragged last chunk by
+    // per-row stores.  D[c % 2] is released to the issuer once read.
+    const int q = warp & 3, t = 32 * q + lane;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    const float sc = p.scale;
+    for (int j = 0; j < n; ++j) {
+      // D[j % 2]'s (j / 2)-th use is complete (one barrier per buffer: these warps may
+      // trail the chain by up to two chunks)
+      const bool got = mbar_wait(smem_u32(&ctl->bar_dO[j & 1]), (uint32_t)(j >> 1) & 1u, ab);
+      if (bar_or_n(4, 64, !got)) break;
+      tc_fence_after();
+      const uint32_t dcol = tmem + 64 * (j & 1) + lane_base;
+      float v0[32], v1[32];
+      tmem_ld32(dcol, v0);
+      tmem_ld32(dcol + 32, v1);
+      tc_wait_ld();
+      // staging buffer j % 2 was last read by the store of chunk j - 2
+      if (warp == 8 && lane == 0) bulk_wait_read<1>();
+      tc_fence_before();
+      bar_sync_n(4, 64);
+      if (warp == 8 && lane == 0) mbar_arrive(smem_u32(&ctl->bar_o[j & 1]));
+      const int tok0 = t_begin + C * j;
+      if (tok0 + C <= t_end) {
+        uint8_t *stg = sm + C_MTL + 8192 * (j & 1);
+        store_row_bf16(stg, t, 0, v0, sc);
+        store_row_bf16(stg, t, 32, v1, sc);
+        fence_proxy_async_smem();
+        bar_sync_n(4, 64);
+        if (warp == 8 && lane == 0) {
+          tma_store_2d(&tm_o, smem_u32(stg), head * p.dv + slice * DVS, tok0);
+          bulk_commit();
+        }
+      } else if (tok0 + t < t_end) {
+        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.o) +
+                                               (size_t)(tok0 + t) * p.o_stride +
+                                               (size_t)head * p.dv + slice * DVS);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          dst[w] = make_uint4(pack_bf16x2(v0[8 * w] * sc, v0[8 * w + 1] * sc),
+                              pack_bf16x2(v0[8 * w + 2] * sc, v0[8 * w + 3] * sc),
+                              pack_bf16x2(v0[8 * w + 4] * sc, v0[8 * w + 5] * sc),
+                              pack_bf16x2(v0[8 * w + 6] * sc, v0[8 * w + 7] * sc));
+          dst[4 + w] = make_uint4(pack_bf16x2(v1[8 * w] * sc, v1[8 * w + 1] * sc),
+                                  pack_bf16x2(v1[8 * w + 2] * sc, v1[8 * w + 3] * sc),
+                                  pack_bf16x2(v1[8 * w + 4] * sc, v1[8 * w + 5] * sc),
+                                  pack_bf16x2(v1[8 * w + 6] * sc, v1[8 * w + 7] * sc));
+        }
+      }
+    }
+    // the outputs are in global memory before the kernel ends
+    if (warp == 8 && lane == 0) bulk_wait<0>();
   }
 
-  if (tid == 0) bulk_wait<0>();
-  if (!failed && !producer) {
-    float *dst = p.S_final + s_off;
-#pragma unroll
-    for (int j = 0; j < kCols; j += 4)
-      *reinterpret_cast<float4 *>(dst + j) = make_float4(Mr[j], Mr[j + 1], Mr[j + 2], Mr[j + 3]);
+  // a CTA that gave up a wait leaves no copy or product in flight behind it
+  __syncwarp();
+  const bool aborted = *ab.flag != 0;
+  if (warp == 0 && lane == 0 && aborted)
+    for (int b = 0; b < 2; ++b)
+      if (last_k[b] >= 0) mbar_wait_drain(smem_u32(&ctl->full[b]), (uint32_t)(last_k[b] >> 1) & 1u);
+  if (warp == 1 && lane == 0 && aborted && mma_pending) {
+    tc_commit(smem_u32(&ctl->drain));
+    mbar_wait_drain(smem_u32(&ctl->drain), 0);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 64);
+    tmem_dealloc(tmem, 256);
   }
 }
 
 __global__ void __launch_bounds__(kChainThreads, 1)
-    scan_chain_kernel(const __grid_constant__ CUtensorMap tm_A, const __grid_constant__ CUtensorMap tm_B,
-                      const __grid_constant__ CUtensorMap tm_M, const __grid_constant__ ScanLaunch p,
-                      const __grid_constant__ ScanWs ws) {
-  chain_body(tm_A, tm_B, tm_M, p, ws, blockIdx.x, blockIdx.y);
+    scan_chain_kernel(const __grid_constant__ ScanMaps mp, const __grid_constant__ ScanLaunch p,
+                      const __grid_constant__ ScanWs ws, const __grid_constant__ ScanPlan plan) {
+  chain_body(mp, p, ws, plan, blockIdx.x, false);
 }
 
-// ========================================================= readout kernel
-// o_c = R_c M_c + O0_c for every (chunk, head) in parallel: one tcgen05 product
-// ([R; unused rows] (128 x 128) times the bf16 chunk-start state M_c (128 x DV)),
-// plus the fp32 O0, scaled and stored as bf16.  128 threads; thread t < 64 owns
-// token row t.
-constexpr uint32_t O_R = 0;          // [half][128 rows][128 B]: rows 0-63 = R
-constexpr uint32_t O_M = 32768;      // [DV/64 blocks][128 d][128 B]: M_c
-constexpr uint32_t O_O = 65536;      // [DV/32 boxes][64 rows][32 fp32]: O0
-constexpr size_t OUT_SMEM = O_O + 32768 + 1024;
-
+// ===================================================== prep beside chain
+// For few chains (a long sequence's heads: the latency-bound case) the chains run in the
+// same launch as the prep, on their own CTAs, each stage waiting for its slots' flags, so
+// the chain starts with the first chunks instead of after the last.  The launch is
+// cooperative: every CTA is resident at once, so a chain never waits on a prep CTA that
+// cannot be scheduled.  CTAs [0, n_chain) run chains, the rest (warps 0-7) the prep.
 template <int DV>
-__global__ void __launch_bounds__(128)
-    scan_out_kernel(const __grid_constant__ CUtensorMap tm_R, const __grid_constant__ CUtensorMap tm_M,
-                    const __grid_constant__ CUtensorMap tm_O, ScanLaunch p, ScanWs ws,
-                    int total_chunks) {
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_t, bar_m;
-  __shared__ uint32_t tmem_s;
-  __shared__ int abort_s;
-  __shared__ int cu_chunks[kMaxSeqsChunked + 1];
-  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                            ~static_cast<uintptr_t>(1023));
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int H = p.H;
-  const int64_t item = blockIdx.x;
-  const int chunk = (int)(item / H), head = (int)(item % H);
-  if (tid == 0) {
-    tma_prefetch_desc(&tm_R);
-    tma_prefetch_desc(&tm_M);
-    tma_prefetch_desc(&tm_O);
-    mbar_init(smem_u32(&bar_t), 1);
-    mbar_init(smem_u32(&bar_m), 1);
-    abort_s = 0;
-    fence_mbar_init();
+__global__ void __launch_bounds__(kChainThreads, 1)
+    scan_fused_kernel(const __grid_constant__ ScanMaps mp, const __grid_constant__ ScanLaunch p,
+                      const __grid_constant__ ScanWs ws, const __grid_constant__ ScanPlan plan,
+                      int n_chain) {
+  if ((int)blockIdx.x < n_chain) {
+    chain_body(mp, p, ws, plan, blockIdx.x, true);
+  } else if (threadIdx.x < kPrepThreads) {
+    prep_body<DV>(mp, p, ws, plan, (int)blockIdx.x - n_chain, (int)gridDim.x - n_chain, true);
   }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(&tmem_s), DV);
-    tmem_relinquish();
+}
+
+// Host-side plan for up to kParamSeqs sequences: chunk offsets and the longest-first order.
+bool host_plan(const ScanLaunch &p, ScanPlan *pl) {
+  pl->in_params = 0;
+  if (p.n_seqs > kParamSeqs) return false;
+  int acc = 0;
+  int nch[kParamSeqs];
+  for (int i = 0; i < p.n_seqs; ++i) {
+    pl->cu_chunks[i] = acc;
+    nch[i] = (p.cu_seqlens_host[i + 1] - p.cu_seqlens_host[i] + C - 1) / C;
+    acc += nch[i];
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  // TMEM is held: let the next kernel launch; then wait for the previous one's outputs
-  pdl_trigger();
-  pdl_wait();
-  if (tid == 0) {
-    int acc = 0;
-    for (int i = 0; i < p.n_seqs; ++i) {
-      cu_chunks[i] = acc;
-      acc += (p.cu_seqlens[i + 1] - p.cu_seqlens[i] + C - 1) / C;
-    }
-    cu_chunks[p.n_seqs] = acc;
-  }
-  __syncthreads();
-  const uint32_t tmem = tmem_s;
-  const AbortFlag ab{&abort_s, p.err_word, ERRBIT_SCAN_TIMEOUT};
-  int lo = 0, hi = p.n_seqs - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (cu_chunks[mid] <= chunk) lo = mid; else hi = mid - 1;
-  }
-  const int seq = lo;
-  const int t0 = p.cu_seqlens[seq] + (chunk - cu_chunks[seq]) * C;
-  const int nv = min(C, p.cu_seqlens[seq + 1] - t0);
-  if (tid == 0) {
-    const uint32_t r_u = smem_u32(sm + O_R), m_u = smem_u32(sm + O_M);
-    mbar_arrive_expect_tx(smem_u32(&bar_t), 16384u + (uint32_t)DV * 256u + (uint32_t)DV * 256u);
-#pragma unroll
-    for (int b = 0; b < DV / 32; ++b)
-      tma_load_2d(smem_u32(sm + O_O) + 8192 * b, &tm_O, 32 * b, (int32_t)(item * 64), smem_u32(&bar_t));
-    tma_load_2d(r_u, &tm_R, 0, (int32_t)(item * 64), smem_u32(&bar_t));
-    tma_load_2d(r_u + 16384, &tm_R, 64, (int32_t)(item * 64), smem_u32(&bar_t));
-#pragma unroll
-    for (int b = 0; b < DV / 64; ++b)
-      tma_load_2d(m_u + 16384 * b, &tm_M, 64 * b, (int32_t)(item * 128), smem_u32(&bar_t));
-  }
-  bool ok = mbar_wait(smem_u32(&bar_t), 0, ab);
-  if (tid == 0 && ok) {
-    tc_fence_after();
-    const uint64_t rd = kmaj(smem_u32(sm + O_R)), md = mnmaj(smem_u32(sm + O_M), 16384);
-#pragma unroll
-    for (int kk = 0; kk < DK / 16; ++kk)
-      tc_mma_bf16(tmem, desc_k(rd, kk, 16384), desc_mn(md, kk), idesc_bf16(128, DV, 0, 1), kk > 0);
-    tc_commit(smem_u32(&bar_m));
-  }
-  ok = ok && mbar_wait(smem_u32(&bar_m), 0, ab);
-  if (__syncthreads_or(!ok)) {
-    // a wait ran out: leave the outputs alone
-  } else {
-    tc_fence_after();
-    if (tid < C) {
-      const float sc = p.scale;
-#pragma unroll 1
-      for (int j = 0; j < DV / 32; ++j) {
-        float v[32], b[32];
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 32 * j, v);
-        load_row32_f32(sm + O_O + 8192 * j, tid, b);
-        tc_wait_ld();
-        if (tid < nv) {
-          uint4 *d4 = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.o) +
-                                                (size_t)(t0 + tid) * p.o_stride + (size_t)head * DV + 32 * j);
-#pragma unroll
-          for (int w = 0; w < 4; ++w)
-            d4[w] = make_uint4(pack_bf16x2((v[8 * w] + b[8 * w]) * sc, (v[8 * w + 1] + b[8 * w + 1]) * sc),
-                               pack_bf16x2((v[8 * w + 2] + b[8 * w + 2]) * sc, (v[8 * w + 3] + b[8 * w + 3]) * sc),
-                               pack_bf16x2((v[8 * w + 4] + b[8 * w + 4]) * sc, (v[8 * w + 5] + b[8 * w + 5]) * sc),
-                               pack_bf16x2((v[8 * w + 6] + b[8 * w + 6]) * sc, (v[8 * w + 7] + b[8 * w + 7]) * sc));
-        }
-      }
-    }
-  }
-  (void)lane;
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, DV);
-  }
+  pl->cu_chunks[p.n_seqs] = acc;
+  std::iota(pl->order, pl->order + p.n_seqs, 0);
+  std::stable_sort(pl->order, pl->order + p.n_seqs,
+                   [&](int a, int b) { return nch[a] > nch[b]; });
+  pl->in_params = 1;
+  return true;
 }
 
 }  // namespace
@@ -1138,9 +1400,20 @@ bool make_tmap_f32_2d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_
                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
                       std::string *err);
 
+// The fused launch serves few chains (at most kFusedMaxChains CTAs, leaving most SMs to the
+// prep) of a plan that travels in the launch.
+constexpr int kFusedMaxChains = 96;
+int64_t fused_chains(const ScanLaunch &p) { return (int64_t)p.n_seqs * p.H * (p.dv / DVS); }
+bool use_fused(const ScanLaunch &p, int sms) {
+  const int64_t n = fused_chains(p);
+  return p.n_seqs <= kParamSeqs && n > 0 && n <= kFusedMaxChains && sms - n >= 32 &&
+         count_chunks(p) > 0;
+}
+constexpr size_t FUSED_SMEM = PREP_SMEM > CHAIN_SMEM ? PREP_SMEM : CHAIN_SMEM;
+
 bool scan_chunked_supported(const ScanLaunch &p) {
   return p.dtype == TR_DTYPE_BF16 && p.dk == DK && (p.dv == 64 || p.dv == 128) &&
-         p.n_seqs <= kMaxSeqsChunked && (p.o == nullptr || p.o_stride % 8 == 0);
+         (p.o == nullptr || p.o_stride % 8 == 0);
 }
 
 size_t scan_chunked_workspace(const ScanLaunch &p) {
@@ -1150,14 +1423,19 @@ size_t scan_chunked_workspace(const ScanLaunch &p) {
 }
 
 std::vector<const char *> scan_chunked_kernel_names(const ScanLaunch &p, bool with_readout) {
-  (void)p;
-  if (with_readout) return {"scan_prep", "scan_chain", "scan_out"};
+  (void)with_readout;   // the readout is part of the chain kernel
+  if (use_fused(p, device_sm_count())) return {"scan_fused"};
+  if (p.n_seqs > kParamSeqs) return {"scan_plan", "scan_prep", "scan_chain"};
   return {"scan_prep", "scan_chain"};
 }
 
 cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string *err,
                                 const std::function<cudaError_t()> &between) {
   if (p.n_seqs == 0) return cudaSuccess;
+  if (p.precise_state && p.o) {
+    if (err) *err = "the precise-state chain produces no readout";
+    return cudaErrorInvalidValue;
+  }
   size_t total = 0;
   ScanWs ws = ws_layout(p, p.ws, &total);
   if (total > p.ws_bytes || (total > 0 && !p.ws)) {
@@ -1165,44 +1443,83 @@ cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string
     return cudaErrorInvalidValue;
   }
   const int64_t items = ws.slots;
-  const int total_chunks = (int)(items / p.H);
-  if (items > 0x7fffffffLL) {
+  if (items * 128 > 0x7fffffffLL) {
     if (err) *err = "too many (chunk, head) work items";
+    return cudaErrorInvalidValue;
+  }
+  const int64_t ctas = (int64_t)p.n_seqs * p.H * (p.dv / DVS);
+  if (ctas > 0x7fffffffLL) {
+    if (err) *err = "too many (sequence, head) pairs";
     return cudaErrorInvalidValue;
   }
   const uint64_t T = (uint64_t)(p.T > 0 ? p.T : 1);
   const uint64_t slots = (uint64_t)(items > 0 ? items : 1);
-  CUtensorMap tq, tk, tv, tA, tR;
+  ScanMaps mp;
   const void *qb = p.q ? p.q : p.k;
-  if (!make_tmap_bf16_2d(&tk, p.k, (uint64_t)p.H * DK, T, (uint64_t)p.k_stride * 2, 64, C, err) ||
-      !make_tmap_bf16_2d(&tq, qb, (uint64_t)p.H * DK, T,
+  if (!make_tmap_bf16_2d(&mp.k, p.k, (uint64_t)p.H * DK, T, (uint64_t)p.k_stride * 2, 64, C, err) ||
+      !make_tmap_bf16_2d(&mp.q, qb, (uint64_t)p.H * DK, T,
                          (uint64_t)(p.q ? p.q_stride : p.k_stride) * 2, 64, C, err) ||
-      !make_tmap_bf16_2d(&tv, p.v, (uint64_t)p.H * p.dv, T, (uint64_t)p.v_stride * 2, 64, C, err) ||
-      !make_tmap_bf16_2d(&tA, ws.A, 128, slots * 128, 256, 64, 128, err) ||
-      !make_tmap_bf16_2d(&tR, ws.R, 128, slots * 64, 256, 64, 64, err))
+      !make_tmap_bf16_2d(&mp.v, p.v, (uint64_t)p.H * p.dv, T, (uint64_t)p.v_stride * 2, 64, C, err) ||
+      !make_tmap_bf16_2d(&mp.QW, ws.QW, 128, slots * 128, 256, 64, 64, err) ||
+      !make_tmap_bf16_2d(&mp.PY, ws.PY, 64, slots * 128, 128, 64, 64, err) ||
+      !make_tmap_bf16_2d(&mp.KT, ws.KT, 128, slots * 64, 256, 64, 64, err) ||
+      !make_tmap_f32_2d(&mp.UT, ws.UT, (uint64_t)p.dv, slots * 64, (uint64_t)p.dv * 4, 32, 64, err))
     return cudaErrorInvalidValue;
-  CUtensorMap tB, tM, tO;
-  if (!make_tmap_f32_2d(&tB, ws.B, (uint64_t)p.dv, slots * 128, (uint64_t)p.dv * 4, 32, 128, err) ||
-      !make_tmap_bf16_2d(&tM, ws.M, (uint64_t)p.dv, slots * 128, (uint64_t)p.dv * 2, 64, 128, err) ||
-      !make_tmap_f32_2d(&tO, ws.O, (uint64_t)p.dv, slots * 64, (uint64_t)p.dv * 4, 32, 64, err))
+  // the readout o [T, H d_v] (token stride o_stride), stored in 64 x 64 boxes
+  if (p.o && !make_tmap_bf16_2d(&mp.o, p.o, (uint64_t)p.H * p.dv, T, (uint64_t)p.o_stride * 2,
+                                64, C, err))
     return cudaErrorInvalidValue;
+  if (!p.o) mp.o = mp.k;
+  ScanPlan plan{};
   cudaError_t e;
-  if (items > 0) {
-    int64_t grid = device_sm_count();
-    if (grid > items) grid = items;
-    if (p.dv == 128) {
-      e = cudaFuncSetAttribute(scan_prep_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)PREP_SMEM);
+  const int sms = device_sm_count();
+  if (use_fused(p, sms)) {
+    // chains and prep in one cooperative launch (all CTAs resident at once)
+    ScanLaunch pf = p;
+    static std::atomic<unsigned long long> epoch_counter{0};
+    pf.epoch = ++epoch_counter;
+    host_plan(pf, &plan);
+    const int grid = sms;
+    auto kern = pf.dv == 128 ? scan_fused_kernel<128> : scan_fused_kernel<64>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FUSED_SMEM);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kChainThreads);
+    cfg.dynamicSmemBytes = FUSED_SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pf.pdl ? 2 : 1;
+    e = cudaLaunchKernelEx(&cfg, kern, mp, pf, ws, plan, (int)fused_chains(p));
+    if (e == cudaSuccess || !pf.pdl) return e;
+    // a runtime that will not combine a cooperative launch with programmatic serialization:
+    // the same launch without the latter
+    (void)cudaGetLastError();
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, mp, pf, ws, plan, (int)fused_chains(p));
+  }
+  if (!host_plan(p, &plan)) {
+    e = launch_kernel(scan_plan_kernel, dim3(1), dim3(kPlanThreads), 0, s, p.pdl, p.cu_seqlens,
+                      p.n_seqs, ws.cu_chunks, ws.order);
+    if (e != cudaSuccess) return e;
+    if (between) {
+      e = between();
       if (e != cudaSuccess) return e;
-      e = launch_kernel(scan_prep_kernel<128>, dim3((unsigned)grid), dim3(kPrepThreads), PREP_SMEM,
-                        s, p.pdl, tq, tk, tv, tA, tB, tR, tO, p, ws, total_chunks);
-    } else {
-      e = cudaFuncSetAttribute(scan_prep_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)PREP_SMEM);
-      if (e != cudaSuccess) return e;
-      e = launch_kernel(scan_prep_kernel<64>, dim3((unsigned)grid), dim3(kPrepThreads), PREP_SMEM,
-                        s, p.pdl, tq, tk, tv, tA, tB, tR, tO, p, ws, total_chunks);
     }
+  }
+  if (items > 0) {
+    int64_t grid = sms;
+    if (grid > items) grid = items;
+    auto kern = p.dv == 128 ? scan_prep_kernel<128> : scan_prep_kernel<64>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PREP_SMEM);
+    if (e != cudaSuccess) return e;
+    e = launch_kernel(kern, dim3((unsigned)grid), dim3(kPrepThreads), PREP_SMEM, s, p.pdl, mp, p,
+                      ws, plan);
     if (e != cudaSuccess) return e;
   }
   if (between) {
@@ -1212,26 +1529,8 @@ cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string
   e = cudaFuncSetAttribute(scan_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)CHAIN_SMEM);
   if (e != cudaSuccess) return e;
-  e = launch_kernel(scan_chain_kernel, dim3((unsigned)(p.n_seqs * p.H), (unsigned)(p.dv / DVS)),
-                    dim3(kChainThreads), CHAIN_SMEM, s, p.pdl, tA, tB, tM, p, ws);
-  if (e != cudaSuccess || !p.o || items == 0) return e;
-  if (between) {
-    e = between();
-    if (e != cudaSuccess) return e;
-  }
-  if (p.dv == 128) {
-    e = cudaFuncSetAttribute(scan_out_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)OUT_SMEM);
-    if (e != cudaSuccess) return e;
-    return launch_kernel(scan_out_kernel<128>, dim3((unsigned)items), dim3(128), OUT_SMEM, s, p.pdl,
-                         tR, tM, tO, p, ws, total_chunks);
-  } else {
-    e = cudaFuncSetAttribute(scan_out_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)OUT_SMEM);
-    if (e != cudaSuccess) return e;
-    return launch_kernel(scan_out_kernel<64>, dim3((unsigned)items), dim3(128), OUT_SMEM, s, p.pdl,
-                         tR, tM, tO, p, ws, total_chunks);
-  }
+  return launch_kernel(scan_chain_kernel, dim3((unsigned)ctas), dim3(kChainThreads), CHAIN_SMEM,
+                       s, p.pdl, mp, p, ws, plan);
 }
 
 }  // namespace tr

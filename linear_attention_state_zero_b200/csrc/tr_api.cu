@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>
@@ -123,6 +124,10 @@ int record_error(int status, const char *fmt, ...) {
   return status;
 }
 
+std::atomic<unsigned long long> g_wait_ns{4000000000ull};
+
+unsigned long long scan_wait_limit_ns() { return g_wait_ns.load(); }
+
 int device_sm_count() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
@@ -211,7 +216,7 @@ tr_status validate_scan(const tr_scan_args *a, tr::ScanLaunch *out) {
   if ((a->d_k != 64 && a->d_k != 128) || (a->d_v != 64 && a->d_v != 128))
     return fail(TR_ERR_UNSUPPORTED, "d_k = %d, d_v = %d: supported values are 64 and 128", a->d_k,
                 a->d_v);
-  if (a->flags & ~(unsigned)(TR_NORMALIZE_QK | TR_SCAN_RECURRENT))
+  if (a->flags & ~(unsigned)(TR_NORMALIZE_QK | TR_SCAN_RECURRENT | TR_SCAN_STALL_TEST))
     return fail(TR_ERR_INVALID_ARG, "unknown scan flags 0x%x", a->flags);
   if (!a->S_final || !a->cu_seqlens)
     return fail(TR_ERR_INVALID_ARG, "a required pointer is NULL");
@@ -261,6 +266,8 @@ tr_status validate_scan(const tr_scan_args *a, tr::ScanLaunch *out) {
   p.ws = nullptr;
   p.ws_bytes = 0;
   p.pdl = true;
+  p.wait_ns = tr::scan_wait_limit_ns();
+  p.precise_state = false;
   return TR_OK;
 }
 
@@ -321,6 +328,8 @@ tr::ScanLaunch group_scan_launch(const tr_group_args *a) {
   sp.flags = 0;
   sp.scale = 1.f;
   sp.cu_seqlens_host = a->cu_seqlens_host;
+  sp.wait_ns = tr::scan_wait_limit_ns();
+  sp.precise_state = false;
   return sp;
 }
 
@@ -679,6 +688,12 @@ extern "C" {
 
 const char *tr_last_error(void) { return g_last_error.c_str(); }
 
+tr_status tr_set_wait_limit_ns(uint64_t ns) {
+  if (ns > 60000000000ull) return fail(TR_ERR_INVALID_ARG, "wait limit above 60 s");
+  tr::g_wait_ns.store(ns ? ns : 4000000000ull);
+  return ok();
+}
+
 const char *tr_version(void) {
   return "libtr (Tail-Replay GDN tail replay), sm_100a";
 }
@@ -762,6 +777,9 @@ tr_status tr_transition_product(const tr_scan_args *args, float *P, void *ws, si
   p.ws = base + L.scan;
   p.ws_bytes = ws_bytes - L.scan;
   p.err_word = errw;
+  // P is the whole result and, under slow decay, keeps every chunk's rounding: the chunked
+  // chain takes the state into its products as a bf16 hi + lo pair
+  p.precise_state = true;
   st = run_scan(p, s);
   return st == TR_OK ? ok() : st;
 }

@@ -85,7 +85,13 @@ struct ScanLaunch {
   void *ws;            // scan workspace (chunked kernels), ws_bytes long
   size_t ws_bytes;
   bool pdl;            // launch with programmatic dependent launch
+  unsigned long long wait_ns;  // bounded-wait limit of the chunked kernels
+  bool precise_state;  // chunked chain: the state enters its products as a bf16 hi + lo pair
+  unsigned long long epoch;    // per-call tag of the chunked scan's ready flags (set at launch)
 };
+
+// The bounded-wait limit the scan kernels get (tr_set_wait_limit_ns; 4 s by default).
+unsigned long long scan_wait_limit_ns();
 
 int device_sm_count();
 

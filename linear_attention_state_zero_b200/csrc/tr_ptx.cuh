@@ -84,11 +84,12 @@ struct AbortFlag {
   volatile int *flag;   // shared memory
   unsigned *err_word;   // global memory (may be nullptr)
   unsigned err_bit;
+  unsigned long long limit_ns = WAIT_LIMIT_NS;   // give up after this much wall-clock time
 };
 
 // Wait for the phase with parity `parity` of the mbarrier to complete.
 // Returns false (and raises the CTA's abort flag and the error word) if it did
-// not complete within WAIT_LIMIT_NS, or if another role already aborted.
+// not complete within ab.limit_ns, or if another role already aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const AbortFlag &ab) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
@@ -97,11 +98,25 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const A
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (*ab.flag) return false;
-    if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+    if (globaltimer_ns() - t0 > ab.limit_ns) {
       *ab.flag = 1;
       if (ab.err_word) atomicOr(ab.err_word, ab.err_bit);
       return false;
     }
+  }
+}
+
+// Drain wait of an abort path: wait for the phase with parity `parity` to complete (the
+// copies or products still in flight behind it), bounded by DRAIN_LIMIT_NS whatever the
+// caller's wait limit.  Returns whether it completed.
+constexpr unsigned long long DRAIN_LIMIT_NS = 200000000ull;
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > DRAIN_LIMIT_NS) return false;
   }
 }
 

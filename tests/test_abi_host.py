@@ -256,3 +256,11 @@ def test_replay_kernel_names_match_the_count():
     assert names.count("short_conv") == 3 and names.count("gated_norm") == 2
     assert names.count("ffn_gate_up") == 2 and names.count("ffn_down") == 2
     assert tr.lib.tr_replay_group_kernel_names(None) == b""
+
+
+def test_wait_limit_setting_is_host_only_and_checked():
+    """tr_set_wait_limit_ns accepts up to 60 s (0 = the default) and rejects more; it only
+    sets a host value that later scan launches carry."""
+    assert tr.lib.tr_set_wait_limit_ns(61_000_000_000) == 1
+    assert tr.lib.tr_set_wait_limit_ns(1_000_000) == 0
+    assert tr.lib.tr_set_wait_limit_ns(0) == 0

@@ -130,3 +130,21 @@ def test_no_readout(cuda_device):
 
 def test_check_reports_clean_state(cuda_device):
     tr.check()
+
+
+@pytest.mark.parametrize("n_seqs,max_len,H", [(100, 300, 2), (1500, 90, 1), (5000, 70, 1)])
+def test_many_sequences(cuda_device, n_seqs, max_len, H):
+    """More sequences than travel in the launch (the plan kernel orders them longest first on
+    the device), more than the old per-block limit of 1024, and more than the sort covers
+    (identity order), with empty and ragged sequences: every output against the oracle."""
+    lens = [int(x) for x in np.random.default_rng(n_seqs).integers(0, max_len, n_seqs)]
+    lens[3] = lens[n_seqs // 2] = 0   # empty sequences among them
+    case = synth.scan_case(lens, H, 128, 128, torch.bfloat16, 0.9, 1.0, seed=600 + n_seqs)
+    o, S = run_gpu(case, cuda_device)
+    torch.cuda.synchronize()
+    tr.check()
+    wo, wS = run_oracle(case)
+    assert rel_fro(o, wo) < TOL_BF16
+    assert rel_fro(S, wS) < TOL_BF16
+    empty = [i for i, n in enumerate(lens) if n == 0]
+    assert empty and not S[empty].any()
