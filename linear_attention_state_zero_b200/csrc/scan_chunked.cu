@@ -157,6 +157,7 @@ __device__ __forceinline__ void scale_row32_bf16(uint8_t *tile, int row, int col
 // chunk count, longest first (ties by index).
 struct ScanPlan {
   int32_t cu_chunks[kParamSeqs + 1];
+  int32_t cu_tokens[kParamSeqs + 1];   // the sequences' token offsets (cu_seqlens)
   int32_t order[kParamSeqs];
   int in_params;     // 1: the arrays above hold the plan; 0: it is in the workspace
 };
@@ -295,6 +296,9 @@ __device__ __forceinline__ const int32_t *plan_cu_chunks(const ScanPlan &pl, con
 __device__ __forceinline__ const int32_t *plan_order(const ScanPlan &pl, const ScanWs &ws) {
   return pl.in_params ? pl.order : ws.order;
 }
+__device__ __forceinline__ const int32_t *plan_cu_tokens(const ScanPlan &pl, const ScanLaunch &p) {
+  return pl.in_params ? pl.cu_tokens : p.cu_seqlens;
+}
 
 // ============================================================ prep kernel
 // 256 threads, persistent over work items (item = chunk_global * H + head, CTA b takes
@@ -328,8 +332,9 @@ struct PrepItem {
 
 struct PrepCtl {
   uint64_t tma_bar[2];
-  uint64_t mma_bar;
-  uint64_t drain_bar;
+  uint64_t mma_bar;     // group 1, then the first part of group 2 (thread 0, thread 64)
+  uint64_t mma_bar2;    // the second part of group 2 (thread 64)
+  uint64_t drain_bar, drain_bar2;
   uint32_t tmem;
   int abort;
   PrepItem cur, nxt;
@@ -345,14 +350,14 @@ struct PrepCtl {
 
 // The item's location given its sequence (cu_chunks[seq] <= chunk < cu_chunks[seq + 1]).
 __device__ __forceinline__ PrepItem item_at(int64_t item, int seq, const ScanLaunch &p,
-                                            const int32_t *cu_chunks) {
+                                            const int32_t *cu_chunks, const int32_t *cu_tokens) {
   PrepItem it;
   const int chunk = (int)(item / p.H);
   it.seq = seq;
   it.c = chunk - cu_chunks[seq];
   it.head = (int)(item % p.H);
-  it.t0 = p.cu_seqlens[seq] + it.c * C;
-  it.nv = min(C, p.cu_seqlens[seq + 1] - it.t0);
+  it.t0 = cu_tokens[seq] + it.c * C;
+  it.nv = min(C, cu_tokens[seq + 1] - it.t0);
   it.has_prev = it.c > 0;
   it.slot = item;
   return it;
@@ -401,7 +406,8 @@ __device__ __forceinline__ void publish_slot(const ScanWs &ws, int64_t slot, uns
 }
 
 // The prep work of CTA `vb` of `vg` (256 threads: warps 0-7).  With `publish`, each item's
-// flag is set once its stores have completed (one item later, so thread 0 never waits).
+// flag is set once its stores have completed: by thread 0 right after it has issued the next
+// item's first products (or after the loop, for the last item).
 template <int DV>
 __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &p, const ScanWs &ws,
                                           const ScanPlan &plan, int vb, int vg, bool publish) {
@@ -422,6 +428,7 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
   const int64_t n_items = ws.slots;
   const int64_t stride = vg;
   const int32_t *cu_chunks = plan_cu_chunks(plan, ws);
+  const int32_t *cu_tokens = plan_cu_tokens(plan, p);
 
   if (tid == 0) {
     tma_prefetch_desc(&tm_q);
@@ -434,7 +441,9 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
     mbar_init(smem_u32(&ctl->tma_bar[0]), 1);
     mbar_init(smem_u32(&ctl->tma_bar[1]), 1);
     mbar_init(smem_u32(&ctl->mma_bar), 1);
+    mbar_init(smem_u32(&ctl->mma_bar2), 1);
     mbar_init(smem_u32(&ctl->drain_bar), 1);
+    mbar_init(smem_u32(&ctl->drain_bar2), 1);
     ctl->abort = 0;
     fence_mbar_init();
   }
@@ -487,12 +496,14 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
   };
 
   int64_t item = vb;
-  int seq_cur = 0;   // thread 0: the sequence of the current item
+  int seq_cur = 0;   // threads 0 and 32: the sequence of the current item
   float la_next = 0.f, b_next = 0.f;
-  if (tid == 0 && item < n_items) {
+  if ((tid == 0 || tid == 32) && item < n_items) {
     seq_cur = seq_of_chunk((int)(item / p.H), p.n_seqs, cu_chunks);
     seq_cur = advance_seq(seq_cur, (int)(item / p.H), cu_chunks);
-    ctl->cur = item_at(item, seq_cur, p, cu_chunks);
+  }
+  if (tid == 0 && item < n_items) {
+    ctl->cur = item_at(item, seq_cur, p, cu_chunks, cu_tokens);
     fence_proxy_async_smem();
     issue(ctl->cur, 0);
   }
@@ -501,7 +512,8 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
 
   const uint32_t mma_bar = smem_u32(&ctl->mma_bar);
   uint32_t mma_phase = 0;
-  bool mma_pending = false;   // thread 0: products issued whose completion was not seen
+  uint32_t mma2_phase = 0;
+  bool mma_pending = false;   // threads 0, 64: products issued whose completion was not seen
   auto mma_wait = [&]() -> bool {
     const bool ok = mbar_wait(mma_bar, mma_phase, ab);
     mma_phase ^= 1u;
@@ -569,14 +581,21 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
                     idesc_bf16(128, 128, 0, 0), kk > 0);
       tc_commit(mma_bar);
       mma_pending = true;
-      // the next item's location (its gates are loaded under the inverse)
-      if (has_next) {
-        seq_cur = advance_seq(seq_cur, (int)((item + stride) / p.H), cu_chunks);
-        ctl->nxt = item_at(item + stride, seq_cur, p, cu_chunks);
+      if (publish && prev_slot >= 0) {
+        // the previous item's three store groups have completed: publish it for the chain
+        bulk_wait<0>();
+        publish_slot(ws, prev_slot, p.epoch);
+        prev_slot = -1;
+      } else {
+        // the previous item's first store group (P, -Y) has read its staging: P and Z are
+        // written below
+        bulk_wait_read<2>();
       }
-      // the previous item's first store group (P, -Y) has read its staging: P and Z are
-      // written below
-      bulk_wait_read<2>();
+    } else if (tid == 32 && has_next) {
+      // the next item's location, beside the products (its gates are loaded under the
+      // inverse, its bands after group 2 is issued)
+      seq_cur = advance_seq(seq_cur, (int)((item + stride) / p.H), cu_chunks);
+      ctl->nxt = item_at(item + stride, seq_cur, p, cu_chunks, cu_tokens);
     }
     if (!mma_wait()) break;
 
@@ -719,12 +738,14 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
       *reinterpret_cast<float4 *>(Xs + r * LDX + c0) = make_float4(x0, x1, x2, x3);
     }
     bar_sync_n(1, kPrepThreads);
-    {  // T21 = -T22 X
+    {  // T21 = -T22 X: thread -> row r, columns c0..c0+3; T22 is lower triangular, so
+       // columns s > r of it contribute nothing (the warp's rows end at 4 warp + 3)
       const int r = tid >> 3, c0 = (tid & 7) * 4;
       float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
       const float *Tr = Ts + (32 + r) * LDA + 32;
-#pragma unroll 4
+#pragma unroll
       for (int s = 0; s < 32; s += 4) {
+        if (s > 4 * warp + 3) break;
         const float4 a = *reinterpret_cast<const float4 *>(Tr + s);
         const float av[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
@@ -760,9 +781,12 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
     fence_proxy_async_smem();
     bar_sync_n(1, kPrepThreads);
 
-    // group 2: [T'; T''] K -> cols [128, 256) (rows 0-63: W); [T'; T''] V (hi + lo) ->
-    // [256, 256 + DV) (rows 64-127: U~); [T'; T''] Z -> [384, 448) (rows 0-63: Y)
-    if (tid == 0) {
+    // group 2, issued by thread 64 in two parts: [T'; T''] K -> cols [128, 256) (rows 0-63:
+    // W) and [T'; T''] Z -> [384, 448) (rows 0-63: Y), committed for the W / Y epilogue; then
+    // [T'; T''] V (hi + lo) -> [256, 256 + DV) (rows 64-127: U~).  Thread 0 meanwhile
+    // prefetches the next item into the other stage, once the previous item's output
+    // stores have finished reading their staging there (issued an item ago: usually done).
+    if (tid == 64) {
       tc_fence_after();
       const uint64_t th = kmaj(smem_u32(sm + P_THI)), tl = kmaj(smem_u32(sm + P_TLO));
       const uint64_t dk_ = mnmaj(st_u + 8192, 32768), dv_ = mnmaj(st_u + 24576, 32768);
@@ -770,30 +794,40 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
 #pragma unroll
       for (int kk = 0; kk < C / 16; ++kk)
         tc_mma_bf16(tmem + 128, desc_k(th, kk, 0), desc_mn(dk_, kk), idesc_bf16(128, 128, 0, 1), kk > 0);
-#pragma unroll
-      for (int kk = 0; kk < C / 16; ++kk)
-        tc_mma_bf16(tmem + 256, desc_k(th, kk, 0), desc_mn(dv_, kk), idesc_bf16(128, DV, 0, 1), kk > 0);
-#pragma unroll
-      for (int kk = 0; kk < C / 16; ++kk)
-        tc_mma_bf16(tmem + 256, desc_k(tl, kk, 0), desc_mn(dv_, kk), idesc_bf16(128, DV, 0, 1), 1u);
       if (it.has_prev) {
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk)
           tc_mma_bf16(tmem + 384, desc_k(th, kk, 0), desc_mn(dz, kk), idesc_bf16(128, 64, 0, 1), kk > 0);
       }
       tc_commit(mma_bar);
+#pragma unroll
+      for (int kk = 0; kk < C / 16; ++kk)
+        tc_mma_bf16(tmem + 256, desc_k(th, kk, 0), desc_mn(dv_, kk), idesc_bf16(128, DV, 0, 1), kk > 0);
+#pragma unroll
+      for (int kk = 0; kk < C / 16; ++kk)
+        tc_mma_bf16(tmem + 256, desc_k(tl, kk, 0), desc_mn(dv_, kk), idesc_bf16(128, DV, 0, 1), 1u);
+      tc_commit(smem_u32(&ctl->mma_bar2));
       mma_pending = true;
-      // prefetch the next item into the other stage once the previous item's output stores
-      // have finished reading their staging there (issued an item ago: usually done)
+    } else if (tid == 0) {
       bulk_wait_read<0>();
       if (has_next) {
         fence_proxy_async_smem();
         issue(ctl->nxt, buf ^ 1);
       }
     }
-    if (!mma_wait()) break;
-
+    // gamma Q in place (thread -> row, 32-column piece): the Q band is no product's operand
     {
+      const int r = tid & 63, pc = tid >> 6, h = pc >> 1, c0 = 32 * (pc & 1);
+      if (want_o) scale_row32_bf16(ST + h * 32768, r, c0, ctl->gq[r]);
+    }
+    // lane quarters 0, 1 (W, Y) wait for the first part, quarters 2, 3 (U~) for the second
+    const bool ok2 = mbar_wait(q4 < 2 ? mma_bar : smem_u32(&ctl->mma_bar2),
+                               q4 < 2 ? mma_phase : mma2_phase, ab);
+    mma_phase ^= 1u;
+    mma2_phase ^= 1u;
+    if (tid == 64 && ok2) mma_pending = false;
+    if (ok2) {
+      tc_fence_after();
       float v[32];
       if (q4 < 2) {
         const int t = q4 * 32 + lane;
@@ -821,10 +855,8 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
           store_row32_f32(sm + P_THI + 8192 * (col >> 5), t, v, 1.f);
         }
       }
-      // gamma Q in place (thread -> row, 32-column piece)
-      const int r = tid & 63, pc = tid >> 6, h = pc >> 1, c0 = 32 * (pc & 1);
-      if (want_o) scale_row32_bf16(ST + h * 32768, r, c0, ctl->gq[r]);
     }
+    if (bar_or_n(1, kPrepThreads, !ok2)) break;
     fence_proxy_async_smem();
     tc_fence_before();
     bar_sync_n(1, kPrepThreads);
@@ -849,14 +881,7 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
       bulk_commit();
       ws.G[slot * 4] = exp_ftz(ctl->g[C - 1]);
       if (has_next) ctl->cur = ctl->nxt;
-      if (publish) {
-        // the previous item's three store groups have completed (this item's three may not)
-        if (prev_slot >= 0) {
-          bulk_wait<3>();
-          publish_slot(ws, prev_slot, p.epoch);
-        }
-        prev_slot = slot;
-      }
+      if (publish) prev_slot = slot;   // published once its stores complete
     }
     if (tid < C) ws.GP[it.slot * C + tid] = ctl->gp[tid];
     bar_sync_n(1, kPrepThreads);
@@ -877,6 +902,10 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
       }
     }
   }
+  if (tid == 64 && item < n_items && mma_pending) {
+    tc_commit(smem_u32(&ctl->drain_bar2));
+    mbar_wait_drain(smem_u32(&ctl->drain_bar2), 0);
+  }
   tc_fence_before();
   bar_sync_n(1, kPrepThreads);
   if (warp == 0) {
@@ -894,16 +923,20 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
 
 // =========================================================== chain kernel
 // One CTA per (sequence, head, 64-column slice of d_v), in longest-first order of the
-// sequences; 320 threads:
+// sequences; 384 threads:
 //   warp 0      TMA producer: stage k (k = 0..n) holds chunk k-1's gamma Q, P, K~ and
-//               gamma_C and chunk k's -gamma_C W, -Y and U~ slice (2 stages)
+//               gamma_C and chunk k's -gamma_C W, -Y and U~ slice (2 stages; the MMA
+//               operands and the epilogue operands each with their own barriers)
 //   warp 1      MMA issuer (one thread)
 //   warps 2-5   state warps: thread (quarter q = warp % 4) owns row d = 32 q + lane of the
 //               fp32 state slice M (64 columns in registers); M_{c+1} = gamma_C M_c + dM
-//   warps 6, 7  U warps (TMEM lanes 64-127): U_{c+1} = U~_{c+1} + D rows 64-127, written as
-//               bf16 and gamma' U_{c+1} as a bf16 hi + lo pair (shared memory)
+//   warps 6, 7, 10, 11  U warps (TMEM lanes 64-127; 6, 7 columns 0-31, 10, 11 columns
+//               32-63): U_{c+1} = U~_{c+1} + D rows 64-127, written as bf16 and
+//               gamma' U_{c+1} as a bf16 hi + lo pair (shared memory)
 //   warps 8, 9  O warps (TMEM lanes 0-63): the chunk's output rows, bf16, stored by TMA
 //               (off the chain's critical path)
+// The state and U warps signal the issuer warp by warp (mbarrier counts of 4), with no CTA
+// barrier on the step's path.
 // Per chunk c the issuer waits for M_c and U_c and issues
 //   D[c % 2] = A1 M_c (8 MMAs; 16 with the state as a hi + lo pair) once M_c is ready, then,
 //   once U_c is, dM = K^T [gamma' U_c hi | lo] (4 MMAs of N = 128), commit S;
@@ -923,11 +956,12 @@ constexpr uint32_t C_GUH = C_UTL + 8192;        // gamma' U, high bf16 parts
 constexpr uint32_t C_GUL = C_GUH + 8192;        // low parts
 constexpr size_t CHAIN_SMEM = C_GUL + 8192 + 1024;
 static_assert(C_MT % 1024 == 0, "swizzled tiles are 1024-byte aligned");
-constexpr int kChainThreads = 320;
+constexpr int kChainThreads = 384;
 static_assert(CHAIN_SMEM <= 232448, "chain shared memory");
 
 struct ChainCtl {
-  uint64_t full[2], empty[2];
+  uint64_t full[2], empty[2];   // the stage's epilogue operands: landed / read
+  uint64_t full_m[2], empty_m[2];   // its MMA operands: landed / read (the issuer's commit)
   uint64_t bar_s, bar_d, bar_m, bar_u, drain;
   uint64_t bar_dO[2];   // D[b] holds a finished chunk output (for the O warps)
   uint64_t bar_o[2];    // the O warps have read D[b]
@@ -963,7 +997,7 @@ __device__ bool wait_slot(const ScanWs &ws, int64_t slot, unsigned long long epo
   return true;
 }
 
-// The chain of CTA `cta` (320 threads); with `wait_flags` each stage's slots are awaited
+// The chain of CTA `cta` (384 threads); with `wait_flags` each stage's slots are awaited
 // first (their prep runs in the same launch).
 __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch &p,
                                            const ScanWs &ws, const ScanPlan &plan, int cta,
@@ -989,12 +1023,14 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
     if (want_o) tma_prefetch_desc(&tm_o);
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&ctl->full[s]), 1);
-      mbar_init(smem_u32(&ctl->empty[s]), 2);   // the state warps and the output warps
+      mbar_init(smem_u32(&ctl->empty[s]), 8);   // each state warp and each U warp
+      mbar_init(smem_u32(&ctl->full_m[s]), 1);
+      mbar_init(smem_u32(&ctl->empty_m[s]), 1);
     }
     mbar_init(smem_u32(&ctl->bar_s), 1);
     mbar_init(smem_u32(&ctl->bar_d), 1);
-    mbar_init(smem_u32(&ctl->bar_m), 1);
-    mbar_init(smem_u32(&ctl->bar_u), 1);
+    mbar_init(smem_u32(&ctl->bar_m), 4);        // each state warp
+    mbar_init(smem_u32(&ctl->bar_u), 4);        // each U warp
     mbar_init(smem_u32(&ctl->drain), 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&ctl->bar_dO[b]), 1);
@@ -1018,44 +1054,58 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
 
   const int seq = plan_order(plan, ws)[pos];
   const int cb = plan_cu_chunks(plan, ws)[seq];
-  const int t_begin = p.cu_seqlens[seq], t_end = p.cu_seqlens[seq + 1];
+  const int32_t *cu_tokens = plan_cu_tokens(plan, p);
+  const int t_begin = cu_tokens[seq], t_end = cu_tokens[seq + 1];
   const int n = (t_end - t_begin + C - 1) / C;
   auto slot_of = [&](int c) -> int64_t { return ((int64_t)cb + c) * H + head; };
   const bool s0 = p.S0 != nullptr;
   const uint32_t mt_u = smem_u32(sm + C_MT), utl_u = smem_u32(sm + C_UTL);
-  int last_k[2] = {-1, -1};   // producer: the last stage loaded into each buffer
+  int last_k[2] = {-1, -1};   // producer: the last stage whose epilogue part was loaded
+  int last_m[2] = {-1, -1};   // ... and whose MMA part was
   bool mma_pending = false;   // issuer: products issued whose completion was not seen
 
   if (warp == 0) {
     // ------------------------------------------------------------- producer
+    // A stage is refilled in two parts: the MMA operands (gamma Q, P, K~, -gamma_C W, -Y)
+    // as soon as the issuer's products of its last use have completed, the epilogue
+    // operands (gamma_C, the U~ slice, gamma') once the state and U warps have read them.
+    // The first part's loads thus run under the last use's epilogues.
     if (lane == 0) {
       for (int k = 0; k <= n; ++k) {
         const int st = k & 1;
-        if (k >= 2 && !mbar_wait(smem_u32(&ctl->empty[st]), (uint32_t)((k - 2) >> 1) & 1u, ab)) break;
         const bool cur = k >= 1, nxt = k <= n - 1;
-        const uint32_t bytes = (cur ? (want_o ? 16384u + 8192u : 0u) + 16384u + 16u : 0u) +
-                               (nxt ? 16384u + (k >= 1 ? 8192u : 0u) + 16384u + 256u : 0u);
+        const uint32_t bytes_m = (cur ? (want_o ? 16384u + 8192u : 0u) + 16384u : 0u) +
+                                 (nxt ? 16384u + (k >= 1 ? 8192u : 0u) : 0u);
+        const uint32_t bytes_e = (cur ? 16u : 0u) + (nxt ? 16384u + 256u : 0u);
         const int64_t sc = cur ? slot_of(k - 1) : 0, sn = nxt ? slot_of(k) : 0;
+        const uint32_t par = (uint32_t)((k - 2) >> 1) & 1u;
+        if (k >= 2 && !mbar_wait(smem_u32(&ctl->empty_m[st]), par, ab)) break;
         if (wait_flags && ((cur && !wait_slot(ws, sc, p.epoch, ab)) ||
                            (nxt && !wait_slot(ws, sn, p.epoch, ab))))
           break;
-        const uint32_t bar = smem_u32(&ctl->full[st]);
+        const uint32_t bar_mm = smem_u32(&ctl->full_m[st]), bar = smem_u32(&ctl->full[st]);
         const uint32_t base = smem_u32(sm + st * C_STAGE);
-        mbar_arrive_expect_tx(bar, bytes);
+        mbar_arrive_expect_tx(bar_mm, bytes_m);
         if (cur) {
           if (want_o) {
-            tma_load_2d(base + C_A1, &tm_QW, 0, (int32_t)(sc * 128), bar);
-            tma_load_2d(base + C_A1 + 16384, &tm_QW, 64, (int32_t)(sc * 128), bar);
-            tma_load_2d(base + C_A2, &tm_PY, 0, (int32_t)(sc * 128), bar);
+            tma_load_2d(base + C_A1, &tm_QW, 0, (int32_t)(sc * 128), bar_mm);
+            tma_load_2d(base + C_A1 + 16384, &tm_QW, 64, (int32_t)(sc * 128), bar_mm);
+            tma_load_2d(base + C_A2, &tm_PY, 0, (int32_t)(sc * 128), bar_mm);
           }
-          tma_load_2d(base + C_KT, &tm_KT, 0, (int32_t)(sc * 64), bar);
-          tma_load_2d(base + C_KT + 8192, &tm_KT, 64, (int32_t)(sc * 64), bar);
-          bulk_load(base + C_G, ws.G + sc * 4, 16u, bar);
+          tma_load_2d(base + C_KT, &tm_KT, 0, (int32_t)(sc * 64), bar_mm);
+          tma_load_2d(base + C_KT + 8192, &tm_KT, 64, (int32_t)(sc * 64), bar_mm);
         }
         if (nxt) {
-          tma_load_2d(base + C_A1 + 8192, &tm_QW, 0, (int32_t)(sn * 128 + 64), bar);
-          tma_load_2d(base + C_A1 + 16384 + 8192, &tm_QW, 64, (int32_t)(sn * 128 + 64), bar);
-          if (k >= 1) tma_load_2d(base + C_A2 + 8192, &tm_PY, 0, (int32_t)(sn * 128 + 64), bar);
+          tma_load_2d(base + C_A1 + 8192, &tm_QW, 0, (int32_t)(sn * 128 + 64), bar_mm);
+          tma_load_2d(base + C_A1 + 16384 + 8192, &tm_QW, 64, (int32_t)(sn * 128 + 64), bar_mm);
+          if (k >= 1)
+            tma_load_2d(base + C_A2 + 8192, &tm_PY, 0, (int32_t)(sn * 128 + 64), bar_mm);
+        }
+        last_m[st] = k;
+        if (k >= 2 && !mbar_wait(smem_u32(&ctl->empty[st]), par, ab)) break;
+        mbar_arrive_expect_tx(bar, bytes_e);
+        if (cur) bulk_load(base + C_G, ws.G + sc * 4, 16u, bar);
+        if (nxt) {
           tma_load_2d(base + C_UT, &tm_UT, slice * DVS, (int32_t)(sn * 64), bar);
           tma_load_2d(base + C_UT + 8192, &tm_UT, slice * DVS + 32, (int32_t)(sn * 64), bar);
           bulk_load(base + C_GP, ws.GP + sn * C, 256u, bar);
@@ -1073,7 +1123,7 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
       const uint64_t gu = mnmaj(smem_u32(sm + C_GUH), 8192);   // [hi | lo] blocks, 8 KB apart
       const uint32_t id_s = idesc_bf16(128, 2 * DVS, 1, 1);
       const uint32_t id_mn = idesc_bf16(128, DVS, 0, 1);
-      bool ok = mbar_wait(smem_u32(&ctl->full[0]), 0, ab);
+      bool ok = mbar_wait(smem_u32(&ctl->full_m[0]), 0, ab);
       if (ok && s0) {
         // U_0 = U~_0 - W_0 M_0: D[1] rows 64-127 = -W_0 M_0
         ok = mbar_wait(smem_u32(&ctl->bar_m), 0, ab);
@@ -1092,6 +1142,13 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
           mma_pending = true;
         }
       }
+      // stage 0's MMA operands (read by the products above, if any) may be refilled
+      if (ok) {
+        if (s0)
+          tc_commit(smem_u32(&ctl->empty_m[0]));
+        else
+          mbar_arrive(smem_u32(&ctl->empty_m[0]));
+      }
       for (int j = 0; ok && j < n; ++j) {
         const int k = j + 1, st = k & 1;
         const uint32_t base = smem_u32(sm + st * C_STAGE);
@@ -1100,7 +1157,7 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
         const uint64_t kt = mnmaj(base + C_KT, 8192);
         // D = A1 M_j as soon as M_j is ready (it does not need U_j), once the O warps have
         // read D[j % 2]'s previous chunk
-        if (!mbar_wait(smem_u32(&ctl->full[st]), (uint32_t)(k >> 1) & 1u, ab)) break;
+        if (!mbar_wait(smem_u32(&ctl->full_m[st]), (uint32_t)(k >> 1) & 1u, ab)) break;
         if (!mbar_wait(smem_u32(&ctl->bar_m), (uint32_t)j & 1u, ab)) break;
         if (want_o && j >= 2 &&
             !mbar_wait(smem_u32(&ctl->bar_o[j & 1]), (uint32_t)((j >> 1) - 1) & 1u, ab))
@@ -1127,6 +1184,7 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
         for (int kk = 0; kk < C / 16; ++kk)
           tc_mma_bf16(dcol, desc_k(a2, kk, 0), desc_mn(ud, kk), id_mn, 1u);
         tc_commit(bar_d);
+        tc_commit(smem_u32(&ctl->empty_m[st]));
         if (want_o) tc_commit(smem_u32(&ctl->bar_dO[j & 1]));
       }
       // the last step's products complete before the final barrier either way: the state
@@ -1159,25 +1217,26 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
         store_row_bf16(sm + C_MT, d, 32, M + 32, 1.f);
       }
     };
+    // each warp signals on its own (no CTA barrier on the step's path); a warp that gives
+    // up a wait leaves, and the abort flag ends every other role's next wait
     if (n > 0) {
       store_state();
       fence_proxy_async_smem();
-      bar_sync_n(2, 128);
+      __syncwarp();
       // (the test hook withholds this signal: every role's bounded wait then runs out)
-      if (warp == 2 && lane == 0 && !(p.flags & TR_SCAN_STALL_TEST))
-        mbar_arrive(smem_u32(&ctl->bar_m));
+      if (lane == 0 && !(p.flags & TR_SCAN_STALL_TEST)) mbar_arrive(smem_u32(&ctl->bar_m));
     }
     for (int j = 0; j < n; ++j) {
       const int k = j + 1, st = k & 1;
-      const bool got = mbar_wait(smem_u32(&ctl->bar_s), (uint32_t)j & 1u, ab) &&
-                       mbar_wait(smem_u32(&ctl->full[st]), (uint32_t)(k >> 1) & 1u, ab);
-      // all four state warps leave together (the named barrier below counts them)
-      if (bar_or_n(2, 128, !got)) {
+      // gamma_C first (it lands long before the product)
+      bool got = mbar_wait(smem_u32(&ctl->full[st]), (uint32_t)(k >> 1) & 1u, ab);
+      const float gC = got ? *reinterpret_cast<const float *>(sm + st * C_STAGE + C_G) : 0.f;
+      got = got && mbar_wait(smem_u32(&ctl->bar_s), (uint32_t)j & 1u, ab);
+      if (!__all_sync(0xffffffffu, got)) {
         failed = true;
         break;
       }
       tc_fence_after();
-      const float gC = *reinterpret_cast<const float *>(sm + st * C_STAGE + C_G);
       float v0[32], v1[32];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -1192,8 +1251,8 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
         fence_proxy_async_smem();
       }
       tc_fence_before();
-      bar_sync_n(2, 128);
-      if (warp == 2 && lane == 0) {
+      __syncwarp();
+      if (lane == 0) {
         if (j + 1 < n) mbar_arrive(smem_u32(&ctl->bar_m));
         mbar_arrive(smem_u32(&ctl->empty[st]));   // gamma_C read
       }
@@ -1204,11 +1263,12 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
       for (int j = 0; j < DVS; j += 4)
         *reinterpret_cast<float4 *>(dst + j) = make_float4(M[j], M[j + 1], M[j + 2], M[j + 3]);
     }
-  } else if (warp < 8) {
+  } else if (warp < 8 || warp >= 10) {
     // ------------------------------------------------------------- U warps
-    // warps 6, 7 (TMEM lanes 64-127): U_{c+1} = U~_{c+1} + D rows 64-127, written as bf16
-    // (for A2 U) and gamma' U as a bf16 hi + lo pair (for dM); then U is announced
-    const int q = warp & 3, t = 32 * (q - 2) + lane;
+    // warps 6, 7 (columns 0-31) and 10, 11 (columns 32-63), TMEM lanes 64-127:
+    // U_{c+1} = U~_{c+1} + D rows 64-127, written as bf16 (for A2 U) and gamma' U as a bf16
+    // hi + lo pair (for dM); each warp then announces its part
+    const int q = warp & 3, t = 32 * (q - 2) + lane, ch = warp >= 10 ? 1 : 0;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     uint32_t d_phase = 0;
     if (n > 0) {
@@ -1217,60 +1277,52 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
         ok = mbar_wait(smem_u32(&ctl->bar_d), d_phase, ab);
         d_phase ^= 1u;
       }
-      if (!bar_or_n(3, 64, !ok)) {
+      if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
         const float gp = reinterpret_cast<const float *>(sm + C_GP)[t];
-        float u0[32], u1[32], v0[32], v1[32];
-        if (s0) {
-          tmem_ld32(tmem + 64 + lane_base, v0);
-          tmem_ld32(tmem + 64 + lane_base + 32, v1);
-        }
-        load_row32_f32(sm + C_UT, t, u0);
-        load_row32_f32(sm + C_UT + 8192, t, u1);
+        float u[32], v[32];
+        if (s0) tmem_ld32(tmem + 64 + lane_base + 32 * ch, v);
+        load_row32_f32(sm + C_UT + 8192 * ch, t, u);
         if (s0) {
           tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) { u0[i] += v0[i]; u1[i] += v1[i]; }
+          for (int i = 0; i < 32; ++i) u[i] += v[i];
         }
-        store_row_bf16(sm + C_UTL, t, 0, u0, 1.f);
-        store_row_bf16(sm + C_UTL, t, 32, u1, 1.f);
-        store_row_split(sm + C_GUH, sm + C_GUL, t, 0, u0, gp);
-        store_row_split(sm + C_GUH, sm + C_GUL, t, 32, u1, gp);
+        store_row_bf16(sm + C_UTL, t, 32 * ch, u, 1.f);
+        store_row_split(sm + C_GUH, sm + C_GUL, t, 32 * ch, u, gp);
         fence_proxy_async_smem();
         tc_fence_before();
-        bar_sync_n(3, 64);
-        if (warp == 6 && lane == 0) {
+        __syncwarp();
+        if (lane == 0) {
           mbar_arrive(smem_u32(&ctl->bar_u));
           mbar_arrive(smem_u32(&ctl->empty[0]));
           mbar_arrive(smem_u32(&ctl->empty[0]));   // stage 0 holds no gamma_C
         }
         for (int j = 0; j < n; ++j) {
           const int k = j + 1, st = k & 1;
-          const bool got = mbar_wait(smem_u32(&ctl->bar_d), d_phase, ab) &&
-                           mbar_wait(smem_u32(&ctl->full[st]), (uint32_t)(k >> 1) & 1u, ab);
-          if (bar_or_n(3, 64, !got)) break;
+          // the stage's U~ row and gamma' first (they land long before the products)
+          bool got = mbar_wait(smem_u32(&ctl->full[st]), (uint32_t)(k >> 1) & 1u, ab);
+          float gq = 0.f;
+          if (got && j + 1 < n) {
+            gq = reinterpret_cast<const float *>(sm + st * C_STAGE + C_GP)[t];
+            load_row32_f32(sm + st * C_STAGE + C_UT + 8192 * ch, t, u);
+          }
+          got = got && mbar_wait(smem_u32(&ctl->bar_d), d_phase, ab);
+          if (!__all_sync(0xffffffffu, got)) break;
           d_phase ^= 1u;
           tc_fence_after();
           if (j + 1 < n) {
-            const uint32_t dcol = tmem + 64 * (j & 1) + lane_base;
-            const uint8_t *ut = sm + st * C_STAGE + C_UT;
-            const float gq = reinterpret_cast<const float *>(sm + st * C_STAGE + C_GP)[t];
-            tmem_ld32(dcol, v0);
-            tmem_ld32(dcol + 32, v1);
-            load_row32_f32(ut, t, u0);
-            load_row32_f32(ut + 8192, t, u1);
+            tmem_ld32(tmem + 64 * (j & 1) + lane_base + 32 * ch, v);
             tc_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) { u0[i] += v0[i]; u1[i] += v1[i]; }
-            store_row_bf16(sm + C_UTL, t, 0, u0, 1.f);
-            store_row_bf16(sm + C_UTL, t, 32, u1, 1.f);
-            store_row_split(sm + C_GUH, sm + C_GUL, t, 0, u0, gq);
-            store_row_split(sm + C_GUH, sm + C_GUL, t, 32, u1, gq);
+            for (int i = 0; i < 32; ++i) u[i] += v[i];
+            store_row_bf16(sm + C_UTL, t, 32 * ch, u, 1.f);
+            store_row_split(sm + C_GUH, sm + C_GUL, t, 32 * ch, u, gq);
             fence_proxy_async_smem();
           }
           tc_fence_before();
-          bar_sync_n(3, 64);
-          if (warp == 6 && lane == 0) {
+          __syncwarp();
+          if (lane == 0) {
             if (j + 1 < n) mbar_arrive(smem_u32(&ctl->bar_u));
             mbar_arrive(smem_u32(&ctl->empty[st]));
           }
@@ -1337,8 +1389,10 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
   __syncwarp();
   const bool aborted = *ab.flag != 0;
   if (warp == 0 && lane == 0 && aborted)
-    for (int b = 0; b < 2; ++b)
+    for (int b = 0; b < 2; ++b) {
+      if (last_m[b] >= 0) mbar_wait_drain(smem_u32(&ctl->full_m[b]), (uint32_t)(last_m[b] >> 1) & 1u);
       if (last_k[b] >= 0) mbar_wait_drain(smem_u32(&ctl->full[b]), (uint32_t)(last_k[b] >> 1) & 1u);
+    }
   if (warp == 1 && lane == 0 && aborted && mma_pending) {
     tc_commit(smem_u32(&ctl->drain));
     mbar_wait_drain(smem_u32(&ctl->drain), 0);
@@ -1383,10 +1437,12 @@ bool host_plan(const ScanLaunch &p, ScanPlan *pl) {
   int nch[kParamSeqs];
   for (int i = 0; i < p.n_seqs; ++i) {
     pl->cu_chunks[i] = acc;
+    pl->cu_tokens[i] = p.cu_seqlens_host[i];
     nch[i] = (p.cu_seqlens_host[i + 1] - p.cu_seqlens_host[i] + C - 1) / C;
     acc += nch[i];
   }
   pl->cu_chunks[p.n_seqs] = acc;
+  pl->cu_tokens[p.n_seqs] = p.cu_seqlens_host[p.n_seqs];
   std::iota(pl->order, pl->order + p.n_seqs, 0);
   std::stable_sort(pl->order, pl->order + p.n_seqs,
                    [&](int a, int b) { return nch[a] > nch[b]; });
