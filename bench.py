@@ -947,7 +947,8 @@ def our_arm(args):
                      "state_updates_per_s": upd / scan_t, "us": scan_t * 1e6,
                      "roofline": {"bound": "hbm", "achieved": scan_gbs, "peak": peaks["hbm_gbs"],
                                   "unit": "GB/s", "frac": scan_gbs / peaks["hbm_gbs"],
-                                  "traffic": None, "alg_bytes": scan_bytes}},
+                                  "traffic": traffic.get("scan_cell"),
+                                  "alg_bytes": scan_bytes}},
             "transfer_overlap": {
                 "workload": "group replay with the FA KV (33.5 MB, pinned host) copied on its own "
                             "stream", "kv_bytes": int(kv_host.numel()), "kv_copy_us": t_kv * 1e3,
