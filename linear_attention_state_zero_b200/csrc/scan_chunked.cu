@@ -969,20 +969,24 @@ struct ChainCtl {
   int abort;
 };
 
-// Wait until the prep running beside this chain (fused launch) has published `slot`: an
-// acquire load of its flag, bounded like every other wait; then order the flag before this
-// thread's TMA loads of the slot's data.
-__device__ bool wait_slot(const ScanWs &ws, int64_t slot, unsigned long long epoch,
-                          const AbortFlag &ab) {
-  const unsigned long long *f = ws.flags + slot;
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
-  if (v != epoch) {
+// Wait until the prep running beside this chain (fused launch) has published the slots a
+// stage reads (`n` of them, 1 or 2): acquire loads of their flags, repeated (bounded like
+// every other wait) until both carry this call's epoch, then a proxy fence that orders them
+// before this thread's TMA loads of the slots' data.  (A generic fence instead of acquire
+// loads made the chain slower: it waited for this thread's bulk copies in flight.)
+__device__ bool wait_slots(const ScanWs &ws, const int64_t (&slot)[2], int n,
+                           unsigned long long epoch, const AbortFlag &ab) {
+  auto ready = [&]() {
+    unsigned long long v[2] = {epoch, epoch};
+    for (int i = 0; i < n; ++i)
+      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v[i]) : "l"(ws.flags + slot[i]) : "memory");
+    return v[0] == epoch && v[1] == epoch;
+  };
+  if (!ready()) {
     const unsigned long long t0 = globaltimer_ns();
     for (int i = 0;; ++i) {
       __nanosleep(64);
-      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
-      if (v == epoch) break;
+      if (ready()) break;
       if ((i & 15) == 15) {
         if (*ab.flag) return false;
         if (globaltimer_ns() - t0 > ab.limit_ns) {
@@ -1079,10 +1083,12 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
         const uint32_t bytes_e = (cur ? 16u : 0u) + (nxt ? 16384u + 256u : 0u);
         const int64_t sc = cur ? slot_of(k - 1) : 0, sn = nxt ? slot_of(k) : 0;
         const uint32_t par = (uint32_t)((k - 2) >> 1) & 1u;
+        // the slots' flags first: their check runs while the stage is still in use
+        if (wait_flags && (cur || nxt)) {
+          const int64_t sl[2] = {cur ? sc : sn, sn};
+          if (!wait_slots(ws, sl, (cur && nxt) ? 2 : 1, p.epoch, ab)) break;
+        }
         if (k >= 2 && !mbar_wait(smem_u32(&ctl->empty_m[st]), par, ab)) break;
-        if (wait_flags && ((cur && !wait_slot(ws, sc, p.epoch, ab)) ||
-                           (nxt && !wait_slot(ws, sn, p.epoch, ab))))
-          break;
         const uint32_t bar_mm = smem_u32(&ctl->full_m[st]), bar = smem_u32(&ctl->full[st]);
         const uint32_t base = smem_u32(sm + st * C_STAGE);
         mbar_arrive_expect_tx(bar_mm, bytes_m);
