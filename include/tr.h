@@ -276,7 +276,10 @@ tr_status tr_replay_group(const tr_group_args *args, void *ws, size_t ws_bytes, 
  */
 int32_t tr_replay_group_kernel_count(const tr_group_args *args);
 /* The names of those kernels, comma-separated, in launch order (a thread-local string,
- * valid until the next call from the same thread; "" for invalid args).  Host-only. */
+ * valid until the next call from the same thread; "" for invalid args).  Host-only.
+ * They describe an uncaptured call: a call made while its stream captures a graph runs
+ * the scan as separate prep and chain kernels (the single-launch form synchronises its
+ * parts through per-call tags, which a replayed graph would repeat). */
 const char *tr_replay_group_kernel_names(const tr_group_args *args);
 tr_status tr_replay_group_profiled(const tr_group_args *args, void *ws, size_t ws_bytes,
                                    void *stream, void *const *events, int32_t n_events);

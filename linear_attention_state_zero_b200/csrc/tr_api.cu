@@ -303,7 +303,7 @@ tr_status run_scan(const tr::ScanLaunch &p, cudaStream_t s,
 
 // ------------------------------------------------------------- replay group
 struct GroupLayout {
-  size_t x, xhat, qkv, post, zbuf, la, beta, o, hmid, scan, total;
+  size_t x, xhat, qkv, post, zbuf, la, beta, o, hmid, scan, tflags, total;
   int64_t ldq;
 };
 
@@ -348,6 +348,10 @@ GroupLayout group_layout(const tr_group_args *a) {
   L.o = off;    off = align256(off + T * H * (size_t)a->d_v * 2);
   L.hmid = off; off = align256(off + T * (size_t)(a->d_ff > 0 ? a->d_ff : 0) * 2);
   L.scan = off; off = align256(off + scan_ws_bytes(group_scan_launch(a)));
+  // the input projection's tile flags (the scan of the layer waits on them)
+  const size_t row_tiles = (T + tr::kGemmTileRows - 1) / tr::kGemmTileRows;
+  const size_t col_tiles = ((size_t)in_rows(a) + tr::kInProjTileCols - 1) / tr::kInProjTileCols;
+  L.tflags = off; off = align256(off + row_tiles * col_tiles * 8);
   L.total = off;
   return L;
 }
@@ -485,6 +489,15 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
   const float rms_eps = a->rms_eps > 0.f ? a->rms_eps : 1e-6f;
   const float norm_eps = a->norm_eps > 0.f ? a->norm_eps : 1e-6f;
   const size_t state_elems = (size_t)a->n_seqs * H * dk * dv;
+  // The scan of a layer starts while its input projection runs and waits, item by item, for
+  // the projection tiles it reads (per-tile flags tagged per launch).  Not beside the short
+  // convolution (the scan reads its output) nor under stream capture (a replayed graph would
+  // repeat the tags).
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  const bool capturing = cudaStreamIsCapturing(s, &cs) == cudaSuccess &&
+                         cs != cudaStreamCaptureStatusNone;
+  auto *tflags = reinterpret_cast<unsigned long long *>(base + L.tflags);
+  static std::atomic<unsigned long long> in_epoch_counter{0};
   std::string err;
   cudaError_t e;
   for (int l = 0; l < a->n_layers; ++l) {
@@ -512,6 +525,10 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
     ep.z = output_gate(a) ? zbuf : nullptr;
     ep.A_log = w.A_log;
     ep.dt_bias = w.dt_bias;
+    const bool by_rows = !conv && !capturing && pdl;
+    const unsigned long long in_epoch = by_rows ? ++in_epoch_counter : 0;
+    ep.tile_flags = by_rows ? tflags : nullptr;
+    ep.flag_epoch = in_epoch;
     const void *Wb = static_cast<const __nv_bfloat16 *>(w.W_in) + (size_t)ep.col_offset * D;
     e = tr::launch_gemm_inproj(xhat, Wb, T, n_in - ep.col_offset, D, ep, err_word, s, pdl, &err);
     if (e != cudaSuccess)
@@ -557,6 +574,9 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
     sp.S_final = a->S_hat + (size_t)l * state_elems;
     sp.err_word = err_word;
     sp.pdl = pdl;
+    sp.in_flags = by_rows ? tflags : nullptr;
+    sp.in_epoch = in_epoch;
+    sp.in_tiles_n = (n_in - ep.col_offset + tr::kInProjTileCols - 1) / tr::kInProjTileCols;
     tr_status st = run_scan(sp, s, [&]() { return mk->mark(s); });
     if (st != TR_OK) return st;
     if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");

@@ -148,3 +148,33 @@ def test_many_sequences(cuda_device, n_seqs, max_len, H):
     assert rel_fro(S, wS) < TOL_BF16
     empty = [i for i, n in enumerate(lens) if n == 0]
     assert empty and not S[empty].any()
+
+
+def test_scan_replayed_from_a_captured_graph(cuda_device):
+    """A scan captured into a CUDA graph recomputes on every replay: the inputs are changed in
+    place between replays and each replay's outputs match the oracle on the new inputs (a
+    single-launch scan synchronising through per-call tags would see the last replay's tags
+    and read stale intermediates)."""
+    lengths = [700]
+    case = synth.scan_case(lengths, 16, 128, 128, torch.bfloat16, 0.97, 1.00, seed=611)
+    g = lambda t: t.to(cuda_device)
+    q, k, v, la, be = (g(case.q), g(case.k), g(case.v), g(case.log_alpha), g(case.beta))
+    cu = tr.seqlens(case.cu_seqlens, cuda_device)
+    o = torch.empty_like(v)
+    S = torch.empty(1, 16, 128, 128, dtype=torch.float32, device=cuda_device)
+    tr.gdn_scan(q, k, v, la, be, cu, o=o, S_final=S)   # uncaptured first call on the device
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        tr.gdn_scan(q, k, v, la, be, cu, o=o, S_final=S)
+    for trial in range(3):
+        new = synth.scan_case(lengths, 16, 128, 128, torch.bfloat16, 0.97, 1.00, seed=612 + trial)
+        v.copy_(g(new.v))
+        la.copy_(g(new.log_alpha))
+        graph.replay()
+        torch.cuda.synchronize()
+        wo, wS = oracle.gdn_scan(case.q, case.k, new.v, new.log_alpha, case.beta,
+                                 case.cu_seqlens)
+        assert rel_fro(S, wS) < TOL_BF16
+        assert rel_fro(o, wo) < TOL_BF16
+    tr.check()
