@@ -52,7 +52,6 @@ struct Ctl {
   uint64_t tempty[2];
   uint32_t tmem_base;
   int abort;
-  int tile_done[2];   // epilogue warps done with the tile in TMEM buffer b (tile flags)
 };
 
 __device__ __forceinline__ void store_bf16x32(__nv_bfloat16 *dst, const float (&v)[32], float s) {
@@ -241,18 +240,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m_tiles = (M + BM - 1) / BM;
   const int n_tiles = (N + BN - 1) / BN;
-  // tile t -> (row tile, column tile): column-major by default (concurrent tiles share B);
-  // row-major when the input projection publishes tile flags, so rows complete in order
-  const bool row_major = EPI == EPI_INPROJ && ip.tile_flags != nullptr;
-  auto tile_rc = [&](int t, int &tm, int &tn) {
-    if (row_major) {
-      tm = t / n_tiles;
-      tn = t % n_tiles;
-    } else {
-      tm = t % m_tiles;
-      tn = t / m_tiles;
-    }
-  };
   const int n_total = m_tiles * n_tiles;
   const int kblocks = (K + BK - 1) / BK;
 
@@ -264,7 +251,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&ctl->tfull[b]), 1);
       mbar_init(smem_u32(&ctl->tempty[b]), kEpiWarps);
-      ctl->tile_done[b] = 0;
     }
     ctl->abort = 0;
     fence_mbar_init();
@@ -293,8 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t ph = 0;
       for (int t = blockIdx.x; t < n_total; t += gridDim.x) {
-        int tm, tn;
-        tile_rc(t, tm, tn);
+        const int tm = t % m_tiles, tn = t / m_tiles;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(smem_u32(&ctl->empty[stage]), ph ^ 1u, ab)) goto producer_done;
           const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
@@ -358,8 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t u = (uint32_t)(it >> 1);
       if (!mbar_wait(smem_u32(&ctl->tfull[b]), u & 1u, ab)) break;
       tc_fence_after();
-      int tm, tn;
-      tile_rc(t, tm, tn);
+      const int tm = t % m_tiles, tn = t / m_tiles;
       const int row = tm * BM + q4 * 32 + lane;
       const uint32_t tbase = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(b * BN);
       if (EPI == EPI_INPROJ)
@@ -368,18 +352,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         epi_swiglu(sw, tbase, tn * (BN / 2), row, M, half);
       else
         epi_resid<BN>(rs, tbase, tn * BN, N, row, M, lo, hi);
-      if (EPI == EPI_INPROJ && ip.tile_flags) {
-        // the last of the tile's epilogue warps to finish publishes its flag: each warp
-        // fences its stores before counting itself, the last fences again and releases
-        __threadfence();
-        __syncwarp();
-        if (lane == 0 && atomicAdd(&ctl->tile_done[b], 1) == kEpiWarps - 1) {
-          ctl->tile_done[b] = 0;
-          __threadfence();
-          asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(ip.tile_flags + t),
-                       "l"(ip.flag_epoch) : "memory");
-        }
-      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&ctl->tempty[b]));
@@ -434,9 +406,7 @@ cudaError_t launch_gemm_inproj(const void *A, const void *B, int M, int N, int K
                                bool pdl, std::string *err) {
   ResidEpi none{};
   SwigluEpi no_sw{};
-  static_assert(BM == kGemmTileRows, "the scan's row tiles are the GEMM's");
-  return launch<kInProjTileCols, EPI_INPROJ>(A, K, B, nullptr, M, N, K, ep, none, no_sw, err_word,
-                                             s, pdl, err);
+  return launch<256, EPI_INPROJ>(A, K, B, nullptr, M, N, K, ep, none, no_sw, err_word, s, pdl, err);
 }
 
 cudaError_t launch_gemm_resid(const void *A, int64_t lda, const void *B, int M, int N, int K,

@@ -398,44 +398,6 @@ struct ScanMaps {
   CUtensorMap q, k, v, QW, PY, KT, UT, o;
 };
 
-// Wait (every lane of the calling warp) until the input projection has written the tiles
-// of tokens [t_lo, t_hi): every column tile of their row tiles (kGemmTileRows tokens each)
-// carries this call's tag.  Relaxed loads, all lanes at once, repeated with a bounded wait; then an acquire
-// fence.  Returns false when the wait gave up (the abort flag and error word are set).
-__device__ bool wait_rows(const ScanLaunch &p, int t_lo, int t_hi, const AbortFlag &ab) {
-  const int lane = threadIdx.x & 31;
-  const int r0 = t_lo / kGemmTileRows, r1 = (t_hi - 1) / kGemmTileRows;
-  const int n = (r1 - r0 + 1) * p.in_tiles_n;
-  const unsigned long long t0 = globaltimer_ns();
-  for (int i = 0;; ++i) {
-    bool ready = true;
-    for (int q = lane; q < n; q += 32) {
-      const unsigned long long *f =
-          p.in_flags + (size_t)(r0 + q / p.in_tiles_n) * p.in_tiles_n + q % p.in_tiles_n;
-      unsigned long long v;
-      asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
-      ready = ready && v == p.in_epoch;
-    }
-    if (__all_sync(0xffffffffu, ready)) break;
-    __nanosleep(64);
-    if ((i & 15) == 15) {
-      int quit = 0;
-      if (lane == 0) {
-        if (*ab.flag) {
-          quit = 1;
-        } else if (globaltimer_ns() - t0 > ab.limit_ns) {
-          *ab.flag = 1;
-          if (ab.err_word) atomicOr(ab.err_word, ab.err_bit);
-          quit = 1;
-        }
-      }
-      if (__shfl_sync(0xffffffffu, quit, 0)) return false;
-    }
-  }
-  asm volatile("fence.acq_rel.gpu;" ::: "memory");
-  return true;
-}
-
 // Publish item `slot` as complete for the chain running beside the prep (fused launch):
 // its output stores have completed; the release store orders them before the flag.
 __device__ __forceinline__ void publish_slot(const ScanWs &ws, int64_t slot, unsigned long long epoch) {
@@ -494,15 +456,9 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
   tc_fence_after();
   const uint32_t tmem = ctl->tmem;
   const AbortFlag ab{&ctl->abort, p.err_word, ERRBIT_SCAN_TIMEOUT, p.wait_ns};
-  // TMEM is held: let the next kernel launch; then wait for the previous one's outputs --
-  // with the projection's tile flags (and the plan in the parameters) only item by item
-  const bool by_rows = p.in_flags != nullptr && plan.in_params;
+  // TMEM is held: let the next kernel launch; then wait for the previous one's outputs
   pdl_trigger();
-  if (!by_rows) pdl_wait();
-  // rows of an item's inputs: its chunk and, for the look-ahead terms, the previous one
-  auto item_rows = [&](const PrepItem &it) {
-    return wait_rows(p, it.t0 - (it.has_prev ? C : 0), it.t0 + (it.nv > 0 ? it.nv : 1), ab);
-  };
+  pdl_wait();
 
   int fills[2] = {0, 0};   // TMA fills issued per stage (thread 0)
   int64_t prev_slot = -1;  // thread 0: the last item whose flag is not yet published
@@ -546,17 +502,10 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
     seq_cur = seq_of_chunk((int)(item / p.H), p.n_seqs, cu_chunks);
     seq_cur = advance_seq(seq_cur, (int)(item / p.H), cu_chunks);
   }
-  if (warp == 0 && item < n_items) {
-    if (tid == 0) ctl->cur = item_at(item, seq_cur, p, cu_chunks, cu_tokens);
-    __syncwarp();
-    if (by_rows) {
-      item_rows(ctl->cur);
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-    }
-    if (tid == 0) {
-      fence_proxy_async_smem();
-      issue(ctl->cur, 0);
-    }
+  if (tid == 0 && item < n_items) {
+    ctl->cur = item_at(item, seq_cur, p, cu_chunks, cu_tokens);
+    fence_proxy_async_smem();
+    issue(ctl->cur, 0);
   }
   bar_sync_n(1, kPrepThreads);
   if (item < n_items) load_gates(ctl->cur, la_next, b_next);
@@ -642,15 +591,11 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
         // written below
         bulk_wait_read<2>();
       }
-    } else if (warp == 1 && has_next) {
+    } else if (tid == 32 && has_next) {
       // the next item's location, beside the products (its gates are loaded under the
-      // inverse, its bands after group 2 is issued), and its input rows' flags
-      if (lane == 0) {
-        seq_cur = advance_seq(seq_cur, (int)((item + stride) / p.H), cu_chunks);
-        ctl->nxt = item_at(item + stride, seq_cur, p, cu_chunks, cu_tokens);
-      }
-      __syncwarp();
-      if (by_rows) item_rows(ctl->nxt);
+      // inverse, its bands after group 2 is issued)
+      seq_cur = advance_seq(seq_cur, (int)((item + stride) / p.H), cu_chunks);
+      ctl->nxt = item_at(item + stride, seq_cur, p, cu_chunks, cu_tokens);
     }
     if (!mma_wait()) break;
 
@@ -866,8 +811,6 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
     } else if (tid == 0) {
       bulk_wait_read<0>();
       if (has_next) {
-        // (the rows' flags were acquired by warp 1 before the barriers since)
-        if (by_rows) asm volatile("fence.proxy.async.global;" ::: "memory");
         fence_proxy_async_smem();
         issue(ctl->nxt, buf ^ 1);
       }
@@ -1111,9 +1054,7 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
   const AbortFlag ab{&ctl->abort, p.err_word, ERRBIT_SCAN_TIMEOUT, p.wait_ns};
   // TMEM is held: let the next kernel launch; then wait for the previous one's outputs
   pdl_trigger();
-  // (beside a prep that waits for the projection's rows, a chain reads only what that prep
-  // published)
-  if (!(wait_flags && p.in_flags)) pdl_wait();
+  pdl_wait();
 
   const int seq = plan_order(plan, ws)[pos];
   const int cb = plan_cu_chunks(plan, ws)[seq];
@@ -1614,26 +1555,15 @@ cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string
     cfg.blockDim = dim3(kChainThreads);
     cfg.dynamicSmemBytes = FUSED_SMEM;
     cfg.stream = s;
-    // Cooperative (every CTA resident at once), except beside a running input projection
-    // (tile flags): then the launch starts on the SMs the projection frees and the rest
-    // follow as it ends.  Either way a chain only waits on prep CTAs that run or will: at
-    // most kFusedMaxChains CTAs are chains, so the other SMs of the grid take prep CTAs.
     cudaLaunchAttribute attr[2];
-    int na = 0;
-    if (!pf.in_flags) {
-      attr[na].id = cudaLaunchAttributeCooperative;
-      attr[na].val.cooperative = 1;
-      ++na;
-    }
-    if (pf.pdl) {
-      attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-      attr[na].val.programmaticStreamSerializationAllowed = 1;
-      ++na;
-    }
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = na;
+    cfg.numAttrs = pf.pdl ? 2 : 1;
     e = cudaLaunchKernelEx(&cfg, kern, mp, pf, ws, plan, (int)fused_chains(p));
-    if (e == cudaSuccess || !pf.pdl || pf.in_flags) return e;
+    if (e == cudaSuccess || !pf.pdl) return e;
     // a runtime that will not combine a cooperative launch with programmatic serialization:
     // the same launch without the latter
     (void)cudaGetLastError();

@@ -240,6 +240,7 @@ tr_status validate_scan(const tr_scan_args *a, tr::ScanLaunch *out) {
   if (!aligned16(a->S_final) || (a->S0 && !aligned16(a->S0)))
     return fail(TR_ERR_ALIGNMENT, "S0/S_final must be 16-byte aligned");
   tr::ScanLaunch &p = *out;
+  p = tr::ScanLaunch{};   // every field not set below is off
   p.n_seqs = a->n_seqs;
   p.H = a->n_heads;
   p.dk = a->d_k;
@@ -303,7 +304,7 @@ tr_status run_scan(const tr::ScanLaunch &p, cudaStream_t s,
 
 // ------------------------------------------------------------- replay group
 struct GroupLayout {
-  size_t x, xhat, qkv, post, zbuf, la, beta, o, hmid, scan, tflags, total;
+  size_t x, xhat, qkv, post, zbuf, la, beta, o, hmid, scan, total;
   int64_t ldq;
 };
 
@@ -348,10 +349,6 @@ GroupLayout group_layout(const tr_group_args *a) {
   L.o = off;    off = align256(off + T * H * (size_t)a->d_v * 2);
   L.hmid = off; off = align256(off + T * (size_t)(a->d_ff > 0 ? a->d_ff : 0) * 2);
   L.scan = off; off = align256(off + scan_ws_bytes(group_scan_launch(a)));
-  // the input projection's tile flags (the scan of the layer waits on them)
-  const size_t row_tiles = (T + tr::kGemmTileRows - 1) / tr::kGemmTileRows;
-  const size_t col_tiles = ((size_t)in_rows(a) + tr::kInProjTileCols - 1) / tr::kInProjTileCols;
-  L.tflags = off; off = align256(off + row_tiles * col_tiles * 8);
   L.total = off;
   return L;
 }
@@ -489,15 +486,6 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
   const float rms_eps = a->rms_eps > 0.f ? a->rms_eps : 1e-6f;
   const float norm_eps = a->norm_eps > 0.f ? a->norm_eps : 1e-6f;
   const size_t state_elems = (size_t)a->n_seqs * H * dk * dv;
-  // The scan of a layer starts while its input projection runs and waits, item by item, for
-  // the projection tiles it reads (per-tile flags tagged per launch).  Not beside the short
-  // convolution (the scan reads its output) nor under stream capture (a replayed graph would
-  // repeat the tags).
-  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-  const bool capturing = cudaStreamIsCapturing(s, &cs) == cudaSuccess &&
-                         cs != cudaStreamCaptureStatusNone;
-  auto *tflags = reinterpret_cast<unsigned long long *>(base + L.tflags);
-  static std::atomic<unsigned long long> in_epoch_counter{0};
   std::string err;
   cudaError_t e;
   for (int l = 0; l < a->n_layers; ++l) {
@@ -525,10 +513,6 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
     ep.z = output_gate(a) ? zbuf : nullptr;
     ep.A_log = w.A_log;
     ep.dt_bias = w.dt_bias;
-    const bool by_rows = !conv && !capturing && pdl;
-    const unsigned long long in_epoch = by_rows ? ++in_epoch_counter : 0;
-    ep.tile_flags = by_rows ? tflags : nullptr;
-    ep.flag_epoch = in_epoch;
     const void *Wb = static_cast<const __nv_bfloat16 *>(w.W_in) + (size_t)ep.col_offset * D;
     e = tr::launch_gemm_inproj(xhat, Wb, T, n_in - ep.col_offset, D, ep, err_word, s, pdl, &err);
     if (e != cudaSuccess)
@@ -574,9 +558,6 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
     sp.S_final = a->S_hat + (size_t)l * state_elems;
     sp.err_word = err_word;
     sp.pdl = pdl;
-    sp.in_flags = by_rows ? tflags : nullptr;
-    sp.in_epoch = in_epoch;
-    sp.in_tiles_n = (n_in - ep.col_offset + tr::kInProjTileCols - 1) / tr::kInProjTileCols;
     tr_status st = run_scan(sp, s, [&]() { return mk->mark(s); });
     if (st != TR_OK) return st;
     if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
@@ -588,7 +569,7 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
         if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
       }
       if (out) {
-        tr::ResidEpi rp;
+        tr::ResidEpi rp{};
         rp.x_res = x_in;
         rp.res_is_bf16 = in_bf16;
         rp.x_out = out;
@@ -607,7 +588,7 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
       e = tr::launch_rmsnorm(xr, 0, w.ffn_gain, T, D, rms_eps, xhat, s, pdl);
       if (e != cudaSuccess) return cuda_fail(e, "FFN rmsnorm");
       if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
-      tr::SwigluEpi sw;
+      tr::SwigluEpi sw{};
       sw.h = hmid;
       sw.ld = a->d_ff;
       e = tr::launch_gemm_swiglu(xhat, w.W_gate, w.W_up, T, a->d_ff, D, sw, err_word, s, pdl,
@@ -616,7 +597,7 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
         return err.empty() ? cuda_fail(e, "FFN gate/up projection")
                            : fail(TR_ERR_CUDA, "%s", err.c_str());
       if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
-      tr::ResidEpi rp;
+      tr::ResidEpi rp{};
       rp.x_res = xr;
       rp.res_is_bf16 = 0;
       rp.x_out = xr;
@@ -1021,7 +1002,7 @@ tr_status tr_out_projection(const void *o, int64_t o_stride, const void *W_o, co
   unsigned *errw;
   std::string err;
   if (!device_state(static_cast<cudaStream_t>(stream), &dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
-  tr::ResidEpi rp;
+  tr::ResidEpi rp{};
   rp.x_res = x_res;
   rp.res_is_bf16 = x_res_dtype == TR_DTYPE_BF16;
   rp.x_out = x_out;

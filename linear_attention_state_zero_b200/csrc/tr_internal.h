@@ -19,10 +19,6 @@ enum : unsigned {
   ERRBIT_SCAN_TIMEOUT = 2u,
 };
 
-// The GEMMs' output tile: 128 rows; the input projection's tiles are 256 columns wide.
-constexpr int kGemmTileRows = 128;
-constexpr int kInProjTileCols = 256;
-
 // Epilogue of the input projection: per-head L2 norm of q and k, bf16 q/k/v,
 // gate activations in fp32.
 struct InProjEpi {
@@ -38,11 +34,6 @@ struct InProjEpi {
   __nv_bfloat16 *z;       // [M, H d_v] bf16: the output gate's input, W_in rows after v
   const float *A_log;     // [H]: log alpha = -exp(A_log) softplus(a + dt_bias)
   const float *dt_bias;   // [H]
-  // optional: per output tile a ready flag (the launch's epoch, release-stored once the
-  // tile's outputs are written), tiles in row-major order [row tile][column tile]; the scan
-  // that follows waits on them instead of on the whole kernel
-  unsigned long long *tile_flags;
-  unsigned long long flag_epoch;
 };
 
 // Short causal depthwise convolution + silu over the bf16 q/k/v projections (zero history
@@ -97,13 +88,6 @@ struct ScanLaunch {
   unsigned long long wait_ns;  // bounded-wait limit of the chunked kernels
   bool precise_state;  // chunked chain: the state enters its products as a bf16 hi + lo pair
   unsigned long long epoch;    // per-call tag of the chunked scan's ready flags (set at launch)
-  // optional: the input projection's tile flags (InProjEpi::tile_flags; 128-token row tiles
-  // of in_tiles_n column tiles, tagged in_epoch).  With them the chunked scan is launched
-  // while the projection runs and its prep waits for the row tiles each item reads, not for
-  // the whole projection (q, k, v and the gates must be that projection's outputs).
-  const unsigned long long *in_flags;
-  unsigned long long in_epoch;
-  int in_tiles_n;
 };
 
 // The bounded-wait limit the scan kernels get (tr_set_wait_limit_ns; 4 s by default).
