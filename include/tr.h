@@ -289,9 +289,23 @@ tr_status tr_replay_group_profiled(const tr_group_args *args, void *ws, size_t w
  * GS "Key Mechanisms").  groups is a HOST array of n_groups tr_group_args; each
  * group carries its own LA weights and its own tails (the hits of one group
  * share its weights and are packed by that group's cu_seqlens).  The workspace
- * is shared: tr_replay_groups_workspace_size() is the largest single group's.
+ * is shared: tr_replay_groups_workspace_size() is the largest single group's, and
+ * with that much the groups run one after another on `stream`.
+ *
+ * Lanes: a workspace of tr_replay_groups_lanes_workspace_size(groups, n, L) bytes
+ * (L slices of the single-group size, L = 2..4) lets the call run the groups on L
+ * lanes at once: group g on lane g % L with its own slice, lane 0 on `stream`, the
+ * others on streams the library keeps per device (created on first use), forked
+ * from `stream` by an event and joined back into it before the call returns, so
+ * work enqueued on `stream` after the call sees every group's results.  The lanes
+ * overlap one group's partly idle phases (a chunk chain on few SMs, a GEMM's last
+ * wave) with another group's kernels; the results are bitwise those of the
+ * sequential call.  The lanes are used as far as the workspace allows, never
+ * while `stream` is being captured into a graph (the groups then run in turn).
  */
 size_t tr_replay_groups_workspace_size(const tr_group_args *groups, int32_t n_groups);
+size_t tr_replay_groups_lanes_workspace_size(const tr_group_args *groups, int32_t n_groups,
+                                             int32_t lanes);
 tr_status tr_replay_groups(const tr_group_args *groups, int32_t n_groups, void *ws,
                            size_t ws_bytes, void *stream);
 

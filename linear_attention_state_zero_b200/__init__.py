@@ -75,6 +75,7 @@ _SIGNATURES = {
     "tr_replay_group_profiled": (ctypes.c_int, [ctypes.POINTER(GroupArgs), c_vp, c_sz, c_vp,
                                                 ctypes.POINTER(c_vp), c_i32]),
     "tr_replay_groups_workspace_size": (c_sz, [ctypes.POINTER(GroupArgs), c_i32]),
+    "tr_replay_groups_lanes_workspace_size": (c_sz, [ctypes.POINTER(GroupArgs), c_i32, c_i32]),
     "tr_replay_groups": (ctypes.c_int, [ctypes.POINTER(GroupArgs), c_i32, c_vp, c_sz, c_vp]),
     "tr_state_error_workspace_size": (c_sz, [c_i64]),
     "tr_state_error": (ctypes.c_int, [c_vp, c_vp, c_i64, c_i32, c_i32, c_vp, c_vp, c_vp, c_sz,
@@ -407,15 +408,21 @@ def replay_group(h_tail, cu_seqlens, layers, n_heads, d_k, d_v, **kw):
 
 
 class GroupsReplay:
-    """A prepared tr_replay_groups call over several GroupReplay descriptions (shared workspace)."""
+    """A prepared tr_replay_groups call over several GroupReplay descriptions (shared workspace).
+    With lanes = 2..4 the workspace holds that many group slices and the groups run on that
+    many streams at once (bitwise the same results)."""
 
-    def __init__(self, groups: Sequence[GroupReplay]):
+    def __init__(self, groups: Sequence[GroupReplay], lanes: int = 1):
         self.groups = list(groups)
         n = len(self.groups)
+        if not 1 <= lanes <= 4:
+            raise ValueError("lanes must be 1..4")
         self._arr = (GroupArgs * n)()
         for i, g in enumerate(self.groups):
             self._arr[i] = g.args
-        self.ws_bytes = lib.tr_replay_groups_workspace_size(self._arr, n)
+        self.lanes = lanes
+        self.ws_bytes = (lib.tr_replay_groups_workspace_size(self._arr, n) if lanes == 1 else
+                         lib.tr_replay_groups_lanes_workspace_size(self._arr, n, lanes))
         dev = self.groups[0].h_tail.device
         for g in self.groups:
             if g.h_tail.device != dev:

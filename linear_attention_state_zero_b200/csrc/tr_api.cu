@@ -661,6 +661,23 @@ tr_status tp_layout(const tr_scan_args *a, TpLayout *L, tr::ScanLaunch *p) {
   return TR_OK;
 }
 
+// Extra streams and fork/join events of tr_replay_groups' lanes, per device (created on
+// first use, kept for the process; a mutex serialises the calls that use them).
+constexpr int kMaxLanes = 4;
+struct LaneSet {
+  cudaStream_t s[kMaxLanes] = {};
+  cudaEvent_t fork = nullptr, join[kMaxLanes] = {};
+  bool ready = false;
+};
+std::mutex g_lane_mu;
+LaneSet g_lanes[64];
+
+size_t single_group_bytes(const tr_group_args *groups, int32_t n_groups) {
+  size_t need = 0;
+  for (int32_t g = 0; g < n_groups; ++g) need = std::max(need, group_layout(&groups[g]).total);
+  return need;
+}
+
 // The group array, every group and the shared workspace of tr_replay_groups.
 tr_status validate_groups(const tr_group_args *groups, int32_t n_groups, const void *ws,
                           size_t ws_bytes) {
@@ -853,6 +870,12 @@ size_t tr_replay_groups_workspace_size(const tr_group_args *groups, int32_t n_gr
   return m;
 }
 
+size_t tr_replay_groups_lanes_workspace_size(const tr_group_args *groups, int32_t n_groups,
+                                             int32_t lanes) {
+  if (lanes < 1 || lanes > kMaxLanes) return 0;
+  return (size_t)lanes * align256(tr_replay_groups_workspace_size(groups, n_groups));
+}
+
 tr_status tr_replay_groups(const tr_group_args *groups, int32_t n_groups, void *ws,
                            size_t ws_bytes, void *stream) {
   tr_status vst = validate_groups(groups, n_groups, ws, ws_bytes);
@@ -860,12 +883,52 @@ tr_status tr_replay_groups(const tr_group_args *groups, int32_t n_groups, void *
   int dev;
   unsigned *errw;
   std::string err;
-  if (!device_state(static_cast<cudaStream_t>(stream), &dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
-  for (int32_t g = 0; g < n_groups; ++g) {
-    tr_status st = replay_group_enqueue(&groups[g], ws, errw, static_cast<cudaStream_t>(stream));
-    if (st != TR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!device_state(s, &dev, &errw, &err)) return fail(TR_ERR_CUDA, "%s", err.c_str());
+  // lanes: as many workspace slices as fit (at most kMaxLanes, at most one per group), none
+  // under capture
+  const size_t slice = align256(single_group_bytes(groups, n_groups));
+  int lanes = slice > 0 ? (int)std::min<size_t>(ws_bytes / slice, kMaxLanes) : 1;
+  lanes = std::max(1, std::min(lanes, (int)n_groups));
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (lanes > 1 && (cudaStreamIsCapturing(s, &cs) != cudaSuccess ||
+                    cs != cudaStreamCaptureStatusNone || dev < 0 || dev >= 64))
+    lanes = 1;
+  if (lanes == 1) {
+    for (int32_t g = 0; g < n_groups; ++g) {
+      tr_status st = replay_group_enqueue(&groups[g], ws, errw, s);
+      if (st != TR_OK) return st;
+    }
+    return ok();
   }
-  return ok();
+  std::lock_guard<std::mutex> lock(g_lane_mu);
+  LaneSet &L = g_lanes[dev];
+  if (!L.ready) {
+    cudaError_t e = cudaEventCreateWithFlags(&L.fork, cudaEventDisableTiming);
+    for (int i = 1; e == cudaSuccess && i < kMaxLanes; ++i) {
+      e = cudaStreamCreateWithFlags(&L.s[i], cudaStreamNonBlocking);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L.join[i], cudaEventDisableTiming);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "lane streams");
+    L.ready = true;
+  }
+  // fork: every extra lane starts after the work already on `stream`
+  cudaError_t e = cudaEventRecord(L.fork, s);
+  for (int i = 1; e == cudaSuccess && i < lanes; ++i) e = cudaStreamWaitEvent(L.s[i], L.fork, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "lane fork");
+  tr_status st = TR_OK;
+  for (int32_t g = 0; g < n_groups && st == TR_OK; ++g) {
+    const int lane = g % lanes;
+    st = replay_group_enqueue(&groups[g], static_cast<uint8_t *>(ws) + (size_t)lane * slice, errw,
+                              lane == 0 ? s : L.s[lane]);
+  }
+  // join (also after a failed enqueue, so `stream` never runs ahead of a lane)
+  for (int i = 1; i < lanes; ++i) {
+    cudaError_t je = cudaEventRecord(L.join[i], L.s[i]);
+    if (je == cudaSuccess) je = cudaStreamWaitEvent(s, L.join[i], 0);
+    if (je != cudaSuccess && st == TR_OK) st = cuda_fail(je, "lane join");
+  }
+  return st == TR_OK ? ok() : st;
 }
 
 tr_status tr_replay_groups_overlapped(const tr_group_args *groups, int32_t n_groups, void *ws,

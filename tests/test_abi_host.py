@@ -218,6 +218,19 @@ def test_overlapped_replay_checks_everything_before_the_copy():
     assert ov(arr, -1, FAKE, need, FAKE, FAKE, 4096, S1, S2) == 1
 
 
+def test_lanes_workspace_is_whole_slices():
+    """tr_replay_groups' lanes: L slices of the single-group workspace (256-byte multiples),
+    1 <= L <= 4; anything else is 0."""
+    a, keep = _group_args()
+    arr = (tr.GroupArgs * 2)(a, a)
+    one = tr.lib.tr_replay_groups_workspace_size(arr, 2)
+    assert one > 0 and one % 256 == 0
+    for lanes in range(1, 5):
+        assert tr.lib.tr_replay_groups_lanes_workspace_size(arr, 2, lanes) == lanes * one
+    assert tr.lib.tr_replay_groups_lanes_workspace_size(arr, 2, 0) == 0
+    assert tr.lib.tr_replay_groups_lanes_workspace_size(arr, 2, 5) == 0
+
+
 def test_replay_workspace_checks():
     a, keep = _group_args()
     need = tr.lib.tr_replay_group_workspace_size(ctypes.byref(a))

@@ -11,7 +11,7 @@ notes, section 2.3).
   states the benchmark's state error is measured against.
 - 8 concurrent hits x 8 groups x 3 LA layers, d_model 2048, 16 heads of 128, m = 32768,
   r in {5%, 10%}: one tr_replay_groups call; the oracle replays all 64 (hit, group) tails,
-  and the full prefill of two units (S_m).
+  and the full prefill of two units (S_m); the call on 4 lanes gives the same states bitwise.
 - a varlen batch of 64 requests with m ~ U[1024, 131072], r = 10%, d_model 4096, 32 heads,
   8 groups x 3 LA layers in one tr_replay_groups call; the oracle replays sampled requests of
   every group, the longest request of one group, and the full prefill (S_m) of the shortest.
@@ -75,11 +75,17 @@ def test_eight_hits_eight_groups(cuda_device):
         host.append((tails, layers, h, cu))
         groups.append(tr.GroupReplay(h.to(cuda_device), cu, to_dev(layers, cuda_device), H, d, d,
                                      skip_last_output=True))
-    outs = tr.GroupsReplay(groups).run()
+    outs = [(S.clone(), x) for S, x in tr.GroupsReplay(groups).run()]
     torch.cuda.synchronize()
     tr.check()
     for g in range(G):
         assert torch.isfinite(outs[g][0]).all()
+    # the same call on 4 lanes (concurrent streams, a workspace slice each): bitwise the same
+    lanes_out = tr.GroupsReplay(groups, lanes=4).run()
+    torch.cuda.synchronize()
+    tr.check()
+    for g in range(G):
+        assert torch.equal(lanes_out[g][0], outs[g][0]), g
     # the oracle on all 64 (hit, group) tails: one packed oracle call per group
     for g in range(G):
         tails, layers, h, cu = host[g]

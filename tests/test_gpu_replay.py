@@ -81,6 +81,32 @@ def test_groups_call_equals_single_calls(cuda_device):
         assert torch.equal(S, S1) and torch.equal(x, x1)
 
 
+@pytest.mark.parametrize("lanes", [2, 3, 4])
+def test_groups_on_lanes_equal_the_sequential_call(cuda_device, lanes):
+    """Groups are independent (reading notes section 2.4): run on 2-4 lanes at once (each
+    with its own workspace slice and stream, forked from and joined into the caller's
+    stream) they give bitwise the states and outputs of the one-after-another call, and work
+    enqueued on the caller's stream after the call sees all of them."""
+    D, H, d, L = 512, 4, 128, 3
+    gs = []
+    for g in range(5):
+        h, layers, cu = make_group([300 + 70 * g, 40, 129], D, H, d, L, seed=350 + g)
+        gs.append(tr.GroupReplay(h.to(cuda_device), cu, to_dev(layers, cuda_device), H, d, d))
+    seq = [(S.clone(), x.clone()) for S, x in tr.GroupsReplay(gs).run()]
+    for g in gs:
+        g.S_hat.zero_()
+        g.x_out.zero_()
+    par = tr.GroupsReplay(gs, lanes=lanes)
+    assert par.ws_bytes >= lanes * tr.GroupsReplay(gs).ws_bytes
+    outs = par.run()
+    after = [(S.sum(), x.sum()) for S, x in outs]   # enqueued after the call on its stream
+    torch.cuda.synchronize()
+    for (S, x), (S0, x0), (sS, sx) in zip(outs, seq, after):
+        assert torch.equal(S, S0) and torch.equal(x, x0)
+        assert torch.equal(sS, S0.sum()) and torch.equal(sx, x0.sum())
+    tr.check()
+
+
 def test_all_empty_tails_give_zero_states(cuda_device):
     D, H, d = 128, 2, 64
     layers = synth.la_layers(2, D, H, d, d, seed=320)
