@@ -679,6 +679,13 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
       }
 #pragma unroll
       for (int i = 0; i < 16; ++i) Ts[(base + i) * LDA + base + c] = Tc[i];
+    } else if (want_o) {
+      // meanwhile the other warps scale Q by gamma in place (64 rows x 4 pieces of 32
+      // columns; the Q band was group 1's operand only)
+      for (int pc = tid - C; pc < 4 * C; pc += kPrepThreads - C) {
+        const int r = pc & 63, q = pc >> 6;
+        scale_row32_bf16(ST + (q >> 1) * 32768, r, 32 * (q & 1), ctl->gq[r]);
+      }
     }
     bar_sync_n(1, kPrepThreads);
     const int mJ = tid >> 7, mr = (tid >> 3) & 15, mc = (tid & 7) * 2;
@@ -814,11 +821,6 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
         fence_proxy_async_smem();
         issue(ctl->nxt, buf ^ 1);
       }
-    }
-    // gamma Q in place (thread -> row, 32-column piece): the Q band is no product's operand
-    {
-      const int r = tid & 63, pc = tid >> 6, h = pc >> 1, c0 = 32 * (pc & 1);
-      if (want_o) scale_row32_bf16(ST + h * 32768, r, c0, ctl->gq[r]);
     }
     // lane quarters 0, 1 (W, Y) wait for the first part, quarters 2, 3 (U~) for the second
     const bool ok2 = mbar_wait(q4 < 2 ? mma_bar : smem_u32(&ctl->mma_bar2),
