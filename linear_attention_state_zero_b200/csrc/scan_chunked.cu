@@ -405,12 +405,37 @@ __device__ __forceinline__ void publish_slot(const ScanWs &ws, int64_t slot, uns
   asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(ws.flags + slot), "l"(epoch) : "memory");
 }
 
-// The prep work of CTA `vb` of `vg` (256 threads: warps 0-7).  With `publish`, each item's
+// The items one prep CTA takes, in increasing order: first the shared rounds (items below
+// shared_end, every `all` CTAs one each: item = cta, cta + all, ...), then, unless the CTA
+// only helps in those rounds, the rest in its own stride (shared_end + own_first, + own_stride
+// ...).  Without shared rounds this is one strided walk.
+struct PrepSched {
+  int64_t shared_end;   // items in the shared rounds (0: none)
+  int cta, all;         // this CTA's place among the shared rounds' CTAs
+  int64_t own_first;    // first item after the shared rounds, relative to shared_end (-1: none)
+  int own_stride;
+  __device__ __forceinline__ int64_t first(int64_t n_items) const {
+    if (cta < shared_end) return cta;
+    return own_first >= 0 ? shared_end + own_first : n_items;
+  }
+  __device__ __forceinline__ int64_t next(int64_t item, int64_t n_items) const {
+    if (item < shared_end) {
+      if (item + all < shared_end) return item + all;
+      return own_first >= 0 ? shared_end + own_first : n_items;
+    }
+    return item + own_stride;
+  }
+};
+
+// The prep work of one CTA (256 threads: warps 0-7) over the items of `sc`.  A CTA that
+// allocates tensor memory again afterwards (a chain CTA of the fused launch) keeps its
+// allocation permit (`last_alloc` false).  With `publish`, each item's
 // flag is set once its stores have completed: by thread 0 right after it has issued the next
 // item's first products (or after the loop, for the last item).
 template <int DV>
 __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &p, const ScanWs &ws,
-                                          const ScanPlan &plan, int vb, int vg, bool publish) {
+                                          const ScanPlan &plan, const PrepSched &sc, bool publish,
+                                          bool last_alloc = true) {
   const CUtensorMap &tm_q = mp.q, &tm_k = mp.k, &tm_v = mp.v, &tm_QW = mp.QW, &tm_PY = mp.PY,
                     &tm_KT = mp.KT, &tm_UT = mp.UT;
   extern __shared__ uint8_t smem_raw[];
@@ -426,7 +451,6 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
   const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
   const bool want_o = p.o != nullptr;
   const int64_t n_items = ws.slots;
-  const int64_t stride = vg;
   const int32_t *cu_chunks = plan_cu_chunks(plan, ws);
   const int32_t *cu_tokens = plan_cu_tokens(plan, p);
 
@@ -449,7 +473,7 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(&ctl->tmem), 512);
-    tmem_relinquish();
+    if (last_alloc) tmem_relinquish();
   }
   tc_fence_before();
   bar_sync_n(1, kPrepThreads);
@@ -495,7 +519,7 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
     }
   };
 
-  int64_t item = vb;
+  int64_t item = sc.first(n_items);
   int seq_cur = 0;   // threads 0 and 32: the sequence of the current item
   float la_next = 0.f, b_next = 0.f;
   if ((tid == 0 || tid == 32) && item < n_items) {
@@ -524,12 +548,12 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
   };
 
   int n = 0;
-  for (; item < n_items; item += stride, ++n) {
+  for (; item < n_items; item = sc.next(item, n_items), ++n) {
     const int buf = n & 1;
     uint8_t *ST = sm + buf * P_STAGE;
     const uint32_t st_u = smem_u32(ST);
     const PrepItem it = ctl->cur;
-    const bool has_next = item + stride < n_items;
+    const bool has_next = sc.next(item, n_items) < n_items;
 
     // gates: g = inclusive cumsum of log alpha (0 past the end), and the previous chunk's
     if (tid < 2 * C) {
@@ -594,8 +618,9 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
     } else if (tid == 32 && has_next) {
       // the next item's location, beside the products (its gates are loaded under the
       // inverse, its bands after group 2 is issued)
-      seq_cur = advance_seq(seq_cur, (int)((item + stride) / p.H), cu_chunks);
-      ctl->nxt = item_at(item + stride, seq_cur, p, cu_chunks, cu_tokens);
+      const int64_t nx = sc.next(item, n_items);
+      seq_cur = advance_seq(seq_cur, (int)(nx / p.H), cu_chunks);
+      ctl->nxt = item_at(nx, seq_cur, p, cu_chunks, cu_tokens);
     }
     if (!mma_wait()) break;
 
@@ -920,7 +945,7 @@ template <int DV>
 __global__ void __launch_bounds__(kPrepThreads, 1)
     scan_prep_kernel(const __grid_constant__ ScanMaps mp, const __grid_constant__ ScanLaunch p,
                      const __grid_constant__ ScanWs ws, const __grid_constant__ ScanPlan plan) {
-  prep_body<DV>(mp, p, ws, plan, blockIdx.x, gridDim.x, false);
+  prep_body<DV>(mp, p, ws, plan, PrepSched{0, 0, 1, (int64_t)blockIdx.x, (int)gridDim.x}, false);
 }
 
 // =========================================================== chain kernel
@@ -1422,19 +1447,27 @@ __global__ void __launch_bounds__(kChainThreads, 1)
 // ===================================================== prep beside chain
 // For few chains (a long sequence's heads: the latency-bound case) the chains run in the
 // same launch as the prep, on their own CTAs, each stage waiting for its slots' flags, so
-// the chain starts with the first chunks instead of after the last.  The launch is
+// the chain starts with the first chunks instead of after the last.  When the prep is the
+// longer part (many heads, long tails) the chain CTAs first help with it for a few rounds
+// (the shared rounds: every CTA of the grid takes one item per round), then run their
+// chains on the chunks those rounds prepared.  The launch is
 // cooperative: every CTA is resident at once, so a chain never waits on a prep CTA that
 // cannot be scheduled.  CTAs [0, n_chain) run chains, the rest (warps 0-7) the prep.
 template <int DV>
 __global__ void __launch_bounds__(kChainThreads, 1)
     scan_fused_kernel(const __grid_constant__ ScanMaps mp, const __grid_constant__ ScanLaunch p,
                       const __grid_constant__ ScanWs ws, const __grid_constant__ ScanPlan plan,
-                      int n_chain) {
-  if ((int)blockIdx.x < n_chain) {
-    chain_body(mp, p, ws, plan, blockIdx.x, true);
-  } else if (threadIdx.x < kPrepThreads) {
-    prep_body<DV>(mp, p, ws, plan, (int)blockIdx.x - n_chain, (int)gridDim.x - n_chain, true);
-  }
+                      int n_chain, int64_t shared_end) {
+  const int b = (int)blockIdx.x, all = (int)gridDim.x;
+  const bool chain = b < n_chain;
+  // a chain CTA first takes its items of the shared rounds (when the prep is the longer
+  // part: then the chain would only wait), then runs its chain (one call site of each body)
+  if (threadIdx.x < kPrepThreads && (!chain || shared_end > 0))
+    prep_body<DV>(mp, p, ws, plan,
+                  PrepSched{shared_end, b, all, chain ? -1 : (int64_t)(b - n_chain),
+                            all - n_chain},
+                  true, !chain);
+  if (chain) chain_body(mp, p, ws, plan, b, true);
 }
 
 // Host-side plan for up to kParamSeqs sequences: chunk offsets and the longest-first order.
@@ -1549,6 +1582,27 @@ cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string
     pf.epoch = ++epoch_counter;
     host_plan(pf, &plan);
     const int grid = sms;
+    // Shared rounds R: the chains start after R item-rounds on all SMs, the prep then goes
+    // on on the other SMs.  Costs in units of a chain step: a prep item about 5.3 steps
+    // (measured: ~14.7k against ~2.8k cycles); R minimises the later of the two ends.
+    const int64_t n_chain = fused_chains(p), pc = grid - n_chain;
+    int64_t longest = 0;
+    for (int i = 0; i < p.n_seqs; ++i)
+      longest = std::max<int64_t>(longest, (p.cu_seqlens_host[i + 1] - p.cu_seqlens_host[i] + C - 1) / C);
+    constexpr double kItem = 5.3, kStep = 1.0;
+    int64_t best_r = 0;
+    double best_t = 1e300;
+    for (int64_t r = 0; r * grid <= items + grid; ++r) {
+      const int64_t rest = std::max<int64_t>(0, items - r * grid);
+      const double prep = kItem * (double)(r + (rest + pc - 1) / pc);
+      const double chain = kItem * (double)(r + 1) + kStep * (double)(longest + 1);
+      const double t = std::max(prep, chain);
+      if (t < best_t - 1e-9) {
+        best_t = t;
+        best_r = r;
+      }
+    }
+    const int64_t shared_end = std::min<int64_t>(best_r * grid, items);
     auto kern = pf.dv == 128 ? scan_fused_kernel<128> : scan_fused_kernel<64>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FUSED_SMEM);
     if (e != cudaSuccess) return e;
@@ -1564,13 +1618,13 @@ cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pf.pdl ? 2 : 1;
-    e = cudaLaunchKernelEx(&cfg, kern, mp, pf, ws, plan, (int)fused_chains(p));
+    e = cudaLaunchKernelEx(&cfg, kern, mp, pf, ws, plan, (int)n_chain, shared_end);
     if (e == cudaSuccess || !pf.pdl) return e;
     // a runtime that will not combine a cooperative launch with programmatic serialization:
     // the same launch without the latter
     (void)cudaGetLastError();
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, mp, pf, ws, plan, (int)fused_chains(p));
+    return cudaLaunchKernelEx(&cfg, kern, mp, pf, ws, plan, (int)n_chain, shared_end);
   }
   if (!host_plan(p, &plan)) {
     e = launch_kernel(scan_plan_kernel, dim3(1), dim3(kPlanThreads), 0, s, p.pdl, p.cu_seqlens,
