@@ -752,22 +752,30 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
           make_float2(-x0, -x1);
     }
     bar_sync_n(1, kPrepThreads);
-    {  // X = A21 T11 (32 x 32): thread -> row r, columns c0..c0+3
+    if (tid < 128) {  // X = A21 T11 (32 x 32): thread -> rows r, r + 16, columns c0..c0+3
+      // (two rows per thread: each T11 row read from shared memory serves 8 products; the
+      // phase is bound by shared-memory bytes, not by threads)
       const int r = tid >> 3, c0 = (tid & 7) * 4;
-      float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
-      const float *Ar = As + (32 + r) * LDA;
-#pragma unroll 4
+      float x[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      const float *Ar0 = As + (32 + r) * LDA, *Ar1 = As + (48 + r) * LDA;
+#pragma unroll 2
       for (int s = 0; s < 32; s += 4) {
-        const float4 a = *reinterpret_cast<const float4 *>(Ar + s);
-        const float av[4] = {a.x, a.y, a.z, a.w};
+        const float4 a0 = *reinterpret_cast<const float4 *>(Ar0 + s);
+        const float4 a1 = *reinterpret_cast<const float4 *>(Ar1 + s);
+        const float av[2][4] = {{a0.x, a0.y, a0.z, a0.w}, {a1.x, a1.y, a1.z, a1.w}};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const float4 t = *reinterpret_cast<const float4 *>(Ts + (s + u) * LDA + c0);
-          x0 = fmaf(av[u], t.x, x0); x1 = fmaf(av[u], t.y, x1);
-          x2 = fmaf(av[u], t.z, x2); x3 = fmaf(av[u], t.w, x3);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            x[h][0] = fmaf(av[h][u], t.x, x[h][0]); x[h][1] = fmaf(av[h][u], t.y, x[h][1]);
+            x[h][2] = fmaf(av[h][u], t.z, x[h][2]); x[h][3] = fmaf(av[h][u], t.w, x[h][3]);
+          }
         }
       }
-      *reinterpret_cast<float4 *>(Xs + r * LDX + c0) = make_float4(x0, x1, x2, x3);
+      *reinterpret_cast<float4 *>(Xs + r * LDX + c0) = make_float4(x[0][0], x[0][1], x[0][2], x[0][3]);
+      *reinterpret_cast<float4 *>(Xs + (r + 16) * LDX + c0) =
+          make_float4(x[1][0], x[1][1], x[1][2], x[1][3]);
     }
     bar_sync_n(1, kPrepThreads);
     {  // T21 = -T22 X: thread -> row r, columns c0..c0+3; T22 is lower triangular, so
