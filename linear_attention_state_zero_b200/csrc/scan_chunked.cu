@@ -344,6 +344,7 @@ struct PrepCtl {
   float gp[C];     // gamma' = e^{g_C - g_t}
   float gpp[C];    // the previous chunk's gamma'
   float gq[C];     // gamma
+  __align__(16) float igq[C];   // 1 / gamma (when the chunk's decay allows it: see p1)
   float gpv[C];    // the previous chunk's cumsum
   float gc_prev;   // the previous chunk's gamma_C (1 without one)
 };
@@ -578,6 +579,7 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
     if (tid < C) {
       const float gt = ctl->g[tid];
       ctl->gq[tid] = exp_ftz(gt);
+      ctl->igq[tid] = exp_ftz(-gt);
       ctl->bg[tid] = ctl->beta[tid] * ctl->gq[tid];
       ctl->gp[tid] = exp_ftz(ctl->g[C - 1] - gt);
     } else if (tid < 2 * C) {
@@ -624,7 +626,11 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
     }
     if (!mma_wait()) break;
 
-    // P (rows 0-63, bf16), A (rows 64-127, fp32) and Z = K K~_prev^T (rows 64-127, bf16)
+    // P (rows 0-63, bf16), A (rows 64-127, fp32) and Z = K K~_prev^T (rows 64-127, bf16).
+    // The decays e^{g_t - g_s} are gamma_t (1 / gamma_s) when the chunk's total decay keeps
+    // 1 / gamma within fp32 (g_C > -80: then e^{-g} < 6e34): two exponentials per token
+    // instead of one per pair; otherwise they are taken pair by pair.
+    const bool factored = ctl->g[C - 1] > -80.f;
     {
       float v[32];
       // warps whose 32 columns all lie right of the diagonal (hsel 1, rows 0-31) write zeros
@@ -638,11 +644,26 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
           } else {
             tmem_ld32(tmem + lane_base + 32 * hsel, v);
             tc_wait_ld();
-            const float gt = ctl->g[t];
+            if (factored) {
+              const float et = ctl->gq[t];
+              const float4 *ig = reinterpret_cast<const float4 *>(ctl->igq + 32 * hsel);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int s = 32 * hsel + i;
-              v[i] = (s <= t) ? exp_ftz(gt - ctl->g[s]) * v[i] : 0.f;
+              for (int w = 0; w < 8; ++w) {
+                const float4 q = ig[w];
+                const float iq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  const int i = 4 * w + u, s = 32 * hsel + i;
+                  v[i] = (s <= t) ? et * iq[u] * v[i] : 0.f;
+                }
+              }
+            } else {
+              const float gt = ctl->g[t];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int s = 32 * hsel + i;
+                v[i] = (s <= t) ? exp_ftz(gt - ctl->g[s]) * v[i] : 0.f;
+              }
             }
           }
           store_row_bf16(sm + P_P, t, 32 * hsel, v, 1.f);
@@ -655,11 +676,26 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
         } else {
           tmem_ld32(tmem + lane_base + 32 * hsel, v);
           tc_wait_ld();
-          const float gt = ctl->g[t], bt = ctl->beta[t];
+          if (factored) {
+            const float bet = ctl->beta[t] * ctl->gq[t];
+            const float4 *ig = reinterpret_cast<const float4 *>(ctl->igq + 32 * hsel);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int s = 32 * hsel + i;
-            v[i] = (s < t) ? bt * exp_ftz(gt - ctl->g[s]) * v[i] : 0.f;
+            for (int w = 0; w < 8; ++w) {
+              const float4 q = ig[w];
+              const float iq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int i = 4 * w + u, s = 32 * hsel + i;
+                v[i] = (s < t) ? bet * iq[u] * v[i] : 0.f;
+              }
+            }
+          } else {
+            const float gt = ctl->g[t], bt = ctl->beta[t];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int s = 32 * hsel + i;
+              v[i] = (s < t) ? bt * exp_ftz(gt - ctl->g[s]) * v[i] : 0.f;
+            }
           }
         }
         float4 *dst = reinterpret_cast<float4 *>(As + t * LDA + 32 * hsel);
