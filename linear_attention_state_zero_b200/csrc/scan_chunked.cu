@@ -192,7 +192,9 @@ ScanWs ws_layout(const ScanLaunch &p, void *base, size_t *total) {
   size_t off = 0;
   const size_t oQW = off; off = align256(off + S * 128 * 128 * 2);
   const size_t oPY = off; off = align256(off + S * 128 * 64 * 2);
-  const size_t oKT = off; off = align256(off + S * 64 * 128 * 2);
+  // K~ is kept only when the scan normalises k itself; otherwise the chain reads k
+  const bool keep_kt = (p.flags & TR_NORMALIZE_QK) != 0;
+  const size_t oKT = off; off = align256(off + (keep_kt ? S * 64 * 128 * 2 : 0));
   const size_t oUT = off; off = align256(off + S * 64 * (size_t)p.dv * 4);
   const size_t oGP = off; off = align256(off + S * 64 * 4);
   const size_t oG = off;  off = align256(off + S * 16);
@@ -947,7 +949,7 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
       for (int h = 0; h < 2; ++h) {
         if (want_o) tma_store_2d(&tm_QW, st_u + h * 32768, 64 * h, y128);
         tma_store_2d(&tm_QW, st_u + h * 32768 + 16384, 64 * h, y128 + 64);
-        tma_store_2d(&tm_KT, st_u + h * 32768 + 8192, 64 * h, y64);
+        if (p.flags & TR_NORMALIZE_QK) tma_store_2d(&tm_KT, st_u + h * 32768 + 8192, 64 * h, y64);
       }
       bulk_commit();
       ws.G[slot * 4] = exp_ftz(ctl->g[C - 1]);
@@ -1077,7 +1079,10 @@ __device__ bool wait_slots(const ScanWs &ws, const int64_t (&slot)[2], int n,
 __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch &p,
                                            const ScanWs &ws, const ScanPlan &plan, int cta,
                                            bool wait_flags) {
-  const CUtensorMap &tm_QW = mp.QW, &tm_PY = mp.PY, &tm_KT = mp.KT, &tm_UT = mp.UT, &tm_o = mp.o;
+  const CUtensorMap &tm_QW = mp.QW, &tm_PY = mp.PY, &tm_KT = mp.KT, &tm_UT = mp.UT, &tm_o = mp.o,
+                    &tm_k = mp.k;
+  // K of a chunk: the prep's normalised copy, or the scan's own k input (no copy made)
+  const bool kt_ws = (p.flags & TR_NORMALIZE_QK) != 0;
   extern __shared__ uint8_t smem_raw[];
   __shared__ ChainCtl ctl_s;
   ChainCtl *ctl = &ctl_s;
@@ -1169,8 +1174,15 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
             tma_load_2d(base + C_A1 + 16384, &tm_QW, 64, (int32_t)(sc * 128), bar_mm);
             tma_load_2d(base + C_A2, &tm_PY, 0, (int32_t)(sc * 128), bar_mm);
           }
-          tma_load_2d(base + C_KT, &tm_KT, 0, (int32_t)(sc * 64), bar_mm);
-          tma_load_2d(base + C_KT + 8192, &tm_KT, 64, (int32_t)(sc * 64), bar_mm);
+          if (kt_ws) {
+            tma_load_2d(base + C_KT, &tm_KT, 0, (int32_t)(sc * 64), bar_mm);
+            tma_load_2d(base + C_KT + 8192, &tm_KT, 64, (int32_t)(sc * 64), bar_mm);
+          } else {
+            // rows past the sequence's end are other tokens or zero fill: their U rows are 0
+            const int32_t t0 = t_begin + C * (k - 1);
+            tma_load_2d(base + C_KT, &tm_k, head * DK, t0, bar_mm);
+            tma_load_2d(base + C_KT + 8192, &tm_k, head * DK + 64, t0, bar_mm);
+          }
         }
         if (nxt) {
           tma_load_2d(base + C_A1 + 8192, &tm_QW, 0, (int32_t)(sn * 128 + 64), bar_mm);
@@ -1603,7 +1615,8 @@ cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string
       !make_tmap_bf16_2d(&mp.v, p.v, (uint64_t)p.H * p.dv, T, (uint64_t)p.v_stride * 2, 64, C, err) ||
       !make_tmap_bf16_2d(&mp.QW, ws.QW, 128, slots * 128, 256, 64, 64, err) ||
       !make_tmap_bf16_2d(&mp.PY, ws.PY, 64, slots * 128, 128, 64, 64, err) ||
-      !make_tmap_bf16_2d(&mp.KT, ws.KT, 128, slots * 64, 256, 64, 64, err) ||
+      !make_tmap_bf16_2d(&mp.KT, (p.flags & TR_NORMALIZE_QK) ? (const void *)ws.KT : p.k, 128,
+                         (p.flags & TR_NORMALIZE_QK) ? slots * 64 : 1, 256, 64, 64, err) ||
       !make_tmap_f32_2d(&mp.UT, ws.UT, (uint64_t)p.dv, slots * 64, (uint64_t)p.dv * 4, 32, 64, err))
     return cudaErrorInvalidValue;
   // the readout o [T, H d_v] (token stride o_stride), stored in 64 x 64 boxes
