@@ -178,3 +178,19 @@ def test_scan_replayed_from_a_captured_graph(cuda_device):
         assert rel_fro(S, wS) < TOL_BF16
         assert rel_fro(o, wo) < TOL_BF16
     tr.check()
+
+
+@pytest.mark.parametrize("alpha_lo,alpha_hi", [(0.05, 0.2), (0.2, 0.6), (0.995, 1.0)])
+def test_decay_regimes(cuda_device, alpha_lo, alpha_hi):
+    """The chunked scan takes a chunk's in-chunk decays e^{g_t - g_s} as gamma_t / gamma_s
+    when the chunk's total decay keeps 1 / gamma within fp32 (g_C > -80), pair by pair
+    otherwise: alpha ~ U[0.05, 0.2] puts every chunk on the second path (g_C ~ -150), U[0.2,
+    0.6] mixes them (g_C ~ -60 .. -70), U[0.995, 1] is the slow-decay first path.  Each agrees
+    with the oracle, on one long sequence (the single-launch form) and on a varlen batch."""
+    for lengths, H in (([777], 16), ([1, 63, 64, 65, 300, 0, 129], 4)):
+        case = synth.scan_case(lengths, H, 128, 128, torch.bfloat16, alpha_lo, alpha_hi,
+                               seed=621)
+        o, S = run_gpu(case, cuda_device)
+        wo, wS = run_oracle(case)
+        assert rel_fro(o, wo) < TOL_BF16, lengths
+        assert rel_fro(S, wS) < TOL_BF16, lengths
