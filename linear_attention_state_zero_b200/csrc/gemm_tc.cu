@@ -226,12 +226,25 @@ __device__ __forceinline__ void epi_swiglu(const SwigluEpi &ep, uint32_t tbase, 
   }
 }
 
+// Work units: tiles [0, whole) run whole; each later tile (a partial last wave) runs as two
+// units of BN / 2 columns (half the B bytes per k-block, so the last wave ends sooner).
+__device__ __forceinline__ void unit_tile(int u, int whole, int &tile, int &half) {
+  if (u < whole) {
+    tile = u;
+    half = -1;
+  } else {
+    tile = whole + (u - whole) / 2;
+    half = (u - whole) % 2;
+  }
+}
+
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmB2, int M, int N, int K,
-                        InProjEpi ip, ResidEpi rs, SwigluEpi sw, unsigned *err_word) {
+                        InProjEpi ip, ResidEpi rs, SwigluEpi sw, int whole,
+                        unsigned *err_word) {
   using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -241,6 +254,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int m_tiles = (M + BM - 1) / BM;
   const int n_tiles = (N + BN - 1) / BN;
   const int n_total = m_tiles * n_tiles;
+  // units: the whole tiles, then two half-width units per remaining tile (whole == n_total:
+  // none split; the half units load B through tmB2, whose box is BN / 2 rows)
+  const int n_units = whole + 2 * (n_total - whole);
   const int kblocks = (K + BK - 1) / BK;
 
   if (threadIdx.x == 0) {
@@ -278,19 +294,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t ph = 0;
-      for (int t = blockIdx.x; t < n_total; t += gridDim.x) {
+      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        int t, hf;
+        unit_tile(u, whole, t, hf);
         const int tm = t % m_tiles, tn = t / m_tiles;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(smem_u32(&ctl->empty[stage]), ph ^ 1u, ab)) goto producer_done;
           const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t fb = smem_u32(&ctl->full[stage]);
-          mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+          mbar_arrive_expect_tx(fb, hf < 0 ? C::STAGE_BYTES : C::A_BYTES + C::B_BYTES / 2);
           tma_load_2d(sa, &tmA, kb * BK, tm * BM, fb);
           if (EPI == EPI_SWIGLU) {  // gate rows, then the same up rows
             tma_load_2d(sa + C::A_BYTES, &tmB, kb * BK, tn * (BN / 2), fb);
             tma_load_2d(sa + C::A_BYTES + C::B_BYTES / 2, &tmB2, kb * BK, tn * (BN / 2), fb);
-          } else {
+          } else if (hf < 0) {
             tma_load_2d(sa + C::A_BYTES, &tmB, kb * BK, tn * BN, fb);
+          } else {
+            tma_load_2d(sa + C::A_BYTES, &tmB2, kb * BK, tn * BN + hf * (BN / 2), fb);
           }
           if (++stage == C::STAGES) {
             stage = 0;
@@ -302,11 +322,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(BM, BN, 0, 0);
+      constexpr uint32_t idesc_full = idesc_bf16(BM, BN, 0, 0);
+      constexpr uint32_t idesc_half = idesc_bf16(BM, BN / 2, 0, 0);
       int stage = 0;
       uint32_t ph = 0;
       int it = 0;
-      for (int t = blockIdx.x; t < n_total; t += gridDim.x, ++it) {
+      for (int un = blockIdx.x; un < n_units; un += gridDim.x, ++it) {
+        int t, hf;
+        unit_tile(un, whole, t, hf);
+        (void)t;
+        const uint32_t idesc = hf < 0 ? idesc_full : idesc_half;
         const int b = it & 1;
         const uint32_t u = (uint32_t)(it >> 1);
         if (!mbar_wait(smem_u32(&ctl->tempty[b]), (u & 1u) ^ 1u, ab)) break;
@@ -338,7 +363,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     static_assert(BN % 64 == 0, "half tiles of whole 32-column groups");
     const int lo = half * (BN / 2), hi = lo + BN / 2;
     int it = 0;
-    for (int t = blockIdx.x; t < n_total; t += gridDim.x, ++it) {
+    for (int un = blockIdx.x; un < n_units; un += gridDim.x, ++it) {
+      int t, hf;
+      unit_tile(un, whole, t, hf);
       const int b = it & 1;
       const uint32_t u = (uint32_t)(it >> 1);
       if (!mbar_wait(smem_u32(&ctl->tfull[b]), u & 1u, ab)) break;
@@ -346,12 +373,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tm = t % m_tiles, tn = t / m_tiles;
       const int row = tm * BM + q4 * 32 + lane;
       const uint32_t tbase = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(b * BN);
-      if (EPI == EPI_INPROJ)
-        epi_inproj<BN>(ip, tbase, tn * BN, N, row, M, lo, hi);
+      // a half unit's BN / 2 columns sit at the accumulator's start: the warps of the first
+      // column half take them all, the others have none
+      const int n0 = tn * BN + (hf < 0 ? 0 : hf * (BN / 2));
+      const bool any = hf < 0 || half == 0;
+      const int ulo = hf < 0 ? lo : 0, uhi = hf < 0 ? hi : BN / 2;
+      if (!any) {
+      } else if (EPI == EPI_INPROJ)
+        epi_inproj<BN>(ip, tbase, n0, N, row, M, ulo, uhi);
       else if (EPI == EPI_SWIGLU)
         epi_swiglu(sw, tbase, tn * (BN / 2), row, M, half);
       else
-        epi_resid<BN>(rs, tbase, tn * BN, N, row, M, lo, hi);
+        epi_resid<BN>(rs, tbase, n0, N, row, M, ulo, uhi);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&ctl->tempty[b]));
@@ -387,6 +420,10 @@ cudaError_t launch(const void *A, int64_t lda, const void *B, const void *B2, in
         !make_tmap_bf16_2d(&tb, B, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN, err))
       return cudaErrorInvalidValue;
     tb2 = tb;
+    // the half-width tail units load BN / 2 rows of B
+    if (EPI == EPI_INPROJ &&
+        !make_tmap_bf16_2d(&tb2, B, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN / 2, err))
+      return cudaErrorInvalidValue;
   }
   auto kern = gemm_bf16_tn_kernel<BN, EPI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -395,8 +432,15 @@ cudaError_t launch(const void *A, int64_t lda, const void *B, const void *B2, in
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   int grid = device_sm_count();
   if (grid > tiles) grid = tiles;
+  // the input projection's partial last wave: its tiles split into two half-width units
+  // when twice as many still fit in one round
+  int whole = tiles;
+  if (EPI == EPI_INPROJ && grid > 0) {
+    const int rest = tiles % grid;
+    if (tiles > grid && rest > 0 && 2 * rest <= grid) whole = tiles - rest;
+  }
   return launch_kernel(kern, dim3((unsigned)grid), dim3(kThreads), C::SMEM, s, pdl, ta, tb, tb2, M,
-                       N, K, ip, rs, sw, err_word);
+                       N, K, ip, rs, sw, whole, err_word);
 }
 
 }  // namespace
