@@ -73,6 +73,44 @@ __device__ __forceinline__ uint64_t desc_mn(uint64_t d0, int kk) {
   return d0 + (uint64_t)kk * 128u;
 }
 
+// Packed fp32 pairs (sm_100a f32x2 arithmetic): one instruction for two lanes, each lane
+// rounded exactly as the scalar operation would be.
+__device__ __forceinline__ uint64_t f32x2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f32x2_unpack(uint64_t r, float &a, float &b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+// (a0, a1) += (b0, b1)
+__device__ __forceinline__ void add_f32x2(float &a0, float &a1, float b0, float b1) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f32x2_pack(a0, a1)), "l"(f32x2_pack(b0, b1)));
+  f32x2_unpack(r, a0, a1);
+}
+// (d0, d1) = (a0, a1) - (b0, b1)
+__device__ __forceinline__ void sub_f32x2(float &d0, float &d1, float a0, float a1, float b0,
+                                          float b1) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f32x2_pack(a0, a1)), "l"(f32x2_pack(b0, b1)));
+  f32x2_unpack(r, d0, d1);
+}
+// (d0, d1) = s (a0, a1)
+__device__ __forceinline__ void mul_f32x2(float &d0, float &d1, float a0, float a1, float s) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f32x2_pack(a0, a1)), "l"(f32x2_pack(s, s)));
+  f32x2_unpack(r, d0, d1);
+}
+// (m0, m1) = g (m0, m1) + (c0, c1), fused
+__device__ __forceinline__ void fma_f32x2(float &m0, float &m1, float g, float c0, float c1) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(r)
+      : "l"(f32x2_pack(g, g)), "l"(f32x2_pack(m0, m1)), "l"(f32x2_pack(c0, c1)));
+  f32x2_unpack(r, m0, m1);
+}
+
 // 32 consecutive bf16 (v[i] * s) into row `row` of a 128-byte-row swizzled tile at col0.
 __device__ __forceinline__ void store_row_bf16(uint8_t *tile, int row, int col0, const float *v,
                                                float s) {
@@ -118,7 +156,9 @@ __device__ __forceinline__ void load_row8_bf16(const uint8_t *tile, int row, int
   }
 }
 
-// hi + lo bf16 split of 32 values (v[i] * s) into two 128-byte-row swizzled tiles.
+// hi + lo bf16 split of 32 values (v[i] * s; v[i] itself without kScale) into two
+// 128-byte-row swizzled tiles.
+template <bool kScale = true>
 __device__ __forceinline__ void store_row_split(uint8_t *hi, uint8_t *lo, int row, int col0,
                                                 const float *v, float s) {
 #pragma unroll
@@ -126,10 +166,12 @@ __device__ __forceinline__ void store_row_split(uint8_t *hi, uint8_t *lo, int ro
     uint32_t h[4], l[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float a = v[8 * w + 2 * i] * s, b = v[8 * w + 2 * i + 1] * s;
+      float a = v[8 * w + 2 * i], b = v[8 * w + 2 * i + 1], ra, rb;
+      if (kScale) mul_f32x2(a, b, a, b, s);
       const __nv_bfloat162 hh = __floats2bfloat162_rn(a, b);
       const float2 hf = __bfloat1622float2(hh);
-      const __nv_bfloat162 ll = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+      sub_f32x2(ra, rb, a, b, hf.x, hf.y);
+      const __nv_bfloat162 ll = __floats2bfloat162_rn(ra, rb);
       h[i] = *reinterpret_cast<const uint32_t *>(&hh);
       l[i] = *reinterpret_cast<const uint32_t *>(&ll);
     }
@@ -854,7 +896,7 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
           v[4 * w + u] = te[u] * (rr < C ? ctl->bg[s] : ctl->beta[s]);
         }
       }
-      store_row_split(sm + P_THI, sm + P_TLO, rr, 32 * half, v, 1.f);
+      store_row_split<false>(sm + P_THI, sm + P_TLO, rr, 32 * half, v, 1.f);
     }
     fence_proxy_async_smem();
     bar_sync_n(1, kPrepThreads);
@@ -1299,8 +1341,8 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
     const bool lo2 = p.precise_state;
     auto store_state = [&]() {
       if (lo2) {
-        store_row_split(sm + C_MT, sm + C_MTL, d, 0, M, 1.f);
-        store_row_split(sm + C_MT, sm + C_MTL, d, 32, M + 32, 1.f);
+        store_row_split<false>(sm + C_MT, sm + C_MTL, d, 0, M, 1.f);
+        store_row_split<false>(sm + C_MT, sm + C_MTL, d, 32, M + 32, 1.f);
       } else {
         store_row_bf16(sm + C_MT, d, 0, M, 1.f);
         store_row_bf16(sm + C_MT, d, 32, M + 32, 1.f);
@@ -1333,7 +1375,10 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
         tmem_ld32(tmem + 192 + lane_base + 32 * h, v1);   // K^T (gamma' U_lo)
         tc_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) M[32 * h + i] = fmaf(gC, M[32 * h + i], v0[i] + v1[i]);
+        for (int i = 0; i < 32; i += 2) {
+          add_f32x2(v0[i], v0[i + 1], v1[i], v1[i + 1]);
+          fma_f32x2(M[32 * h + i], M[32 * h + i + 1], gC, v0[i], v0[i + 1]);
+        }
       }
       if (j + 1 < n) {
         store_state();
@@ -1404,7 +1449,7 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
             tmem_ld32(tmem + 64 * (j & 1) + lane_base + 32 * ch, v);
             tc_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) u[i] += v[i];
+            for (int i = 0; i < 32; i += 2) add_f32x2(u[i], u[i + 1], v[i], v[i + 1]);
             store_row_bf16(sm + C_UTL, t, 32 * ch, u, 1.f);
             store_row_split(sm + C_GUH, sm + C_GUL, t, 32 * ch, u, gq);
             fence_proxy_async_smem();
