@@ -19,6 +19,15 @@
 //              stores; overlaps the next tile's MMAs
 // Every mbarrier wait is bounded (see tr_ptx.cuh); a timeout ends all roles of
 // the CTA, frees its TMEM and raises the library's error word.
+//
+// Pair variant (the input projection): a cluster of two CTAs on two SMs computes a
+// 256 x BN tile with tcgen05.mma.cta_group::2.  Each CTA loads its own 128 rows of A and
+// its own BN / 2 rows of B (plain TMA loads, no multicast) into its shared memory, and
+// those loads complete on the leader CTA's barrier; the leader's single thread issues the
+// products (M = 256), whose completion is committed to both CTAs' barriers; each CTA's
+// epilogue reads its 128 accumulator rows out of its own TMEM.  Per SM and k-block that
+// is 32 KB of operands instead of 48 KB for a 128 x 256 tile: the L2-to-SM traffic that
+// bounds the single-CTA tile drops by a third.
 #include <cuda_bf16.h>
 
 #include "tr_internal.h"
@@ -399,6 +408,229 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ CTA pairs
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The shared::cluster address of `addr` (a shared::cta address) in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+// Arrive on an mbarrier of either CTA of the cluster (a shared::cluster address).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
+               : "memory");
+}
+// Tiled TMA load into this CTA's shared memory whose transaction count completes on an
+// mbarrier of either CTA of the pair (no multicast).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *tm, int32_t x,
+                                                 int32_t y, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.cta_group::2"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+// D[tmem] (+)= A * B^T over the pair: M = 256 (128 rows of A in each CTA), N columns (N / 2
+// rows of B in each CTA), operands at the same shared-memory offsets in both CTAs.
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on the mbarrier at shared offset `bar` in both CTAs of the pair when every
+// product issued so far by this thread is done.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"((uint16_t)3)
+      : "memory");
+}
+
+template <int BN>
+struct PairCfg {
+  static constexpr uint32_t A_BYTES = BM * BK * 2;            // this CTA's 128 rows
+  static constexpr uint32_t B_BYTES = (BN / 2) * BK * 2;      // this CTA's BN / 2 rows
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (200 * 1024 / STAGE_BYTES) < 8 ? (200 * 1024 / STAGE_BYTES) : 8;
+  static constexpr uint32_t TMEM_COLS = BN <= 128 ? 2 * BN : 512;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+};
+
+// Units as in the single-CTA kernel, over pair tiles (256 x BN); a half unit is 256 x BN / 2.
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                     const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmB2, int M, int N, int K,
+                     InProjEpi ip, ResidEpi rs, int whole, unsigned *err_word) {
+  using C = PairCfg<BN>;
+  static_assert(EPI != EPI_SWIGLU, "the pair kernel has no SwiGLU operand split");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  Ctl *ctl = reinterpret_cast<Ctl *>(smem + C::STAGES * C::STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int m_tiles = (M + 2 * BM - 1) / (2 * BM);
+  const int n_tiles = (N + BN - 1) / BN;
+  const int n_total = m_tiles * n_tiles;
+  const int n_units = whole + 2 * (n_total - whole);
+  const int kblocks = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(smem_u32(&ctl->full[s]), 1);    // the leader's: its expect-tx arrival
+      mbar_init(smem_u32(&ctl->empty[s]), 1);   // the leader's commit, in both CTAs
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&ctl->tfull[b]), 1);                // the leader's commit
+      mbar_init(smem_u32(&ctl->tempty[b]), 2 * kEpiWarps);   // both CTAs' epilogue warps
+    }
+    ctl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmB2);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&ctl->tmem_base)),
+                 "r"(C::TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  // both CTAs' barriers are initialised before either CTA's loads or arrivals reach them
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  const AbortFlag ab{&ctl->abort, err_word, ERRBIT_GEMM_TIMEOUT};
+  pdl_trigger();
+  pdl_wait();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph = 0;
+      for (int u = pair; u < n_units; u += n_pairs) {
+        int t, hf;
+        unit_tile(u, whole, t, hf);
+        const int tm = t % m_tiles, tn = t / m_tiles;
+        const int row_a = tm * 2 * BM + (int)rank * BM;
+        // this CTA's rows of B: half of the tile's (or of the half unit's) columns
+        const int row_b = hf < 0 ? tn * BN + (int)rank * (BN / 2)
+                                 : tn * BN + hf * (BN / 2) + (int)rank * (BN / 4);
+        const uint32_t pair_bytes = 2u * (hf < 0 ? C::STAGE_BYTES : C::A_BYTES + C::B_BYTES / 2);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(smem_u32(&ctl->empty[stage]), ph ^ 1u, ab)) goto producer_done;
+          const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t fb = cluster_map(smem_u32(&ctl->full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(smem_u32(&ctl->full[stage]), pair_bytes);
+          tma_load_2d_pair(sa, &tmA, kb * BK, row_a, fb);
+          tma_load_2d_pair(sa + C::A_BYTES, hf < 0 ? &tmB : &tmB2, kb * BK, row_b, fb);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+    producer_done:;
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc_full = idesc_bf16(2 * BM, BN, 0, 0);
+      constexpr uint32_t idesc_half = idesc_bf16(2 * BM, BN / 2, 0, 0);
+      int stage = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      for (int un = pair; un < n_units; un += n_pairs, ++it) {
+        int t, hf;
+        unit_tile(un, whole, t, hf);
+        (void)t;
+        const uint32_t idesc = hf < 0 ? idesc_full : idesc_half;
+        const int b = it & 1;
+        const uint32_t u = (uint32_t)(it >> 1);
+        if (!mbar_wait(smem_u32(&ctl->tempty[b]), (u & 1u) ^ 1u, ab)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(b * BN);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(smem_u32(&ctl->full[stage]), ph, ab)) goto mma_done;
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint64_t ad0 = sw128_desc(sa, 16, 1024);
+          const uint64_t bd0 = sw128_desc(sa + C::A_BYTES, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_pair(d, ad0 + 2u * kk, bd0 + 2u * kk, idesc, (kb | kk) ? 1u : 0u);
+          tc_commit_pair(smem_u32(&ctl->empty[stage]));
+          if (++stage == C::STAGES) {
+            stage = 0;
+            ph ^= 1u;
+          }
+        }
+        tc_commit_pair(smem_u32(&ctl->tfull[b]));
+      }
+    mma_done:;
+    }
+  } else {
+    const int q4 = warp & 3;
+    const int half = (warp - 2) >> 2;
+    static_assert(BN % 64 == 0, "half tiles of whole 32-column groups");
+    const int lo = half * (BN / 2), hi = lo + BN / 2;
+    const uint32_t tempty0 = cluster_map(smem_u32(&ctl->tempty[0]), 0);
+    const uint32_t tempty1 = cluster_map(smem_u32(&ctl->tempty[1]), 0);
+    int it = 0;
+    for (int un = pair; un < n_units; un += n_pairs, ++it) {
+      int t, hf;
+      unit_tile(un, whole, t, hf);
+      const int b = it & 1;
+      const uint32_t u = (uint32_t)(it >> 1);
+      if (!mbar_wait(smem_u32(&ctl->tfull[b]), u & 1u, ab)) break;
+      tc_fence_after();
+      const int tm = t % m_tiles, tn = t / m_tiles;
+      const int row = tm * 2 * BM + (int)rank * BM + q4 * 32 + lane;
+      const uint32_t tbase = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(b * BN);
+      const int n0 = tn * BN + (hf < 0 ? 0 : hf * (BN / 2));
+      const bool any = hf < 0 || half == 0;
+      const int ulo = hf < 0 ? lo : 0, uhi = hf < 0 ? hi : BN / 2;
+      if (!any) {
+      } else if (EPI == EPI_INPROJ)
+        epi_inproj<BN>(ip, tbase, n0, N, row, M, ulo, uhi);
+      else
+        epi_resid<BN>(rs, tbase, n0, N, row, M, ulo, uhi);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(b ? tempty1 : tempty0);
+    }
+  }
+
+  // no CTA leaves while its peer may still signal its barriers or read its operands
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(C::TMEM_COLS));
+  }
+}
+
 // N counts the tile's output columns; for the FFN gate/up product N = 2 d_ff, B = W_gate
 // and B2 = W_up ([d_ff, K] each).
 template <int BN, int EPI>
@@ -443,6 +675,63 @@ cudaError_t launch(const void *A, int64_t lda, const void *B, const void *B2, in
                        N, K, ip, rs, sw, whole, err_word);
 }
 
+// The pair kernel: clusters of two CTAs, as many as can be resident at once (each needs two
+// SMs of one TPC); tiles of 256 x BN, a partial last round as 256 x BN / 2 half units.
+template <int BN, int EPI>
+cudaError_t launch_pair(const void *A, int64_t lda, const void *B, int M, int N, int K,
+                        const InProjEpi &ip, const ResidEpi &rs, unsigned *err_word,
+                        cudaStream_t s, bool pdl, std::string *err) {
+  using C = PairCfg<BN>;
+  if (M <= 0 || N <= 0) return cudaSuccess;
+  CUtensorMap ta, tb, tb2;
+  if (!make_tmap_bf16_2d(&ta, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 2, BK, BM, err) ||
+      !make_tmap_bf16_2d(&tb, B, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN / 2, err) ||
+      !make_tmap_bf16_2d(&tb2, B, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN / 4, err))
+    return cudaErrorInvalidValue;
+  auto kern = gemm_pair_kernel<BN, EPI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)C::SMEM);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  // resident pairs (queried once per device; the SM count halved if the query fails)
+  constexpr int kDevices = 64;
+  static int resident[kDevices] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int pairs = device_sm_count() / 2;
+  if (dev >= 0 && dev < kDevices) {
+    if (resident[dev] == 0) {
+      cfg.gridDim = dim3((unsigned)(2 * pairs));
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0)
+        resident[dev] = n;
+      else
+        resident[dev] = pairs;
+      cudaGetLastError();
+    }
+    pairs = resident[dev] < pairs ? resident[dev] : pairs;
+  }
+  const int tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + BN - 1) / BN);
+  if (pairs > tiles) pairs = tiles;
+  int whole = tiles;
+  const int rest = tiles % pairs;
+  if (tiles > pairs && rest > 0 && 2 * rest <= pairs) whole = tiles - rest;
+  cfg.gridDim = dim3((unsigned)(2 * pairs));
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, tb2, M, N, K, ip, rs, whole, err_word);
+}
+
 }  // namespace
 
 cudaError_t launch_gemm_inproj(const void *A, const void *B, int M, int N, int K,
@@ -450,6 +739,8 @@ cudaError_t launch_gemm_inproj(const void *A, const void *B, int M, int N, int K
                                bool pdl, std::string *err) {
   ResidEpi none{};
   SwigluEpi no_sw{};
+  // more than one 128-row tile: 256-row tiles on CTA pairs
+  if (M > BM) return launch_pair<256, EPI_INPROJ>(A, K, B, M, N, K, ep, none, err_word, s, pdl, err);
   return launch<256, EPI_INPROJ>(A, K, B, nullptr, M, N, K, ep, none, no_sw, err_word, s, pdl, err);
 }
 

@@ -26,7 +26,11 @@ def test_rmsnorm(cuda_device, in_dtype, T, D):
     assert rel_fro(got, want) < 1e-3
 
 
-@pytest.mark.parametrize("T,D,H,d", [(300, 256, 2, 128), (129, 512, 4, 64), (1639, 2048, 16, 128)])
+# T <= 128: one CTA per 128-row tile; T > 128: 256-row tiles on CTA pairs, whose second CTA
+# may hold no valid row (T = 129, 300) and whose partial last round runs as half-width units
+# (T = 1639: 175 pair tiles)
+@pytest.mark.parametrize("T,D,H,d", [(100, 256, 2, 128), (300, 256, 2, 128), (129, 512, 4, 64),
+                                     (1639, 2048, 16, 128)])
 @pytest.mark.parametrize("skip_q", [False, True])
 def test_in_projection(cuda_device, T, D, H, d, skip_q):
     x_hat = synth.normal((T, D), 102, 1).to(torch.bfloat16)
