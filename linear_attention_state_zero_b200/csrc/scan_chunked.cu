@@ -1117,10 +1117,18 @@ __device__ bool wait_slots(const ScanWs &ws, const int64_t (&slot)[2], int n,
 }
 
 // The chain of CTA `cta` (384 threads); with `wait_flags` each stage's slots are awaited
-// first (their prep runs in the same launch).
+// first (their prep runs in the same launch).  SPL CTAs share one 64-column tile of d_v:
+// with SPL = 2 each carries 32 of its state columns (the columns of M, U and the products
+// are independent): the products still run over the whole tile (at the tensor pipe's
+// per-instruction floor N = 32 and N = 64 cost the same), the other half's columns are
+// zero, and each CTA's epilogues do half the work, on two U warps.
+template <int SPL>
 __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch &p,
                                            const ScanWs &ws, const ScanPlan &plan, int cta,
                                            bool wait_flags) {
+  static_assert(SPL == 1 || SPL == 2, "one or two CTAs per 64-column tile");
+  constexpr int CN = DVS / SPL;     // state columns this CTA carries
+  constexpr int NU = 4 / SPL;       // U warps
   const CUtensorMap &tm_QW = mp.QW, &tm_PY = mp.PY, &tm_KT = mp.KT, &tm_UT = mp.UT, &tm_o = mp.o,
                     &tm_k = mp.k;
   // K of a chunk: the prep's normalised copy, or the scan's own k input (no copy made)
@@ -1133,9 +1141,18 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int NS = p.dv / DVS;
   const int H = p.H;
-  const int pos = cta / (H * NS);
-  const int head = (cta / NS) % H, slice = cta % NS;
+  const int per_head = NS * SPL;
+  const int pos = cta / (H * per_head);
+  const int head = (cta / per_head) % H, sub = cta % per_head;
+  const int slice = sub / SPL, part = sub % SPL;
+  const int c_lo = part * CN;       // this CTA's first column within the tile
   const bool want_o = p.o != nullptr;
+  if (SPL > 1) {
+    // the other half of the MMA operand tiles stays zero
+    for (uint32_t o = 16u * (uint32_t)tid; o < C_GUL + 8192 - C_MT; o += 16u * kChainThreads)
+      *reinterpret_cast<uint4 *>(sm + C_MT + o) = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
 
   if (tid == 0) {
     tma_prefetch_desc(&tm_QW);
@@ -1145,14 +1162,14 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
     if (want_o) tma_prefetch_desc(&tm_o);
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&ctl->full[s]), 1);
-      mbar_init(smem_u32(&ctl->empty[s]), 8);   // each state warp and each U warp
+      mbar_init(smem_u32(&ctl->empty[s]), 4 + NU);   // each state warp and each U warp
       mbar_init(smem_u32(&ctl->full_m[s]), 1);
       mbar_init(smem_u32(&ctl->empty_m[s]), 1);
     }
     mbar_init(smem_u32(&ctl->bar_s), 1);
     mbar_init(smem_u32(&ctl->bar_d), 1);
     mbar_init(smem_u32(&ctl->bar_m), 4);        // each state warp
-    mbar_init(smem_u32(&ctl->bar_u), 4);        // each U warp
+    mbar_init(smem_u32(&ctl->bar_u), NU);       // each U warp
     mbar_init(smem_u32(&ctl->drain), 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&ctl->bar_dO[b]), 1);
@@ -1198,7 +1215,7 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
         const bool cur = k >= 1, nxt = k <= n - 1;
         const uint32_t bytes_m = (cur ? (want_o ? 16384u + 8192u : 0u) + 16384u : 0u) +
                                  (nxt ? 16384u + (k >= 1 ? 8192u : 0u) : 0u);
-        const uint32_t bytes_e = (cur ? 16u : 0u) + (nxt ? 16384u + 256u : 0u);
+        const uint32_t bytes_e = (cur ? 16u : 0u) + (nxt ? 16384u / SPL + 256u : 0u);
         const int64_t sc = cur ? slot_of(k - 1) : 0, sn = nxt ? slot_of(k) : 0;
         const uint32_t par = (uint32_t)((k - 2) >> 1) & 1u;
         // the slots' flags first: their check runs while the stage is still in use
@@ -1237,8 +1254,10 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
         mbar_arrive_expect_tx(bar, bytes_e);
         if (cur) bulk_load(base + C_G, ws.G + sc * 4, 16u, bar);
         if (nxt) {
-          tma_load_2d(base + C_UT, &tm_UT, slice * DVS, (int32_t)(sn * 64), bar);
-          tma_load_2d(base + C_UT + 8192, &tm_UT, slice * DVS + 32, (int32_t)(sn * 64), bar);
+          // the U~ columns this CTA carries (boxes of 32)
+          for (int bx = c_lo / 32; bx < (c_lo + CN) / 32; ++bx)
+            tma_load_2d(base + C_UT + 8192 * bx, &tm_UT, slice * DVS + 32 * bx, (int32_t)(sn * 64),
+                        bar);
           bulk_load(base + C_GP, ws.GP + sn * C, 256u, bar);
         }
         last_k[st] = k;
@@ -1325,27 +1344,28 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
     // ---------------------------------------------------------- state warps
     const int q = warp & 3, d = 32 * q + lane;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    float M[DVS];
-    const size_t s_off = ((size_t)(seq * H + head) * DK + d) * p.dv + (size_t)slice * DVS;
+    float M[CN];
+    const size_t s_off =
+        ((size_t)(seq * H + head) * DK + d) * p.dv + (size_t)slice * DVS + (size_t)c_lo;
     if (s0) {
 #pragma unroll
-      for (int j = 0; j < DVS; j += 4) {
+      for (int j = 0; j < CN; j += 4) {
         const float4 a = *reinterpret_cast<const float4 *>(p.S0 + s_off + j);
         M[j] = a.x; M[j + 1] = a.y; M[j + 2] = a.z; M[j + 3] = a.w;
       }
     } else {
 #pragma unroll
-      for (int j = 0; j < DVS; ++j) M[j] = 0.f;
+      for (int j = 0; j < CN; ++j) M[j] = 0.f;
     }
     bool failed = false;
     const bool lo2 = p.precise_state;
     auto store_state = [&]() {
-      if (lo2) {
-        store_row_split<false>(sm + C_MT, sm + C_MTL, d, 0, M, 1.f);
-        store_row_split<false>(sm + C_MT, sm + C_MTL, d, 32, M + 32, 1.f);
-      } else {
-        store_row_bf16(sm + C_MT, d, 0, M, 1.f);
-        store_row_bf16(sm + C_MT, d, 32, M + 32, 1.f);
+#pragma unroll
+      for (int h = 0; h < CN / 32; ++h) {
+        if (lo2)
+          store_row_split<false>(sm + C_MT, sm + C_MTL, d, c_lo + 32 * h, M + 32 * h, 1.f);
+        else
+          store_row_bf16(sm + C_MT, d, c_lo + 32 * h, M + 32 * h, 1.f);
       }
     };
     // each warp signals on its own (no CTA barrier on the step's path); a warp that gives
@@ -1370,9 +1390,9 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
       tc_fence_after();
       float v0[32], v1[32];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        tmem_ld32(tmem + 128 + lane_base + 32 * h, v0);   // K^T (gamma' U_hi)
-        tmem_ld32(tmem + 192 + lane_base + 32 * h, v1);   // K^T (gamma' U_lo)
+      for (int h = 0; h < CN / 32; ++h) {
+        tmem_ld32(tmem + 128 + lane_base + c_lo + 32 * h, v0);   // K^T (gamma' U_hi)
+        tmem_ld32(tmem + 192 + lane_base + c_lo + 32 * h, v1);   // K^T (gamma' U_lo)
         tc_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
@@ -1394,15 +1414,16 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
     if (!failed) {
       float *dst = p.S_final + s_off;
 #pragma unroll
-      for (int j = 0; j < DVS; j += 4)
+      for (int j = 0; j < CN; j += 4)
         *reinterpret_cast<float4 *>(dst + j) = make_float4(M[j], M[j + 1], M[j + 2], M[j + 3]);
     }
-  } else if (warp < 8 || warp >= 10) {
+  } else if (SPL == 1 ? (warp < 8 || warp >= 10) : warp < 8) {
     // ------------------------------------------------------------- U warps
     // warps 6, 7 (columns 0-31) and 10, 11 (columns 32-63), TMEM lanes 64-127:
     // U_{c+1} = U~_{c+1} + D rows 64-127, written as bf16 (for A2 U) and gamma' U as a bf16
     // hi + lo pair (for dM); each warp then announces its part
-    const int q = warp & 3, t = 32 * (q - 2) + lane, ch = warp >= 10 ? 1 : 0;
+    // with SPL = 2 warps 6 and 7 take this CTA's 32 columns; warps 10 and 11 have no role
+    const int q = warp & 3, t = 32 * (q - 2) + lane, ch = SPL == 1 ? (warp >= 10 ? 1 : 0) : part;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     uint32_t d_phase = 0;
     if (n > 0) {
@@ -1429,8 +1450,8 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(smem_u32(&ctl->bar_u));
-          mbar_arrive(smem_u32(&ctl->empty[0]));
-          mbar_arrive(smem_u32(&ctl->empty[0]));   // stage 0 holds no gamma_C
+          // its own arrival, and the state warps' share: stage 0 holds no gamma_C
+          for (int i = 0; i < 1 + 4 / NU; ++i) mbar_arrive(smem_u32(&ctl->empty[0]));
         }
         for (int j = 0; j < n; ++j) {
           const int k = j + 1, st = k & 1;
@@ -1463,7 +1484,7 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
         }
       }
     }
-  } else if (want_o) {
+  } else if (want_o && warp < 10) {
     // ------------------------------------------------------------- O warps
     // warps 8, 9 (TMEM lanes 0-63): O_c = D rows 0-63 (scaled, bf16).  Full chunks go out
     // by one TMA store from a double-buffered staging tile; the ragged last chunk by
@@ -1479,8 +1500,8 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
       tc_fence_after();
       const uint32_t dcol = tmem + 64 * (j & 1) + lane_base;
       float v0[32], v1[32];
-      tmem_ld32(dcol, v0);
-      tmem_ld32(dcol + 32, v1);
+      tmem_ld32(dcol + c_lo, v0);
+      if (SPL == 1) tmem_ld32(dcol + 32, v1);
       tc_wait_ld();
       // staging buffer j % 2 was last read by the store of chunk j - 2
       if (warp == 8 && lane == 0) bulk_wait_read<1>();
@@ -1488,7 +1509,20 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
       bar_sync_n(4, 64);
       if (warp == 8 && lane == 0) mbar_arrive(smem_u32(&ctl->bar_o[j & 1]));
       const int tok0 = t_begin + C * j;
-      if (tok0 + C <= t_end) {
+      if (SPL > 1) {
+        // half a tile's columns: row stores (a tile store would cover the other CTA's half)
+        if (tok0 + t < t_end) {
+          uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.o) +
+                                                 (size_t)(tok0 + t) * p.o_stride +
+                                                 (size_t)head * p.dv + slice * DVS + c_lo);
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            dst[w] = make_uint4(pack_bf16x2(v0[8 * w] * sc, v0[8 * w + 1] * sc),
+                                pack_bf16x2(v0[8 * w + 2] * sc, v0[8 * w + 3] * sc),
+                                pack_bf16x2(v0[8 * w + 4] * sc, v0[8 * w + 5] * sc),
+                                pack_bf16x2(v0[8 * w + 6] * sc, v0[8 * w + 7] * sc));
+        }
+      } else if (tok0 + C <= t_end) {
         uint8_t *stg = sm + C_MTL + 8192 * (j & 1);
         store_row_bf16(stg, t, 0, v0, sc);
         store_row_bf16(stg, t, 32, v1, sc);
@@ -1542,7 +1576,7 @@ __device__ __forceinline__ void chain_body(const ScanMaps &mp, const ScanLaunch 
 __global__ void __launch_bounds__(kChainThreads, 1)
     scan_chain_kernel(const __grid_constant__ ScanMaps mp, const __grid_constant__ ScanLaunch p,
                       const __grid_constant__ ScanWs ws, const __grid_constant__ ScanPlan plan) {
-  chain_body(mp, p, ws, plan, blockIdx.x, false);
+  chain_body<1>(mp, p, ws, plan, blockIdx.x, false);
 }
 
 // ===================================================== prep beside chain
@@ -1554,7 +1588,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
 // chains on the chunks those rounds prepared.  The launch is
 // cooperative: every CTA is resident at once, so a chain never waits on a prep CTA that
 // cannot be scheduled.  CTAs [0, n_chain) run chains, the rest (warps 0-7) the prep.
-template <int DV>
+template <int DV, int SPL>
 __global__ void __launch_bounds__(kChainThreads, 1)
     scan_fused_kernel(const __grid_constant__ ScanMaps mp, const __grid_constant__ ScanLaunch p,
                       const __grid_constant__ ScanWs ws, const __grid_constant__ ScanPlan plan,
@@ -1568,7 +1602,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
                   PrepSched{shared_end, b, all, chain ? -1 : (int64_t)(b - n_chain),
                             all - n_chain},
                   true, !chain);
-  if (chain) chain_body(mp, p, ws, plan, b, true);
+  if (chain) chain_body<SPL>(mp, p, ws, plan, b, true);
 }
 
 // Host-side plan for up to kParamSeqs sequences: chunk offsets and the longest-first order.
@@ -1601,6 +1635,7 @@ bool make_tmap_f32_2d(CUtensorMap *tm, const void *base, uint64_t inner, uint64_
 // The fused launch serves few chains (at most kFusedMaxChains CTAs, leaving most SMs to the
 // prep) of a plan that travels in the launch.
 constexpr int kFusedMaxChains = 96;
+constexpr int kSplitMaxChains = 64;
 int64_t fused_chains(const ScanLaunch &p) { return (int64_t)p.n_seqs * p.H * (p.dv / DVS); }
 bool use_fused(const ScanLaunch &p, int sms) {
   const int64_t n = fused_chains(p);
@@ -1687,7 +1722,10 @@ cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string
     // Shared rounds R: the chains start after R item-rounds on all SMs, the prep then goes
     // on on the other SMs.  Costs in units of a chain step: a prep item about 5.3 steps
     // (measured: ~14.7k against ~2.8k cycles); R minimises the later of the two ends.
-    const int64_t n_chain = fused_chains(p), pc = grid - n_chain;
+    // few chains: two CTAs per 64-column tile, each carrying 32 state columns (half the
+    // epilogue work on the chain's critical path; the prep keeps at least 84 SMs)
+    const bool split = !p.precise_state && 2 * fused_chains(p) <= kSplitMaxChains;
+    const int64_t n_chain = fused_chains(p) * (split ? 2 : 1), pc = grid - n_chain;
     int64_t longest = 0;
     for (int i = 0; i < p.n_seqs; ++i)
       longest = std::max<int64_t>(longest, (p.cu_seqlens_host[i + 1] - p.cu_seqlens_host[i] + C - 1) / C);
@@ -1705,7 +1743,8 @@ cudaError_t launch_scan_chunked(const ScanLaunch &p, cudaStream_t s, std::string
       }
     }
     const int64_t shared_end = std::min<int64_t>(best_r * grid, items);
-    auto kern = pf.dv == 128 ? scan_fused_kernel<128> : scan_fused_kernel<64>;
+    auto kern = pf.dv == 128 ? (split ? scan_fused_kernel<128, 2> : scan_fused_kernel<128, 1>)
+                             : (split ? scan_fused_kernel<64, 2> : scan_fused_kernel<64, 1>);
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FUSED_SMEM);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
