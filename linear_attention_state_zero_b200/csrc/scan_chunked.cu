@@ -383,10 +383,10 @@ struct PrepCtl {
   int abort;
   PrepItem cur, nxt;
   float g[C];      // inclusive cumsum of log alpha over the chunk
-  float beta[C];
-  float bg[C];     // beta * gamma
+  __align__(16) float beta[C];
+  __align__(16) float bg[C];     // beta * gamma
   float gp[C];     // gamma' = e^{g_C - g_t}
-  float gpp[C];    // the previous chunk's gamma'
+  __align__(16) float gpp[C];    // the previous chunk's gamma'
   float gq[C];     // gamma
   __align__(16) float igq[C];   // 1 / gamma (when the chunk's decay allows it: see p1)
   float gpv[C];    // the previous chunk's cumsum
@@ -748,8 +748,15 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
         if (it.has_prev) {
           tmem_ld32(tmem + lane_base + 64 + 32 * hsel, v);
           tc_wait_ld();
+          const float4 *gp4 = reinterpret_cast<const float4 *>(ctl->gpp + 32 * hsel);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= ctl->gpp[32 * hsel + i];
+          for (int w = 0; w < 8; ++w) {
+            const float4 g = gp4[w];
+            v[4 * w] *= g.x;
+            v[4 * w + 1] *= g.y;
+            v[4 * w + 2] *= g.z;
+            v[4 * w + 3] *= g.w;
+          }
           store_row_bf16(sm + P_Z, t, 32 * hsel, v, 1.f);
         }
       }
@@ -884,17 +891,19 @@ __device__ __forceinline__ void prep_body(const ScanMaps &mp, const ScanLaunch &
        // consecutive rows (conflict-free reads of T and swizzled stores)
       const int rr = tid & 127, half = tid >> 7, t = rr & 63;
       const bool zero = t < 32 && half == 1;  // T is lower triangular: T12 = 0
+      // the column scales, four per (broadcast) read
+      const float4 *sc4 =
+          reinterpret_cast<const float4 *>((rr < C ? ctl->bg : ctl->beta) + 32 * half);
       float v[32];
 #pragma unroll
       for (int w = 0; w < 8; ++w) {
         const float4 tv = zero ? make_float4(0.f, 0.f, 0.f, 0.f)
                                : *reinterpret_cast<const float4 *>(Ts + t * LDA + 32 * half + 4 * w);
-        const float te[4] = {tv.x, tv.y, tv.z, tv.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int s = 32 * half + 4 * w + u;
-          v[4 * w + u] = te[u] * (rr < C ? ctl->bg[s] : ctl->beta[s]);
-        }
+        const float4 sv = sc4[w];
+        v[4 * w] = tv.x * sv.x;
+        v[4 * w + 1] = tv.y * sv.y;
+        v[4 * w + 2] = tv.z * sv.z;
+        v[4 * w + 3] = tv.w * sv.w;
       }
       store_row_split<false>(sm + P_THI, sm + P_TLO, rr, 32 * half, v, 1.f);
     }
