@@ -206,9 +206,11 @@ def kernel_rooflines(names, avg_ms, k, peaks):
     KERNELS_SEEN.clear()
     KERNELS_SEEN.update(names)
     for n, t in zip(names, avg_ms):
-        if n == "rmsnorm":
+        # a layer starts at its input projection; an RMSNorm launch (the first layer's; the
+        # later layers' is folded into the residual GEMM before them) precedes it
+        if n == "in_proj":
             layer += 1
-        b, w = kernel_work(n, layer, k)
+        b, w = kernel_work(n, layer + 1 if n == "rmsnorm" else layer, k)
         bound[n] = b
         work[n] = work.get(n, 0.0) + w
         ms[n] = ms.get(n, 0.0) + t

@@ -89,6 +89,13 @@ __device__ __forceinline__ void epi_inproj(const InProjEpi &ep, uint32_t tbase, 
   const int nq = 2 * ep.H * dk;          // q and k features
   const int nv = nq + ep.H * ep.dv;      // end of the v features
   const int nz = nv + (ep.z ? ep.H * ep.dv : 0);  // end of the z features
+  // the folded RMSNorm's 1/rms of this row (1 without it)
+  float rs = 1.f;
+  if (ep.ssq_part && row < M) {
+    float ss = 0.f;
+    for (int i = 0; i < ep.n_part; ++i) ss += ep.ssq_part[(int64_t)i * ep.part_ld + row];
+    rs = rsqrtf(ss * ep.inv_d + ep.rms_eps);
+  }
   for (int blk = lo / dk; blk < hi / dk; ++blk) {
     const int c0 = n0 + blk * dk;  // GEMM column
     if (c0 >= N) break;
@@ -105,7 +112,10 @@ __device__ __forceinline__ void epi_inproj(const InProjEpi &ep, uint32_t tbase, 
           tmem_ld32(tb + 32 * j, v);
           tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ssq = fmaf(v[i], v[i], ssq);
+          for (int i = 0; i < 32; ++i) {
+            v[i] *= rs;
+            ssq = fmaf(v[i], v[i], ssq);
+          }
         }
         inv = rsqrtf(ssq + ep.norm_eps);
       }
@@ -113,7 +123,7 @@ __device__ __forceinline__ void epi_inproj(const InProjEpi &ep, uint32_t tbase, 
         float v[32];
         tmem_ld32(tb + 32 * j, v);
         tc_wait_ld();
-        if (row < M) store_bf16x32(ep.qkv + (int64_t)row * ep.ldq + g0 + 32 * j, v, inv);
+        if (row < M) store_bf16x32(ep.qkv + (int64_t)row * ep.ldq + g0 + 32 * j, v, rs * inv);
       }
     } else {
       for (int j = 0; j < dk / 32; ++j) {
@@ -124,6 +134,8 @@ __device__ __forceinline__ void epi_inproj(const InProjEpi &ep, uint32_t tbase, 
         tmem_ld32(tb + 32 * j, v);
         tc_wait_ld();
         if (row >= M) continue;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= rs;
         if (g + 32 <= nv) {
           store_bf16x32(ep.qkv + (int64_t)row * ep.ldq + g, v, 1.f);
         } else if (g + 32 <= nz) {
@@ -195,6 +207,7 @@ __device__ __forceinline__ void epi_resid(const ResidEpi &ep, uint32_t tbase, in
                                           int row, int M, int lo, int hi) {
   const bool live = row < M;
   Res32 cur, nxt;
+  float ss = 0.f;   // the folded RMSNorm's partial sum of squares of this row
   if (live && n0 + lo < N) load_res32(ep, row, n0 + lo, cur);
 #pragma unroll 1
   for (int j = lo / 32; j < hi / 32; ++j) {
@@ -207,14 +220,33 @@ __device__ __forceinline__ void epi_resid(const ResidEpi &ep, uint32_t tbase, in
     if (live) {
       float r[32];
       res32_to_f32(ep, cur, r);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] += r[i];
       float4 *out = reinterpret_cast<float4 *>(ep.x_out + (int64_t)row * ep.ld + c);
 #pragma unroll
       for (int w = 0; w < 8; ++w)
-        out[w] = make_float4(r[4 * w] + v[4 * w], r[4 * w + 1] + v[4 * w + 1],
-                             r[4 * w + 2] + v[4 * w + 2], r[4 * w + 3] + v[4 * w + 3]);
+        out[w] = make_float4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]);
+      if (ep.xhat_out) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
+        if (ep.gain) {
+          const float4 *gp = reinterpret_cast<const float4 *>(ep.gain + c);
+#pragma unroll
+          for (int w = 0; w < 8; ++w) {
+            const float4 g = gp[w];
+            v[4 * w] *= g.x;
+            v[4 * w + 1] *= g.y;
+            v[4 * w + 2] *= g.z;
+            v[4 * w + 3] *= g.w;
+          }
+        }
+        store_bf16x32(ep.xhat_out + (int64_t)row * ep.ld + c, v, 1.f);
+      }
     }
     cur = nxt;
   }
+  // one partial per (row, column group), written even when the group holds no column
+  if (ep.xhat_out && live) ep.ssq_part[(int64_t)((n0 + lo) / (BN / 2)) * ep.part_ld + row] = ss;
 }
 
 // FFN epilogue for one tile of 128 gate (TMEM columns 0-127) and 128 up columns
@@ -733,6 +765,11 @@ cudaError_t launch_pair(const void *A, int64_t lda, const void *B, int M, int N,
 }
 
 }  // namespace
+
+// The residual GEMM's tiles (launch<192, EPI_RESID>) are 192 columns wide, each half taken
+// by its own epilogue warps: one partial sum of squares per row and half tile, the last
+// tile's halves included even where they hold no column
+int resid_ssq_partials(int N) { return 2 * ((N + 191) / 192); }
 
 cudaError_t launch_gemm_inproj(const void *A, const void *B, int M, int N, int K,
                                const InProjEpi &ep, unsigned *err_word, cudaStream_t s,

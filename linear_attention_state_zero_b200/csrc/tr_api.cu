@@ -304,7 +304,7 @@ tr_status run_scan(const tr::ScanLaunch &p, cudaStream_t s,
 
 // ------------------------------------------------------------- replay group
 struct GroupLayout {
-  size_t x, xhat, qkv, post, zbuf, la, beta, o, hmid, scan, total;
+  size_t x, xhat, qkv, post, zbuf, la, beta, o, hmid, ssq, scan, total;
   int64_t ldq;
 };
 
@@ -348,6 +348,8 @@ GroupLayout group_layout(const tr_group_args *a) {
   L.beta = off; off = align256(off + T * H * 4);
   L.o = off;    off = align256(off + T * H * (size_t)a->d_v * 2);
   L.hmid = off; off = align256(off + T * (size_t)(a->d_ff > 0 ? a->d_ff : 0) * 2);
+  // the folded RMSNorm's per-row partial sums of squares (layers after the first)
+  L.ssq = off;  off = align256(off + (a->n_layers > 1 ? T * (size_t)tr::resid_ssq_partials((int)D) * 4 : 0));
   L.scan = off; off = align256(off + scan_ws_bytes(group_scan_launch(a)));
   L.total = off;
   return L;
@@ -438,7 +440,8 @@ std::vector<const char *> group_kernel_names(const tr_group_args *a) {
   for (int l = 0; l < a->n_layers; ++l) {
     const bool last = l == a->n_layers - 1;
     const bool skip = last && (a->flags & TR_SKIP_LAST_OUTPUT);
-    n.push_back("rmsnorm");
+    // later layers' RMSNorm is folded into the previous layer's last residual GEMM
+    if (l == 0) n.push_back("rmsnorm");
     n.push_back("in_proj");
     if (a->conv_width > 0) n.push_back("short_conv");
     for (const char *k : scan_kernel_names(group_scan_launch(a), !skip)) n.push_back(k);
@@ -478,6 +481,7 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
   auto *hmid = reinterpret_cast<__nv_bfloat16 *>(base + L.hmid);
   auto *post = reinterpret_cast<__nv_bfloat16 *>(base + L.post);
   auto *zbuf = reinterpret_cast<__nv_bfloat16 *>(base + L.zbuf);
+  float *ssq = reinterpret_cast<float *>(base + L.ssq);
   const int T = (int)a->total_tokens, D = a->d_model, H = a->n_heads, dk = a->d_k, dv = a->d_v;
   const int n_in = in_rows(a);
   const bool conv = a->conv_width > 0;
@@ -496,10 +500,31 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
     const bool skip_q = skip && !a->conv_state;
     const void *x_in = l == 0 ? a->h_tail : static_cast<const void *>(x);
     const int in_bf16 = l == 0 ? 1 : 0;
-    e = tr::launch_rmsnorm(x_in, in_bf16, w.rms_gain, T, D, rms_eps, xhat, s, pdl);
-    if (e != cudaSuccess) return cuda_fail(e, "rmsnorm");
-    if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
+    // the RMSNorm of layers after the first was folded into the residual GEMM that wrote x
+    // (xhat = bf16(x * gain) and the rows' partial sums of squares); the projection's
+    // epilogue applies 1/rms
+    const bool folded = l > 0;
+    if (!folded) {
+      e = tr::launch_rmsnorm(x_in, in_bf16, w.rms_gain, T, D, rms_eps, xhat, s, pdl);
+      if (e != cudaSuccess) return cuda_fail(e, "rmsnorm");
+      if (mk->mark(s) != cudaSuccess) return fail(TR_ERR_CUDA, "cudaEventRecord");
+    }
+    // the residual GEMM that writes the next layer's input folds that layer's RMSNorm in
+    auto fold_next = [&](tr::ResidEpi &rp) {
+      if (l + 1 >= a->n_layers) return;
+      rp.xhat_out = static_cast<__nv_bfloat16 *>(xhat);
+      rp.gain = a->layers[l + 1].rms_gain;
+      rp.ssq_part = ssq;
+      rp.part_ld = T;
+    };
     tr::InProjEpi ep{};
+    if (folded) {
+      ep.ssq_part = ssq;
+      ep.n_part = tr::resid_ssq_partials(D);
+      ep.part_ld = T;
+      ep.inv_d = 1.f / (float)D;
+      ep.rms_eps = rms_eps;
+    }
     ep.qkv = qkv;
     ep.ldq = L.ldq;
     ep.log_alpha = la;
@@ -574,6 +599,7 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
         rp.res_is_bf16 = in_bf16;
         rp.x_out = out;
         rp.ld = D;
+        if (!runs_ffn(a, l)) fold_next(rp);
         e = tr::launch_gemm_resid(obuf, (int64_t)H * dv, w.W_o, T, D, H * dv, rp, err_word, s,
                                   pdl, &err);
         if (e != cudaSuccess)
@@ -602,6 +628,7 @@ tr_status replay_group_enqueue(const tr_group_args *a, void *ws, unsigned *err_w
       rp.res_is_bf16 = 0;
       rp.x_out = xr;
       rp.ld = D;
+      fold_next(rp);
       e = tr::launch_gemm_resid(hmid, a->d_ff, w.W_down, T, D, a->d_ff, rp, err_word, s, pdl,
                                 &err);
       if (e != cudaSuccess)

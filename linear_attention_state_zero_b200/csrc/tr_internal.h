@@ -34,6 +34,13 @@ struct InProjEpi {
   __nv_bfloat16 *z;       // [M, H d_v] bf16: the output gate's input, W_in rows after v
   const float *A_log;     // [H]: log alpha = -exp(A_log) softplus(a + dt_bias)
   const float *dt_bias;   // [H]
+  // RMSNorm folded in (NULL: not used): A is bf16(x * gain) without the 1/rms factor, and
+  // every output of row r is first multiplied by 1/sqrt(ss_r / d_model + rms_eps), ss_r the
+  // sum of the row's n_part partial sums ssq_part[i * part_ld + r], added in order of i
+  const float *ssq_part;
+  int n_part;
+  int64_t part_ld;
+  float inv_d, rms_eps;
 };
 
 // Short causal depthwise convolution + silu over the bf16 q/k/v projections (zero history
@@ -59,7 +66,17 @@ struct ResidEpi {
   int res_is_bf16;
   float *x_out;        // [M, ld] fp32
   int64_t ld;
+  // the next layer's RMSNorm, folded in (NULL: not used): bf16(x_out * gain) to xhat_out
+  // [M, ld] and, per row, one partial sum of x_out^2 per column group (each half of a
+  // 192-column tile; groups past N hold 0), group i to ssq_part[i * part_ld + row]
+  __nv_bfloat16 *xhat_out;
+  const float *gain;   // [ld] (NULL: 1)
+  float *ssq_part;
+  int64_t part_ld;
 };
+
+// Number of per-row partial sums of squares the residual GEMM writes for N columns.
+int resid_ssq_partials(int N);
 
 // Epilogue of the FFN's gate/up projection: h = bf16(silu(gate) * up).
 struct SwigluEpi {

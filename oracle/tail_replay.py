@@ -25,7 +25,12 @@ RN section 2.3 says no model dimensions are to be made up from Eq. (1)):
   * bf16 cast points of the boundary (``emulate_casts``): the projection
     operands x_hat and o (and the FFN's pre-norm output and hidden activation)
     and the stored q, k, v are rounded to bf16
-    (round-to-nearest-even); everything else stays fp64 here.
+    (round-to-nearest-even); everything else stays fp64 here.  For the LA layers
+    after a group's first, the RMSNorm's 1/rms factor sits after the projection
+    (``fold_norm``): the operand rounded to bf16 is x * gain, and the projection's
+    outputs are multiplied by the row's 1/rms, the same value in exact arithmetic
+    with the bf16 rounding taken before the scale (the implementation computes the
+    norm inside the residual and projection GEMMs there).
 """
 from __future__ import annotations
 
@@ -356,8 +361,12 @@ def replay_layer(x, W_in, W_o, rms_gain, cu_seqlens, n_heads: int, d_k: int, d_v
                  want_output: bool = True, emulate_casts: bool = True,
                  rms_eps: float = 1e-6, norm_eps: float = 1e-6, n_threads=None, ffn=None,
                  conv_w=None, A_log=None, dt_bias=None, output_gate: bool = False,
-                 o_norm_gain=None, conv_states: Optional[list] = None):
+                 o_norm_gain=None, conv_states: Optional[list] = None,
+                 fold_norm: bool = False):
     """One LA layer of the replay from a zero state: returns (S_hat, x_next or None).
+
+    ``fold_norm``: the RMSNorm's cast point of the layers after a group's first (module
+    docstring): x_hat = bf16(x * gain), and the projection's outputs times 1/rms.
 
     ``ffn`` = (W_gate, W_up, W_down, ffn_gain) runs the FFN sublayer on x_next
     (``ffn_residual``); None leaves it out.  The Gated DeltaNet details the pages
@@ -370,8 +379,16 @@ def replay_layer(x, W_in, W_o, rms_gain, cu_seqlens, n_heads: int, d_k: int, d_v
     """
     x = _f64(x)
     cast = bf16_round if emulate_casts else (lambda a: a)
-    x_hat = cast(rmsnorm(x, rms_gain, rms_eps))
-    proj = in_projection(x_hat, W_in, n_heads, d_k, d_v, output_gate)
+    if fold_norm:
+        # RMSNorm(x) W_in^T = (1 / rms) ((x * gain) W_in^T), the rounding taken on x * gain
+        inv_rms = 1.0 / np.sqrt(np.mean(x * x, axis=-1) + rms_eps)
+        x_g = x * _f64(rms_gain) if rms_gain is not None else x
+        proj = in_projection(cast(x_g), W_in, n_heads, d_k, d_v, output_gate)
+        proj = tuple(a * (inv_rms[:, None, None] if a.ndim == 3 else inv_rms[:, None])
+                     for a in proj)
+    else:
+        x_hat = cast(rmsnorm(x, rms_gain, rms_eps))
+        proj = in_projection(x_hat, W_in, n_heads, d_k, d_v, output_gate)
     if output_gate:
         q, k, v, z, a_alpha, a_beta = proj
     else:
@@ -445,7 +462,7 @@ def replay_group(h_tail, cu_seqlens, layers: Sequence, n_heads: int, d_k: int, d
                                      dt_bias=getattr(lw, "dt_bias", None),
                                      output_gate=output_gate,
                                      o_norm_gain=getattr(lw, "o_norm_gain", None),
-                                     conv_states=conv_states)
+                                     conv_states=conv_states, fold_norm=i > 0)
         S_all.append(S_hat)
         x = x_next
     return np.stack(S_all, 0), x

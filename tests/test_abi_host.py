@@ -251,13 +251,14 @@ def test_state_error_workspace_and_args():
 
 def test_replay_kernel_names_match_the_count():
     """tr_replay_group_kernel_names lists exactly the launches tr_replay_group_kernel_count
-    counts, in launch order: per layer the RMSNorm, the input projection, the scan's kernels
-    and the output projection (not after the last layer without x_out), plus the options'."""
+    counts, in launch order: the first layer's RMSNorm (later layers' is folded into the
+    residual GEMM before them), per layer the input projection, the scan's kernels and the
+    output projection (not after the last layer without x_out), plus the options'."""
     a, keep = _group_args()
     names = tr.lib.tr_replay_group_kernel_names(ctypes.byref(a)).decode().split(",")
     assert len(names) == tr.lib.tr_replay_group_kernel_count(ctypes.byref(a))
     assert names[:2] == ["rmsnorm", "in_proj"] and names[-1] != "out_proj"
-    assert names.count("rmsnorm") == 3 and names.count("out_proj") == 2
+    assert names.count("rmsnorm") == 1 and names.count("out_proj") == 2
     assert all(n.startswith("scan") for n in names if n not in ("rmsnorm", "in_proj", "out_proj"))
     a.d_ff = 1024
     a.conv_width = 4

@@ -113,7 +113,7 @@ def test_group_with_ffn_paper_shape(cuda_device):
         lw = layers[l]
         ffn = (lw.W_gate, lw.W_up, lw.W_down, lw.ffn_gain)
         wS_l, wx_l = oracle.replay_layer(f64(x_in), lw.W_in, lw.W_o, lw.rms_gain, cu, H, d, d,
-                                         ffn=ffn)
+                                         ffn=ffn, fold_norm=l > 0)
         assert rel_fro(S[l], wS_l) < TOL, l
         if l == L - 1:
             assert rel_fro(x, wx_l) < TOL

@@ -118,7 +118,7 @@ def test_group_all_options_paper_shape(cuda_device):
         wS_l, wx_l = oracle.replay_layer(f64(x_in), lw.W_in, lw.W_o, lw.rms_gain, cu, H, d, d,
                                          conv_w=lw.conv_w, A_log=lw.A_log, dt_bias=lw.dt_bias,
                                          output_gate=True, o_norm_gain=lw.o_norm_gain,
-                                         conv_states=st)
+                                         conv_states=st, fold_norm=l > 0)
         assert rel_fro(S[l], wS_l) < TOL, l
         assert rel_fro(g.conv_state[l], st[0]) < TOL, l
         if l == L - 1:

@@ -616,6 +616,26 @@ def test_replay_cast_points_are_small():
     assert 0 < tot < 2e-2
 
 
+def test_folded_norm_cast_point_is_the_same_math():
+    """The layers after a group's first take RMSNorm(x) W_in^T as (1/rms) ((x * gain) W_in^T),
+    the bf16 rounding on x * gain: in exact arithmetic (no casts) that is the plain RMSNorm
+    and projection to fp64 rounding, with the gain and the 1/rms both in play; with the
+    casts the two orders differ by bf16 rounding only."""
+    h, layers, cu = _tiny_group([40, 25], D=64, H=2, dk=16, dv=16)
+    lw = layers[1]
+    x = synth.normal((65, 64), 17, 3).double() * 3.0     # rows of very different rms
+    gain = torch.linspace(0.5, 1.5, 64, dtype=torch.float64)
+    for g in (None, gain):
+        S_a, x_a = oracle.replay_layer(x, lw.W_in, lw.W_o, g, cu, 2, 16, 16, emulate_casts=False)
+        S_b, x_b = oracle.replay_layer(x, lw.W_in, lw.W_o, g, cu, 2, 16, 16, emulate_casts=False,
+                                       fold_norm=True)
+        np.testing.assert_allclose(S_b, S_a, rtol=1e-10, atol=1e-13)
+        np.testing.assert_allclose(x_b, x_a, rtol=1e-10, atol=1e-12)
+        S_c, _ = oracle.replay_layer(x, lw.W_in, lw.W_o, g, cu, 2, 16, 16, fold_norm=True)
+        _, tot = oracle.state_error(S_a, S_c)
+        assert 0 < tot < 2e-2
+
+
 def _tiny_ffn_group(lengths, D=48, H=2, dk=8, dv=8, L=3, F=64, seed=11):
     layers = synth.la_layers(L, D, H, dk, dv, seed=seed, std=0.2, with_gain=True, d_ff=F)
     h = torch.cat([synth.hidden_prefix(n, D, seed + i) for i, n in enumerate(lengths)])
