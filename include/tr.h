@@ -180,6 +180,10 @@ tr_status tr_transition_product(const tr_scan_args *args, float *P, void *ws, si
  * Per LA layer (the pages give no layer internals; this is the reading used):
  *   x_hat = bf16(RMSNorm(x) * gain)            eps = rms_eps (0 -> 1e-6)
  *   [q|k|v|a_alpha|a_beta] = x_hat W_in^T      fp32 accumulate
+ *     (for the layers after the first the norm is computed inside the residual GEMM
+ *     before the layer and the projection: x_hat = bf16(x * gain) and the projection's
+ *     outputs are multiplied by the row's 1 / sqrt(mean x^2 + rms_eps); the same value,
+ *     the bf16 rounding taken before the scale)
  *   q, k <- bf16(x / sqrt(sum x^2 + norm_eps)) per head (norm_eps 0 -> 1e-6)
  *   v <- bf16(v); log alpha = -softplus(a_alpha), beta = sigmoid(a_beta) (fp32)
  *   o, S_hat[layer] = tr_gdn_scan(q, k, v, log alpha, beta), zero start
@@ -270,8 +274,8 @@ tr_status tr_replay_group(const tr_group_args *args, void *ws, size_t ws_bytes, 
  * The same replay with timing marks: `events` is a HOST array of n_events
  * created cudaEvent_t handles (passed as void*).  events[0] is recorded on
  * `stream` before the first kernel and events[i] after the i-th kernel launch,
- * in launch order (per layer: RMSNorm, input projection, scan, then the output
- * projection when it runs).  n_events must be at least
+ * in launch order (the first layer's RMSNorm, then per layer the input projection,
+ * the scan, and the output projection when it runs).  n_events must be at least
  * 1 + tr_replay_group_kernel_count(args); the rest are left alone.
  */
 int32_t tr_replay_group_kernel_count(const tr_group_args *args);
@@ -368,7 +372,8 @@ tr_status tr_state_error_noalloc(const float *S, const float *S_hat, int64_t n_m
 /*
  * ---------------------------------------------- steps of one LA layer, alone
  * The three dense steps of tr_replay_group, exposed so that each can be checked
- * on its own.  Same arithmetic and cast points as inside tr_replay_group.
+ * on its own.  Same arithmetic and cast points as inside tr_replay_group (the
+ * group's first layer: its later layers fold the RMSNorm into the GEMMs, see above).
  *
  * tr_rmsnorm: x_hat[t] = bf16(x[t] / sqrt(mean_j x[t,j]^2 + eps) * gain)
  *   x [n_rows, D] of x_dtype (bf16 or fp32); gain [D] fp32 or NULL;
