@@ -87,6 +87,25 @@ def test_kernel_rooflines_aggregate_one_step():
         assert v["us_per_step"] > 0
 
 
+def test_kernel_rooflines_with_the_folded_norm():
+    """The step as launched now: the first layer's RMSNorm only (the later layers' is folded
+    into the residual GEMM before them), then per layer the projection, the fused scan and
+    (but for the last) the output projection.  Layers still count from the projections: the
+    last one's projection and scan use the last layer's work."""
+    names = ["rmsnorm"]
+    for l in range(L):
+        names += ["in_proj", "scan_fused"] + (["out_proj"] if l < L - 1 else [])
+    avg_ms = [0.01 * (i + 1) for i in range(len(names))]
+    r = bench.kernel_rooflines(names, avg_ms, K, {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0})
+    assert r["rmsnorm"]["launches_per_step"] == 1
+    assert r["rmsnorm"]["bytes_per_launch"] == K * D * (2 + 2)    # bf16 h in, bf16 out
+    fl = (L - 1) * bench.flops_inproj(K, False) + bench.flops_inproj(K, True)
+    assert r["in_proj"]["flops_per_launch"] == pytest.approx(fl / L)
+    by = sum(bench.kernel_work("scan_fused", l, K)[1] for l in range(L))
+    assert r["scan_fused"]["bytes_per_launch"] == pytest.approx(by / L)
+    assert bench.kernel_work("scan_fused", L - 1, K)[1] < bench.kernel_work("scan_fused", 0, K)[1]
+
+
 def test_job_throughput_is_all_ranks_over_the_slowest():
     assert bench.job_throughput(K, 4, 2.0) == pytest.approx(4 * K / 2e-3)
 
